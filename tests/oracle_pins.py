@@ -1,0 +1,409 @@
+"""Pins for the oracle: checks against what the pages and the mathematics fix, not
+against the oracle's own formulas.
+
+Each ``pin_*(impl)`` raises ``AssertionError`` when ``impl`` is wrong.  The pins are:
+
+* closed-form groups whose scale, zero and codes follow by hand (exact grids, exact
+  half-way ties, clamped zero points, constant groups, each bit-width);
+* brute force: for tiny random groups, enumeration of all 2^b reconstruction levels
+  in exact rational arithmetic must give the same code as the RTN formula (the
+  VBQ/CellFill codes are nearest-level codes);
+* the invariants the CellFill abstract states: dequantize -> requantize returns the
+  codes; a zero or projected residual leaves the artifact bit-identical; dropping the
+  residual revokes exactly; drift stays within the cell;
+* a negative control whose mismatch count is predicted in exact rational arithmetic;
+* layout facts of packed storage (LSB-first codes, plain nibbles for 4-bit);
+* the fp64 matmul against NumPy's BLAS and closed forms.
+"""
+from fractions import Fraction
+
+import numpy as np
+
+GROUP = 64
+
+
+def _f16(bits):
+    return float(np.uint16(bits).view(np.float16))
+
+
+def _q1(impl, w, b):
+    """quantize one 64-weight group of width b."""
+    w = np.asarray(w, np.float32).reshape(1, GROUP)
+    codes, scale, zero, st = impl.quantize(w, np.array([b], np.uint8))
+    return codes, int(scale[0]), int(zero[0]), st
+
+
+def _expect(impl, w, b, s16, z, q):
+    codes, s, zz, st = _q1(impl, w, b)
+    assert st == 0, f"status {st}"
+    assert s == s16, f"scale {s:#06x} != {s16:#06x}"
+    assert zz == z, f"zero {zz} != {z}"
+    assert np.array_equal(codes, np.asarray(q, np.uint8)), f"codes {codes.tolist()} != {list(q)}"
+
+
+def _fill(vals, rest):
+    w = np.full(GROUP, rest, np.float32)
+    w[:len(vals)] = vals
+    return w
+
+
+# ---- closed-form quantize cases ------------------------------------------------------------
+
+def pin_quant_exact_grid(impl):
+    # w_i = 0.25*(i mod 16) - 2: wmin=-2, wmax=1.75, range/15 = 0.25 exactly (fp16 0x3400),
+    # z = rne(2/0.25) = 8, q_i = (i mod 16) - 8 + 8 = i mod 16.
+    i = np.arange(GROUP)
+    w = (0.25 * (i % 16) - 2.0).astype(np.float32)
+    _expect(impl, w, 4, 0x3400, 8, i % 16)
+
+
+def pin_quant_ties_half_even(impl):
+    # wmin=0, wmax=3.75 -> s=0.25, z=0; w/s lands exactly on .5: 2.5->2, 3.5->4, 0.5->0,
+    # 1.5->2, 14.5->14, 13.5->14, 4.5->4, 5.5->6; the filler 1.0 -> 4.
+    w = _fill([0.0, 3.75, 0.625, 0.875, 0.125, 0.375, 3.625, 3.375, 1.125, 1.375], 1.0)
+    q = [0, 15, 2, 4, 0, 2, 14, 14, 4, 6] + [4] * 54
+    _expect(impl, w, 4, 0x3400, 0, q)
+
+
+def pin_quant_zero_tie(impl):
+    # wmin=-0.625, wmax=3.125 -> s=0.25; z = rne(2.5) = 2.  -2.5->-2 (q 0), -1.5->-2 (q 0),
+    # -0.5->0 (q 2), 0.5->0 (q 2), 12.5->12 (q 14), 1.5->2 (q 4); filler 0 -> q 2.
+    w = _fill([-0.625, 3.125, -0.375, -0.125, 0.125, 0.375], 0.0)
+    q = [0, 14, 0, 2, 2, 4] + [2] * 58
+    _expect(impl, w, 4, 0x3400, 2, q)
+
+
+def pin_quant_clamped_zero(impl):
+    # all positive: range 1.875 -> s=0.125 (0x3000); z = rne(-8) -> clamp 0;
+    # 1->8, 2.875->23->15, 1.5->12, 2->16->15, filler 1.25->10.
+    w = _fill([1.0, 2.875, 1.5, 2.0], 1.25)
+    _expect(impl, w, 4, 0x3000, 0, [8, 15, 12, 15] + [10] * 60)
+    # all negative: z = rne(23) -> clamp 15; -1->7, -2.875->-8->0, -1.5->3, -2->-1->0, -1.25->5.
+    _expect(impl, -w, 4, 0x3000, 15, [7, 0, 3, 0] + [5] * 60)
+
+
+def pin_quant_constant_groups(impl):
+    # range 0 -> s floors at 2^-14 (0x0400).  0.5: z = rne(-8192) -> 0, q = 8192 -> 15.
+    _expect(impl, np.full(GROUP, 0.5, np.float32), 4, 0x0400, 0, [15] * GROUP)
+    _expect(impl, np.zeros(GROUP, np.float32), 4, 0x0400, 0, [0] * GROUP)
+    _expect(impl, np.full(GROUP, -0.5, np.float32), 4, 0x0400, 15, [0] * GROUP)
+
+
+def pin_quant_each_width(impl):
+    # 1 bit: w in {-1, 3}: s = 4/1 = 4 (0x4400), z = rne(0.25) = 0, q(-1)=rne(-0.25)=0, q(3)=rne(0.75)=1
+    w = np.tile(np.array([-1.0, 3.0], np.float32), 32)
+    _expect(impl, w, 1, 0x4400, 0, np.tile([0, 1], 32))
+    # 1 bit: w in {-1, 1}: s = 2 (0x4000), z = rne(0.5) = 0 (tie to even), q = rne(+-0.5) = 0
+    _expect(impl, np.tile(np.array([-1.0, 1.0], np.float32), 32), 1, 0x4000, 0, [0] * GROUP)
+    # 2 bits: {-0.75,-0.25,0.25,0.75}: s = 1.5/3 = 0.5 (0x3800), z = rne(1.5) = 2;
+    # q = -2+2, 0+2, 0+2, 2+2->3
+    w = np.tile(np.array([-0.75, -0.25, 0.25, 0.75], np.float32), 16)
+    _expect(impl, w, 2, 0x3800, 2, np.tile([0, 2, 2, 3], 16))
+    # 8 bits: w_j = v_j / 256 with v = 4j and v_63 = 255: s = (255/256)/255 = 2^-8 (0x1C00), z = 0,
+    # q_j = v_j
+    v = 4 * np.arange(GROUP)
+    v[63] = 255
+    _expect(impl, (v / 256.0).astype(np.float32), 8, 0x1C00, 0, v)
+
+
+def pin_quant_fp16_scale_rounding(impl):
+    # range 1: RN32(1/15) rounds to fp16 0x2C44 = 0.066650390625 (1/15*1024/0.0625... hand:
+    # 1/15 = 0.0625 * 1.0666.., mantissa 0.0666..*1024 = 68.27 -> 68).  z = rne(0.5/s) =
+    # rne(7.5018) = 8; q(0.5) = 8+8 -> 15, q(-0.5) = 0, q(0) = 8, q(0.1) = rne(1.50037)+8 = 10.
+    w = _fill([-0.5, 0.5, 0.1], 0.0)
+    _expect(impl, w, 4, 0x2C44, 8, [0, 15, 10] + [8] * 61)
+
+
+def pin_quant_status(impl):
+    w = np.zeros((4, GROUP), np.float32)
+    w[0, 5] = np.nan
+    w[1, 7] = np.inf
+    w[2, 0], w[2, 1] = -3e38, 3e38            # range overflows binary32 -> scale overflow
+    w[3] = np.linspace(-1, 1, GROUP)
+    codes, scale, zero, st = impl.quantize(w.reshape(1, -1), np.array([4, 4, 4, 4], np.uint8))
+    assert st == 1 | 2, st
+    assert scale[:3].tolist() == [0, 0, 0] and zero[:3].tolist() == [0, 0, 0]
+    assert not codes[:3 * GROUP].any() and scale[3] != 0
+    codes, scale, zero, st = impl.quantize(w[3:].reshape(1, -1), np.array([3], np.uint8))
+    assert st == 4 and scale[0] == 0
+
+
+# ---- brute force against all 2^b levels (exact rationals) -----------------------------------
+
+def _tiny_groups(rng, n):
+    out = []
+    for t in range(n):
+        kind = t % 5
+        if kind == 0:
+            w = rng.standard_normal(GROUP) * 0.02
+        elif kind == 1:
+            w = rng.uniform(-1, 1, GROUP) * 10.0 ** rng.integers(-3, 3)
+        elif kind == 2:
+            w = rng.standard_t(3, GROUP) * 0.05
+        elif kind == 3:
+            w = rng.uniform(0.1, 0.3, GROUP)          # all positive
+        else:
+            w = np.round(rng.standard_normal(GROUP) * 8) / 32.0   # many duplicates
+        out.append(w.astype(np.float32))
+    return out
+
+
+def pin_quant_bruteforce(impl, n_groups=60, seed=1234):
+    rng = np.random.default_rng(seed)
+    near_ties = 0
+    for idx, w in enumerate(_tiny_groups(rng, n_groups)):
+        b = (1, 2, 4, 8)[idx % 4]
+        L = (1 << b) - 1
+        codes, s16, z, st = _q1(impl, w, b)
+        assert st == 0
+        S = Fraction(_f16(s16))
+        W = [Fraction(float(v)) for v in w]
+        # scale: within half an fp16 ulp (plus one binary32 rounding) of range/L, floored at 2^-14
+        exact = (max(W) - min(W)) / L
+        if exact >= Fraction(1, 2 ** 14):
+            e = Fraction(2) ** (int(np.floor(np.log2(float(exact)))) - 10)
+            assert abs(S - exact) <= e / 2 + exact / 2 ** 23, (float(S), float(exact))
+        else:
+            assert S == Fraction(1, 2 ** 14) or abs(S - exact) <= Fraction(1, 2 ** 24)
+        # zero point: nearest integer to -wmin/S, clamped
+        zt = -min(W) / S
+        zr = int(np.floor(float(zt) + 0.5))
+        if abs(zt - Fraction(2 * int(np.floor(float(zt))) + 1, 2)) > Fraction(1, 2 ** 20):
+            assert z == min(max(zr, 0), L), (z, float(zt))
+        # codes: exhaustive nearest level among the 2^b levels S*(j - z)
+        for i, wi in enumerate(W):
+            dists = [abs(wi - S * (j - z)) for j in range(L + 1)]
+            best = min(dists)
+            arg = [j for j in range(L + 1) if dists[j] == best]
+            t = wi / S
+            half = Fraction(2 * int(np.floor(float(t))) + 1, 2)
+            if abs(t - half) <= abs(t) / 2 ** 22 + Fraction(1, 2 ** 40):
+                near_ties += 1
+                assert int(codes[i]) in (min(max(int(np.floor(float(t))) + z, 0), L),
+                                         min(max(int(np.floor(float(t))) + 1 + z, 0), L))
+                continue
+            assert int(codes[i]) in arg, (b, i, float(wi), float(S), z, int(codes[i]), arg)
+    return near_ties
+
+
+def pin_quant_min_maps_to_zero(impl, seed=7):
+    # rne(a) + rne(-a) = 0, so the group minimum lands on code 0 whenever z is not clamped.
+    rng = np.random.default_rng(seed)
+    w = (rng.standard_normal((64, GROUP)) * 0.02).astype(np.float32)
+    codes, scale, zero, _ = impl.quantize(w, np.full(64, 4, np.uint8))
+    codes = codes.reshape(64, GROUP)
+    for g in range(64):
+        sf = Fraction(_f16(scale[g]))
+        zt = -Fraction(float(w[g].min())) / sf
+        if 0 < zt < 15:
+            assert codes[g, int(np.argmin(w[g]))] == 0
+
+
+def pin_quant_reconstruction_error(impl, seed=11):
+    # |w - s(q - z)| <= s/2 (+ binary32 rounding) for every code that is not clamped.
+    rng = np.random.default_rng(seed)
+    w = (rng.standard_t(5, (128, GROUP)) * 0.02).astype(np.float32)
+    codes, scale, zero, _ = impl.quantize(w, np.full(128, 4, np.uint8))
+    s = np.asarray(scale, np.uint16).view(np.float16).astype(np.float64)[:, None]
+    q = codes.reshape(128, GROUP).astype(np.float64)
+    err = np.abs(w.astype(np.float64) - s * (q - zero[:, None]))
+    inner = (q > 0) & (q < 15)
+    assert (err[inner] <= s.repeat(GROUP, 1)[inner] * (0.5 + 2 ** -20)).all()
+
+
+# ---- packed storage ------------------------------------------------------------------------
+
+def pin_pack_lsb_first(impl):
+    # b=2: codes 1,2,3,0 -> byte 0 = 1 | 2<<2 | 3<<4 | 0<<6 = 0x39;  b=1: 0,1,0,1.. -> 0xAA;
+    # b=8: bytes are the codes; b=4: low nibble first.
+    codes = np.zeros((4, GROUP), np.uint8)
+    codes[0] = np.tile([0, 1], 32)
+    codes[1, :4] = [1, 2, 3, 0]
+    codes[2, :2] = [0xA, 0x5]
+    codes[3] = np.arange(GROUP) * 3
+    bits = np.array([1, 2, 4, 8], np.uint8)
+    planes = impl.pack(codes.ravel(), bits)
+    assert planes[0][:8].tolist() == [0xAA] * 8
+    assert planes[1][0] == 0x39 and not planes[1][1:16].any()
+    assert planes[2][0] == 0x5A and not planes[2][1:32].any()
+    assert planes[3][:64].tolist() == (np.arange(GROUP) * 3).tolist()
+
+
+def pin_pack_fixed4_is_plain_nibbles(impl, seed=3):
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 16, 8 * 256, dtype=np.uint8)
+    planes = impl.pack(codes, None)
+    expect = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)
+    assert np.array_equal(planes[2][:expect.size], expect)
+    assert np.array_equal(impl.unpack(planes, codes.size // GROUP, None), codes)
+
+
+def pin_pack_roundtrip_and_totals(impl, seed=5):
+    rng = np.random.default_rng(seed)
+    G = 777
+    bits = rng.choice(np.array([1, 2, 4, 8], np.uint8), G, p=[0.69, 0.15, 0.12, 0.04])
+    codes = (rng.integers(0, 256, G * GROUP) & ((1 << bits.repeat(GROUP).astype(np.int64)) - 1)).astype(np.uint8)
+    off, pbytes = impl.varbits_index(bits)
+    for slot, b in enumerate((1, 2, 4, 8)):
+        sel = bits == b
+        assert pbytes[slot] == 8 * b * int(sel.sum())
+        o = np.sort(np.asarray(off)[sel].astype(np.int64))
+        assert np.array_equal(o, 8 * b * np.arange(sel.sum()))
+    planes = impl.pack(codes, bits)
+    assert np.array_equal(impl.unpack(planes, G, bits), codes)
+
+
+# ---- the CellFill invariants -------------------------------------------------------------------
+
+def _random_artifact(rng, G, bits=None, subnormal_scales=False):
+    b = np.full(G, 4, np.int64) if bits is None else np.asarray(bits, np.int64)
+    L = (1 << b) - 1
+    codes = (rng.integers(0, 256, (G, GROUP)) % (L[:, None] + 1)).astype(np.uint8)
+    zero = (rng.integers(0, 256, G) % (L + 1)).astype(np.uint8)
+    if subnormal_scales:
+        scale = rng.integers(1, 0x7BFF, G).astype(np.uint16)      # every positive finite fp16
+    else:
+        scale = np.asarray(rng.uniform(1e-3, 1e-1, G), np.float16).view(np.uint16)
+    return codes.ravel(), scale.astype(np.uint16), zero
+
+
+def pin_roundtrip_dequant_requant(impl, seed=21):
+    # W = s(q - z) is exact, and (s k)/s = k exactly: requantizing returns every code.
+    rng = np.random.default_rng(seed)
+    for bits in (None, rng.choice(np.array([1, 2, 4, 8], np.uint8), 300)):
+        G = 300
+        codes, scale, zero = _random_artifact(rng, G, bits, subnormal_scales=True)
+        planes = impl.pack(codes, bits)
+        m, fb, mask = impl.verify(planes, scale, zero, bits)
+        assert m == 0 and fb == -1 and not mask.any()
+        m, fb, _ = impl.verify(planes, scale, zero, bits, r=np.zeros(G * GROUP, np.float32))
+        assert m == 0 and fb == -1
+
+
+def _boundary_residuals(rng, scale):
+    sf = np.asarray(scale, np.uint16).view(np.float16).astype(np.float32)
+    G = sf.size
+    mult = rng.uniform(-3, 3, (G, GROUP)).astype(np.float32)
+    mult[:, 0] = 0.5
+    mult[:, 1] = -0.5
+    mult[:, 2] = 0.5 - 2 ** -10
+    mult[:, 3] = 0.5 + 2 ** -10
+    mult[:, 4] = 1e30
+    mult[:, 5] = -1e30
+    return (mult * sf[:, None]).astype(np.float32).ravel()
+
+
+def pin_projected_residual_f32(impl, seed=31):
+    rng = np.random.default_rng(seed)
+    G = 400
+    codes, scale, zero = _random_artifact(rng, G)
+    planes = impl.pack(codes, None)
+    r = _boundary_residuals(rng, scale)
+    rp, n = impl.project_f32(r, scale)
+    sf = np.asarray(scale, np.uint16).view(np.float16).astype(np.float64).repeat(GROUP)
+    bound = (0.5 - 2 ** -10) * sf
+    assert (np.abs(rp.astype(np.float64)) <= bound).all()                    # drift bounded
+    inside = np.abs(r.astype(np.float64)) <= bound
+    assert np.array_equal(rp[inside].view(np.uint32), r[inside].view(np.uint32))
+    assert n == int((~inside).sum())
+    m, fb, _ = impl.verify(planes, scale, zero, None, r=rp)
+    assert m == 0 and fb == -1
+    m, fb, _ = impl.verify(planes, scale, zero, None)                         # revoke
+    assert m == 0 and fb == -1
+
+
+def pin_projected_residual_bf16(impl, seed=41):
+    rng = np.random.default_rng(seed)
+    G = 2000
+    codes, scale, zero = _random_artifact(rng, G, subnormal_scales=False)
+    scale = rng.integers(0x0400, 0x7800, G).astype(np.uint16)   # wide spread of fp16 mantissas
+    planes = impl.pack(codes, None)
+    r = _boundary_residuals(rng, scale)
+    rb = (r.view(np.uint32) >> 16).astype(np.uint16)           # any bf16 values
+    rp, n = impl.project_bf16(rb, scale)
+    sf = np.asarray(scale, np.uint16).view(np.float16).astype(np.float64).repeat(GROUP)
+    rv = (rp.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert (np.abs(rv) <= (0.5 - 2 ** -10) * sf).all()
+    assert (np.abs(rv).reshape(G, GROUP).max(axis=1) >= 0.4952 * sf[::GROUP]).all()
+    m, fb, _ = impl.verify(planes, scale, zero, None, r=rp, r_dtype="bf16")
+    assert m == 0 and fb == -1
+
+
+def _expected_mismatch(codes, scale, zero, bits, r_f64):
+    """Exact-rational prediction of the requant decision, away from rounding ties."""
+    G = scale.size
+    b = np.full(G, 4, np.int64) if bits is None else np.asarray(bits, np.int64)
+    L = ((1 << b) - 1).repeat(GROUP)
+    sf = np.asarray(scale, np.uint16).view(np.float16).astype(np.float64).repeat(GROUP)
+    z = np.asarray(zero, np.int64).repeat(GROUP)
+    q = np.asarray(codes, np.int64)
+    t = (q - z) + r_f64 / sf                          # exact to ~1e-16 in binary64
+    frac = t - np.floor(t)
+    tie = np.abs(frac - 0.5) < 2 ** -12
+    qp = np.clip(np.floor(t + 0.5).astype(np.int64) + z, 0, L)
+    return qp != q, tie
+
+
+def pin_negative_control(impl, seed=51):
+    # unprojected residuals: the predicted count (exact arithmetic, far from ties) must match
+    rng = np.random.default_rng(seed)
+    for bits in (None, rng.choice(np.array([1, 2, 4, 8], np.uint8), 500)):
+        G = 500
+        codes, scale, zero = _random_artifact(rng, G, bits)
+        planes = impl.pack(codes, bits)
+        sf = np.asarray(scale, np.uint16).view(np.float16).astype(np.float32)
+        u = rng.uniform(-0.6, 0.6, (G, GROUP)).astype(np.float32)
+        for lim in (0.5, -0.5):
+            near = np.abs(u - lim) < 1e-3
+            u[near] = 0.0
+        r = (u * sf[:, None]).astype(np.float32).ravel()
+        bad, tie = _expected_mismatch(codes, scale, zero, bits, r.astype(np.float64))
+        assert not tie.any()
+        m, fb, mask = impl.verify(planes, scale, zero, bits, r=r)
+        assert m == int(bad.sum()) and m > 0
+        assert fb == int(np.argmax(bad))
+        assert np.array_equal(mask, bad.reshape(G, GROUP).any(axis=1))
+
+
+def pin_bad_scale_flags(impl):
+    codes = np.full(4 * GROUP, 3, np.uint8)
+    scale = np.array([0x0000, 0x7C00, 0x7E00, 0x3C00], np.uint16)   # 0, inf, NaN, 1.0
+    zero = np.array([1, 1, 1, 1], np.uint8)
+    planes = impl.pack(codes, None)
+    m, fb, mask = impl.verify(planes, scale, zero, None)
+    assert m == 3 * GROUP and fb == 0 and mask.tolist() == [True, True, True, False]
+
+
+# ---- fp64 dequantize-and-multiply ------------------------------------------------------------
+
+def pin_matmul(impl, seed=61):
+    rng = np.random.default_rng(seed)
+    rows, cols = 24, 192
+    G = rows * cols // GROUP
+    bits = rng.choice(np.array([1, 2, 4, 8], np.uint8), G)
+    codes, scale, zero = _random_artifact(rng, G, bits)
+    planes = impl.pack(codes, bits)
+    r = rng.standard_normal(rows * cols).astype(np.float32) * 1e-3
+    x = rng.standard_normal((3, cols)).astype(np.float32)
+    y = impl.dequant_matmul_f64(planes, scale, zero, rows, cols, x, "f32", bits, r)
+    # independent dense construction + BLAS
+    sf = np.asarray(scale, np.uint16).view(np.float16).astype(np.float64)
+    W = (sf[:, None] * (codes.reshape(G, GROUP).astype(np.float64) - zero[:, None])).reshape(rows, cols)
+    W = W + r.reshape(rows, cols)
+    ref = x.astype(np.float64) @ W.T
+    assert y.shape == (3, rows)
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+    # closed forms: x = e_k picks column k of W; codes == zero gives exactly r.x
+    for k in (0, 63, 64, cols - 1):
+        e = np.zeros((1, cols), np.float32)
+        e[0, k] = 1.0
+        yk = impl.dequant_matmul_f64(planes, scale, zero, rows, cols, e, "f32", bits, r)
+        assert np.array_equal(yk[0], W[:, k])
+    flat = np.asarray(zero).repeat(GROUP).astype(np.uint8)
+    planes0 = impl.pack(flat, bits)
+    y0 = impl.dequant_matmul_f64(planes0, scale, zero, rows, cols, x, "f32", bits, r)
+    assert np.allclose(y0, x.astype(np.float64) @ r.reshape(rows, cols).astype(np.float64).T,
+                       rtol=1e-12, atol=1e-15)
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
