@@ -1,0 +1,305 @@
+// k_pack.cu -- packed low-bit storage for per-group widths.
+//
+// [VBQ] "In-Cell Learning: Language Models That Update Their Own Weights in Sequence
+// Without Changing the File They Ship", abstract: the per-group allocation maps directly
+// to packed low-bit storage. The layout (one plane per width, row-major rank of the group
+// among groups of its width, LSB-first codes) is defined in include/cq.h.
+//
+// Work unit: eight lanes per group, one lane per eight consecutive codes. Lane `sub` of a
+// group of width b owns exactly b bytes of the plane (8 codes * b bits), so packing and
+// unpacking are single stores/loads of 1, 2, 4 or 8 bytes with no read-modify-write.
+#include "cq_internal.cuh"
+
+namespace cq {
+namespace {
+
+constexpr int kThreads = 256;
+
+// 8 codes (one per byte of v) -> 8*b bits, code j at bits [j*b, (j+1)*b)
+__device__ __forceinline__ uint64_t pack8(uint64_t v, int b) {
+  uint64_t out = 0;
+  const uint64_t mask = (1ull << b) - 1ull;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) out |= ((v >> (8 * j)) & mask) << (j * b);
+  return out;
+}
+
+__device__ __forceinline__ uint64_t unpack8(uint64_t p, int b) {
+  uint64_t out = 0;
+  const uint64_t mask = (1ull << b) - 1ull;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) out |= ((p >> (j * b)) & mask) << (8 * j);
+  return out;
+}
+
+__device__ __forceinline__ void store_bytes(uint8_t *dst, uint64_t v, int b) {
+  switch (b) {
+    case 1: *dst = static_cast<uint8_t>(v); break;
+    case 2: *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(v); break;
+    case 4: *reinterpret_cast<uint32_t *>(dst) = static_cast<uint32_t>(v); break;
+    default: *reinterpret_cast<uint2 *>(dst) = make_uint2(static_cast<uint32_t>(v), static_cast<uint32_t>(v >> 32)); break;
+  }
+}
+
+__device__ __forceinline__ uint64_t load_bytes(const uint8_t *src, int b) {
+  switch (b) {
+    case 1: return __ldg(src);
+    case 2: return __ldg(reinterpret_cast<const uint16_t *>(src));
+    case 4: return __ldg(reinterpret_cast<const uint32_t *>(src));
+    default: {
+      const uint2 t = __ldg(reinterpret_cast<const uint2 *>(src));
+      return static_cast<uint64_t>(t.x) | (static_cast<uint64_t>(t.y) << 32);
+    }
+  }
+}
+
+struct Planes {
+  uint8_t *p[4];
+};
+
+__global__ void __launch_bounds__(kThreads)
+pack_kernel(const uint8_t *__restrict__ codes, int64_t n_units, const uint8_t *__restrict__ bits,
+            const uint32_t *__restrict__ offset, Planes planes) {
+  for (int64_t u = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; u < n_units;
+       u += static_cast<int64_t>(gridDim.x) * kThreads) {
+    const int64_t g = u >> 3;
+    const int sub = static_cast<int>(u & 7);
+    const uint2 c = __ldcs(reinterpret_cast<const uint2 *>(codes) + u);
+    const uint64_t v = static_cast<uint64_t>(c.x) | (static_cast<uint64_t>(c.y) << 32);
+    int b = 4;
+    uint8_t *base;
+    if (bits) {
+      b = __ldg(bits + g);
+      if (!width_ok(b)) continue;   // nothing to store; quantize reports the width
+      base = planes.p[width_slot(b)] + __ldg(offset + g);
+    } else {
+      base = planes.p[2] + g * 32;
+    }
+    store_bytes(base + sub * b, pack8(v, b), b);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+unpack_kernel(uint8_t *__restrict__ codes, int64_t n_units, const uint8_t *__restrict__ bits,
+              const uint32_t *__restrict__ offset, Planes planes) {
+  for (int64_t u = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; u < n_units;
+       u += static_cast<int64_t>(gridDim.x) * kThreads) {
+    const int64_t g = u >> 3;
+    const int sub = static_cast<int>(u & 7);
+    int b = 4;
+    const uint8_t *base;
+    uint64_t v = 0;
+    if (bits) {
+      b = __ldg(bits + g);
+      if (width_ok(b)) {
+        base = planes.p[width_slot(b)] + __ldg(offset + g);
+        v = unpack8(load_bytes(base + sub * b, b), b);
+      }
+    } else {
+      base = planes.p[2] + g * 32;
+      v = unpack8(load_bytes(base + sub * 4, 4), 4);
+    }
+    reinterpret_cast<uint2 *>(codes)[u] = make_uint2(static_cast<uint32_t>(v), static_cast<uint32_t>(v >> 32));
+  }
+}
+
+// ---- group -> byte offset index: three passes, no scratch beyond the offset array ------
+//
+// pass 1: every full tile but the last writes its four width counts into the first four
+//         offset slots of its own range;
+// pass 2: one block turns those counts into exclusive prefixes in place, counts the last
+//         tile itself and writes the plane sizes;
+// pass 3: every tile reads its four bases (before any thread overwrites them) and writes
+//         the offsets of its groups. A tile only ever touches its own slots across passes.
+constexpr int kIndexThreads = 512;
+constexpr int kIndexPer = 8;
+constexpr int64_t kTile = kIndexThreads * kIndexPer;  // 4096 groups
+
+__device__ __forceinline__ uint64_t width_onehot16(int b) {
+  // one 16-bit counter field per width slot
+  return width_ok(b) ? (1ull << (16 * width_slot(b))) : 0ull;
+}
+
+// counts of the (up to) kIndexPer groups this thread owns in tile t, packed 4 x 16 bits
+__device__ __forceinline__ uint64_t thread_counts(const uint8_t *bits, int64_t G, int64_t t,
+                                                  int tid, int widths[kIndexPer]) {
+  uint64_t c = 0;
+  const int64_t g0 = t * kTile + static_cast<int64_t>(tid) * kIndexPer;
+#pragma unroll
+  for (int j = 0; j < kIndexPer; ++j) {
+    const int64_t g = g0 + j;
+    widths[j] = g < G ? static_cast<int>(__ldg(bits + g)) : 0;
+    c += width_onehot16(widths[j]);
+  }
+  return c;
+}
+
+// exclusive scan of a packed 4x16-bit counter over the block; returns the block total too
+__device__ __forceinline__ uint64_t block_exclusive_scan(uint64_t v, uint64_t *total) {
+  __shared__ uint64_t warp_sums[kIndexThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint64_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint64_t s = lane < kIndexThreads / 32 ? warp_sums[lane] : 0;
+    uint64_t si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t n = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += n;
+    }
+    if (lane < kIndexThreads / 32) warp_sums[lane] = si - s;   // exclusive warp prefix
+  }
+  __syncthreads();
+  const uint64_t excl = warp_sums[warp] + incl - v;
+  // total = exclusive prefix of the last thread + its own value
+  __shared__ uint64_t tot;
+  if (threadIdx.x == kIndexThreads - 1) tot = excl + v;
+  __syncthreads();
+  *total = tot;
+  __syncthreads();
+  return excl;
+}
+
+__device__ __forceinline__ uint32_t field16(uint64_t v, int slot) {
+  return static_cast<uint32_t>((v >> (16 * slot)) & 0xFFFFu);
+}
+
+__global__ void __launch_bounds__(kIndexThreads)
+index_count_kernel(const uint8_t *__restrict__ bits, int64_t G, uint32_t *__restrict__ offset) {
+  const int64_t t = blockIdx.x;   // a full tile that is not the last one
+  int widths[kIndexPer];
+  uint64_t total;
+  block_exclusive_scan(thread_counts(bits, G, t, threadIdx.x, widths), &total);
+  if (threadIdx.x < 4) offset[t * kTile + threadIdx.x] = field16(total, threadIdx.x);
+}
+
+__global__ void __launch_bounds__(kIndexThreads)
+index_scan_kernel(const uint8_t *__restrict__ bits, int64_t G, int64_t n_tiles,
+                  uint32_t *__restrict__ offset, uint64_t *__restrict__ plane_bytes) {
+  // prefix over the first n_tiles-1 tiles, 32-bit counts (G <= 2^26 keeps them exact)
+  __shared__ uint32_t base[4];
+  if (threadIdx.x < 4) base[threadIdx.x] = 0;
+  __syncthreads();
+  const int64_t full = n_tiles - 1;
+  for (int64_t c0 = 0; c0 < full; c0 += kIndexThreads) {
+    const int64_t t = c0 + threadIdx.x;
+    uint32_t cnt[4] = {0, 0, 0, 0};
+    if (t < full)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) cnt[w] = offset[t * kTile + w];
+    // two 64-bit scans with 32-bit fields (prefix <= 2^26)
+    uint64_t lo = cnt[0] | (static_cast<uint64_t>(cnt[1]) << 32);
+    uint64_t hi = cnt[2] | (static_cast<uint64_t>(cnt[3]) << 32);
+    uint64_t tlo, thi;
+    // reuse the 4x16 scan machinery on 2x32 fields: additions never carry between fields
+    const uint64_t elo = block_exclusive_scan(lo, &tlo);
+    const uint64_t ehi = block_exclusive_scan(hi, &thi);
+    if (t < full) {
+      offset[t * kTile + 0] = base[0] + static_cast<uint32_t>(elo);
+      offset[t * kTile + 1] = base[1] + static_cast<uint32_t>(elo >> 32);
+      offset[t * kTile + 2] = base[2] + static_cast<uint32_t>(ehi);
+      offset[t * kTile + 3] = base[3] + static_cast<uint32_t>(ehi >> 32);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      base[0] += static_cast<uint32_t>(tlo);
+      base[1] += static_cast<uint32_t>(tlo >> 32);
+      base[2] += static_cast<uint32_t>(thi);
+      base[3] += static_cast<uint32_t>(thi >> 32);
+    }
+    __syncthreads();
+  }
+  int widths[kIndexPer];
+  uint64_t last;
+  block_exclusive_scan(thread_counts(bits, G, n_tiles - 1, threadIdx.x, widths), &last);
+  if (threadIdx.x < 4) {
+    const int b = 1 << threadIdx.x;
+    plane_bytes[threadIdx.x] = static_cast<uint64_t>(base[threadIdx.x] + field16(last, threadIdx.x)) * 8u * b;
+  }
+}
+
+__global__ void __launch_bounds__(kIndexThreads)
+index_write_kernel(const uint8_t *__restrict__ bits, int64_t G, int64_t n_tiles,
+                   uint32_t *__restrict__ offset, const uint64_t *__restrict__ plane_bytes) {
+  const int64_t t = blockIdx.x;
+  int widths[kIndexPer];
+  uint64_t total;
+  const uint64_t excl = block_exclusive_scan(thread_counts(bits, G, t, threadIdx.x, widths), &total);
+  __shared__ uint32_t base[4];
+  if (threadIdx.x < 4) {
+    if (t < n_tiles - 1) {
+      base[threadIdx.x] = offset[t * kTile + threadIdx.x];
+    } else {
+      const uint32_t per = 8u << threadIdx.x;   // bytes per group of width 2^slot
+      base[threadIdx.x] = static_cast<uint32_t>(plane_bytes[threadIdx.x] / per) - field16(total, threadIdx.x);
+    }
+  }
+  __syncthreads();   // every base is read before any slot of this tile is overwritten
+  uint32_t run[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) run[w] = base[w] + field16(excl, w);
+  const int64_t g0 = t * kTile + static_cast<int64_t>(threadIdx.x) * kIndexPer;
+#pragma unroll
+  for (int j = 0; j < kIndexPer; ++j) {
+    const int64_t g = g0 + j;
+    if (g >= G) break;
+    const int b = widths[j];
+    if (width_ok(b)) {
+      const int sl = width_slot(b);
+      offset[g] = run[sl] * 8u * static_cast<uint32_t>(b);
+      run[sl] += 1;
+    } else {
+      offset[g] = 0;
+    }
+  }
+}
+
+int grid_for(int64_t units) {
+  const int64_t need = (units + kThreads - 1) / kThreads;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  return static_cast<int>(need < cap ? need : cap);
+}
+
+}  // namespace
+
+cq_status launch_varbits_index(const uint8_t *bits, int64_t G, uint32_t *offset,
+                               uint64_t *plane_bytes, cudaStream_t s) {
+  if (G == 0) return cuda_check(cudaMemsetAsync(plane_bytes, 0, 4 * sizeof(uint64_t), s), "cq_varbits_index");
+  const int64_t n_tiles = (G + kTile - 1) / kTile;
+  if (n_tiles > 1) {
+    index_count_kernel<<<static_cast<unsigned>(n_tiles - 1), kIndexThreads, 0, s>>>(bits, G, offset);
+    cq_status st = launch_check("cq_varbits_index: count");
+    if (st != CQ_OK) return st;
+  }
+  index_scan_kernel<<<1, kIndexThreads, 0, s>>>(bits, G, n_tiles, offset, plane_bytes);
+  cq_status st = launch_check("cq_varbits_index: scan");
+  if (st != CQ_OK) return st;
+  index_write_kernel<<<static_cast<unsigned>(n_tiles), kIndexThreads, 0, s>>>(bits, G, n_tiles, offset, plane_bytes);
+  return launch_check("cq_varbits_index: write");
+}
+
+cq_status launch_pack(const uint8_t *codes, int64_t G, const uint8_t *bits, const uint32_t *offset,
+                      uint8_t *const plane[4], cudaStream_t s) {
+  if (G == 0) return CQ_OK;
+  Planes P{{plane[0], plane[1], plane[2], plane[3]}};
+  pack_kernel<<<grid_for(G * 8), kThreads, 0, s>>>(codes, G * 8, bits, offset, P);
+  return launch_check("cq_pack_varbits");
+}
+
+cq_status launch_unpack(const cq_qweight &qw, uint8_t *codes, cudaStream_t s) {
+  const int64_t G = qw.rows * (qw.cols / kGroup);
+  if (G == 0) return CQ_OK;
+  Planes P{{const_cast<uint8_t *>(qw.plane[0]), const_cast<uint8_t *>(qw.plane[1]),
+            const_cast<uint8_t *>(qw.plane[2]), const_cast<uint8_t *>(qw.plane[3])}};
+  unpack_kernel<<<grid_for(G * 8), kThreads, 0, s>>>(codes, G * 8, qw.bits, qw.offset, P);
+  return launch_check("cq_unpack_varbits");
+}
+
+}  // namespace cq

@@ -1,0 +1,93 @@
+// k_project.cu -- projection of the per-weight residual into its quantization cell.
+//
+// [CF] "Nothing Changed but the Model: CellFill -- Bounded In-Cell Learning for
+// Bit-Identical, Revocable Updates to Quantized LLMs", Abstract: the residual must stay
+// strictly inside each decision cell; the constrained dense path projects into the cells.
+// Reading: half-width c = (0.5 - 2^-10) * s (exact in binary32: 9 x 11 significant bits);
+// a bf16 residual uses c rounded toward zero to bf16, so the clamp never rounds outward.
+// The clamp is written with comparisons so that a NaN residual passes through unchanged.
+//
+// Layout: one lane per eight residuals (one 16-byte load for bf16, two for fp32); eight
+// lanes share a group scale. Streaming, in place.
+#include "cq_internal.cuh"
+
+namespace cq {
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float cell_bound(uint16_t s16) {
+  return __fmul_rn(0.5f - 0x1p-10f, f16_bits_to_f32(s16));
+}
+
+__device__ __forceinline__ float clamp_cell(float r, float c) {
+  return r > c ? c : (r < -c ? -c : r);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads)
+project_kernel(void *__restrict__ rv, const uint16_t *__restrict__ scale, int64_t n_units,
+               unsigned long long *__restrict__ n_clamped) {
+  uint32_t changed = 0;
+  for (int64_t u = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; u < n_units;
+       u += static_cast<int64_t>(gridDim.x) * kThreads) {
+    const float c = cell_bound(__ldg(scale + (u >> 3)));
+    if (BF16) {
+      // c rounded toward zero to bf16: drop the low 16 bits (c >= 0 or NaN)
+      const float cb = __uint_as_float(__float_as_uint(c) & 0xFFFF0000u);
+      uint4 *p = reinterpret_cast<uint4 *>(rv) + u;
+      const uint4 in = __ldcs(p);
+      uint32_t w[4] = {in.x, in.y, in.z, in.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xFFFF0000u);
+        const uint32_t nlo = __float_as_uint(clamp_cell(lo, cb)) >> 16;
+        const uint32_t nhi = __float_as_uint(clamp_cell(hi, cb)) & 0xFFFF0000u;
+        const uint32_t nw = nlo | nhi;
+        changed += ((nw ^ w[j]) & 0xFFFFu) != 0;
+        changed += ((nw ^ w[j]) & 0xFFFF0000u) != 0;
+        w[j] = nw;
+      }
+      __stcs(p, make_uint4(w[0], w[1], w[2], w[3]));
+    } else {
+      float4 *p = reinterpret_cast<float4 *>(rv) + 2 * u;
+      float4 a = __ldcs(p), b = __ldcs(p + 1);
+      float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float o = clamp_cell(v[j], c);
+        changed += __float_as_uint(o) != __float_as_uint(v[j]);
+        v[j] = o;
+      }
+      __stcs(p, make_float4(v[0], v[1], v[2], v[3]));
+      __stcs(p + 1, make_float4(v[4], v[5], v[6], v[7]));
+    }
+  }
+  if (n_clamped) {
+    changed = __reduce_add_sync(0xffffffffu, changed);
+    if ((threadIdx.x & 31) == 0 && changed) atomicAdd(n_clamped, static_cast<unsigned long long>(changed));
+  }
+}
+
+}  // namespace
+
+cq_status launch_project(void *r, cq_dtype dt, const uint16_t *scale, int64_t n, uint64_t *n_clamped,
+                         cudaStream_t s) {
+  if (n_clamped) {
+    cq_status st = cuda_check(cudaMemsetAsync(n_clamped, 0, sizeof(uint64_t), s), "cq_project_residual: clear count");
+    if (st != CQ_OK) return st;
+  }
+  if (n == 0) return CQ_OK;
+  const int64_t units = n / 8;
+  const int64_t need = (units + kThreads - 1) / kThreads;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  const int blocks = static_cast<int>(need < cap ? need : cap);
+  auto *cnt = reinterpret_cast<unsigned long long *>(n_clamped);
+  if (dt == CQ_BF16)
+    project_kernel<true><<<blocks, kThreads, 0, s>>>(r, scale, units, cnt);
+  else
+    project_kernel<false><<<blocks, kThreads, 0, s>>>(r, scale, units, cnt);
+  return launch_check("cq_project_residual");
+}
+
+}  // namespace cq

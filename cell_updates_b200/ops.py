@@ -1,0 +1,100 @@
+"""Convenience wrappers over the C ABI: allocate the outputs with torch, then call libcq.
+
+No arithmetic of the method happens here; every value is produced by a libcq kernel.
+"""
+import torch
+
+from . import cq
+
+GROUP = 64
+
+
+def empty_u8(n, device):
+    return torch.empty(int(n), dtype=torch.uint8, device=device)
+
+
+def quantize(w, bits=None, stream=None):
+    """fp32 [rows, cols] on the GPU -> (codes u8 [rows*cols], scale int16 [G] (fp16 bits), zero u8 [G], status)."""
+    rows, cols = w.shape
+    G = rows * cols // GROUP
+    dev = w.device
+    codes = empty_u8(rows * cols, dev)
+    scale = torch.empty(G, dtype=torch.int16, device=dev)
+    zero = empty_u8(G, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    cq.cq_quantize(w, bits, codes, scale, zero, status, stream)
+    return codes, scale, zero, status
+
+
+def varbits_index(bits, stream=None):
+    """-> (offset int32 [G], plane_bytes list of 4 ints).  Reads plane_bytes back (synchronizes)."""
+    dev = bits.device
+    offset = torch.empty(bits.numel(), dtype=torch.int32, device=dev)
+    pb = torch.empty(4, dtype=torch.int64, device=dev)
+    cq.cq_varbits_index(bits, offset, pb, stream)
+    return offset, [int(v) for v in pb.cpu()]
+
+
+def pack(codes, rows, cols, bits=None, offset=None, plane_bytes=None, stream=None):
+    """codes -> list of 4 planes (None where unused)."""
+    G = rows * cols // GROUP
+    dev = codes.device
+    if bits is None:
+        planes = [None, None, empty_u8(32 * G, dev), None]
+    else:
+        planes = [empty_u8(max(16, n), dev) for n in plane_bytes]
+    cq.cq_pack_varbits(codes, G, bits, offset, planes, stream)
+    return planes
+
+
+def quantize_and_pack(w, bits=None, stream=None):
+    """fp32 weights -> (QWeight, codes, status)."""
+    rows, cols = w.shape
+    codes, scale, zero, status = quantize(w, bits, stream)
+    offset = pb = None
+    if bits is not None:
+        offset, pb = varbits_index(bits, stream)
+    planes = pack(codes, rows, cols, bits, offset, pb, stream)
+    return cq.QWeight(rows, cols, planes, scale, zero, bits, offset), codes, status
+
+
+def unpack(qw, stream=None):
+    codes = empty_u8(qw.rows * qw.cols, qw.scale.device)
+    cq.cq_unpack_varbits(qw, codes, stream)
+    return codes
+
+
+def project(r, scale, stream=None):
+    n = torch.zeros(1, dtype=torch.int64, device=r.device)
+    cq.cq_project_residual(r, scale, n, stream)
+    return n
+
+
+def verify(qw, first_w=0, n_w=None, flags=False, stream=None):
+    """-> (mismatches int64[1], first_bad int64[1], group_flags int32[...] or None), on the device."""
+    dev = qw.scale.device
+    if n_w is None:
+        n_w = qw.rows * qw.cols - first_w
+    mism = torch.empty(1, dtype=torch.int64, device=dev)
+    first = torch.empty(1, dtype=torch.int64, device=dev)
+    gf = None
+    if flags:
+        gf = torch.empty(max(1, (n_w // GROUP + 31) // 32), dtype=torch.int32, device=dev)
+    cq.cq_requant_verify(qw, first_w, n_w, mism, first, gf, stream)
+    return mism, first, gf
+
+
+def gemv(qw, x, stream=None):
+    y = torch.empty((x.shape[0], qw.rows), dtype=torch.float32, device=x.device)
+    cq.cq_dequant_gemv(qw, x, y, stream)
+    return y
+
+
+def gemm(qw, x, workspace=None, stream=None):
+    m = x.shape[0]
+    y = torch.empty((m, qw.rows), dtype=torch.float32, device=x.device)
+    need = cq.cq_gemm_workspace(qw.rows, qw.cols, m)
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    cq.cq_dequant_gemm(qw, x, y, workspace if need else None, stream)
+    return y

@@ -1,0 +1,183 @@
+/*
+ * cq.h -- C ABI of libcq: group-wise low-bit weight quantization for NVIDIA B200 (sm_100a).
+ *
+ * The method follows two abstracts (cited by page title and section):
+ *   [VBQ] "In-Cell Learning: Language Models That Update Their Own Weights in Sequence
+ *         Without Changing the File They Ship" (thelatestinai.com/papers/2608.20873),
+ *         abstract: every contiguous group of 64 weights has its own bit-width from
+ *         {1,2,4,8}; the allocation maps onto packed low-bit storage; fused
+ *         dequantize-and-multiply kernels serve memory-bound decode.
+ *   [CF]  "Nothing Changed but the Model: CellFill -- Bounded In-Cell Learning for
+ *         Bit-Identical, Revocable Updates to Quantized LLMs", Abstract: a 4-bit release
+ *         whose integer codes and scales stay frozen; updates live in a per-weight
+ *         residual strictly inside each quantization cell; re-quantization returns the
+ *         release bit for bit; dropping the residual revokes the update; drift is bounded.
+ *   [SLQ] listing page thelatestinai.com/papers/2512.18934, SLQ abstract: asymmetric
+ *         quantization (hence the zero point).
+ *
+ * Quantizer (the pages do not print it; this is the reading every entry point uses):
+ * a group of 64 consecutive weights along a row has an fp16 scale s, a uint8 zero z
+ * and a width b; L = 2^b - 1;
+ *     s = RN_fp16(RN32(RN32(wmax - wmin) / L)), floored at 2^-14
+ *     z = clamp(rne(RN32(-wmin / s)), 0, L)
+ *     q = clamp(rne(RN32(w / s)) + z, 0, L)                 (rne: ties to even)
+ * and the served weight is W = s * (q - z) + r, r an optional per-weight residual.
+ *
+ * Conventions for every call:
+ *  - Every pointer is a DEVICE pointer owned by the caller, unless the comment says host.
+ *  - Matrices are row-major [rows, cols]; groups run along cols (the input dimension), so
+ *    there are G = rows * cols / 64 groups, group g = row * (cols/64) + col/64.
+ *  - Arguments are validated on the host before anything is enqueued; a bad argument
+ *    returns a non-zero cq_status, launches nothing and sets cq_last_error().
+ *  - Work is enqueued asynchronously on `stream` (NULL = legacy default stream). The
+ *    library never synchronizes and never allocates device memory; results that the
+ *    device computes (counts, flags, status words) land in caller memory.
+ *  - A launch failure returns CQ_ERR_CUDA with the CUDA error text in cq_last_error().
+ *  - Calls on different streams that write the same buffers race, as usual in CUDA.
+ */
+#ifndef CQ_H
+#define CQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ABI-identical to cudaStream_t, without pulling in the CUDA headers. */
+typedef struct CUstream_st *cq_stream_t;
+
+typedef enum {
+    CQ_OK = 0,
+    CQ_ERR_ARG = 1,         /* NULL where a pointer is required, bad enum, m out of range */
+    CQ_ERR_SHAPE = 2,       /* negative sizes, cols % 64 != 0, chunk not on group bounds */
+    CQ_ERR_BITS = 3,        /* a host-visible bit-width outside {1,2,4,8}                 */
+    CQ_ERR_ALIGN = 4,       /* a pointer that must be 16-byte aligned is not              */
+    CQ_ERR_NONFINITE = 5,   /* reserved: non-finite input reported synchronously          */
+    CQ_ERR_RANGE = 6,       /* a size beyond what the format or a workspace can address   */
+    CQ_ERR_CUDA = 7,        /* a CUDA launch or memset failed                             */
+    CQ_ERR_UNSUPPORTED = 8  /* a valid combination this build has no kernel for           */
+} cq_status;
+
+typedef enum { CQ_F32 = 0, CQ_BF16 = 1 } cq_dtype;
+
+/* bits of the device status word written by cq_quantize */
+#define CQ_QSTATUS_NONFINITE 1u /* a group held a NaN or infinity: written as s=+0, z=0, q=0 */
+#define CQ_QSTATUS_RANGE 2u     /* a group's scale overflowed fp16: written as s=+0, z=0, q=0 */
+#define CQ_QSTATUS_BADBITS 4u   /* bits[g] not in {1,2,4,8}: written as s=+0, z=0, q=0        */
+
+/*
+ * A quantized weight matrix ([VBQ] packed low-bit storage, [CF] frozen codes + scales).
+ * Packed layout: one plane per width b in {1,2,4,8} (plane[0..3] for b = 1,2,4,8). Group g
+ * of width b occupies 8*b bytes of plane b starting at byte offset[g]; code j of the group
+ * is in bits [j*b, (j+1)*b) of that little-endian byte string, least significant bit first.
+ * offset[g] = 8*b * (number of earlier groups, in row-major group order, of the same width).
+ * Fixed 4-bit ([CF] 4-bit release): bits = offset = NULL, plane[2] holds plain row-major
+ * nibbles (offset 32*g; even column in the low nibble); the other planes are unused.
+ */
+typedef struct {
+    int64_t rows, cols;       /* N (outputs) x K (inputs); cols % 64 == 0                  */
+    const uint8_t *bits;      /* [G] widths in {1,2,4,8}, or NULL for all-4                */
+    const uint32_t *offset;   /* [G] byte offsets into plane[width], NULL when bits NULL   */
+    const uint8_t *plane[4];  /* planes for b = 1, 2, 4, 8; 16-byte aligned when used      */
+    const uint16_t *scale;    /* [G] fp16 bit patterns                                     */
+    const uint8_t *zero;      /* [G]                                                       */
+    const void *residual;     /* [rows*cols] of residual_dtype, or NULL (revoked / none)   */
+    cq_dtype residual_dtype;
+} cq_qweight;
+
+/*
+ * cq_quantize -- [VBQ] per-group widths, [CF] 4-bit codes and scales, [SLQ] asymmetry.
+ * w: [rows, cols] fp32 (16-byte aligned). bits: [G] widths or NULL (= 4 for every group).
+ * codes: [rows*cols] one code per byte (8-byte aligned); scale: [G] fp16 bits; zero: [G].
+ * status_word: one uint32 (device) that receives the OR of CQ_QSTATUS_* over all groups;
+ * it is cleared by the call; may be NULL. Groups with a non-finite weight, an fp16-overflowing
+ * scale or a bad width are written as s=+0, z=0, q=0 and flagged; the call still returns CQ_OK.
+ */
+cq_status cq_quantize(const float *w, int64_t rows, int64_t cols, const uint8_t *bits,
+                      uint8_t *codes, uint16_t *scale, uint8_t *zero, uint32_t *status_word,
+                      cq_stream_t stream);
+
+/*
+ * cq_varbits_index -- [VBQ] "maps directly to packed low-bit storage": builds offset[G] (byte
+ * offsets as in cq_qweight) and plane_bytes[4] (device, uint64: bytes needed by each plane).
+ * bits: [G]. Device-side, widths outside {1,2,4,8} count as width 0 (offset 0, no bytes);
+ * pack and quantize flag them. n_groups <= 2^26 (byte offsets are 32-bit) else CQ_ERR_RANGE.
+ * The offset array also serves as the call's temporary storage, so it must not alias bits.
+ */
+cq_status cq_varbits_index(const uint8_t *bits, int64_t n_groups, uint32_t *offset,
+                           uint64_t *plane_bytes, cq_stream_t stream);
+
+/*
+ * cq_pack_varbits -- codes (one per byte, [n_groups*64]) -> planes, in the cq_qweight layout.
+ * bits/offset NULL: fixed 4-bit into plane[2]. Only the low b bits of each code are stored.
+ * plane[i] must hold plane_bytes[i] bytes and be 16-byte aligned when used; codes 16-byte aligned.
+ */
+cq_status cq_pack_varbits(const uint8_t *codes, int64_t n_groups, const uint8_t *bits,
+                          const uint32_t *offset, uint8_t *const plane[4], cq_stream_t stream);
+
+/* cq_unpack_varbits -- the inverse of cq_pack_varbits: qw's planes -> codes [rows*cols]. */
+cq_status cq_unpack_varbits(const cq_qweight *qw, uint8_t *codes, cq_stream_t stream);
+
+/*
+ * cq_project_residual -- [CF] "projecting into the cells": in place,
+ *     r <- c if r > c;  -c if r < -c;  r otherwise,   c = (0.5 - 2^-10) * s_group,
+ * for fp32 r; for bf16 r the bound is c rounded toward zero to bf16 (never outward).
+ * A NaN residual is left as it is (requant-verify then reports it). r: [n] (16-byte aligned),
+ * n % 64 == 0, element i belongs to group i/64 of scale. n_clamped: one uint64 (device) that
+ * receives the number of elements whose bits changed; cleared by the call; may be NULL.
+ */
+cq_status cq_project_residual(void *r, cq_dtype dtype, const uint16_t *scale, int64_t n,
+                              uint64_t *n_clamped, cq_stream_t stream);
+
+/*
+ * cq_requant_verify -- [CF] "re-quantization returns the released artifact bit-for-bit" and
+ * "exactly revocable by dropping the residual" (qw->residual = NULL). For each weight i in
+ * [first_w, first_w + n_w) with code q, scale s, zero z, width b:
+ *     w' = RN32(RN32(s*(q-z)) + r_i);  t = RN32(w'/s);  q' = clamp(rne(t) + z, 0, 2^b-1)
+ * and a mismatch is q' != q (a NaN t is a mismatch). first_w and n_w are multiples of 64
+ * and the range lies inside the matrix (chunks let a 2.4e10-weight check run piecewise).
+ * mismatches: one uint64 (device) <- count; first_bad: one int64 (device) <- smallest
+ * mismatching index or -1; group_flags: NULL or ceil(n_w/64/32) uint32 (device), bit j set
+ * when group first_w/64 + j holds a mismatch. All three are cleared by the call. A mismatch
+ * is a result, not an error. The residual must be 16-byte aligned.
+ */
+cq_status cq_requant_verify(const cq_qweight *qw, int64_t first_w, int64_t n_w,
+                            uint64_t *mismatches, int64_t *first_bad, uint32_t *group_flags,
+                            cq_stream_t stream);
+
+/*
+ * cq_dequant_gemv -- [VBQ] fused dequantize-and-multiply for decode:
+ *     y[i, n] = sum_k (s*(q-z) + r)[n, k] * x[i, k],   i < m, 1 <= m <= 8,
+ * products accumulated in fp32. x: [m, cols] of x_dtype (16-byte aligned); y: [m, rows] fp32.
+ * y is overwritten. Fixed-4 weights with bf16 x and no residual run on the tensor-core
+ * path (integer codes are exact bf16 operands; scales and zero points are applied in fp32
+ * per group); other combinations run on an fp32 CUDA-core path.
+ */
+cq_status cq_dequant_gemv(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m,
+                          float *y, cq_stream_t stream);
+
+/*
+ * cq_dequant_gemm -- the same contraction for a batch, 1 <= m <= 256. Fixed-4 weights with
+ * bf16 x, no residual and m >= 16 run on the sm_100a tcgen05 tensor cores with accumulators
+ * in tensor memory; m < 16 goes to the GEMV kernels, as do other formats (in slices of 8).
+ * workspace: caller-owned device scratch of at least cq_gemm_workspace(rows, cols, m) bytes
+ * (may be NULL when that is 0), 16-byte aligned. y: [m, rows] fp32, overwritten.
+ */
+cq_status cq_dequant_gemm(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m,
+                          float *y, void *workspace, size_t workspace_bytes, cq_stream_t stream);
+
+/* Bytes of workspace cq_dequant_gemm needs for this shape (host function, no GPU work). */
+size_t cq_gemm_workspace(int64_t rows, int64_t cols, int m);
+
+/* Text of the last non-OK status returned on the calling thread (thread-local, host). */
+const char *cq_last_error(void);
+
+/* Name of a status code (host). */
+const char *cq_status_string(cq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CQ_H */

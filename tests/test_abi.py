@@ -1,0 +1,71 @@
+"""The C-ABI libraries load and export every symbol their headers declare, and reject bad
+arguments on the host before touching a GPU (no compute call runs here)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from cell_updates_b200 import build, cq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+
+
+def _declared(header):
+    text = open(os.path.join(ROOT, "include", header)).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(cqs?_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_libcq_exports_header_symbols():
+    names = _declared("cq.h")
+    assert names == sorted(cq.EXPORTS)
+    lib = C.CDLL(cq.LIBCQ_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_libcq_synth_exports_header_symbols():
+    names = _declared("cq_synth.h")
+    assert names == sorted(cq.SYNTH_EXPORTS)
+    lib = C.CDLL(cq.LIBSYNTH_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_host_validation_rejects_bad_arguments():
+    L = cq.lib()
+    p = C.c_void_p(16)   # never dereferenced: validation fails first
+    assert L.cq_quantize(p, 4, 63, None, p, p, p, None, None) == 2          # cols % 64
+    assert L.cq_quantize(p, -1, 64, None, p, p, p, None, None) == 2         # negative
+    assert L.cq_quantize(C.c_void_p(8), 4, 64, None, p, p, p, None, None) == 4   # misaligned w
+    assert L.cq_quantize(None, 4, 64, None, p, p, p, None, None) == 1       # NULL w
+    assert L.cq_project_residual(p, 0, p, 100, None, None) == 2             # n % 64
+    assert L.cq_project_residual(p, 5, p, 64, None, None) == 1              # bad dtype
+    assert L.cq_varbits_index(p, (1 << 26) + 1, p, p, None) == 6            # 32-bit offsets
+    qw = cq.cq_qweight()
+    qw.rows, qw.cols = 4, 64
+    qw.scale, qw.zero = 16, 16
+    qw.plane[2] = 16
+    assert L.cq_requant_verify(C.byref(qw), 32, 64, p, p, None, None) == 2  # not whole groups
+    assert L.cq_requant_verify(C.byref(qw), 0, 512, p, p, None, None) == 2  # past the end
+    assert L.cq_dequant_gemv(C.byref(qw), p, 1, 9, p, None) == 1            # m > 8
+    qw.plane[2] = 8
+    assert L.cq_dequant_gemv(C.byref(qw), p, 1, 1, p, None) == 4            # misaligned plane
+    qw.plane[2] = 16
+    qw.bits = 16                                                             # bits without offset
+    assert L.cq_dequant_gemv(C.byref(qw), p, 1, 1, p, None) == 1
+    assert "offset" in cq.cq_last_error()
+    assert L.cq_gemm_workspace(8192, 28672, 8) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(cq, "_lib", None)
+    monkeypatch.setattr(cq, "LIBCQ_PATH", "/nonexistent/libcq.so")
+    with pytest.raises(cq.CQError):
+        cq.lib()

@@ -1,0 +1,276 @@
+"""GPU (CUDA path through the C ABI) against the CPU oracle on the same seeded inputs.
+
+Bit-exact: codes, scales, zeros, status, group offsets, plane bytes, unpacked codes,
+projected residuals and clamp counts, verify counts / first index / group flags.
+Tolerance (benchmark spec): the matmuls vs the fp64 oracle, relative Frobenius
+error <= 2e-3 and per-element |err| <= 1e-2 * rms(y).
+Sizes span several tiles plus ragged tails; the config-0 shape is included.
+"""
+import numpy as np
+import pytest
+import torch
+
+from cell_updates_b200 import cq, ops, synth
+from gpu_util import bf16_dev, check_matmul, dev, host, planes_host, u16_dev
+from oracle import c_oracle as co
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(cuda_ok):
+    from cell_updates_b200 import build
+    build.build()
+    cq.lib()
+
+
+def _oracle_qw(codes, scale, zero, bits):
+    """the oracle's own packing of its own codes"""
+    if bits is None:
+        return co.pack(codes), None
+    off, pb = co.varbits_index(bits)
+    return co.pack(codes, bits, off, pb), off
+
+
+def _quantize_both(w, bits=None):
+    bits_d = dev(bits) if bits is not None else None
+    qw, codes_d, st_d = ops.quantize_and_pack(dev(w), bits_d)
+    torch.cuda.synchronize()
+    oc = co.quantize(w, bits)
+    return qw, codes_d, st_d, oc
+
+
+def _assert_quant_equal(codes_d, qw, st_d, oc):
+    codes, scale, zero, st = oc
+    assert np.array_equal(host(codes_d), codes)
+    assert np.array_equal(host(qw.scale, np.uint16), scale)
+    assert np.array_equal(host(qw.zero), zero)
+    assert int(host(st_d)[0]) == st
+
+
+# ---- quantize ------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape,seed", [((256, 512), 0), ((37, 64 * 13), 3), ((1, 64), 4)])
+def test_quantize_fixed4_bit_exact(shape, seed):
+    w = synth.normal_weights(*shape, seed=seed)
+    qw, codes_d, st_d, oc = _quantize_both(w)
+    _assert_quant_equal(codes_d, qw, st_d, oc)
+
+
+def test_quantize_edge_groups_bit_exact():
+    rng = np.random.default_rng(8)
+    rows = []
+    i = np.arange(64)
+    rows.append((0.25 * (i % 16) - 2.0))                                  # exact grid
+    t = np.full(64, 1.0); t[:10] = [0, 3.75, .625, .875, .125, .375, 3.625, 3.375, 1.125, 1.375]
+    rows.append(t)                                                         # ties
+    rows.append(np.full(64, 0.5)); rows.append(np.zeros(64)); rows.append(np.full(64, -0.5))
+    rows.append(rng.uniform(1, 3, 64)); rows.append(-rng.uniform(1, 3, 64))
+    r = np.zeros(64); r[3] = np.nan; rows.append(r)
+    r = np.zeros(64); r[9] = -np.inf; rows.append(r)
+    r = np.zeros(64); r[0], r[1] = -3e38, 3e38; rows.append(r)
+    r = np.zeros(64); r[0], r[1] = 0.0, 1e6; rows.append(r)             # fp16 overflow of s
+    rows.append(rng.standard_t(2, 64) * 1e-6)                              # sub-2^-14 scales
+    rows.append(rng.standard_normal(64) * 1e4)
+    w = np.stack([np.asarray(v, np.float32) for v in rows]).reshape(1, -1)
+    w = np.repeat(w, 3, axis=0)
+    G = w.size // 64
+    bits = np.tile(np.array([1, 2, 4, 8], np.uint8), G // 4 + 1)[:G]
+    bits[5] = 3                                                            # bad width
+    for b in (None, bits):
+        qw_codes = _quantize_both(w, b) if b is None else None
+        if b is None:
+            qw, codes_d, st_d, oc = qw_codes
+            _assert_quant_equal(codes_d, qw, st_d, oc)
+        else:
+            codes_d, scale_d, zero_d, st_d = ops.quantize(dev(w), dev(b))
+            torch.cuda.synchronize()
+            oc = co.quantize(w, b)
+            assert np.array_equal(host(codes_d), oc[0])
+            assert np.array_equal(host(scale_d, np.uint16), oc[1])
+            assert np.array_equal(host(zero_d), oc[2])
+            assert int(host(st_d)[0]) == oc[3] == 7
+
+
+def test_quantize_vbq_config2_bit_exact():
+    # 2048 x 8192 ~ N(0, 0.02^2), widths drawn with the VBQ allocation statistics
+    w = synth.normal_weights(2048, 8192, seed=2)
+    bits = synth.vbq_bits(2048 * 8192 // 64, seed=2)
+    qw, codes_d, st_d, oc = _quantize_both(w, bits)
+    _assert_quant_equal(codes_d, qw, st_d, oc)
+    off, pb = co.varbits_index(bits)
+    assert np.array_equal(host(qw.offset, np.uint32), off)
+    planes = co.pack(oc[0], bits, off, pb)
+    for slot in range(4):
+        assert np.array_equal(host(qw.planes[slot])[:pb[slot]], planes[slot][:pb[slot]])
+    assert np.array_equal(host(ops.unpack(qw)), oc[0])
+
+
+# ---- pack / index -------------------------------------------------------------------------
+
+@pytest.mark.parametrize("G", [1, 3, 4095, 4096, 4097, 3 * 4096 + 5, 70000])
+def test_varbits_index_and_pack_bit_exact(G):
+    rng = np.random.default_rng(G)
+    bits = synth.vbq_bits(G, seed=G)
+    L = (1 << bits.astype(np.int64)) - 1
+    codes = (rng.integers(0, 256, (G, 64)) & L[:, None]).astype(np.uint8).ravel()
+    off, pb = co.varbits_index(bits)
+    off_d, pb_d = ops.varbits_index(dev(bits))
+    assert np.array_equal(host(off_d, np.uint32), off) and pb_d == pb
+    planes_d = ops.pack(dev(codes), G, 64, dev(bits), off_d, pb_d)
+    planes = co.pack(codes, bits, off, pb)
+    for slot in range(4):
+        assert np.array_equal(host(planes_d[slot])[:pb[slot]], planes[slot][:pb[slot]])
+    qw = cq.QWeight(G, 64, planes_d, u16_dev(np.zeros(G, np.uint16)), dev(np.zeros(G, np.uint8)), dev(bits), off_d)
+    assert np.array_equal(host(ops.unpack(qw)), codes)
+
+
+# ---- projection ---------------------------------------------------------------------------------
+
+def _residual_cases(scale, seed):
+    rng = np.random.default_rng(seed)
+    sf = np.asarray(scale, np.uint16).view(np.float16).astype(np.float32)
+    G = sf.size
+    mult = rng.uniform(-0.8, 0.8, (G, 64)).astype(np.float32)
+    mult[:, :6] = [0.5, -0.5, 0.5 - 2 ** -10, 0.5 + 2 ** -10, 1e30, -1e30]
+    r = (mult * sf[:, None]).astype(np.float32)
+    r[0, 7] = np.nan
+    r[1, 8] = -0.0
+    return r.ravel()
+
+
+def test_project_f32_bit_exact():
+    w = synth.normal_weights(256, 512, seed=0)
+    _, scale, _, _ = co.quantize(w)
+    r = _residual_cases(scale, 1)
+    rp, n = co.project_f32(r, scale)
+    r_d = dev(r)
+    n_d = ops.project(r_d, u16_dev(scale))
+    torch.cuda.synchronize()
+    assert np.array_equal(host(r_d).view(np.uint32), rp.view(np.uint32))
+    assert int(host(n_d)[0]) == n
+
+
+def test_project_bf16_bit_exact():
+    rng = np.random.default_rng(5)
+    G = 3001
+    scale = rng.integers(0x0001, 0x7C01, G).astype(np.uint16)        # incl. subnormal and +inf
+    r = _residual_cases(scale, 2)
+    rb = (r.view(np.uint32) >> 16).astype(np.uint16)
+    rp, n = co.project_bf16(rb, scale)
+    r_d = bf16_dev(rb)
+    n_d = ops.project(r_d, u16_dev(scale))
+    torch.cuda.synchronize()
+    assert np.array_equal(host(r_d, np.uint16), rp)
+    assert int(host(n_d)[0]) == n
+
+
+# ---- requant verify --------------------------------------------------------------------------
+
+def _verify_both(qw, planes, scale, zero, bits, off, r, r_dtype, first_w=0, n_w=None):
+    total = qw.rows * qw.cols
+    if n_w is None:
+        n_w = total - first_w
+    m_d, f_d, g_d = ops.verify(qw, first_w, n_w, flags=True)
+    torch.cuda.synchronize()
+    m, f, flags = co.verify(planes, scale, zero, bits, off, r, r_dtype, first_w, n_w, want_flags=True)
+    assert int(host(m_d)[0]) == m
+    assert int(host(f_d)[0]) == f
+    assert np.array_equal(host(g_d, np.uint32)[:flags.size], flags)
+    return m
+
+
+@pytest.mark.parametrize("varbits", [False, True])
+def test_verify_config0_and_controls(varbits):
+    w = synth.normal_weights(256, 512, seed=0)
+    G = 256 * 512 // 64
+    bits = synth.vbq_bits(G, seed=9) if varbits else None
+    codes, scale, zero, _ = co.quantize(w, bits)
+    planes, off = _oracle_qw(codes, scale, zero, bits)
+    qw, _, _, _ = _quantize_both(w, bits)
+    # negative control: r ~ U(-0.6 s, 0.6 s) unprojected
+    r = synth.uniform_residual_f32(scale, seed=10)
+    m = _verify_both(qw.with_residual(dev(r)), planes, scale, zero, bits, off, r, "f32")
+    assert m > 0
+    # chunks of whole groups give the same answer piecewise
+    for first, n in [(0, 64 * 100), (64 * 100, 64 * 37), (64 * 1000, w.size - 64 * 1000)]:
+        _verify_both(qw.with_residual(dev(r)), planes, scale, zero, bits, off, r, "f32", first, n)
+    # projected: bit-identical; dropped: revoked
+    rp, _ = co.project_f32(r, scale)
+    assert _verify_both(qw.with_residual(dev(rp)), planes, scale, zero, bits, off, rp, "f32") == 0
+    assert _verify_both(qw, planes, scale, zero, bits, off, None, "f32") == 0
+    # bf16 residual, projected and not
+    rb = synth.normal_residual_bf16(scale, seed=11, rel_sigma=0.3)
+    assert _verify_both(qw.with_residual(bf16_dev(rb)), planes, scale, zero, bits, off, rb, "bf16") > 0
+    rbp, _ = co.project_bf16(rb, scale)
+    assert _verify_both(qw.with_residual(bf16_dev(rbp)), planes, scale, zero, bits, off, rbp, "bf16") == 0
+
+
+def test_verify_boundary_and_corrupt_scales():
+    rng = np.random.default_rng(12)
+    G = 4096 + 17
+    codes = rng.integers(0, 16, G * 64).astype(np.uint8)
+    zero = rng.integers(0, 16, G).astype(np.uint8)
+    scale = rng.integers(0x0001, 0x7C00, G).astype(np.uint16)
+    scale[:4] = [0x0000, 0x7C00, 0x7E00, 0xBC00]                        # 0, inf, NaN, -1
+    planes = co.pack(codes)
+    r = _residual_cases(scale, 13)
+    qw = cq.QWeight(G, 64, [None, None, dev(planes[2]), None], u16_dev(scale), dev(zero))
+    m = _verify_both(qw.with_residual(dev(r)), planes, scale, zero, None, None, r, "f32")
+    assert m > 0
+
+
+# ---- matmuls ------------------------------------------------------------------------------------
+
+def _matmul_case(rows, cols, m, x_dtype, bits=None, r=None, seed=0):
+    w = synth.normal_weights(rows, cols, seed=seed)
+    qw, _, _, oc = _quantize_both(w, bits)
+    codes, scale, zero, _ = oc
+    planes, off = _oracle_qw(codes, scale, zero, bits)
+    x = synth.activations(m, cols, seed=seed + 1, dtype=x_dtype)
+    x_d = bf16_dev(x) if x_dtype == "bf16" else dev(x)
+    r_dtype = None
+    if r is not None:
+        r_dtype = "bf16" if r.dtype == np.uint16 else "f32"
+        qw = qw.with_residual(bf16_dev(r) if r_dtype == "bf16" else dev(r))
+    y_ref = co.dequant_matmul_f64(planes, scale, zero, rows, cols, x, x_dtype, bits, off, r, r_dtype or "f32")
+    return qw, x_d, y_ref, scale
+
+
+def test_gemv_config0_fp32_with_projected_residual():
+    w = synth.normal_weights(256, 512, seed=0)
+    _, scale, _, _ = co.quantize(w)
+    rp, _ = co.project_f32(synth.uniform_residual_f32(scale, seed=10), scale)
+    qw, x_d, y_ref, _ = _matmul_case(256, 512, 1, "f32", r=rp)
+    check_matmul(host(ops.gemv(qw, x_d)), y_ref, "cfg0 r")
+    qw0, x0, y0, _ = _matmul_case(256, 512, 1, "f32")
+    check_matmul(host(ops.gemv(qw0, x0)), y0, "cfg0 revoked")
+
+
+@pytest.mark.parametrize("rows,cols", [(256, 512), (16, 64), (47, 64 * 9), (300, 64 * 21), (1000, 4096)])
+@pytest.mark.parametrize("m", [1, 3, 8])
+def test_gemv_tensor_core_4bit(rows, cols, m):
+    qw, x_d, y_ref, _ = _matmul_case(rows, cols, m, "bf16", seed=rows + m)
+    check_matmul(host(ops.gemv(qw, x_d)), y_ref, f"{rows}x{cols} m={m}")
+
+
+@pytest.mark.parametrize("m", [1, 8])
+def test_gemv_varbits(m):
+    G = 512 * 1024 // 64
+    bits = synth.vbq_bits(G, seed=3)
+    qw, x_d, y_ref, _ = _matmul_case(512, 1024, m, "bf16", bits=bits, seed=5)
+    check_matmul(host(ops.gemv(qw, x_d)), y_ref, f"vbq m={m}")
+
+
+@pytest.mark.parametrize("m", [16, 64])
+def test_gemm_batches(m):
+    qw, x_d, y_ref, _ = _matmul_case(384, 64 * 40, m, "bf16", seed=m)
+    check_matmul(host(ops.gemm(qw, x_d)), y_ref, f"gemm m={m}")
+
+
+def test_gemm_bf16_residual_uses_exact_formula():
+    w = synth.normal_weights(128, 1024, seed=21)
+    _, scale, _, _ = co.quantize(w)
+    rb, _ = co.project_bf16(synth.normal_residual_bf16(scale, seed=22), scale)
+    qw, x_d, y_ref, _ = _matmul_case(128, 1024, 20, "bf16", r=rb, seed=21)
+    check_matmul(host(ops.gemm(qw, x_d)), y_ref, "gemm r bf16")
