@@ -1,0 +1,540 @@
+"""Benchmark of the group-wise quantization hot path on B200.
+
+One step = one pass of every hot-path row over the decode workload of the 4-bit GEMV
+configuration (three weight matrices 4096x4096, 11008x4096, 4096x11008, drawn as
+0.02 * Student-t(5) with 0.1% of entries x10):
+
+    quantize (fp32 -> 4-bit codes, fp16 scales, u8 zeros)   -> pack into the 4-bit plane
+    -> project a bf16 residual ~ N(0, (0.3 s)^2) into the cells -> requant-verify with it
+    -> requant-verify without it (revocation) -> dequant-GEMV at batch 1 (decode)
+    -> dequant-GEMM at batch 64
+
+for each matrix.  The step is captured once as a CUDA graph and replayed; per-kernel
+durations come from event-record nodes inside the same graph (the timed region).
+Printed: one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cq|reference]
+       (N > 1: launch with torch.distributed.run, one process per GPU)
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+GROUP = 64
+SHAPES = [(4096, 4096), (11008, 4096), (4096, 11008)]       # rows (out) x cols (in)
+LAYER_MIX = [4, 2, 1]       # per layer of a 7B-shaped decoder: q,k,v,o | gate,up | down
+N_LAYERS = 32
+GEMM_M = 64
+METRIC = "dequant-GEMV weight GB/s & tokens/s vs HBM peak; requant-verify weights/s"
+WORKLOAD = "4-bit g=64 decode matrices 4096x4096, 11008x4096, 4096x11008 (0.02*t5, 0.1% outliers x10)"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# algorithmic bytes per weight of each step (what the method must move)
+def kernel_bytes(n):
+    G = n // GROUP
+    meta = 3 * G                      # fp16 scale + u8 zero per group
+    return {
+        "quantize": 4 * n + n + meta,                 # read fp32 W, write u8 codes + meta
+        "pack": n + n // 2,                           # read codes, write nibbles
+        "project": 2 * n + 2 * n + 2 * G,             # read + write bf16 r, read scales
+        "verify": n // 2 + meta + 2 * n,              # codes + meta + bf16 r
+        "revoke_verify": n // 2 + meta,               # codes + meta
+        "gemv": n // 2 + meta,                        # weights (x, y negligible)
+        "gemm": n // 2 + meta,
+    }
+
+
+KERNELS = ["quantize", "pack", "project", "verify", "revoke_verify", "gemv", "gemm"]
+
+
+# ---------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------------------
+def count_kernel_nodes(graph):
+    """Number of kernel nodes in a captured graph (all of them are libcq kernels)."""
+    from cuda.bindings import driver as drv
+    h = drv.CUgraph(graph.raw_cuda_graph())
+    err, _, n = drv.cuGraphGetNodes(h, 0)
+    if err != drv.CUresult.CUDA_SUCCESS:
+        return None
+    err, nodes, n = drv.cuGraphGetNodes(h, n)
+    kinds = [drv.cuGraphNodeGetType(nd)[1] for nd in nodes]
+    return sum(1 for k in kinds if k == drv.CUgraphNodeType.CU_GRAPH_NODE_TYPE_KERNEL)
+
+
+class Workload:
+    def __init__(self, torch, cq, ops, synth, device, seed_base=1):
+        self.torch, self.cq, self.ops = torch, cq, ops
+        self.mats = []
+        for idx, (N, K) in enumerate(SHAPES):
+            w = synth.student_t_weights(N, K, seed=seed_base + 1000 * idx)
+            w_host = torch.from_numpy(w).pin_memory()
+            w_dev = w_host.to(device)
+            qw, codes, status = ops.quantize_and_pack(w_dev)
+            scale_np = qw.scale.cpu().view(torch.int16).numpy().view(np.uint16)
+            r = synth.normal_residual_bf16(scale_np, seed=seed_base + 1000 * idx + 7, rel_sigma=0.3)
+            r_host = torch.from_numpy(r.view(np.int16)).view(torch.bfloat16).pin_memory()
+            x = synth.activations(1, K, seed=seed_base + 1000 * idx + 11, dtype="bf16")
+            X = synth.activations(GEMM_M, K, seed=seed_base + 1000 * idx + 13, dtype="bf16")
+            x_host = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+            X_host = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).pin_memory()
+            m = dict(N=N, K=K, n=N * K, w_host=w_host, w=w_dev, codes=codes, qw=qw,
+                     r_host=r_host, r=r_host.to(device), x_host=x_host, x=x_host.to(device),
+                     X_host=X_host, X=X_host.to(device),
+                     y=torch.empty(1, N, device=device), Y=torch.empty(GEMM_M, N, device=device),
+                     status=torch.zeros(1, dtype=torch.int32, device=device),
+                     mism=torch.zeros(1, dtype=torch.int64, device=device),
+                     first=torch.zeros(1, dtype=torch.int64, device=device),
+                     mism0=torch.zeros(1, dtype=torch.int64, device=device),
+                     first0=torch.zeros(1, dtype=torch.int64, device=device),
+                     nclamp=torch.zeros(1, dtype=torch.int64, device=device))
+            need = cq.cq_gemm_workspace(N, K, GEMM_M)
+            m["ws"] = torch.empty(max(need, 16), dtype=torch.uint8, device=device) if need else None
+            self.mats.append(m)
+        torch.cuda.synchronize()
+
+    def step(self, stream, marks=None):
+        """Enqueue one step. marks[(matrix, kernel)] = (start, end) external events: recorded
+        inside a graph capture they become event nodes that time each launch on replay."""
+        cq = self.cq
+        for mi, m in enumerate(self.mats):
+            qw = m["qw"]
+            def mark(name, which):
+                if marks is not None:
+                    marks[(mi, name)][which].record(stream)
+            mark("quantize", 0)
+            cq.cq_quantize(m["w"], None, m["codes"], qw.scale, qw.zero, m["status"], stream)
+            mark("quantize", 1)
+            mark("pack", 0)
+            cq.cq_pack_varbits(m["codes"], m["n"] // GROUP, None, None, qw.planes, stream)
+            mark("pack", 1)
+            mark("project", 0)
+            cq.cq_project_residual(m["r"], qw.scale, m["nclamp"], stream)
+            mark("project", 1)
+            qwr = qw.with_residual(m["r"])
+            mark("verify", 0)
+            cq.cq_requant_verify(qwr, 0, m["n"], m["mism"], m["first"], None, stream)
+            mark("verify", 1)
+            mark("revoke_verify", 0)
+            cq.cq_requant_verify(qw, 0, m["n"], m["mism0"], m["first0"], None, stream)
+            mark("revoke_verify", 1)
+            mark("gemv", 0)
+            cq.cq_dequant_gemv(qw, m["x"], m["y"], stream)
+            mark("gemv", 1)
+            mark("gemm", 0)
+            cq.cq_dequant_gemm(qw, m["X"], m["Y"], m["ws"], stream)
+            mark("gemm", 1)
+
+    def n_weights(self):
+        return sum(m["n"] for m in self.mats)
+
+    def step_bytes(self):
+        tot = {k: 0 for k in KERNELS}
+        for m in self.mats:
+            for k, v in kernel_bytes(m["n"]).items():
+                tot[k] += v
+        return tot
+
+
+def time_graph(torch, graph, reps, stream):
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def isolated_components(torch, cq, ops, device, peaks, stream):
+    """Cold-L2 component rates: GEMV (rotating > 2x L2), the 32-layer decode proxy, verify."""
+    out = {}
+    L2 = torch.cuda.get_device_properties(device).L2_cache_size
+    # 32-layer 7B-shaped decode: distinct weights per layer (3.54 GB), one graph per token
+    base = []
+    for (N, K) in SHAPES:
+        w = torch.randn(N, K, device=device) * 0.02
+        qw, _, _ = ops.quantize_and_pack(w)
+        base.append(qw)
+        del w
+    layers = []
+    for l in range(N_LAYERS):
+        for qw, mult in zip(base, LAYER_MIX):
+            for _ in range(mult):
+                layers.append(cq.QWeight(qw.rows, qw.cols, [None, None, qw.planes[2].clone(), None],
+                                         qw.scale.clone(), qw.zero.clone()))
+    xs = {K: torch.randn(1, K, device=device).to(torch.bfloat16) for (_, K) in SHAPES}
+    ys = {N: torch.empty(1, N, device=device) for (N, _) in SHAPES}
+    token_bytes = sum(q.rows * q.cols // 2 + 3 * q.rows * q.cols // GROUP for q in layers)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        for q in layers:     # warm-up outside capture
+            cq.cq_dequant_gemv(q, xs[q.cols], ys[q.rows], stream)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for q in layers:
+                cq.cq_dequant_gemv(q, xs[q.cols], ys[q.rows], stream)
+    for _ in range(3):
+        g.replay()
+    t_ms = time_graph(torch, g, 20, stream)
+    out["decode_32_layers"] = {"tokens_per_s": 1e3 / t_ms, "ms_per_token": t_ms, "weight_bytes_per_token": token_bytes,
+                               "GBps": token_bytes / t_ms / 1e6, "frac_hbm": token_bytes / t_ms / 1e6 / peaks["hbm_gbs"],
+                               "ceiling_tokens_per_s": peaks["hbm_gbs"] * 1e9 / token_bytes,
+                               "launches_per_token": len(layers)}
+    # per shape, the same pool (rotation over 32 copies > 2 x L2)
+    per = {}
+    for si, (N, K) in enumerate(SHAPES):
+        pool = [q for q in layers if q.rows == N and q.cols == K]
+        g1 = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g1, stream=stream):
+                for q in pool:
+                    cq.cq_dequant_gemv(q, xs[K], ys[N], stream)
+        g1.replay()
+        t = time_graph(torch, g1, 10, stream) / len(pool)
+        b = N * K // 2 + 3 * N * K // GROUP
+        per[f"{N}x{K}"] = {"us": t * 1e3, "GBps": b / t / 1e6, "frac_hbm": b / t / 1e6 / peaks["hbm_gbs"]}
+        del g1
+    out["gemv_m1_cold"] = per
+    out["l2_bytes"] = L2
+    del g, layers
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    from cell_updates_b200 import cq, ops, synth
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    peaks = load_peaks()
+    cq.lib()
+    wl = Workload(torch, cq, ops, synth, device, seed_base=1 + 100000 * rank)
+    stream = torch.cuda.Stream(device)
+    # eager run, then a one-step graph for the warm-up and a K-step graph for the timed
+    # region, each launch of the K-step graph bracketed by its own event pair
+    with torch.cuda.stream(stream):
+        wl.step(stream)
+    torch.cuda.synchronize()
+    g1 = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g1, stream=stream):
+            wl.step(stream)
+    launches_per_step = count_kernel_nodes(g1)
+    marks = [{(mi, k): (torch.cuda.Event(enable_timing=True, external=True),
+                        torch.cuda.Event(enable_timing=True, external=True))
+              for mi in range(len(wl.mats)) for k in KERNELS} for _ in range(args.steps)]
+    gK = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(gK, stream=stream):
+            for s_i in range(args.steps):
+                wl.step(stream, marks[s_i])
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        g1.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        gK.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    t_step = start.elapsed_time(end) / args.steps
+    per_kernel = {k: 0.0 for k in KERNELS}           # ms summed over every launch
+    for mk in marks:
+        for (mi, k), (a, b) in mk.items():
+            per_kernel[k] += a.elapsed_time(b)
+    if dist:
+        t = torch.tensor([t_step], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_step = float(t.item())
+    checks = [int(m["mism"].item()) for m in wl.mats] + [int(m["mism0"].item()) for m in wl.mats] + \
+             [int(m["status"].item()) for m in wl.mats]
+    assert all(c == 0 for c in checks), f"hot-path results not clean: {checks}"
+
+    bytes_step = wl.step_bytes()
+    total_bytes = sum(bytes_step.values())
+    n_w = wl.n_weights()
+    value = total_bytes * world / (t_step * 1e-3) / 1e9      # GB/s over all ranks
+    comps = {}
+    for k in KERNELS:
+        t_k = per_kernel[k] / args.steps                  # ms per step for this kernel
+        comps[k] = {"us_per_step": t_k * 1e3, "GBps": bytes_step[k] / (t_k * 1e-3) / 1e9,
+                    "frac_hbm": bytes_step[k] / (t_k * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                    "share": per_kernel[k] / max(sum(per_kernel.values()), 1e-12)}
+    dominant = max(KERNELS, key=lambda k: per_kernel[k])
+    achieved = comps[dominant]["GBps"]
+    roofline = {"kernel": dominant, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": peaks["source"],
+                "algorithmic_bytes_per_launch": bytes_step[dominant] / len(wl.mats),
+                "launches_timed": args.steps * len(wl.mats)}
+    t_unmarked = time_graph(torch, g1, args.steps, stream)
+    iso = isolated_components(torch, cq, ops, device, peaks, stream) if args.components else None
+
+    # end to end: pinned host inputs -> device, the step, results -> host
+    e2e = run_e2e(torch, wl, g1, stream, args.steps)
+    if dist:
+        t = torch.tensor([e2e["ms_per_step"]], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e["ms_per_step"] = float(t.item())
+    e2e_value = total_bytes * world / (e2e["ms_per_step"] * 1e-3) / 1e9
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_step, "ms_per_step_without_event_nodes": t_unmarked,
+            "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "u4 codes / fp32 quantize / bf16 x, fp32 accumulate",
+            "data": "synthetic (seeded Student-t weights, N(0,1) activations, N(0,(0.3s)^2) bf16 residuals)",
+            "config": {"workload": WORKLOAD, "weights_per_step": n_w, "gemv_batch": 1, "gemm_batch": GEMM_M,
+                       "residual": "bf16", "l2": "inputs larger than L2 (377 MB fp32 weights per step)",
+                       "parallelism": f"replicas x{world}", "step": "+".join(KERNELS)},
+            "roofline": roofline,
+            "requant_verify_weights_per_s": n_w / (per_kernel["verify"] / args.steps * 1e-3),
+            "revoke_verify_weights_per_s": n_w / (per_kernel["revoke_verify"] / args.steps * 1e-3),
+            "dequant_gemv_GBps_in_step": comps["gemv"]["GBps"],
+            "components": comps,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
+                    "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e["ms_per_step"]},
+            "gpu_launches": launches_per_step * args.steps if launches_per_step is not None else None,
+            "clocks": clk,
+        }
+        if iso:
+            line["isolated"] = iso
+            line["tokens_per_s"] = iso["decode_32_layers"]["tokens_per_s"]
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_sample_rows)
+    if dist:
+        g1.reset()
+        gK.reset()
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+def run_e2e(torch, wl, graph, stream, steps):
+    """Same step with host buffers: H2D of W, r, x, X before and D2H of y, Y, counts after."""
+    h2d = d2h = 0
+    for m in wl.mats:
+        h2d += sum(t.numel() * t.element_size() for t in (m["w_host"], m["r_host"], m["x_host"], m["X_host"]))
+        d2h += m["y"].numel() * 4 + m["Y"].numel() * 4 + 2 * 8 * 2 + 4
+    outs = [{k: torch.empty_like(m[k], device="cpu").pin_memory() for k in ("y", "Y", "mism", "mism0", "status")}
+            for m in wl.mats]
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(steps):
+            for m in wl.mats:
+                m["w"].copy_(m["w_host"], non_blocking=True)
+                m["r"].copy_(m["r_host"], non_blocking=True)
+                m["x"].copy_(m["x_host"], non_blocking=True)
+                m["X"].copy_(m["X_host"], non_blocking=True)
+            graph.replay()
+            for m, o in zip(wl.mats, outs):
+                for k in o:
+                    o[k].copy_(m[k], non_blocking=True)
+        b.record(stream)
+    torch.cuda.synchronize()
+    return {"ms_per_step": a.elapsed_time(b) / steps, "h2d": h2d, "d2h": d2h}
+
+
+# ---------------------------------------------------------------------------------------
+# the CPU oracle (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------------------
+_SAMPLE_CACHE = {}
+
+
+def _sample_inputs(rows_per_matrix):
+    """Inputs of the CPU sample (built once, not timed): the first rows of each matrix."""
+    if rows_per_matrix in _SAMPLE_CACHE:
+        return _SAMPLE_CACHE[rows_per_matrix]
+    from cell_updates_b200 import synth
+    from oracle import c_oracle as co
+    out = []
+    for idx, (N, K) in enumerate(SHAPES):
+        rows = min(rows_per_matrix, N)
+        w = np.ascontiguousarray(synth.student_t_weights(N, K, seed=1 + 1000 * idx)[:rows])
+        _, scale, _, _ = co.quantize(w)
+        r = synth.normal_residual_bf16(scale, seed=1 + 1000 * idx + 7, rel_sigma=0.3)
+        x = synth.activations(1, K, seed=1 + 1000 * idx + 11, dtype="bf16")
+        X = synth.activations(GEMM_M, K, seed=1 + 1000 * idx + 13, dtype="bf16")
+        out.append((rows, K, w, r, x, X))
+    _SAMPLE_CACHE[rows_per_matrix] = out
+    return out
+
+
+def cpu_sample(rows_per_matrix):
+    """The same step on a row sample of each matrix, on the host cores, with the oracle."""
+    from oracle import c_oracle as co
+    threads = co.default_threads()
+    inputs = _sample_inputs(rows_per_matrix)
+    nbytes = n_w = 0
+    t0 = time.perf_counter()
+    for rows, K, w, r, x, X in inputs:
+        codes, scale, zero, st = co.quantize(w, nthreads=threads)
+        planes = co.pack(codes)
+        rp, _ = co.project_bf16(r, scale)
+        co.verify(planes, scale, zero, r=rp, r_dtype="bf16", nthreads=threads)
+        co.verify(planes, scale, zero, nthreads=threads)
+        co.dequant_matmul_f64(planes, scale, zero, rows, K, x, "bf16", nthreads=threads)
+        co.dequant_matmul_f64(planes, scale, zero, rows, K, X, "bf16", nthreads=threads)
+        n = rows * K
+        n_w += n
+        nbytes += sum(kernel_bytes(n).values())
+    dt = time.perf_counter() - t0
+    return nbytes, n_w, dt, threads
+
+
+def cpu_baseline(rows, min_seconds=10.0):
+    """The oracle as it stands, repeated on the row sample until ~min_seconds of CPU work."""
+    nbytes = n_w = 0
+    dt = 0.0
+    reps = 0
+    while dt < min_seconds:
+        b, n, t, threads = cpu_sample(rows)
+        nbytes, n_w, dt, reps = nbytes + b, n_w + n, dt + t, reps + 1
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {rows} rows of each of the 3 matrices ({n_w // reps} weights), the whole step, "
+                      f"repeated {reps}x ({dt:.1f} s)",
+            "seconds": dt}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    t_all = []
+    warm = max(0, args.warmup)
+    for i in range(warm + args.steps):
+        nbytes, n_w, dt, threads = cpu_sample(args.cpu_sample_rows)
+        if i >= warm:
+            t_all.append(dt)
+    ms = float(np.mean(t_all)) * 1e3
+    value = nbytes / (ms * 1e-3) / 1e9
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp32 / fp64 (CPU oracle)", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample_rows_per_matrix": args.cpu_sample_rows,
+                       "weights_per_step": n_w, "step": "+".join(KERNELS)},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": f"first {args.cpu_sample_rows} rows of each matrix ({n_w} weights)"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="cq", choices=["cq", "reference"])
+    ap.add_argument("--cpu-sample-rows", type=int, default=1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-components", dest="components", action="store_false")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "cq" else args.warmup
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", args.gpus if args.gpus == 1 else 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        line = run_gpu(args, rank, world, local_rank)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

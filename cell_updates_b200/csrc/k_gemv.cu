@@ -12,11 +12,11 @@
 //    128 + q is built from a nibble with one LOP3 as the bf16 bit pattern 0x4300 | q (exact;
 //    bf16 has 8 significant bits), x is bf16 already, so the tensor-core products are exact
 //    and accumulate in fp32 (mma.sync m16n8k16). Scale and zero point are applied per group
-//    in fp32. The contraction over k is a sum, so the kernel may pair any code with any
-//    activation as long as both operands use the same order: each lane feeds the MMA with
-//    the 16 codes it loaded contiguously (one 8-byte load per row and group), and the
-//    activations are staged once per CTA in shared memory in that same order, together
-//    with their per-group sums.
+//    in fp32; the per-group activation sums come from one more MMA with an all-ones A
+//    operand, so the correction is exact for any zero point. The contraction over k is a
+//    sum, so the kernel may pair any code with any activation as long as both operands
+//    use the same order: each lane feeds the MMA with the 16 codes it loaded contiguously
+//    (one 8-byte load per row and group) and permutes its 16 activations to match (PRMT).
 //  * gemv_generic: any format (per-group widths), fp32 or bf16 x, optional residual; one
 //    warp per row, fp32 CUDA-core math. Used for the small fp32-activation cases and for
 //    residual-carrying weights.
@@ -28,12 +28,13 @@ namespace {
 // ------------------------------------------------------------------------------------
 // tensor-core path
 // ------------------------------------------------------------------------------------
-constexpr int kMmaWarps = 4;
-constexpr int kMmaThreads = kMmaWarps * 32;
-constexpr int kKCH = 8;                       // groups per k-chunk (512 columns)
-constexpr int kTilesPerWarp = 1;              // 16-row tiles per warp
-constexpr int kTilesPerCta = kMmaWarps * kTilesPerWarp;
-constexpr int kXRowBytes = kKCH * 64 * 2 + 16;   // padded: conflict-free 16-byte fragment loads
+// One CTA owns a 16-row tile and the whole K range; its warps split K and meet in shared
+// memory at the end, so every output is written once (no atomics, no zero-fill, and the
+// summation order is fixed). Weight and scale loads do not depend on earlier kernels, so
+// they are issued before the programmatic-dependent-launch wait: back-to-back GEMVs in a
+// stream overlap one kernel's weight streaming with the previous kernel's tail.
+constexpr int kTileRows = 16;
+constexpr int kChunk = 8;                      // groups per register batch and warp
 
 __device__ __forceinline__ void mma_bf16_16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -50,100 +51,124 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
   return out;   // (w & 0x000F000F) | 0x43004300
 }
 
-// position of column offset o (0..15 inside a lane's 16 columns) in fragment order:
-// pairs (0,4) (1,5) (2,6) (3,7) (8,12) (9,13) (10,14) (11,15)
-__device__ __forceinline__ int frag_pos(int o) { return (o & 8) + 2 * (o & 3) + ((o >> 2) & 1); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::); }
 
-__global__ void __launch_bounds__(kMmaThreads)
+// 16 consecutive bf16 activations (columns c..c+15) -> the 8 B-fragment registers in the
+// order the codes are fed: pairs (0,4) (1,5) (2,6) (3,7) (8,12) (9,13) (10,14) (11,15)
+__device__ __forceinline__ void x_fragments(const __nv_bfloat16 *p, uint32_t b[8]) {
+  const uint4 lo = __ldg(reinterpret_cast<const uint4 *>(p));
+  const uint4 hi = __ldg(reinterpret_cast<const uint4 *>(p) + 1);
+  b[0] = __byte_perm(lo.x, lo.z, 0x5410); b[1] = __byte_perm(lo.x, lo.z, 0x7632);
+  b[2] = __byte_perm(lo.y, lo.w, 0x5410); b[3] = __byte_perm(lo.y, lo.w, 0x7632);
+  b[4] = __byte_perm(hi.x, hi.z, 0x5410); b[5] = __byte_perm(hi.x, hi.z, 0x7632);
+  b[6] = __byte_perm(hi.y, hi.w, 0x5410); b[7] = __byte_perm(hi.y, hi.w, 0x7632);
+}
+
+template <int W>
+__global__ void __launch_bounds__(W * 32)
 gemv4_mma_kernel(const uint8_t *__restrict__ plane4, const uint16_t *__restrict__ scale,
                  const uint8_t *__restrict__ zero, const __nv_bfloat16 *__restrict__ x, int m,
                  int64_t N, int64_t K, float *__restrict__ y) {
-  __shared__ __align__(16) uint8_t xs[8 * kXRowBytes];   // [n][fragment-ordered columns]
-  __shared__ __align__(16) float xsum[kKCH][8];            // per group, per batch column
+  __shared__ float red[W][kTileRows][8];
+  pdl_launch_dependents();
   const int KG = static_cast<int>(K >> 6);
-  const int kc = blockIdx.x;
-  const int gk0 = kc * kKCH;
-  const int ng = min(kKCH, KG - gk0);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-
-  // ---- stage x[:, chunk] in fragment order, plus per-group sums -------------------------
-  for (int p = warp; p < 8 * kKCH; p += kMmaWarps) {
-    const int n = p / kKCH, gl = p % kKCH;
-    float v0 = 0.0f, v1 = 0.0f;
-    uint32_t raw = 0;
-    if (n < m && gl < ng) {
-      raw = __ldg(reinterpret_cast<const uint32_t *>(x + static_cast<int64_t>(n) * K + (gk0 + gl) * 64) + lane);
-      v0 = __uint_as_float(raw << 16);
-      v1 = __uint_as_float(raw & 0xFFFF0000u);
-    }
-    const int c0 = 2 * lane;                 // columns c0, c0+1 of this group
-    const int blk = c0 >> 4, o0 = c0 & 15;
-    uint16_t *row = reinterpret_cast<uint16_t *>(xs + n * kXRowBytes) + gl * 64 + blk * 16;
-    row[frag_pos(o0)] = static_cast<uint16_t>(raw & 0xFFFFu);
-    row[frag_pos(o0 + 1)] = static_cast<uint16_t>(raw >> 16);
-    float sum = v0 + v1;
-#pragma unroll
-    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0) xsum[gl][n] = sum;
-  }
-  __syncthreads();
-
   const int gid = lane >> 2, tig = lane & 3;
+  const int64_t tile = blockIdx.x;
+  const int64_t r0 = tile * kTileRows + gid, r1 = r0 + 8;
+  const int64_t lr0 = r0 < N ? r0 : N - 1, lr1 = r1 < N ? r1 : N - 1;
   const int64_t half_k = K >> 1;
-  for (int t = 0; t < kTilesPerWarp; ++t) {
-    const int64_t tile = static_cast<int64_t>(blockIdx.y) * kTilesPerCta + warp * kTilesPerWarp + t;
-    const int64_t r0 = tile * 16 + gid, r1 = r0 + 8;
-    if (tile * 16 >= N) break;
-    const int64_t lr0 = r0 < N ? r0 : N - 1, lr1 = r1 < N ? r1 : N - 1;
-    // issue every weight load of the chunk first (16 bytes per row and group per lane)
-    uint2 a0[kKCH], a1[kKCH];
-    float s0[kKCH], s1[kKCH], zc0[kKCH], zc1[kKCH];
+  const int per = (KG + W - 1) / W;
+  const int g_begin = min(warp * per, KG), g_end = min(g_begin + per, KG);
+  const uint8_t *row0 = plane4 + lr0 * half_k + tig * 8;
+  const uint8_t *row1 = plane4 + lr1 * half_k + tig * 8;
+  const uint16_t *srow0 = scale + lr0 * KG, *srow1 = scale + lr1 * KG;
+  const uint8_t *zrow0 = zero + lr0 * KG, *zrow1 = zero + lr1 * KG;
+  const bool has_x = gid < m;
+  const __nv_bfloat16 *xrow = x + static_cast<int64_t>(has_x ? gid : 0) * K + tig * 16;
+  const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};   // bf16 1.0
+
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  bool waited = false;
+  for (int c0 = g_begin; c0 < g_end; c0 += kChunk) {
+    const int nc = min(kChunk, g_end - c0);
+    uint2 a0[kChunk], a1[kChunk];
+    float s0[kChunk], s1[kChunk], zc0[kChunk], zc1[kChunk];
 #pragma unroll
-    for (int j = 0; j < kKCH; ++j) {
-      if (j < ng) {
-        const int64_t gk = gk0 + j;
-        a0[j] = __ldcs(reinterpret_cast<const uint2 *>(plane4 + lr0 * half_k + gk * 32 + tig * 8));
-        a1[j] = __ldcs(reinterpret_cast<const uint2 *>(plane4 + lr1 * half_k + gk * 32 + tig * 8));
-        s0[j] = f16_bits_to_f32(__ldg(scale + lr0 * KG + gk));
-        s1[j] = f16_bits_to_f32(__ldg(scale + lr1 * KG + gk));
-        zc0[j] = 128.0f + static_cast<float>(__ldg(zero + lr0 * KG + gk));
-        zc1[j] = 128.0f + static_cast<float>(__ldg(zero + lr1 * KG + gk));
+    for (int j = 0; j < kChunk; ++j) {
+      if (j < nc) {
+        const int gk = c0 + j;
+        a0[j] = __ldcs(reinterpret_cast<const uint2 *>(row0 + gk * 32));
+        a1[j] = __ldcs(reinterpret_cast<const uint2 *>(row1 + gk * 32));
+        s0[j] = f16_bits_to_f32(__ldg(srow0 + gk));
+        s1[j] = f16_bits_to_f32(__ldg(srow1 + gk));
+        zc0[j] = 128.0f + static_cast<float>(__ldg(zrow0 + gk));
+        zc1[j] = 128.0f + static_cast<float>(__ldg(zrow1 + gk));
       }
     }
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (!waited) {
+      pdl_wait();        // x may be the output of the previous kernel in the stream
+      waited = true;
+    }
 #pragma unroll
-    for (int j = 0; j < kKCH; ++j) {
-      if (j < ng) {
-        const uint4 *bp = reinterpret_cast<const uint4 *>(xs + gid * kXRowBytes + (j * 64 + tig * 16) * 2);
-        const uint4 bA = bp[0], bB = bp[1];
-        const uint32_t bx[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
+    for (int j = 0; j < kChunk; ++j) {
+      if (j < nc) {
+        const int gk = c0 + j;
+        uint32_t bx[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (has_x) x_fragments(xrow + gk * 64, bx);
         float p[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        float xs[4] = {0.0f, 0.0f, 0.0f, 0.0f};     // per-column sums of x over the group
         const uint32_t w0[2] = {a0[j].x, a0[j].y}, w1[2] = {a1[j].x, a1[j].y};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          // codes k..k+7 of row r0 in w0[h], of row r1 in w1[h]; two MMAs per word
           const uint32_t A0[4] = {nib_pair(w0[h]), nib_pair(w1[h]), nib_pair(w0[h] >> 4), nib_pair(w1[h] >> 4)};
           mma_bf16_16816(p, A0, bx[4 * h + 0], bx[4 * h + 1]);
+          mma_bf16_16816(xs, ones, bx[4 * h + 0], bx[4 * h + 1]);
           const uint32_t A1[4] = {nib_pair(w0[h] >> 8), nib_pair(w1[h] >> 8), nib_pair(w0[h] >> 12), nib_pair(w1[h] >> 12)};
           mma_bf16_16816(p, A1, bx[4 * h + 2], bx[4 * h + 3]);
+          mma_bf16_16816(xs, ones, bx[4 * h + 2], bx[4 * h + 3]);
         }
-        const float2 X = *reinterpret_cast<const float2 *>(&xsum[j][2 * tig]);
-        acc[0] = fmaf(s0[j], fmaf(-zc0[j], X.x, p[0]), acc[0]);
-        acc[1] = fmaf(s0[j], fmaf(-zc0[j], X.y, p[1]), acc[1]);
-        acc[2] = fmaf(s1[j], fmaf(-zc1[j], X.x, p[2]), acc[2]);
-        acc[3] = fmaf(s1[j], fmaf(-zc1[j], X.y, p[3]), acc[3]);
+        // sum_k (q - z) x = sum_k (128 + q) x - (128 + z) sum_k x, in fp32
+        acc[0] = fmaf(s0[j], fmaf(-zc0[j], xs[0], p[0]), acc[0]);
+        acc[1] = fmaf(s0[j], fmaf(-zc0[j], xs[1], p[1]), acc[1]);
+        acc[2] = fmaf(s1[j], fmaf(-zc1[j], xs[2], p[2]), acc[2]);
+        acc[3] = fmaf(s1[j], fmaf(-zc1[j], xs[3], p[3]), acc[3]);
       }
     }
-    const int c0 = 2 * tig, c1 = c0 + 1;
-    if (r0 < N) {
-      if (c0 < m) atomicAdd(y + static_cast<int64_t>(c0) * N + r0, acc[0]);
-      if (c1 < m) atomicAdd(y + static_cast<int64_t>(c1) * N + r0, acc[1]);
-    }
-    if (r1 < N) {
-      if (c0 < m) atomicAdd(y + static_cast<int64_t>(c0) * N + r1, acc[2]);
-      if (c1 < m) atomicAdd(y + static_cast<int64_t>(c1) * N + r1, acc[3]);
+  }
+  if (!waited) pdl_wait();
+  red[warp][gid][2 * tig] = acc[0];
+  red[warp][gid][2 * tig + 1] = acc[1];
+  red[warp][gid + 8][2 * tig] = acc[2];
+  red[warp][gid + 8][2 * tig + 1] = acc[3];
+  __syncthreads();
+  if (threadIdx.x < kTileRows * 8) {
+    const int row = threadIdx.x & 15, col = threadIdx.x >> 4;
+    const int64_t r = tile * kTileRows + row;
+    if (col < m && r < N) {
+      float v = 0.0f;
+#pragma unroll
+      for (int w = 0; w < W; ++w) v += red[w][row][col];
+      y[static_cast<int64_t>(col) * N + r] = v;
     }
   }
+}
+
+template <int W>
+cudaError_t launch_gemv4(const cq_qweight &qw, const void *x, int m, float *y, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((qw.rows + kTileRows - 1) / kTileRows));
+  cfg.blockDim = dim3(W * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv4_mma_kernel<W>, qw.plane[2], qw.scale, qw.zero,
+                            static_cast<const __nv_bfloat16 *>(x), m, qw.rows, qw.cols, y);
 }
 
 // ------------------------------------------------------------------------------------
@@ -225,14 +250,11 @@ cq_status launch_gemv(const cq_qweight &qw, const void *x, cq_dtype xdt, int m, 
   if (K == 0) return cuda_check(cudaMemsetAsync(y, 0, sizeof(float) * m * N, s), "cq_dequant_gemv: zero y");
   const bool tc = qw.bits == nullptr && qw.residual == nullptr && xdt == CQ_BF16;
   if (tc) {
-    cq_status st = cuda_check(cudaMemsetAsync(y, 0, sizeof(float) * m * N, s), "cq_dequant_gemv: zero y");
-    if (st != CQ_OK) return st;
+    // warps per tile: enough K-slices to keep ~8 groups (4 KiB of codes) per warp in flight
     const int64_t KG = K >> 6;
-    dim3 grid(static_cast<unsigned>((KG + kKCH - 1) / kKCH),
-              static_cast<unsigned>((N + 16 * kTilesPerCta - 1) / (16 * kTilesPerCta)));
-    gemv4_mma_kernel<<<grid, kMmaThreads, 0, s>>>(qw.plane[2], qw.scale, qw.zero,
-                                                  static_cast<const __nv_bfloat16 *>(x), m, N, K, y);
-    return launch_check("cq_dequant_gemv");
+    (void)KG;
+    const cudaError_t e = launch_gemv4<8>(qw, x, m, y, s);
+    return cuda_check(e, "cq_dequant_gemv");
   }
   const int64_t need = (N + 7) / 8;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;

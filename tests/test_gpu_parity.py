@@ -262,10 +262,17 @@ def test_gemv_varbits(m):
     check_matmul(host(ops.gemv(qw, x_d)), y_ref, f"vbq m={m}")
 
 
-@pytest.mark.parametrize("m", [16, 64])
-def test_gemm_batches(m):
-    qw, x_d, y_ref, _ = _matmul_case(384, 64 * 40, m, "bf16", seed=m)
-    check_matmul(host(ops.gemm(qw, x_d)), y_ref, f"gemm m={m}")
+@pytest.mark.parametrize("rows,cols,m", [(384, 64 * 40, 16), (384, 64 * 40, 64), (200, 64 * 7, 17),
+                                         (1000, 4096, 33), (128, 64, 100), (2500, 2048, 256),
+                                         (4096, 4096, 64)])
+def test_gemm_tensor_core(rows, cols, m):
+    qw, x_d, y_ref, _ = _matmul_case(rows, cols, m, "bf16", seed=rows + m)
+    check_matmul(host(ops.gemm(qw, x_d)), y_ref, f"gemm {rows}x{cols} m={m}")
+
+
+def test_gemm_small_batch_uses_gemv_slices():
+    qw, x_d, y_ref, _ = _matmul_case(300, 64 * 21, 12, "bf16", seed=12)
+    check_matmul(host(ops.gemm(qw, x_d)), y_ref, "gemm m=12")
 
 
 def test_gemm_bf16_residual_uses_exact_formula():
