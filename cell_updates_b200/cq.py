@@ -23,7 +23,7 @@ QSTATUS_NONFINITE, QSTATUS_RANGE, QSTATUS_BADBITS = 1, 2, 4
 # every symbol include/cq.h declares
 EXPORTS = ["cq_quantize", "cq_varbits_index", "cq_pack_varbits", "cq_unpack_varbits",
            "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemm",
-           "cq_gemm_workspace", "cq_last_error", "cq_status_string"]
+           "cq_dequant_gemm_static", "cq_gemm_workspace", "cq_last_error", "cq_status_string"]
 SYNTH_EXPORTS = ["cqs_normal_f32", "cqs_code_words", "cqs_scales", "cqs_zeros", "cqs_residual_bf16"]
 
 
@@ -59,13 +59,15 @@ def lib():
         L.cq_requant_verify.argtypes = [p, i64, i64, p, p, p, p]
         L.cq_dequant_gemv.argtypes = [p, p, i32, i32, p, p]
         L.cq_dequant_gemm.argtypes = [p, p, i32, i32, p, p, C.c_size_t, p]
+        L.cq_dequant_gemm_static.argtypes = [p, p, i32, i32, p, p]
         L.cq_gemm_workspace.argtypes = [i64, i64, i32]
         L.cq_gemm_workspace.restype = C.c_size_t
         L.cq_last_error.restype = C.c_char_p
         L.cq_status_string.argtypes = [i32]
         L.cq_status_string.restype = C.c_char_p
         for name in ("cq_quantize", "cq_varbits_index", "cq_pack_varbits", "cq_unpack_varbits",
-                     "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemm"):
+                     "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemm",
+                     "cq_dequant_gemm_static"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -195,6 +197,13 @@ def cq_dequant_gemm(qw, x, y, workspace=None, stream=None):
     nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib().cq_dequant_gemm(C.byref(s), _ptr(x), _dtype_code(x), m, _ptr(y), _ptr(workspace), nbytes,
                                  _stream(stream)), "cq_dequant_gemm")
+
+
+def cq_dequant_gemm_static(qw, x, y, stream=None):
+    """cq_dequant_gemm without a workspace: the library's own static scratch (see include/cq.h)."""
+    s = qw.struct()
+    _check(lib().cq_dequant_gemm_static(C.byref(s), _ptr(x), _dtype_code(x), x.shape[0], _ptr(y), _stream(stream)),
+           "cq_dequant_gemm_static")
 
 
 def cq_last_error():

@@ -403,3 +403,59 @@ cq_status launch_gemm_tc(const cq_qweight &qw, const void *x, int m, float *y, v
 }
 
 }  // namespace cq
+
+// ---- entry point for callers that cannot allocate device memory --------------------------
+//
+// cq_dequant_gemm_static runs the same GEMM with its scratch in this file-scope device
+// array instead of a caller-provided workspace. Each GPU that loads the library keeps the
+// array until the process exits. In host code the array's name only stands in for it, so the
+// device address is looked up once per device (cudaGetSymbolAddress, with that device
+// current) and passed to the kernel.
+namespace cq {
+namespace {
+
+constexpr size_t kStaticScratchBytes = 4096;
+__device__ __align__(256) unsigned char g_gemm_scratch[kStaticScratchBytes];
+
+constexpr int kMaxScratchDevices = 64;
+void *g_scratch_ptr[kMaxScratchDevices];
+cudaError_t g_scratch_err[kMaxScratchDevices];
+std::once_flag g_scratch_once[kMaxScratchDevices];
+
+cq_status static_scratch(void **out) {
+  int dev = 0;
+  cq_status st = cuda_check(cudaGetDevice(&dev), "cq_dequant_gemm_static: current device");
+  if (st != CQ_OK) return st;
+  if (dev < 0 || dev >= kMaxScratchDevices)
+    return fail(CQ_ERR_RANGE, "cq_dequant_gemm_static: device %d beyond the %d supported", dev, kMaxScratchDevices);
+  std::call_once(g_scratch_once[dev], [dev] {
+    void *p = nullptr;
+    g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_gemm_scratch);
+    g_scratch_ptr[dev] = g_scratch_err[dev] == cudaSuccess ? p : nullptr;
+  });
+  if (g_scratch_err[dev] != cudaSuccess || !g_scratch_ptr[dev])
+    return fail(CQ_ERR_CUDA, "cq_dequant_gemm_static: scratch address on device %d: %s", dev,
+                cudaGetErrorString(g_scratch_err[dev]));
+  *out = g_scratch_ptr[dev];
+  return CQ_OK;
+}
+
+}  // namespace
+}  // namespace cq
+
+extern "C" cq_status cq_dequant_gemm_static(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m, float *y,
+                                            cq_stream_t stream) {
+  using namespace cq;
+  const char *fn = "cq_dequant_gemm_static";
+  void *scratch = nullptr;
+  cq_status st = static_scratch(&scratch);
+  if (st != CQ_OK) return st;
+  if (qw && x_dtype == CQ_BF16 && m >= 16 && gemm_tc_eligible(*qw, x_dtype, m)) {
+    const size_t need = gemm_tc_workspace(qw->rows, qw->cols, m);
+    if (need > kStaticScratchBytes)
+      return fail(CQ_ERR_RANGE, "%s: this shape needs %zu bytes of scratch, the static buffer holds %zu", fn, need,
+                  kStaticScratchBytes);
+  }
+  // the regular entry point does the validation and dispatch; the scratch is the static array
+  return cq_dequant_gemm(qw, x, x_dtype, m, y, scratch, kStaticScratchBytes, stream);
+}

@@ -168,6 +168,24 @@ cq_status cq_dequant_gemv(const cq_qweight *qw, const void *x, cq_dtype x_dtype,
 cq_status cq_dequant_gemm(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m,
                           float *y, void *workspace, size_t workspace_bytes, cq_stream_t stream);
 
+/*
+ * cq_dequant_gemm_static -- cq_dequant_gemm for callers that cannot allocate device memory:
+ * no workspace argument, and no cudaMalloc, cudaFree or other allocating call inside. It is
+ * meant for code that runs where allocation is not allowed or not wanted after start-up: a
+ * plug-in that is handed device buffers by a host framework that owns all device memory, or a
+ * serving loop with a fixed memory budget where an allocation could block on the device or
+ * fail at the worst moment. The pages have no counterpart to this call.
+ * Its scratch is a 4096-byte array inside the library that every GPU which loads the library
+ * keeps until the process exits. A shape that would need more scratch than that is refused
+ * with CQ_ERR_RANGE (no shape does today: the GEMM needs 16 bytes). The first call on a device
+ * looks up the array's device address with that device current; make that first call before
+ * any stream capture. All calls share the array and the call clears what must start at zero,
+ * but calls that overlap on the GPU (other streams, other threads) race on it.
+ * Arguments, results and errors are otherwise those of cq_dequant_gemm.
+ */
+cq_status cq_dequant_gemm_static(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m,
+                                 float *y, cq_stream_t stream);
+
 /* Bytes of workspace cq_dequant_gemm needs for this shape (host function, no GPU work). */
 size_t cq_gemm_workspace(int64_t rows, int64_t cols, int m);
 
