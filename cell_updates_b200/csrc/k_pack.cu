@@ -1,8 +1,8 @@
-// k_pack.cu -- packed low-bit storage for per-group widths.
+// k_pack.cu -- bit-packed planes for per-group widths.
 //
 // [VBQ] "In-Cell Learning: Language Models That Update Their Own Weights in Sequence
-// Without Changing the File They Ship", abstract: the per-group allocation maps directly
-// to packed low-bit storage. The layout (one plane per width, row-major rank of the group
+// Without Changing the File They Ship", abstract: because widths are chosen per group, the
+// codes can be stored densely packed at their own widths. The layout (one plane per width, row-major rank of the group
 // among groups of its width, LSB-first codes) is defined in include/cq.h.
 //
 // Work unit: eight lanes per group, one lane per eight consecutive codes. Lane `sub` of a

@@ -1,8 +1,9 @@
 // k_project.cu -- projection of the per-weight residual into its quantization cell.
 //
 // [CF] "Nothing Changed but the Model: CellFill -- Bounded In-Cell Learning for
-// Bit-Identical, Revocable Updates to Quantized LLMs", Abstract: the residual must stay
-// strictly inside each decision cell; the constrained dense path projects into the cells.
+// Bit-Identical, Revocable Updates to Quantized LLMs", Abstract: an update is carried by a
+// residual that may not leave the rounding cell of its weight; the constrained training path
+// enforces this by clamping (projecting) the residual back into the cell.
 // Reading: half-width c = (0.5 - 2^-10) * s (exact in binary32: 9 x 11 significant bits);
 // a bf16 residual uses c rounded toward zero to bf16, so the clamp never rounds outward.
 // The clamp is written with comparisons so that a NaN residual passes through unchanged.

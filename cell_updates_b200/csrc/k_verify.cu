@@ -1,9 +1,9 @@
 // k_verify.cu -- bit-exact re-quantization check of a quantized release (+ residual).
 //
 // [CF] "Nothing Changed but the Model: CellFill -- Bounded In-Cell Learning for
-// Bit-Identical, Revocable Updates to Quantized LLMs", Abstract: re-quantization of the
-// served weights returns the released artifact bit for bit (a machine-checkable
-// guarantee), and dropping the residual revokes the update exactly. For every weight:
+// Bit-Identical, Revocable Updates to Quantized LLMs", Abstract: rounding the served
+// weights again with the frozen grid must reproduce the released codes exactly, which a
+// program can check, and removing the residual must undo the update. For every weight:
 //     k = q - z;  w' = RN32(RN32(s*k) + r);  t = RN32(w'/s);  q' = clamp(rne(t) + z, 0, L)
 // and a mismatch is q' != q, a NaN t included.
 //

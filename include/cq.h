@@ -5,13 +5,14 @@
  *   [VBQ] "In-Cell Learning: Language Models That Update Their Own Weights in Sequence
  *         Without Changing the File They Ship" (thelatestinai.com/papers/2608.20873),
  *         abstract: every contiguous group of 64 weights has its own bit-width from
- *         {1,2,4,8}; the allocation maps onto packed low-bit storage; fused
+ *         {1,2,4,8}; the codes are kept bit-packed at their widths; fused
  *         dequantize-and-multiply kernels serve memory-bound decode.
  *   [CF]  "Nothing Changed but the Model: CellFill -- Bounded In-Cell Learning for
  *         Bit-Identical, Revocable Updates to Quantized LLMs", Abstract: a 4-bit release
  *         whose integer codes and scales stay frozen; updates live in a per-weight
- *         residual strictly inside each quantization cell; re-quantization returns the
- *         release bit for bit; dropping the residual revokes the update; drift is bounded.
+ *         residual confined to the rounding cell of each weight; rounding again gives the
+ *         released codes exactly; removing the residual undoes the update; the change
+ *         of every weight is limited.
  *   [SLQ] listing page thelatestinai.com/papers/2512.18934, SLQ abstract: asymmetric
  *         quantization (hence the zero point).
  *
@@ -68,7 +69,7 @@ typedef enum { CQ_F32 = 0, CQ_BF16 = 1 } cq_dtype;
 #define CQ_QSTATUS_BADBITS 4u   /* bits[g] not in {1,2,4,8}: written as s=+0, z=0, q=0        */
 
 /*
- * A quantized weight matrix ([VBQ] packed low-bit storage, [CF] frozen codes + scales).
+ * A quantized weight matrix ([VBQ] bit-packed per-group widths, [CF] frozen codes + scales).
  * Packed layout: one plane per width b in {1,2,4,8} (plane[0..3] for b = 1,2,4,8). Group g
  * of width b occupies 8*b bytes of plane b starting at byte offset[g]; code j of the group
  * is in bits [j*b, (j+1)*b) of that little-endian byte string, least significant bit first.
@@ -100,7 +101,7 @@ cq_status cq_quantize(const float *w, int64_t rows, int64_t cols, const uint8_t 
                       cq_stream_t stream);
 
 /*
- * cq_varbits_index -- [VBQ] "maps directly to packed low-bit storage": builds offset[G] (byte
+ * cq_varbits_index -- [VBQ] codes stored bit-packed at their group widths: builds offset[G] (byte
  * offsets as in cq_qweight) and plane_bytes[4] (device, uint64: bytes needed by each plane).
  * bits: [G]. Device-side, widths outside {1,2,4,8} count as width 0 (offset 0, no bytes);
  * pack and quantize flag them. n_groups <= 2^26 (byte offsets are 32-bit) else CQ_ERR_RANGE.
@@ -121,7 +122,7 @@ cq_status cq_pack_varbits(const uint8_t *codes, int64_t n_groups, const uint8_t 
 cq_status cq_unpack_varbits(const cq_qweight *qw, uint8_t *codes, cq_stream_t stream);
 
 /*
- * cq_project_residual -- [CF] "projecting into the cells": in place,
+ * cq_project_residual -- [CF] clamping the residual back into its rounding cell, in place:
  *     r <- c if r > c;  -c if r < -c;  r otherwise,   c = (0.5 - 2^-10) * s_group,
  * for fp32 r; for bf16 r the bound is c rounded toward zero to bf16 (never outward).
  * A NaN residual is left as it is (requant-verify then reports it). r: [n] (16-byte aligned),
@@ -132,8 +133,8 @@ cq_status cq_project_residual(void *r, cq_dtype dtype, const uint16_t *scale, in
                               uint64_t *n_clamped, cq_stream_t stream);
 
 /*
- * cq_requant_verify -- [CF] "re-quantization returns the released artifact bit-for-bit" and
- * "exactly revocable by dropping the residual" (qw->residual = NULL). For each weight i in
+ * cq_requant_verify -- [CF] rounding the served weights again must give the released codes
+ * exactly, and with the residual removed (qw->residual = NULL) the update is undone. For weight i in
  * [first_w, first_w + n_w) with code q, scale s, zero z, width b:
  *     w' = RN32(RN32(s*(q-z)) + r_i);  t = RN32(w'/s);  q' = clamp(rne(t) + z, 0, 2^b-1)
  * and a mismatch is q' != q (a NaN t is a mismatch). first_w and n_w are multiples of 64

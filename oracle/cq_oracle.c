@@ -10,13 +10,13 @@
  *   [VBQ]  "In-Cell Learning: Language Models That Update Their Own Weights in Sequence
  *          Without Changing the File They Ship" (thelatestinai.com/papers/2608.20873),
  *          abstract: contiguous groups of 64 weights, each group with its own bit-width
- *          from {1,2,4,8}; the allocation maps to packed low-bit storage; fused
+ *          from {1,2,4,8}; codes are stored bit-packed at their widths; fused
  *          dequantize-and-multiply kernels for memory-bound decode.
  *   [CF]   "Nothing Changed but the Model: CellFill -- Bounded In-Cell Learning for
  *          Bit-Identical, Revocable Updates to Quantized LLMs", Abstract: 4-bit release
  *          with frozen integer codes and scales; a per-weight residual kept strictly
  *          inside each quantization decision cell; re-quantization returns the release
- *          bit for bit; dropping the residual revokes the update; drift is bounded.
+ *          exactly; removing the residual undoes the update; the weight change is limited.
  *   [SLQ]  same listing page 2 (thelatestinai.com/papers/2512.18934), SLQ abstract:
  *          asymmetric quantization (the reason for the zero point z).
  * The quantizer formula itself is not printed on the pages.  The oracle takes the
@@ -195,7 +195,7 @@ uint32_t oq_quantize_group(const float *w, int b, uint8_t *q, uint16_t *s_out, u
 }
 
 /* ------------------------------------------------------------------------------
- * Packed storage ([VBQ]: the per-group allocation maps to packed low-bit storage).
+ * Packed storage ([VBQ]: per-group widths are stored bit-packed).
  * One plane per bit-width b in {1,2,4,8}.  A group of width b occupies 8*b bytes of
  * plane b, starting at byte offset[g]; code j of the group sits in bits
  * [j*b, (j+1)*b) of that little-endian byte string, least significant bit first.
@@ -276,7 +276,7 @@ int oq_unpack(const uint8_t *plane1, const uint8_t *plane2, const uint8_t *plane
 
 /* ------------------------------------------------------------------------------
  * Projection of the residual into the cell ([CF]: new knowledge lives only in a
- * per-weight residual strictly inside each decision cell; the dense path projects
+ * per-weight residual that may not leave its rounding cell; the dense path clamps
  * into the cells).  Reading: the cell half-width is c = (0.5 - 2^-10) * s for every
  * code (the strict margin 2^-10), c = RN32(0.5-2^-10) * s is exact (9 x 11 bits).
  *   fp32 r:  r <- c if r > c;  -c if r < -c;  r otherwise (a NaN is left as it is)

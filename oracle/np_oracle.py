@@ -9,10 +9,10 @@ bit-plane layout.  It never calls the C oracle.
 Sources (cited by page title and section):
   [VBQ] "In-Cell Learning: Language Models That Update Their Own Weights in Sequence
         Without Changing the File They Ship", abstract: groups of 64 weights, per-group
-        width from {1,2,4,8}, packed low-bit storage, fused dequantize-and-multiply.
+        width from {1,2,4,8}, bit-packed storage, fused dequantize-and-multiply.
   [CF]  "Nothing Changed but the Model: CellFill -- Bounded In-Cell Learning for
         Bit-Identical, Revocable Updates to Quantized LLMs", Abstract: frozen 4-bit codes
-        and scales, residual strictly inside each cell, bit-for-bit re-quantization,
+        and scales, residual confined to its rounding cell, exact re-quantization,
         revocation by dropping the residual, bounded drift.
   [SLQ] page 2 listing, SLQ abstract: asymmetric quantization.
 """
@@ -21,7 +21,7 @@ import numpy as np
 GROUP = 64
 ST_NONFINITE, ST_RANGE, ST_BADBITS = 1, 2, 4
 WIDTHS = (1, 2, 4, 8)
-CELL = np.float32(0.5 - 2.0 ** -10)   # [CF] strictly inside the cell, margin 2^-10
+CELL = np.float32(0.5 - 2.0 ** -10)   # [CF] inside the rounding cell with a 2^-10 margin
 SMIN = np.float32(2.0 ** -14)         # smallest normal fp16: floor of the scale
 
 
@@ -56,7 +56,7 @@ def _zero_point(wmin, sf, L):
 
 
 def _cell_halfwidth_f32(sf):
-    """(0.5 - 2^-10) * s: strictly inside the decision cell"""
+    """(0.5 - 2^-10) * s: the cell half-width less a 2^-10 margin"""
     return CELL * sf
 
 
@@ -117,7 +117,7 @@ def quantize(w, bits=None):
     return codes, scale, zero, status
 
 
-# ---- packed storage ([VBQ]: allocation maps to packed low-bit storage) ----------------
+# ---- packed storage ([VBQ]: per-group widths stored bit-packed) ----------------------
 
 def varbits_index(bits):
     bits = np.asarray(bits, np.int64)
