@@ -110,7 +110,7 @@ cq_status cq_quantize(const float *w, int64_t rows, int64_t cols, const uint8_t 
   if (G > 0) {
     if (!w || !codes || !scale || !zero) return fail(CQ_ERR_ARG, "%s: NULL buffer", fn);
     if (!aligned16(w)) return fail(CQ_ERR_ALIGN, "%s: w is not 16-byte aligned", fn);
-    if (!aligned8(codes)) return fail(CQ_ERR_ALIGN, "%s: codes is not 8-byte aligned", fn);
+    if (!aligned16(codes)) return fail(CQ_ERR_ALIGN, "%s: codes is not 16-byte aligned", fn);
   }
   return launch_quantize(w, G, bits, codes, scale, zero, status_word, reinterpret_cast<cudaStream_t>(stream));
 }

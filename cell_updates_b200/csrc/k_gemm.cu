@@ -11,14 +11,15 @@
 //
 // Structure (one CTA per SM, persistent; work = (128-row tile, group) items split evenly
 // over the CTAs in row-major order, so a CTA covers a contiguous K range of one or two tiles):
-//   warp 0     TMA producer: the tile's 4-bit codes (128 rows x 32 B) and the activations of
-//              the group (m rows x 64 bf16, 128-byte swizzled = the UMMA K-major layout)
-//   warp 1     MMA issuer: four tcgen05.mma (M=128, N=NT, K=16) per group into one of two
-//              tensor-memory accumulators; commits release the stage and publish the group
-//   warps 2-5  dequantize: thread r turns row r's 64 codes into bf16 (q - z) and writes them
-//              in the 128-byte swizzled K-major layout the MMA descriptor expects
-//   warps 6-9  epilogue: tcgen05.ld the group's 128 x NT fp32 sums (one row per thread),
-//              acc += s * sum; at the end of a tile (or of the CTA's range) add to y
+//   warp 0      TMA producer: code blocks of 8 groups (two adjacent 128-byte-wide boxes per
+//               row, 128-byte swizzled: long DRAM runs and conflict-free shared reads), and per
+//               group the activations (m rows x 64 bf16, swizzled = the UMMA K-major layout)
+//   warp 1      MMA issuer: four tcgen05.mma (M=128, N=NT, K=16) per group into one of four
+//               tensor-memory accumulators; commits release the A and x stages and publish
+//   warps 2-9   dequantize: each thread turns half a row of the group's codes into bf16
+//               (q - z) in the 128-byte swizzled K-major layout the MMA descriptor expects
+//   warps 10-17 epilogue: tcgen05.ld the group's fp32 sums (one row and half the columns per
+//               thread), acc += s * sum; at the end of a tile (or of the CTA's range) add to y
 // y is zeroed first; tiles split between two CTAs are combined with fp32 atomics.
 // Every barrier wait is bounded: on timeout the CTA raises a status flag, drains what it
 // issued, frees its tensor memory and returns.
@@ -33,20 +34,24 @@ namespace cq {
 namespace {
 
 constexpr int kTileM = 128;
-constexpr int kThreads = 320;
-constexpr uint32_t kCodeBytes = kTileM * 32;      // one group of 4-bit codes for 128 rows
+constexpr int kDeqWarps = 8;                       // two per row quarter: half a row each
+constexpr int kEpiWarps = 8;                       // two per TMEM lane quarter: half the columns each
+constexpr int kThreads = 32 * (2 + kDeqWarps + kEpiWarps);
+constexpr int kBlockGroups = 8;                    // groups per code block (two 128-byte boxes per row)
+constexpr uint32_t kCodeBox = kTileM * 128;        // one swizzled box: 128 rows x 4 groups
+constexpr uint32_t kCodeStage = 2 * kCodeBox;      // 32 KiB
 constexpr uint32_t kABytes = kTileM * 128;         // bf16 A tile: 128 rows x 64 columns
+constexpr int kCodeStages = 2, kAStages = 4, kXStages = 8, kAccBufs = 4;
 constexpr uint32_t kSpinLimit = 1u << 22;          // try_wait rounds before giving up
 
 template <int NT>
 struct Cfg {
   static constexpr uint32_t kXBytes = NT * 128;
-  static constexpr uint32_t kStageBytes = kABytes + kXBytes + kCodeBytes;
-  static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
-  static constexpr uint32_t kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
-  static constexpr uint32_t kSmem = 1024 + kStages * kStageBytes + (4 * kStages + 8) * 8 + 16;
+  static constexpr uint32_t kTmemCols = kAccBufs * NT < 32 ? 32 : kAccBufs * NT;
+  static constexpr int kBars = 2 * kCodeStages + 2 * kAStages + 2 * kXStages + 2 * kAccBufs + 1;
+  static constexpr uint32_t kSmem =
+      1024 + kCodeStages * kCodeStage + kAStages * kABytes + kXStages * kXBytes + kBars * 8 + 16;
 };
-
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -134,6 +139,11 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t *r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
 // (128 + q) pairs in natural column order from one word of 8 nibbles: pair j = columns 2j, 2j+1
@@ -149,21 +159,93 @@ __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
   return d;
 }
 
+// the items of one CTA: (tile, group) pairs, grouped into code blocks of up to 8 groups
+struct ItemWalk {
+  int64_t i;          // current item (tile * KG + g)
+  int tile, g;
+  int block;          // index of the current code block
+  int block_g0;       // first group of the current block
+  bool block_start, block_end, tile_end;
+};
+
+__device__ __forceinline__ void walk_init(ItemWalk &w, int64_t it_begin, int KG) {
+  w.i = it_begin;
+  w.tile = static_cast<int>(it_begin / KG);
+  w.g = static_cast<int>(it_begin % KG);
+  w.block = 0;
+  w.block_g0 = w.g;
+  w.block_start = true;
+}
+
+// flags of the current item, given the CTA's end
+// blocks end on multiples of 8 groups (and at tile and range ends), so every block after the
+// first one of a range starts on an 8-group boundary
+__device__ __forceinline__ void walk_flags(ItemWalk &w, int64_t it_end, int KG) {
+  const bool last = w.i + 1 >= it_end;
+  w.tile_end = (w.g == KG - 1) || last;
+  w.block_end = w.tile_end || (((w.g + 1) & (kBlockGroups - 1)) == 0);
+}
+
+// first (tile, group) of the block after the current one (valid when it exists)
+__device__ __forceinline__ void walk_next_block(const ItemWalk &w, int KG, int &tile, int &g) {
+  const int g_end = (w.block_g0 | (kBlockGroups - 1)) + 1;     // next multiple of 8
+  if (g_end >= KG) {
+    tile = w.tile + 1;
+    g = 0;
+  } else {
+    tile = w.tile;
+    g = g_end;
+  }
+}
+
+// the (up to) 8 per-group bytes / halves of one row for the block starting at group g
+__device__ __forceinline__ void load_block_zeros(const uint8_t *zero, int64_t row, int KG, int g, uint32_t &lo,
+                                                 uint32_t &hi) {
+  uint32_t v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = (g + j < KG && ((g + j) & ~7) == (g & ~7)) ? __ldg(zero + row * KG + g + j) : 0u;
+  lo = v[0] | (v[1] << 8) | (v[2] << 16) | (v[3] << 24);
+  hi = v[4] | (v[5] << 8) | (v[6] << 16) | (v[7] << 24);
+}
+__device__ __forceinline__ void load_block_scales(const uint16_t *scale, int64_t row, int KG, int g, uint32_t (&s)[4]) {
+  uint32_t v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = (g + j < KG && ((g + j) & ~7) == (g & ~7)) ? __ldg(scale + row * KG + g + j) : 0u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) s[j] = v[2 * j] | (v[2 * j + 1] << 16);
+}
+
+__device__ __forceinline__ void walk_next(ItemWalk &w, int KG) {
+  const bool new_block = w.block_end;
+  ++w.i;
+  if (++w.g == KG) {
+    w.g = 0;
+    ++w.tile;
+  }
+  w.block_start = new_block;
+  if (new_block) {
+    ++w.block;
+    w.block_g0 = w.g;
+  }
+}
+
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
                 const uint16_t *__restrict__ scale, const uint8_t *__restrict__ zero, float *__restrict__ y,
                 int m, int64_t N, int KG, int64_t n_items, uint32_t *__restrict__ status) {
   using C = Cfg<NT>;
-  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sA = smem;                               // S x 16 KiB, 1024-aligned
-  uint8_t *sX = sA + S * kABytes;                   // S x NT*128 B, 1024-aligned
-  uint8_t *sC = sX + S * C::kXBytes;                // S x 4 KiB
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sC + S * kCodeBytes);
-  uint64_t *full = bars, *afull = bars + S, *empty = bars + 2 * S, *accf = bars + 3 * S, *acce = accf + 2;
-  uint64_t *drain = acce + 2;
+  uint8_t *sC = smem;                                   // code blocks (1024-aligned, swizzled)
+  uint8_t *sA = sC + kCodeStages * kCodeStage;          // bf16 A tiles (1024-aligned)
+  uint8_t *sX = sA + kAStages * kABytes;                // activation tiles (1024-aligned)
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sX + kXStages * C::kXBytes);
+  uint64_t *c_full = bars, *c_empty = c_full + kCodeStages;
+  uint64_t *a_full = c_empty + kCodeStages, *a_empty = a_full + kAStages;
+  uint64_t *x_full = a_empty + kAStages, *x_empty = x_full + kXStages;
+  uint64_t *acc_full = x_empty + kXStages, *acc_empty = acc_full + kAccBufs;
+  uint64_t *drain = acc_empty + kAccBufs;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile uint32_t *abort_flag = tmem_slot + 1;
 
@@ -173,14 +255,21 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
   const int n_local = static_cast<int>(it_end - it_begin);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(full + s, 1);
-      mbar_init(afull + s, 4);
-      mbar_init(empty + s, 1);
+    for (int i = 0; i < kCodeStages; ++i) {
+      mbar_init(c_full + i, 1);
+      mbar_init(c_empty + i, kDeqWarps);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(accf + b, 1);
-      mbar_init(acce + b, 4);
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(a_full + i, kDeqWarps);
+      mbar_init(a_empty + i, 1);
+    }
+    for (int i = 0; i < kXStages; ++i) {
+      mbar_init(x_full + i, 1);
+      mbar_init(x_empty + i, 1);
+    }
+    for (int i = 0; i < kAccBufs; ++i) {
+      mbar_init(acc_full + i, 1);
+      mbar_init(acc_empty + i, kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0u;
@@ -197,117 +286,178 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer: code blocks and activation tiles ----------------
     if (lane == 0) {
-      int issued = 0;
-      for (int li = 0; li < n_local; ++li) {
-        const int s = li % S;
-        if (!mbar_wait(empty + s, ((li / S) & 1) ^ 1, abort_flag, status)) break;
-        const int64_t i = it_begin + li;
-        const int tile = static_cast<int>(i / KG), g = static_cast<int>(i % KG);
-        mbar_arrive_expect_tx(full + s, kCodeBytes + C::kXBytes);
-        tma_load_2d(sC + s * kCodeBytes, &tm_codes, g * 32, tile * kTileM, full + s);
-        tma_load_2d(sX + s * C::kXBytes, &tm_x, g * 64, 0, full + s);
-        issued = li + 1;
+      ItemWalk w;
+      walk_init(w, it_begin, KG);
+      int code_issued = 0, x_issued = 0;
+      bool ok = true;
+      for (int li = 0; li < n_local && ok; ++li) {
+        walk_flags(w, it_end, KG);
+        if (w.block_start) {
+          const int cs = w.block % kCodeStages;
+          if (!(ok = mbar_wait(c_empty + cs, ((w.block / kCodeStages) & 1) ^ 1, abort_flag, status))) break;
+          mbar_arrive_expect_tx(c_full + cs, kCodeStage);
+          uint8_t *dst = sC + cs * kCodeStage;
+          tma_load_2d(dst, &tm_codes, w.block_g0 * 32, w.tile * kTileM, c_full + cs);
+          tma_load_2d(dst + kCodeBox, &tm_codes, w.block_g0 * 32 + 128, w.tile * kTileM, c_full + cs);
+          code_issued = w.block + 1;
+        }
+        const int xs = li % kXStages;
+        if (!(ok = mbar_wait(x_empty + xs, ((li / kXStages) & 1) ^ 1, abort_flag, status))) break;
+        mbar_arrive_expect_tx(x_full + xs, C::kXBytes);
+        tma_load_2d(sX + xs * C::kXBytes, &tm_x, w.g * 64, 0, x_full + xs);
+        x_issued = li + 1;
+        walk_next(w, KG);
       }
       // every copy this thread started has landed before the CTA may exit
-      for (int li = issued - S > 0 ? issued - S : 0; li < issued; ++li)
-        mbar_wait(full + (li % S), (li / S) & 1, abort_flag, status, false);
+      for (int b = code_issued - kCodeStages > 0 ? code_issued - kCodeStages : 0; b < code_issued; ++b)
+        mbar_wait(c_full + (b % kCodeStages), (b / kCodeStages) & 1, abort_flag, status, false);
+      for (int li = x_issued - kXStages > 0 ? x_issued - kXStages : 0; li < x_issued; ++li)
+        mbar_wait(x_full + (li % kXStages), (li / kXStages) & 1, abort_flag, status, false);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc<NT>();
-      int done = 0;
       for (int li = 0; li < n_local; ++li) {
-        const int s = li % S, b = li & 1;
-        if (!mbar_wait(afull + s, (li / S) & 1, abort_flag, status)) break;
-        if (!mbar_wait(full + s, (li / S) & 1, abort_flag, status)) break;
-        if (!mbar_wait(acce + b, ((li >> 1) & 1) ^ 1, abort_flag, status)) break;
+        const int as = li % kAStages, xs = li % kXStages, b = li % kAccBufs;
+        if (!mbar_wait(a_full + as, (li / kAStages) & 1, abort_flag, status)) break;
+        if (!mbar_wait(x_full + xs, (li / kXStages) & 1, abort_flag, status)) break;
+        if (!mbar_wait(acc_empty + b, ((li / kAccBufs) & 1) ^ 1, abort_flag, status)) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + s * kABytes), b0 = smem_u32(sX + s * C::kXBytes);
+        const uint32_t a0 = smem_u32(sA + as * kABytes), b0 = smem_u32(sX + xs * C::kXBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_bf16(tmem + b * NT, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), idesc, kk > 0);
-        umma_commit(empty + s);
-        umma_commit(accf + b);
-        done = li + 1;
+        umma_commit(a_empty + as);
+        umma_commit(x_empty + xs);
+        umma_commit(acc_full + b);
       }
       // all issued MMAs have completed before tensor memory is released
       umma_commit(drain);
       mbar_wait(drain, 0, abort_flag, status, false);
-      (void)done;
     }
-  } else if (warp < 6) {
-    // ---------------- dequantize: row r of every tile ----------------
-    const int r = (warp - 2) * 32 + lane;
+  } else if (warp < 2 + kDeqWarps) {
+    // ---------------- dequantize: half a row per thread ----------------
+    const int dw = warp - 2;
+    const int r = (dw & 3) * 32 + lane;          // tile row
+    const int half = dw >> 2;                     // columns 32*half .. 32*half+31 of the group
+    ItemWalk w;
+    walk_init(w, it_begin, KG);
+    auto clamp_row = [&](int tile) {
+      const int64_t row = static_cast<int64_t>(tile) * kTileM + r;
+      return row < N ? row : N - 1;
+    };
+    // zero points of the current block and, one block ahead, of the next one
+    uint32_t zlo, zhi, nzlo = 0, nzhi = 0;
+    load_block_zeros(zero, clamp_row(w.tile), KG, w.g, zlo, zhi);
     for (int li = 0; li < n_local; ++li) {
-      const int s = li % S;
-      if (!mbar_wait(full + s, (li / S) & 1, abort_flag, status)) break;
-      const int64_t i = it_begin + li;
-      const int64_t tile = i / KG;
-      const int g = static_cast<int>(i % KG);
-      int64_t row = tile * kTileM + r;
-      row = row < N ? row : N - 1;
-      const uint32_t z = __ldg(zero + row * KG + g);
+      walk_flags(w, it_end, KG);
+      const int cs = w.block % kCodeStages;
+      if (w.block_start) {
+        if (li > 0) {
+          zlo = nzlo;
+          zhi = nzhi;
+        }
+        int nt, ng;
+        walk_next_block(w, KG, nt, ng);
+        if (static_cast<int64_t>(nt) * KG + ng < it_end) load_block_zeros(zero, clamp_row(nt), KG, ng, nzlo, nzhi);
+        if (!mbar_wait(c_full + cs, (w.block / kCodeStages) & 1, abort_flag, status)) break;
+      }
+      const int as = li % kAStages;
+      if (!mbar_wait(a_empty + as, ((li / kAStages) & 1) ^ 1, abort_flag, status)) break;
+      const int jz = w.g - w.block_g0;
+      const uint32_t z = ((jz < 4 ? zlo : zhi) >> (8 * (jz & 3))) & 0xFFu;
       const uint32_t zz = 0x43004300u | z | (z << 16);      // (128 + z) in both halves
-      const uint4 *src = reinterpret_cast<const uint4 *>(sC + s * kCodeBytes + r * 32);
-      const uint4 c0 = src[0], c1 = src[1];
-      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-      uint8_t *dst_row = sA + s * kABytes + r * 128;
+      // group j of the block sits in box j/4, 16-byte chunk (2*(j%4) + half) of the row, swizzled
+      const int j = w.g - w.block_g0;
+      const int chunk = ((j & 3) << 1) | half;
+      const uint4 cw = *reinterpret_cast<const uint4 *>(sC + cs * kCodeStage + (j >> 2) * kCodeBox + r * 128 +
+                                                        ((chunk ^ (r & 7)) << 4));
+      const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+      uint8_t *dst_row = sA + as * kABytes + r * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {       // 16-byte chunk c = columns 8c .. 8c+7
-        const uint32_t w = words[c], w4 = w >> 4;
+      for (int c = 0; c < 4; ++c) {       // A chunk 4*half + c = columns 8(4*half+c) .. +7
+        const uint32_t wd = words[c], w4 = wd >> 4;
         uint4 v;
-        v.x = bf16x2_sub(nat_pair(w, w4, 0x4400u), zz);
-        v.y = bf16x2_sub(nat_pair(w, w4, 0x5511u), zz);
-        v.z = bf16x2_sub(nat_pair(w, w4, 0x6622u), zz);
-        v.w = bf16x2_sub(nat_pair(w, w4, 0x7733u), zz);
-        *reinterpret_cast<uint4 *>(dst_row + ((c ^ (r & 7)) << 4)) = v;
+        v.x = bf16x2_sub(nat_pair(wd, w4, 0x4400u), zz);
+        v.y = bf16x2_sub(nat_pair(wd, w4, 0x5511u), zz);
+        v.z = bf16x2_sub(nat_pair(wd, w4, 0x6622u), zz);
+        v.w = bf16x2_sub(nat_pair(wd, w4, 0x7733u), zz);
+        *reinterpret_cast<uint4 *>(dst_row + ((((half << 2) | c) ^ (r & 7)) << 4)) = v;
       }
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
       __syncwarp();
-      if (lane == 0) mbar_arrive(afull + s);
+      if (lane == 0) {
+        mbar_arrive(a_full + as);
+        if (w.block_end) mbar_arrive(c_empty + cs);
+      }
+      walk_next(w, KG);
     }
   } else {
-    // ---------------- epilogue: row r = TMEM lane ----------------
+    // ---------------- epilogue: row r = TMEM lane, half of the columns ----------------
+    const int ew = warp - 2 - kDeqWarps;
     const int quad = warp & 3;                 // this warp may read TMEM lanes 32*quad .. +31
+    const int chalf = ew >> 2;                 // columns chalf*NT/2 .. +NT/2
+    constexpr int NH = NT / 2;
     const int r = quad * 32 + lane;
-    float acc[NT];
+    float acc[NH];
 #pragma unroll
-    for (int c = 0; c < NT; ++c) acc[c] = 0.0f;
+    for (int c = 0; c < NH; ++c) acc[c] = 0.0f;
+    ItemWalk w;
+    walk_init(w, it_begin, KG);
+    auto clamp_row = [&](int tile) {
+      const int64_t row = static_cast<int64_t>(tile) * kTileM + r;
+      return row < N ? row : N - 1;
+    };
+    // scales of the current block and, one block ahead, of the next one
+    uint32_t sc[4], nsc[4] = {0, 0, 0, 0};
+    load_block_scales(scale, clamp_row(w.tile), KG, w.g, sc);
     for (int li = 0; li < n_local; ++li) {
-      const int b = li & 1;
-      const int64_t i = it_begin + li;
-      const int64_t tile = i / KG;
-      const int g = static_cast<int>(i % KG);
-      int64_t row = tile * kTileM + r;
-      const int64_t lrow = row < N ? row : N - 1;
-      const float sf = f16_bits_to_f32(__ldg(scale + lrow * KG + g));
-      if (!mbar_wait(accf + b, (li >> 1) & 1, abort_flag, status)) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + b * NT;
+      walk_flags(w, it_end, KG);
+      const int b = li % kAccBufs;
+      const int64_t row = static_cast<int64_t>(w.tile) * kTileM + r;
+      if (w.block_start) {
+        if (li > 0) {
 #pragma unroll
-      for (int c0 = 0; c0 < NT; c0 += 16) {
-        uint32_t d[16];
-        tmem_ld16(tbase + c0, d);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) acc[c0 + j] = fmaf(sf, __uint_as_float(d[j]), acc[c0 + j]);
+          for (int j = 0; j < 4; ++j) sc[j] = nsc[j];
+        }
+        int nt, ng;
+        walk_next_block(w, KG, nt, ng);
+        if (static_cast<int64_t>(nt) * KG + ng < it_end) load_block_scales(scale, clamp_row(nt), KG, ng, nsc);
       }
+      const int js = w.g - w.block_g0;
+      const uint32_t sw = js < 2 ? sc[0] : js < 4 ? sc[1] : js < 6 ? sc[2] : sc[3];   // no local-memory indexing
+      const float sf = f16_bits_to_f32(static_cast<uint16_t>(sw >> (16 * (js & 1))));
+      if (!mbar_wait(acc_full + b, (li / kAccBufs) & 1, abort_flag, status)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + b * NT + chalf * NH;
+      uint32_t d[NH];
+      if constexpr (NH >= 16) {
+#pragma unroll
+        for (int c0 = 0; c0 < NH; c0 += 16) tmem_ld16(tbase + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
+      } else {
+        tmem_ld8(tbase, d);
+      }
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce + b);
-      const bool last = (g == KG - 1) || (li == n_local - 1);
-      if (last) {
+      if (lane == 0) mbar_arrive(acc_empty + b);
+#pragma unroll
+      for (int c = 0; c < NH; ++c) acc[c] = fmaf(sf, __uint_as_float(d[c]), acc[c]);
+      if (w.tile_end) {
         if (row < N) {
 #pragma unroll
-          for (int c = 0; c < NT; ++c)
-            if (c < m) atomicAdd(y + static_cast<int64_t>(c) * N + row, acc[c]);
+          for (int c = 0; c < NH; ++c) {
+            const int col = chalf * NH + c;
+            if (col < m) atomicAdd(y + static_cast<int64_t>(col) * N + row, acc[c]);
+          }
         }
 #pragma unroll
-        for (int c = 0; c < NT; ++c) acc[c] = 0.0f;
+        for (int c = 0; c < NH; ++c) acc[c] = 0.0f;
       }
+      walk_next(w, KG);
     }
   }
   __syncthreads();
@@ -342,10 +492,10 @@ cq_status launch_nt(const cq_qweight &qw, const void *x, int m, float *y, uint32
   {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-    cuuint32_t box[2] = {32, kTileM};
+    cuuint32_t box[2] = {128, kTileM};
     cuuint32_t es[2] = {1, 1};
     CUresult r = encode(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(qw.plane[2]), dims, strides,
-                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(CQ_ERR_CUDA, "cq_dequant_gemm: code tensor map (%d)", (int)r);
   }

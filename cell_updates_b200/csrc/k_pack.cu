@@ -55,6 +55,8 @@ __device__ __forceinline__ uint64_t load_bytes(const uint8_t *src, int b) {
 
 struct Planes {
   uint8_t *p[4];
+  // select without indexing the parameter array (which would move it to local memory)
+  __device__ __forceinline__ uint8_t *of(int b) const { return b == 1 ? p[0] : b == 2 ? p[1] : b == 4 ? p[2] : p[3]; }
 };
 
 __global__ void __launch_bounds__(kThreads)
@@ -71,7 +73,7 @@ pack_kernel(const uint8_t *__restrict__ codes, int64_t n_units, const uint8_t *_
     if (bits) {
       b = __ldg(bits + g);
       if (!width_ok(b)) continue;   // nothing to store; quantize reports the width
-      base = planes.p[width_slot(b)] + __ldg(offset + g);
+      base = planes.of(b) + __ldg(offset + g);
     } else {
       base = planes.p[2] + g * 32;
     }
@@ -92,7 +94,7 @@ unpack_kernel(uint8_t *__restrict__ codes, int64_t n_units, const uint8_t *__res
     if (bits) {
       b = __ldg(bits + g);
       if (width_ok(b)) {
-        base = planes.p[width_slot(b)] + __ldg(offset + g);
+        base = planes.of(b) + __ldg(offset + g);
         v = unpack8(load_bytes(base + sub * b, b), b);
       }
     } else {
@@ -100,6 +102,40 @@ unpack_kernel(uint8_t *__restrict__ codes, int64_t n_units, const uint8_t *__res
       v = unpack8(load_bytes(base + sub * 4, 4), 4);
     }
     reinterpret_cast<uint2 *>(codes)[u] = make_uint2(static_cast<uint32_t>(v), static_cast<uint32_t>(v >> 32));
+  }
+}
+
+// fixed 4-bit: one lane packs 32 codes (two 16-byte loads) into one 16-byte store, two such
+// units per iteration so each lane keeps 64 bytes of loads in flight
+__device__ __forceinline__ uint32_t nibbles_of4(uint32_t w) {
+  // four codes (one per byte, low nibble used) -> 16 bits, code j at bits [4j, 4j+4)
+  w &= 0x0F0F0F0Fu;
+  w = (w | (w >> 4)) & 0x00FF00FFu;
+  return (w | (w >> 8)) & 0x0000FFFFu;
+}
+
+__device__ __forceinline__ uint32_t pack8codes(uint32_t lo, uint32_t hi) {
+  return nibbles_of4(lo) | (nibbles_of4(hi) << 16);
+}
+
+__global__ void __launch_bounds__(kThreads)
+pack4_kernel(const uint8_t *__restrict__ codes, int64_t n32, uint8_t *__restrict__ plane) {
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kThreads;
+  for (int64_t u = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; u < n32; u += 2 * step) {
+    const int64_t u2 = u + step;
+    const uint4 *src = reinterpret_cast<const uint4 *>(codes);
+    const uint4 a0 = __ldcs(src + 2 * u), a1 = __ldcs(src + 2 * u + 1);
+    uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
+    if (u2 < n32) {
+      b0 = __ldcs(src + 2 * u2);
+      b1 = __ldcs(src + 2 * u2 + 1);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(plane);
+    __stcs(dst + u, make_uint4(pack8codes(a0.x, a0.y), pack8codes(a0.z, a0.w), pack8codes(a1.x, a1.y),
+                               pack8codes(a1.z, a1.w)));
+    if (u2 < n32)
+      __stcs(dst + u2, make_uint4(pack8codes(b0.x, b0.y), pack8codes(b0.z, b0.w), pack8codes(b1.x, b1.y),
+                                  pack8codes(b1.z, b1.w)));
   }
 }
 
@@ -288,6 +324,11 @@ cq_status launch_varbits_index(const uint8_t *bits, int64_t G, uint32_t *offset,
 cq_status launch_pack(const uint8_t *codes, int64_t G, const uint8_t *bits, const uint32_t *offset,
                       uint8_t *const plane[4], cudaStream_t s) {
   if (G == 0) return CQ_OK;
+  if (!bits) {
+    const int64_t n32 = G * 2;
+    pack4_kernel<<<grid_for((n32 + 1) / 2), kThreads, 0, s>>>(codes, n32, plane[2]);
+    return launch_check("cq_pack_varbits");
+  }
   Planes P{{plane[0], plane[1], plane[2], plane[3]}};
   pack_kernel<<<grid_for(G * 8), kThreads, 0, s>>>(codes, G * 8, bits, offset, P);
   return launch_check("cq_pack_varbits");

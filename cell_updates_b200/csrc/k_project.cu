@@ -25,47 +25,82 @@ __device__ __forceinline__ float clamp_cell(float r, float c) {
   return r > c ? c : (r < -c ? -c : r);
 }
 
+constexpr int kUnroll = 4;    // units per lane and iteration: 64 bytes of bf16 in flight
+
+__device__ __forceinline__ uint32_t project_pair(uint32_t w, float cb, uint32_t &changed) {
+  const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
+  const uint32_t nlo = __float_as_uint(clamp_cell(lo, cb)) >> 16;
+  const uint32_t nhi = __float_as_uint(clamp_cell(hi, cb)) & 0xFFFF0000u;
+  const uint32_t nw = nlo | nhi;
+  changed += ((nw ^ w) & 0xFFFFu) != 0;
+  changed += ((nw ^ w) & 0xFFFF0000u) != 0;
+  return nw;
+}
+
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads)
 project_kernel(void *__restrict__ rv, const uint16_t *__restrict__ scale, int64_t n_units,
                unsigned long long *__restrict__ n_clamped) {
   uint32_t changed = 0;
-  for (int64_t u = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; u < n_units;
-       u += static_cast<int64_t>(gridDim.x) * kThreads) {
-    const float c = cell_bound(__ldg(scale + (u >> 3)));
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kThreads;
+  for (int64_t u0 = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; u0 < n_units; u0 += kUnroll * step) {
     if (BF16) {
-      // c rounded toward zero to bf16: drop the low 16 bits (c >= 0 or NaN)
-      const float cb = __uint_as_float(__float_as_uint(c) & 0xFFFF0000u);
-      uint4 *p = reinterpret_cast<uint4 *>(rv) + u;
-      const uint4 in = __ldcs(p);
-      uint32_t w[4] = {in.x, in.y, in.z, in.w};
+      uint4 in[kUnroll];
+      float cb[kUnroll];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xFFFF0000u);
-        const uint32_t nlo = __float_as_uint(clamp_cell(lo, cb)) >> 16;
-        const uint32_t nhi = __float_as_uint(clamp_cell(hi, cb)) & 0xFFFF0000u;
-        const uint32_t nw = nlo | nhi;
-        changed += ((nw ^ w[j]) & 0xFFFFu) != 0;
-        changed += ((nw ^ w[j]) & 0xFFFF0000u) != 0;
-        w[j] = nw;
+      for (int t = 0; t < kUnroll; ++t) {
+        const int64_t u = u0 + t * step;
+        if (u < n_units) {
+          in[t] = __ldcs(reinterpret_cast<const uint4 *>(rv) + u);
+          // c rounded toward zero to bf16: drop the low 16 bits (c >= 0 or NaN)
+          cb[t] = __uint_as_float(__float_as_uint(cell_bound(__ldg(scale + (u >> 3)))) & 0xFFFF0000u);
+        }
       }
-      __stcs(p, make_uint4(w[0], w[1], w[2], w[3]));
+#pragma unroll
+      for (int t = 0; t < kUnroll; ++t) {
+        const int64_t u = u0 + t * step;
+        if (u < n_units) {
+          uint4 o;
+          o.x = project_pair(in[t].x, cb[t], changed);
+          o.y = project_pair(in[t].y, cb[t], changed);
+          o.z = project_pair(in[t].z, cb[t], changed);
+          o.w = project_pair(in[t].w, cb[t], changed);
+          __stcs(reinterpret_cast<uint4 *>(rv) + u, o);
+        }
+      }
     } else {
-      float4 *p = reinterpret_cast<float4 *>(rv) + 2 * u;
-      float4 a = __ldcs(p), b = __ldcs(p + 1);
-      float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      float4 in[kUnroll][2];
+      float c[kUnroll];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float o = clamp_cell(v[j], c);
-        changed += __float_as_uint(o) != __float_as_uint(v[j]);
-        v[j] = o;
+      for (int t = 0; t < kUnroll; ++t) {
+        const int64_t u = u0 + t * step;
+        if (u < n_units) {
+          const float4 *p = reinterpret_cast<const float4 *>(rv) + 2 * u;
+          in[t][0] = __ldcs(p);
+          in[t][1] = __ldcs(p + 1);
+          c[t] = cell_bound(__ldg(scale + (u >> 3)));
+        }
       }
-      __stcs(p, make_float4(v[0], v[1], v[2], v[3]));
-      __stcs(p + 1, make_float4(v[4], v[5], v[6], v[7]));
+#pragma unroll
+      for (int t = 0; t < kUnroll; ++t) {
+        const int64_t u = u0 + t * step;
+        if (u < n_units) {
+          float v[8] = {in[t][0].x, in[t][0].y, in[t][0].z, in[t][0].w, in[t][1].x, in[t][1].y, in[t][1].z, in[t][1].w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float o = clamp_cell(v[j], c[t]);
+            changed += __float_as_uint(o) != __float_as_uint(v[j]);
+            v[j] = o;
+          }
+          float4 *p = reinterpret_cast<float4 *>(rv) + 2 * u;
+          __stcs(p, make_float4(v[0], v[1], v[2], v[3]));
+          __stcs(p + 1, make_float4(v[4], v[5], v[6], v[7]));
+        }
+      }
     }
   }
   if (n_clamped) {
-    changed = __reduce_add_sync(0xffffffffu, changed);
+    changed = __reduce_add_sync(0xffffffffu, changed);   // every lane of the warp reaches this point
     if ((threadIdx.x & 31) == 0 && changed) atomicAdd(n_clamped, static_cast<unsigned long long>(changed));
   }
 }
@@ -80,7 +115,7 @@ cq_status launch_project(void *r, cq_dtype dt, const uint16_t *scale, int64_t n,
   }
   if (n == 0) return CQ_OK;
   const int64_t units = n / 8;
-  const int64_t need = (units + kThreads - 1) / kThreads;
+  const int64_t need = (units + kUnroll * kThreads - 1) / (kUnroll * kThreads);
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const int blocks = static_cast<int>(need < cap ? need : cap);
   auto *cnt = reinterpret_cast<unsigned long long *>(n_clamped);

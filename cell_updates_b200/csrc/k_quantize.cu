@@ -6,8 +6,6 @@
 // Abstract: 4-bit integer codes and scales. [SLQ] abstract (page 2 listing): asymmetric
 // grids. Reading of the formula: see include/cq.h.
 //
-// Layout: eight lanes own one group (8 fp32 each, two 16-byte loads), a warp covers four
-// consecutive groups = 1 KiB of contiguous input; codes leave as one 8-byte store per lane.
 // Every fp32 operation is an explicit round-to-nearest intrinsic, so nothing is contracted.
 #include "cq_internal.cuh"
 
@@ -15,47 +13,38 @@ namespace cq {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kGroupsPerBlock = kThreads / 8;
 
+// One thread owns one group of 64 weights: the group's scale and zero point (two IEEE
+// divisions, a reciprocal) are paid once per 64 weights, the 256 bytes it loads are all in
+// flight at once, and min/max need no shuffles. Loads go through L1 (ld.global.nc), so the
+// second half of each 32-byte sector is an L1 hit for the next 16-byte load.
 __global__ void __launch_bounds__(kThreads)
 quantize_kernel(const float *__restrict__ w, int64_t G, const uint8_t *__restrict__ bits,
                 uint8_t *__restrict__ codes, uint16_t *__restrict__ scale,
                 uint8_t *__restrict__ zero, uint32_t *__restrict__ status) {
-  const int lane = threadIdx.x & 31;
-  const int sub = lane & 7;
   uint32_t flags = 0;
-  const int64_t step = static_cast<int64_t>(gridDim.x) * kGroupsPerBlock;
-  // warp-uniform trip count: every lane takes part in the shuffles of every iteration
-  const int64_t warp_first = static_cast<int64_t>(blockIdx.x) * kGroupsPerBlock + ((threadIdx.x >> 5) << 2);
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kThreads;
+  // warp-uniform trip count (the exact path below votes across the warp)
+  const int64_t warp_first = static_cast<int64_t>(blockIdx.x) * kThreads + (threadIdx.x & ~31);
   for (int64_t g0 = warp_first; g0 < G; g0 += step) {
-    const int64_t g = g0 + (lane >> 3);
+    const int64_t g = g0 + (threadIdx.x & 31);
     const bool valid = g < G;
-    float v[8];
-    if (valid) {
-      const float4 *p = reinterpret_cast<const float4 *>(w + g * kGroup + sub * 8);
-      const float4 a = __ldcs(p), c = __ldcs(p + 1);
-      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-      v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
-    } else {
+    float v[64];
+    const float4 *p = reinterpret_cast<const float4 *>(w + (valid ? g : 0) * kGroup);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+      const float4 t = __ldg(p + i);
+      v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
     }
-    bool finite = true;
+    // NaN-propagating min/max: a NaN or an infinity shows up as a non-finite extreme
     float lo = v[0], hi = v[0];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      finite = finite && isfinite(v[j]);
-      lo = fminf(lo, v[j]);
-      hi = fmaxf(hi, v[j]);
+    for (int j = 1; j < 64; ++j) {
+      asm("min.NaN.f32 %0, %0, %1;\n" : "+f"(lo) : "f"(v[j]));
+      asm("max.NaN.f32 %0, %0, %1;\n" : "+f"(hi) : "f"(v[j]));
     }
-#pragma unroll
-    for (int o = 4; o; o >>= 1) {
-      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-      finite = __shfl_xor_sync(0xffffffffu, static_cast<int>(finite), o) && finite;
-    }
-    if (!valid) continue;
-    const int b = bits ? static_cast<int>(__ldg(bits + g)) : 4;
+    const bool finite = isfinite(lo) && isfinite(hi);
+    const int b = (bits && valid) ? static_cast<int>(__ldg(bits + g)) : 4;
     const bool width_good = width_ok(b);
     const int L = width_good ? (1 << b) - 1 : 15;
     // s = RN_fp16(RN32(RN32(wmax - wmin) / L)), floored at the smallest normal fp16
@@ -70,29 +59,50 @@ quantize_kernel(const float *__restrict__ w, int64_t G, const uint8_t *__restric
     }
     const float rc = __frcp_rn(sf);
     const int z = clamp_code(rne_quotient(-lo, sf, rc), L);
-    uint64_t packed = 0;
+    // t_j = rne(RN32(w_j / s)) through the division-free filter: with qt = RN32(w_j * rc),
+    // |RN32(w_j / s) - qt| < |qt| * 2^-21, so |qt - rint(qt)| + |qt| * 2^-20 < 0.4999 decides
+    // the rounding; the rest (near a half-way point, huge, non-finite) is redone with the
+    // IEEE division in a branch of its own
+    uint64_t need_exact = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float t = rne_quotient(v[j], sf, rc);
-      const int q = clamp_code(__fadd_rn(t, static_cast<float>(z)), L);
-      packed |= static_cast<uint64_t>(q) << (8 * j);
+    for (int j = 0; j < 64; ++j) {
+      const float qt = __fmul_rn(v[j], rc);
+      const float t = rintf(qt);
+      need_exact |= static_cast<uint64_t>(!(__fmaf_rn(fabsf(qt), 0x1p-20f, fabsf(__fsub_rn(qt, t))) < 0.4999f)) << j;
+      v[j] = t;                                 // v now holds the rounded quotients
+    }
+    if (__any_sync(0xffffffffu, need_exact != 0)) {
+      // rare: re-read the weights and divide
+#pragma unroll 1
+      for (int j = 0; j < 64; ++j)
+        if ((need_exact >> j) & 1u) v[j] = rintf(__fdiv_rn(__ldg(w + (valid ? g : 0) * kGroup + j), sf));
     }
     const bool bad = !width_good || !finite || overflow;
-    if (bad) {
-      flags |= !width_good ? CQ_QSTATUS_BADBITS : (!finite ? CQ_QSTATUS_NONFINITE : CQ_QSTATUS_RANGE);
-      packed = 0;
-      s16 = 0;
-    }
-    *reinterpret_cast<uint2 *>(codes + g * kGroup + sub * 8) =
-        make_uint2(static_cast<uint32_t>(packed), static_cast<uint32_t>(packed >> 32));
-    if (sub == 0) {
-      scale[g] = s16;
+    if (valid) {
+      if (bad) flags |= !width_good ? CQ_QSTATUS_BADBITS : (!finite ? CQ_QSTATUS_NONFINITE : CQ_QSTATUS_RANGE);
+      const float zf = static_cast<float>(z), Lf = static_cast<float>(L);
+      uint4 *dst = reinterpret_cast<uint4 *>(codes + g * kGroup);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t wd[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float q = fminf(fmaxf(__fadd_rn(v[16 * c + 4 * k + e], zf), 0.0f), Lf);
+            word |= static_cast<uint32_t>(static_cast<int>(q)) << (8 * e);
+          }
+          wd[k] = bad ? 0u : word;
+        }
+        __stcs(dst + c, make_uint4(wd[0], wd[1], wd[2], wd[3]));
+      }
+      scale[g] = bad ? 0 : s16;
       zero[g] = bad ? 0 : static_cast<uint8_t>(z);
     }
   }
-  // the lanes that returned no flags still reach this point (no early exit above)
   flags = __reduce_or_sync(0xffffffffu, flags);
-  if (lane == 0 && flags && status) atomicOr(status, flags);
+  if ((threadIdx.x & 31) == 0 && flags && status) atomicOr(status, flags);
 }
 
 }  // namespace
@@ -104,7 +114,7 @@ cq_status launch_quantize(const float *w, int64_t G, const uint8_t *bits, uint8_
     if (st != CQ_OK) return st;
   }
   if (G == 0) return CQ_OK;
-  const int64_t need = (G + kGroupsPerBlock - 1) / kGroupsPerBlock;
+  const int64_t need = (G + kThreads - 1) / kThreads;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const int blocks = static_cast<int>(need < cap ? need : cap);
   quantize_kernel<<<blocks, kThreads, 0, s>>>(w, G, bits, codes, scale, zero, status);

@@ -94,7 +94,9 @@ __global__ void __launch_bounds__(kThreads) verify_kernel(VerifyArgs a) {
         b = __ldg(a.bits + g);
         if (!width_ok(b)) b = 0;
         if (b) {
-          const uint8_t *src = a.plane[width_slot(b)] + __ldg(a.offset + g) + ((i0 >> 3) & 7) * b;
+          // select the plane without indexing the parameter array (keeps it out of local memory)
+          const uint8_t *pl = b == 1 ? a.plane[0] : b == 2 ? a.plane[1] : b == 4 ? a.plane[2] : a.plane[3];
+          const uint8_t *src = pl + __ldg(a.offset + g) + ((i0 >> 3) & 7) * b;
           switch (b) {
             case 1: word = __ldg(src); break;
             case 2: word = __ldg(reinterpret_cast<const uint16_t *>(src)); break;
@@ -129,7 +131,7 @@ __global__ void __launch_bounds__(kThreads) verify_kernel(VerifyArgs a) {
       if (VAR && b == 0) {
         bad = 0xFFu;   // a width outside {1,2,4,8}: no code of the group can be re-derived
       } else if (slow) {
-#pragma unroll 1
+#pragma unroll
         for (int j = 0; j < 8; ++j) {
           if (!((slow >> j) & 1)) continue;
           const int q = static_cast<int>((word >> (j * b)) & mask);
@@ -160,12 +162,148 @@ __global__ void __launch_bounds__(kThreads) verify_kernel(VerifyArgs a) {
   if (first != INT64_MAX) atomicMin(a.first_bad, static_cast<unsigned long long>(first));
 }
 
+// ---- fixed 4-bit fast kernel ------------------------------------------------------------
+// One lane per 32 consecutive weights (16 bytes of codes, 64 bytes of bf16 residual), so each
+// lane keeps 80 bytes in flight; pairs of weights go through the packed fp32x2 pipe. The
+// filter here is d = RN32(w' * rc - k) in one fused step: w' * rc is within |w'/s| * 2^-24 of
+// w'/s, so |d| < 0.5 - 2^-11 again leaves RN32(w'/s) within 0.4996 of k. The per-weight test
+// is folded into a NaN-propagating running maximum of |d|; a lane whose maximum reaches the
+// threshold re-derives its 32 weights with the exact IEEE definition. Without a residual the
+// bound needs no per-weight arithmetic: w' = s*k is exact, |d| <= |k| * |s*rc - 1| (1 + 2^-24),
+// and |k| <= max(qor - z, z) with qor the bitwise OR of the lane's 32 codes bounds all 32.
+__device__ __forceinline__ float max_nan_abs(float m, float d) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;\n" : "=f"(r) : "f"(m), "f"(fabsf(d)));
+  return r;
+}
+
+// -(2^23 + q) as a float, for a nibble q already in the low bits
+__device__ __forceinline__ float neg_magic_code(uint32_t bits) { return __uint_as_float(0xCB000000u | bits); }
+
+template <int RK>
+__global__ void __launch_bounds__(kThreads) verify4_kernel(VerifyArgs a) {
+  const int lane = threadIdx.x & 31;
+  uint32_t count = 0;
+  int64_t first = INT64_MAX;
+  const int64_t n32 = a.n_units >> 2;            // units of 32 weights
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kThreads;
+  const int64_t base_u = blockIdx.x * static_cast<int64_t>(kThreads) + (threadIdx.x & ~31);
+  for (int64_t u0 = base_u; u0 < n32; u0 += step) {
+    const int64_t u = u0 + lane;
+    const bool valid = u < n32;
+    uint32_t bad = 0;
+    int64_t i0 = 0;
+    int64_t g = 0;
+    if (valid) {
+      i0 = a.first_w + 32 * u;
+      g = i0 >> 6;
+      const uint4 cw = __ldcs(reinterpret_cast<const uint4 *>(a.plane[2] + (i0 >> 1)));
+      const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+      uint32_t rw[16];
+      if (RK == kBF16) {
+        const uint4 *rp = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(a.r) + i0);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 t = __ldcs(rp + v);
+          rw[4 * v] = t.x; rw[4 * v + 1] = t.y; rw[4 * v + 2] = t.z; rw[4 * v + 3] = t.w;
+        }
+      }
+      float rf[32];
+      if (RK == kF32) {
+        const float4 *rp = reinterpret_cast<const float4 *>(static_cast<const float *>(a.r) + i0);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 t = __ldcs(rp + v);
+          rf[4 * v] = t.x; rf[4 * v + 1] = t.y; rf[4 * v + 2] = t.z; rf[4 * v + 3] = t.w;
+        }
+      }
+      const float sf = f16_bits_to_f32(__ldg(a.scale + g));
+      const int z = __ldg(a.zero + g);
+      const float rc = __frcp_rn(sf);
+      const float kb = 8388608.0f + static_cast<float>(z);     // 2^23 + z, exact
+      const float2 kb2 = make_float2(kb, kb), ns2 = make_float2(-sf, -sf), rc2 = make_float2(rc, rc);
+      float m = 0.0f;
+      if (RK == kNoR) {
+        // No residual: w' = s*k exactly, so |RN32(w' * rc - k)| <= |k| * |s * rc - 1| (1 + 2^-24).
+        // |k| = |q - z| <= max(qor - z, z), qor = the OR of the lane's 32 codes (>= each code).
+        uint32_t qor = words[0] | words[1] | words[2] | words[3];
+        qor = (qor | (qor >> 4)) & 0x0F0F0F0Fu;
+        qor |= qor >> 16;
+        qor = (qor | (qor >> 8)) & 0xFu;
+        const float kmax = static_cast<float>(max(static_cast<int>(qor) - z, z));
+        const float eps = fabsf(__fmaf_rn(sf, rc, -1.0f));      // |s * rc - 1|, exact in one fma
+        m = __fmul_rn(__fmul_rn(kmax, eps), 1.0f + 0x1p-22f);   // NaN when s is 0, inf or NaN
+      } else {
+#pragma unroll
+      for (int wi = 0; wi < 4; ++wi) {
+        const uint32_t w = words[wi];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const int j = 8 * wi + 2 * p;                          // weights j, j+1
+          // nk = z - q = -k exactly; w' = (-s) * nk + r = RN32(s*k + r); d = RN32(w' * rc - k)
+          const float2 nk = __fadd2_rn(make_float2(neg_magic_code((w >> (8 * p)) & 0xFu),
+                                                   neg_magic_code((w >> (8 * p + 4)) & 0xFu)), kb2);
+          float2 wp;
+          if (RK == kBF16) {
+            const uint32_t r2 = rw[j >> 1];
+            wp = __ffma2_rn(ns2, nk, make_float2(__uint_as_float(r2 << 16), __uint_as_float(r2 & 0xFFFF0000u)));
+          } else if (RK == kF32) {
+            wp = __ffma2_rn(ns2, nk, make_float2(rf[j], rf[j + 1]));
+          } else {
+            wp = __fmul2_rn(ns2, nk);
+          }
+          const float2 d = __ffma2_rn(wp, rc2, nk);
+          m = max_nan_abs(m, d.x);
+          m = max_nan_abs(m, d.y);
+        }
+      }
+      }
+      if (!(m < 0.49951171875f)) {
+        // the exact definition, weight by weight, on inputs re-read from memory (rare path)
+#pragma unroll 1
+        for (int j = 0; j < 32; ++j) {
+          const int64_t i = i0 + j;
+          const int q = static_cast<int>((__ldg(a.plane[2] + (i >> 1)) >> (4 * (i & 1))) & 0xFu);
+          float r = 0.0f;
+          if (RK == kBF16) r = bf16_bits_to_f32(__ldg(static_cast<const uint16_t *>(a.r) + i));
+          if (RK == kF32) r = __ldg(static_cast<const float *>(a.r) + i);
+          if (!exact_match<RK != kNoR>(q, z, 15, sf, r)) bad |= 1u << j;
+        }
+      }
+    }
+    const uint32_t any = __ballot_sync(0xffffffffu, bad != 0);
+    if (any) {
+      count += __popc(bad);
+      if (bad) {
+        const int64_t fi = i0 + (__ffs(bad) - 1);
+        first = fi < first ? fi : first;
+      }
+      if (a.flags && bad) {
+        // the two lanes of a group may both publish; atomicOr makes that harmless
+        const int64_t gl = g - (a.first_w >> 6);
+        atomicOr(a.flags + (gl >> 5), 1u << (gl & 31));
+      }
+    }
+  }
+  count = __reduce_add_sync(0xffffffffu, count);
+  if (lane == 0 && count) atomicAdd(a.mism, static_cast<unsigned long long>(count));
+  if (first != INT64_MAX) atomicMin(a.first_bad, static_cast<unsigned long long>(first));
+}
+
 template <bool VAR>
 void dispatch(int rk, VerifyArgs a, int blocks, cudaStream_t s) {
   switch (rk) {
     case kNoR: verify_kernel<VAR, kNoR><<<blocks, kThreads, 0, s>>>(a); break;
     case kF32: verify_kernel<VAR, kF32><<<blocks, kThreads, 0, s>>>(a); break;
     default: verify_kernel<VAR, kBF16><<<blocks, kThreads, 0, s>>>(a); break;
+  }
+}
+
+void dispatch4(int rk, VerifyArgs a, int blocks, cudaStream_t s) {
+  switch (rk) {
+    case kNoR: verify4_kernel<kNoR><<<blocks, kThreads, 0, s>>>(a); break;
+    case kF32: verify4_kernel<kF32><<<blocks, kThreads, 0, s>>>(a); break;
+    default: verify4_kernel<kBF16><<<blocks, kThreads, 0, s>>>(a); break;
   }
 }
 
@@ -200,10 +338,13 @@ cq_status launch_verify(const cq_qweight &qw, int64_t first_w, int64_t n_w, uint
   const int64_t need = (a.n_units + kThreads - 1) / kThreads;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const int blocks = static_cast<int>(need < cap ? need : cap);
-  if (qw.bits)
+  if (qw.bits) {
     dispatch<true>(rk, a, blocks, s);
-  else
-    dispatch<false>(rk, a, blocks, s);
+  } else {
+    // 32 weights per lane; n_w is a multiple of 64
+    const int64_t need4 = (a.n_units / 4 + kThreads - 1) / kThreads;
+    dispatch4(rk, a, static_cast<int>(need4 < cap ? need4 : cap), s);
+  }
   return launch_check("cq_requant_verify");
 }
 

@@ -91,7 +91,7 @@ typedef struct {
 /*
  * cq_quantize -- [VBQ] per-group widths, [CF] 4-bit codes and scales, [SLQ] asymmetry.
  * w: [rows, cols] fp32 (16-byte aligned). bits: [G] widths or NULL (= 4 for every group).
- * codes: [rows*cols] one code per byte (8-byte aligned); scale: [G] fp16 bits; zero: [G].
+ * codes: [rows*cols] one code per byte (16-byte aligned); scale: [G] fp16 bits; zero: [G].
  * status_word: one uint32 (device) that receives the OR of CQ_QSTATUS_* over all groups;
  * it is cleared by the call; may be NULL. Groups with a non-finite weight, an fp16-overflowing
  * scale or a bad width are written as s=+0, z=0, q=0 and flagged; the call still returns CQ_OK.
