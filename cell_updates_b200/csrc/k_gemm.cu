@@ -23,12 +23,7 @@
 // y is zeroed first; tiles split between two CTAs are combined with fp32 atomics.
 // Every barrier wait is bounded: on timeout the CTA raises a status flag, drains what it
 // issued, frees its tensor memory and returns.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
-#include "cq_internal.cuh"
+#include "cq_async.cuh"
 
 namespace cq {
 namespace {
@@ -42,7 +37,6 @@ constexpr uint32_t kCodeBox = kTileM * 128;        // one swizzled box: 128 rows
 constexpr uint32_t kCodeStage = 2 * kCodeBox;      // 32 KiB
 constexpr uint32_t kABytes = kTileM * 128;         // bf16 A tile: 128 rows x 64 columns
 constexpr int kCodeStages = 2, kAStages = 4, kXStages = 8, kAccBufs = 4;
-constexpr uint32_t kSpinLimit = 1u << 22;          // try_wait rounds before giving up
 
 template <int NT>
 struct Cfg {
@@ -52,52 +46,6 @@ struct Cfg {
   static constexpr uint32_t kSmem =
       1024 + kCodeStages * kCodeStage + kAStages * kABytes + kXStages * kXBytes + kBars * 8 + 16;
 };
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(b)), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(b)) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// bounded wait on the phase of the given parity; false on timeout or when another role gave up
-__device__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile uint32_t *abort_flag, uint32_t *status,
-                          bool honour_abort = true) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(b, parity)) return true;
-    if ((i & 63) == 63) {
-      if (honour_abort && *abort_flag) return false;
-      __nanosleep(64);
-    }
-  }
-  *abort_flag = 1u;
-  if (status) atomicOr(status, 1u);
-  return false;
-}
-
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
-          smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // UMMA shared-memory descriptor: K-major operand in the 128-byte swizzled canonical layout
 // (8-row groups of 128-byte rows, 1024 bytes apart), sm_100 descriptor version 1.
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
@@ -469,19 +417,6 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
 
 // ---- host side ---------------------------------------------------------------------------
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 template <int NT>
 cq_status launch_nt(const cq_qweight &qw, const void *x, int m, float *y, uint32_t *status, cudaStream_t s) {
   using C = Cfg<NT>;
@@ -489,16 +424,8 @@ cq_status launch_nt(const cq_qweight &qw, const void *x, int m, float *y, uint32
   if (!encode) return fail(CQ_ERR_CUDA, "cq_dequant_gemm: cuTensorMapEncodeTiled unavailable");
   const int64_t N = qw.rows, K = qw.cols;
   CUtensorMap tm_codes, tm_x;
-  {
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-    cuuint32_t box[2] = {128, kTileM};
-    cuuint32_t es[2] = {1, 1};
-    CUresult r = encode(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(qw.plane[2]), dims, strides,
-                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(CQ_ERR_CUDA, "cq_dequant_gemm: code tensor map (%d)", (int)r);
-  }
+  cq_status cs = code_tensor_map(&tm_codes, qw.plane[2], N, K, kTileM, "cq_dequant_gemm");
+  if (cs != CQ_OK) return cs;
   {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(m)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * 2)};

@@ -20,12 +20,7 @@
 //  * gemv_generic: any format (per-group widths), fp32 or bf16 x, optional residual; one
 //    warp per row, fp32 CUDA-core math. Used for the small fp32-activation cases and for
 //    residual-carrying weights.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
-#include "cq_internal.cuh"
+#include "cq_async.cuh"
 
 namespace cq {
 namespace {
@@ -48,6 +43,30 @@ __device__ __forceinline__ void mma_bf16_16816(float d[4], const uint32_t a[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma_f16_16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// the same with a zero accumulator in
+__device__ __forceinline__ void mma_f16_16816_z(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};\n"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+// (w & mask) | magic in one LOP3
+template <uint32_t kMask, uint32_t kMagic>
+__device__ __forceinline__ uint32_t lop_or(uint32_t w) {
+  uint32_t out;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(out) : "r"(w), "n"(kMask), "n"(kMagic));
+  return out;
+}
+
 // nibbles i and i+4 of w (i = 0..3 after the shift) -> bf16 pair (128 + q_i, 128 + q_{i+4})
 __device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
   uint32_t out;
@@ -59,65 +78,54 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::); }
 
 // ---- the kernel -------------------------------------------------------------------------------
-// One CTA per 16-row tile and the whole K range, 8 warps. Chunks of 4 groups (128 bytes per
-// row) are dealt to the warps round-robin, so at any moment a CTA's loads cover ~1 KiB of
-// each of its 16 rows: long DRAM runs with few rows in flight (measured on this part: ~6 TB/s
-// for 16-row tiles with >= 512-byte runs, against ~3 TB/s when every row of the matrix is in
-// flight at once). Each warp double-buffers its codes, scales and zero points in registers:
-// the next chunk's loads are issued before the current one is computed. The activations are
-// staged once per CTA in shared memory, in the order the codes are fed to the MMA, together
-// with their exact per-group sums; when they do not fit, each warp reads them from L1 and
-// takes the sums from one more MMA with an all-ones operand. Warps meet in shared memory at
-// the end, so every output is written once (no atomics, no zero-fill, fixed order). Codes
-// and scales do not depend on earlier kernels and are requested before the programmatic-
-// dependent-launch wait; activations are read, and y written, only after it.
-constexpr int kWarps = 8;
+// Persistent CTAs of 16 warps, one per SM; CTA b owns the 16-row tiles b, b + G, b + 2G, ...
+// Each tile is cut into chunks of 4 groups (16 rows x 128 bytes), and the CTA's chunks, tile
+// after tile, are dealt to its warps round-robin, so every warp gets the same share (+-1)
+// whatever the shape, and at any moment the CTA's loads cover a few KiB of each of 16 rows:
+// long DRAM runs with few rows open. Every warp runs its own ring of kStages chunk buffers,
+// filled by one TMA box per chunk (lane 0) plus per-lane cp.async copies of the chunk's scales
+// and zero points; the same warp consumes them, so a buffer is refilled right after the warp
+// has read it, without any cross-warp handshake. When a warp leaves a tile it stores its
+// partial sums; the last of the tile's warps to arrive adds the partials in warp order and
+// writes y (no atomics on y, no zero-fill, a fixed summation order, and no warp ever waits for
+// another to finish a tile unless four tiles apart).
+//
+// Per group, sum_k W x = s * (sum_k (128 + q) x - (128 + z) sum_k x). The operand 128 + q is
+// the bf16 bit pattern 0x4300 | q, made from a nibble pair with one LOP3; the activations are
+// bf16 already, so the tensor-core products are exact and accumulate in fp32 (mma.sync
+// m16n8k16). The correction enters the same accumulator through one more MMA: its A operand
+// holds -(128 + z) (bit pattern 0xC300 | z, exact for z <= 127) and its B operand the group sum
+// of x split into three bf16 parts (hi + mid + lo = the fp32 sum exactly), so the per-group
+// result s * (...) needs only the scale multiply. When the activations are too large to
+// stage, lanes read them from L1 and the group sums come from an MMA with an all-ones A.
+// The contraction over k is a sum, so codes and activations may be paired in any order that
+// both operands share: each lane feeds the 16 codes of one 8-byte word run and the staged
+// activations are stored permuted to match.
+constexpr int kWarps = 16;
 constexpr int kGemvThreads = 32 * kWarps;
-constexpr int kCG = 4;                                  // groups per chunk
-constexpr int kXStageMax = 64 * 1024;                   // staged activations + sums, at most
-constexpr int kRedBytes = kWarps * kTileRows * 8 * 4;
+constexpr int kCG = 8;                                    // groups per chunk (two TMA boxes)
+constexpr int kStages = 2;                                // chunk buffers per warp
+constexpr int kBoxBytes = kTileRows * 4 * 32;             // one box: 16 rows x 4 groups
+constexpr int kChunkBytes = 2 * kBoxBytes;
+constexpr int kMetaBytes = 384;                           // [16][8] fp16 scales, then [16][8] zeros
+constexpr int kRedSlots = 2;                              // tiles in reduction at once
+constexpr int kRedFloats = kWarps * kTileRows * 8;        // one slot: every warp's 16 x 8 partials
+// shared memory: [code rings | meta rings | barriers | reduction slots | counters | group sums |
+//                 staged x]
+constexpr int kOffMeta = kWarps * kStages * kChunkBytes;
+constexpr int kOffBars = kOffMeta + kWarps * kStages * kMetaBytes;
+constexpr int kOffRed = kOffBars + kWarps * kStages * 8;
+constexpr int kOffCnt = kOffRed + kRedSlots * kRedFloats * 4;
+constexpr int kOffSums = kOffCnt + 64;
+constexpr int kSmemCap = 227 * 1024;
+static_assert(kOffSums % 16 == 0 && kOffRed % 16 == 0, "shared-memory carve-up must keep 16-byte alignment");
 
 // staged activations: m rows of K bf16 in fragment order, row pitch padded by 16 bytes so the
-// rows a warp reads fall in different banks, followed by fp32 sums [KG][8]
+// rows a warp reads fall in different banks; group sums [m][KG] as three words (six fp16)
 __host__ __device__ constexpr int64_t xstage_pitch(int64_t K) { return K * 2 + 16; }
-__host__ __device__ constexpr int64_t xstage_bytes(int m, int64_t K) { return m * xstage_pitch(K) + (K / 64) * 32; }
-
-struct Chunk {
-  uint2 a0[kCG], a1[kCG];      // 8 code bytes per row and group for rows gid, gid+8
-  uint2 s0, s1;                // 4 fp16 scales per row
-  uint32_t z0, z1;             // 4 zero points per row
-};
-
-template <bool META4>
-__device__ __forceinline__ void load_chunk(Chunk &ck, const uint8_t *row0, const uint8_t *row1, const uint16_t *srow0,
-                                           const uint16_t *srow1, const uint8_t *zrow0, const uint8_t *zrow1, int g0,
-                                           int ng) {
-#pragma unroll
-  for (int j = 0; j < kCG; ++j) {
-    if (j < ng) {
-      ck.a0[j] = __ldcs(reinterpret_cast<const uint2 *>(row0 + (g0 + j) * 32));
-      ck.a1[j] = __ldcs(reinterpret_cast<const uint2 *>(row1 + (g0 + j) * 32));
-    }
-  }
-  if (META4 && ng == kCG) {
-    ck.s0 = __ldg(reinterpret_cast<const uint2 *>(srow0 + g0));
-    ck.s1 = __ldg(reinterpret_cast<const uint2 *>(srow1 + g0));
-    ck.z0 = __ldg(reinterpret_cast<const uint32_t *>(zrow0 + g0));
-    ck.z1 = __ldg(reinterpret_cast<const uint32_t *>(zrow1 + g0));
-  } else {
-    uint32_t sv0[kCG], sv1[kCG], zv0[kCG], zv1[kCG];
-#pragma unroll
-    for (int j = 0; j < kCG; ++j) {
-      sv0[j] = j < ng ? __ldg(srow0 + g0 + j) : 0u;
-      sv1[j] = j < ng ? __ldg(srow1 + g0 + j) : 0u;
-      zv0[j] = j < ng ? __ldg(zrow0 + g0 + j) : 0u;
-      zv1[j] = j < ng ? __ldg(zrow1 + g0 + j) : 0u;
-    }
-    ck.s0 = make_uint2(sv0[0] | (sv0[1] << 16), sv0[2] | (sv0[3] << 16));
-    ck.s1 = make_uint2(sv1[0] | (sv1[1] << 16), sv1[2] | (sv1[3] << 16));
-    ck.z0 = zv0[0] | (zv0[1] << 8) | (zv0[2] << 16) | (zv0[3] << 24);
-    ck.z1 = zv1[0] | (zv1[1] << 8) | (zv1[2] << 16) | (zv1[3] << 24);
-  }
+__host__ __device__ constexpr int64_t sums_bytes(int m, int64_t K) { return ((K / 64) * m * 12 + 15) & ~int64_t(15); }
+__host__ __device__ constexpr int64_t gemv_smem(int m, int64_t K, bool xs) {
+  return 1024 + kOffSums + sums_bytes(m, K) + (xs ? m * xstage_pitch(K) : 0);
 }
 
 // 16 consecutive bf16 activations -> the 8 B-fragment registers in code-feeding order:
@@ -129,54 +137,130 @@ __device__ __forceinline__ void permute16(const uint4 &lo, const uint4 &hi, uint
   b[6] = __byte_perm(hi.y, hi.w, 0x5410); b[7] = __byte_perm(hi.y, hi.w, 0x7632);
 }
 
-template <bool META4, bool XS>
-__global__ void __launch_bounds__(kGemvThreads, 2)
-gemv4_kernel(const uint8_t *__restrict__ plane4, const uint16_t *__restrict__ scale,
+__device__ __forceinline__ float half_lo(uint32_t w) { return __low2float(*reinterpret_cast<const __half2 *>(&w)); }
+__device__ __forceinline__ float half_hi(uint32_t w) { return __high2float(*reinterpret_cast<const __half2 *>(&w)); }
+__device__ __forceinline__ uint32_t word4(const uint4 &v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// a warp's place in the CTA's chunk stream: local tile index, chunk within the tile
+struct Cursor {
+  int lt, c;
+};
+__device__ __forceinline__ void advance(Cursor &cu, int n_chunks) {
+  cu.c += kWarps;
+  while (cu.c >= n_chunks) {
+    cu.c -= n_chunks;
+    ++cu.lt;
+  }
+}
+
+template <bool FULL, bool XS>
+__global__ void __launch_bounds__(kGemvThreads, 1)
+gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__restrict__ scale,
              const uint8_t *__restrict__ zero, const __nv_bfloat16 *__restrict__ x, int m, int64_t N,
              int64_t K, float *__restrict__ y) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  float (*red)[kTileRows][8] = reinterpret_cast<float (*)[kTileRows][8]>(smem);
-  uint8_t *xst = smem + kRedBytes;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   pdl_launch_dependents();
   const int KG = static_cast<int>(K >> 6);
   const int n_chunks = (KG + kCG - 1) / kCG;
+  const int64_t n_tiles = (N + kTileRows - 1) / kTileRows;
+  const int n_local = static_cast<int>((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gid = lane >> 2, tig = lane & 3;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kTileRows;
-  const int64_t lr0 = row0 + gid < N ? row0 + gid : N - 1;
-  const int64_t lr1 = row0 + gid + 8 < N ? row0 + gid + 8 : N - 1;
-  const int64_t half_k = K >> 1;
-  const uint8_t *crow0 = plane4 + lr0 * half_k + tig * 8, *crow1 = plane4 + lr1 * half_k + tig * 8;
-  const uint16_t *srow0 = scale + lr0 * KG, *srow1 = scale + lr1 * KG;
-  const uint8_t *zrow0 = zero + lr0 * KG, *zrow1 = zero + lr1 * KG;
+  // MMA row gid <-> tile row rho, MMA row gid + 8 <-> tile row rho + 8: with this order the
+  // 8-byte code reads of a half-warp hit all 32 banks of the 128-byte swizzled box
+  const int rho = 2 * (gid & 3) + (gid >> 2);
+  uint8_t *ring = smem + warp * kStages * kChunkBytes;
+  uint8_t *meta = smem + kOffMeta + warp * kStages * kMetaBytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars) + warp * kStages;
+  float *red = reinterpret_cast<float *>(smem + kOffRed);
+  uint32_t *cnt = reinterpret_cast<uint32_t *>(smem + kOffCnt);            // [kRedSlots] arrivals
+  volatile uint32_t *uses = reinterpret_cast<volatile uint32_t *>(smem + kOffCnt + 16);   // reductions done
+  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + kOffCnt + 32);
+  uint32_t *sums = reinterpret_cast<uint32_t *>(smem + kOffSums);          // [m][KG][2]
+  uint8_t *xst = smem + kOffSums + sums_bytes(m, K);
   const int64_t xpitch = xstage_pitch(K);
-  float *xsum = reinterpret_cast<float *>(xst + m * xpitch);          // [KG][8]
-  auto chunk_range = [&](int c, int &g0, int &ng) {
-    g0 = c * kCG;
-    ng = KG - g0 < kCG ? KG - g0 : kCG;
-  };
+  const int total = n_local * n_chunks;                                      // chunks of this CTA
 
-  // first chunk of this warp: codes and scales before the dependency wait
-  Chunk cur, nxt;
-  {
-    int g0, ng;
-    chunk_range(warp, g0, ng);
-    if (warp < n_chunks) load_chunk<META4>(cur, crow0, crow1, srow0, srow1, zrow0, zrow1, g0, ng);
+  if (lane == 0) {
+    for (int i = 0; i < kStages; ++i) mbar_init(bars + i, FULL ? 33u : 1u);
+    mbar_init_fence();
   }
-  pdl_wait();                 // x may be the output of the previous kernel in the stream
-  const bool has_x = gid < m;
-  const __nv_bfloat16 *xrow = x + static_cast<int64_t>(has_x ? gid : 0) * K + tig * 16;
+  for (int i = threadIdx.x; i < kRedSlots * kRedFloats; i += kGemvThreads) red[i] = 0.0f;
+  if (threadIdx.x < kRedSlots) { cnt[threadIdx.x] = 0u; uses[threadIdx.x] = 0u; }
+  if (threadIdx.x == 0) *abort_flag = 0u;
+  __syncthreads();
+
+  // ---- producer side: the warp's own ring ----
+  // lane l copies the scales (8 bytes) and zero points (4 bytes) of groups 4h..4h+3 of the
+  // chunk for tile row l & 15, h = l >> 4; groups past the row's end are zero-filled
+  const int prow = lane & 15, phalf = lane >> 4;
+  Cursor prod = {0, warp};       // chunk number `warp` of the stream may lie beyond the first tile
+  while (prod.c >= n_chunks) { prod.c -= n_chunks; ++prod.lt; }
+  int prod_lt = -1, prod_y = 0;
+  const uint16_t *ps = scale;
+  const uint8_t *pz = zero;
+  auto issue = [&](int slot) {
+    if (prod.lt != prod_lt) {
+      prod_lt = prod.lt;
+      const int64_t tile = blockIdx.x + static_cast<int64_t>(prod_lt) * gridDim.x;
+      int64_t row = tile * kTileRows + prow;
+      row = row < N ? row : N - 1;
+      ps = scale + row * KG + phalf * 4;
+      pz = zero + row * KG + phalf * 4;
+      prod_y = static_cast<int>(tile * kTileRows);
+    }
+    uint64_t *bar = bars + slot;
+    const int g0 = prod.c * kCG;
+    const bool second = g0 + 4 < KG;
+    if (FULL) {
+      const bool valid = g0 + phalf * 4 < KG;
+      uint8_t *ms = meta + slot * kMetaBytes;
+      cp_async_8z(ms + prow * 16 + phalf * 8, valid ? ps + g0 : ps, valid ? 8u : 0u);
+      cp_async_4z(ms + 256 + prow * 8 + phalf * 4, valid ? pz + g0 : pz, valid ? 4u : 0u);
+      cp_async_arrive_noinc(bar);
+    }
+    if (lane == 0) {
+      uint8_t *dst = ring + slot * kChunkBytes;
+      mbar_arrive_expect_tx(bar, second ? kChunkBytes : kBoxBytes);
+      tma_load_2d(dst, &tm_codes, prod.c * 256, prod_y, bar);
+      if (second) tma_load_2d(dst + kBoxBytes, &tm_codes, prod.c * 256 + 128, prod_y, bar);
+    }
+  };
+  int n_issued = 0;
+  for (int e = warp; n_issued < kStages && e < total; e += kWarps, ++n_issued) {
+    issue(n_issued);
+    advance(prod, n_chunks);
+  }
+
+  pdl_wait();   // x may be the output of the previous kernel in the stream; y is written below
+  // Staged activations (XS): x' = x * 2^-e in fp16, e a power of two that puts max|x'| in
+  // [256, 512): every bf16 value down to max|x| * 2^-18 converts exactly, the fp16 group sums
+  // below stay finite, and y is scaled back by 2^e at the end (exact). Thread t owns the
+  // 16-element blocks t, t + 512, ... of the flattened [m][K/16]; four lanes make one group.
+  // Pass 1 stores the bf16 words in fragment order and the fp32 group sums (all elements,
+  // odd-position elements); pass 2 converts both in place once the maximum is known.
+  float out_scale = 1.0f;
   if (XS) {
-    // stage x: thread t owns 16-element blocks t, t + 256, ...; four lanes make one group
-    const int nblk = m * (KG * 4);
+    float *wmax = reinterpret_cast<float *>(smem + kOffCnt + 48);          // [1] block maximum
+    const int bpr = KG * 4;                 // 16-element blocks per activation row
+    const int nblk = m * bpr;
+    float amax = 0.0f;
     for (int b0 = 0; b0 < nblk; b0 += kGemvThreads * 4) {
       uint4 v[4][2];
+      int nn[4], kk[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int b = b0 + u * kGemvThreads + threadIdx.x;
+        int n = 0;
+#pragma unroll
+        for (int i = 1; i < 8; ++i) n += b >= i * bpr ? 1 : 0;      // m <= 8: no division
+        nn[u] = n;
+        kk[u] = b - n * bpr;
         if (b < nblk) {
-          const int n = b / (KG * 4), kb = b - n * (KG * 4);
-          const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(n) * K + kb * 16);
+          const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(n) * K + kk[u] * 16);
           v[u][0] = __ldg(src);
           v[u][1] = __ldg(src + 1);
         }
@@ -184,117 +268,329 @@ gemv4_kernel(const uint8_t *__restrict__ plane4, const uint16_t *__restrict__ sc
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int b = b0 + u * kGemvThreads + threadIdx.x;
-        float sum = 0.0f;
+        float se = 0.0f, so = 0.0f;
         if (b < nblk) {
-          const int n = b / (KG * 4), kb = b - n * (KG * 4);
           uint32_t f[8];
           permute16(v[u][0], v[u][1], f);
-          uint4 *dst = reinterpret_cast<uint4 *>(xst + n * xpitch + kb * 32);
+          uint4 *dst = reinterpret_cast<uint4 *>(xst + nn[u] * xpitch + kk[u] * 32);
           dst[0] = make_uint4(f[0], f[1], f[2], f[3]);
           dst[1] = make_uint4(f[4], f[5], f[6], f[7]);
-          const uint32_t w[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w, v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+          const uint32_t w[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
+                                 v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
+          for (int e = 0; e < 8; ++e) {
+            const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
+            se += lo;
+            so += hi;
+            amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+          }
         }
-        // blocks 4j..4j+3 (one group) sit on lanes 4j..4j+3 of a warp (256 threads, group-aligned)
-        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        float sx = se + so;
+        sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+        sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+        so += __shfl_xor_sync(0xffffffffu, so, 1);
+        so += __shfl_xor_sync(0xffffffffu, so, 2);
         if (b < nblk && (threadIdx.x & 3) == 0) {
-          const int n = b / (KG * 4), kb = b - n * (KG * 4);
-          xsum[(kb >> 2) * 8 + n] = sum;
+          float *dst = reinterpret_cast<float *>(sums + (nn[u] * KG + (kk[u] >> 2)) * 3);
+          dst[0] = sx;
+          dst[1] = so;
         }
       }
     }
-    for (int p = threadIdx.x; p < KG * 8; p += kGemvThreads)
-      if ((p & 7) >= m) xsum[p] = 0.0f;
+    // block maximum (NaNs are skipped here; they reach y through the products)
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+    if (threadIdx.x == 0) *wmax = 0.0f;
     __syncthreads();
+    if (lane == 0) atomicMax(reinterpret_cast<int *>(wmax), __float_as_int(amax));   // amax >= 0: int order
+    __syncthreads();
+    const float gmax = *wmax;
+    int e = 0;
+    if (gmax > 0.0f && gmax <= 3.0e38f) {
+      e = static_cast<int>((__float_as_uint(gmax) >> 23) & 0xFFu) - 127 - 8;
+      e = e < -100 ? -100 : (e > 100 ? 100 : e);
+    }
+    const float in_scale = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+    const float in_scale16 = in_scale * 0.0625f;
+    out_scale = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+    for (int b0 = 0; b0 < nblk; b0 += kGemvThreads * 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int b = b0 + u * kGemvThreads + threadIdx.x;
+        if (b < nblk) {
+          int n = 0;
+#pragma unroll
+          for (int i = 1; i < 8; ++i) n += b >= i * bpr ? 1 : 0;
+          const int kb = b - n * bpr;
+          uint4 *dst = reinterpret_cast<uint4 *>(xst + n * xpitch + kb * 32);
+#pragma unroll
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            uint4 q = dst[hlf];
+            uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              // words 1 and 3 of each half feed codes that carry a factor 16 (see below)
+              const float sc = (i & 1) ? in_scale16 : in_scale;
+              const __half2 h2 = __floats2half2_rn(__uint_as_float(wv[i] << 16) * sc,
+                                                   __uint_as_float(wv[i] & 0xFFFF0000u) * sc);
+              wv[i] = *reinterpret_cast<const uint32_t *>(&h2);
+            }
+            dst[hlf] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+          if ((threadIdx.x & 3) == 0) {
+            // exact three-way fp16 splits of the scaled sums: hi + mid + lo == value
+            uint32_t *sw = sums + (n * KG + (kb >> 2)) * 3;
+            const float sx = reinterpret_cast<const float *>(sw)[0] * in_scale;
+            const float so = reinterpret_cast<const float *>(sw)[1] * in_scale;
+            uint16_t hx[3], ho[3];
+            float rx = sx, ro = so;
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+              const __half a = __float2half_rn(rx), c = __float2half_rn(ro);
+              hx[i] = __half_as_ushort(a);
+              ho[i] = __half_as_ushort(c);
+              rx -= __half2float(a);
+              ro -= __half2float(c);
+            }
+            sw[0] = hx[0] | (static_cast<uint32_t>(hx[1]) << 16);
+            sw[1] = hx[2] | (static_cast<uint32_t>(ho[0]) << 16);
+            sw[2] = ho[1] | (static_cast<uint32_t>(ho[2]) << 16);
+          }
+        }
+      }
+    }
   }
+  __syncthreads();
 
+  // per-lane constants. Lanes whose B column n = gid is past the batch read row 0's data: the
+  // MMA columns they feed are never stored, so no predicates or zero buffers are needed.
+  uint32_t off[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) off[j] = rho * 128 + ((((2 * j) + (tig >> 1)) ^ rho) << 4) + (tig & 1) * 8;
+  const bool has_x = gid < m;
+  const int xrow_s = has_x ? gid : 0;
+  const uint8_t *xs_base = xst + xrow_s * xpitch + tig * 32;
+  const uint32_t *sum_base = sums + xrow_s * KG * 3 + (tig < 2 ? tig : 2);
+  // correction operand per lane (k = 2 tig, 2 tig + 1), fp16 halves: tig 0 (Z, Z), tig 1
+  // (Z, 960), tig 2 (960, 960), tig 3 (0, 0), Z = -(1024 + z) = 0xE400 | z (byte j of the
+  // zero word); constant bytes 4..7 = E4 80 63 00
+  const uint32_t csel_base = tig == 0 ? 0x4040u : (tig == 1 ? 0x6540u : (tig == 2 ? 0x6565u : 0x7777u));
+  const uint32_t csel_mul = tig == 0 ? 0x0101u : (tig == 1 ? 0x0001u : 0u);
+  const __nv_bfloat16 *xrow = x + static_cast<int64_t>(has_x ? gid : 0) * K + tig * 16;
   const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};   // bf16 1.0
+  const int arrivals = n_chunks < kWarps ? n_chunks : kWarps;
+
+  // store this warp's partials of local tile lt; the last arrival reduces and writes y
+  auto flush = [&](int lt, const float acc[4]) {
+    const int slot = lt % kRedSlots;
+    const uint32_t use = static_cast<uint32_t>(lt / kRedSlots);
+    // the slot's previous tile must be reduced (and its partials zeroed) first; lane 0 polls,
+    // the warp follows its verdict
+    uint32_t go = 1u;
+    if (lane == 0) {
+      for (uint32_t i = 0; uses[slot] != use; ++i) {
+        if (*abort_flag) { go = 0u; break; }
+        if (i > kSuspendLimit * 16u) { *abort_flag = 1u; go = 0u; break; }
+        __nanosleep(32);
+      }
+      __threadfence_block();
+    }
+    if (!__shfl_sync(0xffffffffu, go, 0)) return;
+    // partials of the m live columns only, column-major: [col][16 rows]
+    float *rs = red + slot * kRedFloats;
+    float *rw = rs + warp * (kTileRows * 8);
+    if (2 * tig < m) {
+      rw[(2 * tig) * 16 + rho] = acc[0];
+      rw[(2 * tig) * 16 + rho + 8] = acc[2];
+    }
+    if (2 * tig + 1 < m) {
+      rw[(2 * tig + 1) * 16 + rho] = acc[1];
+      rw[(2 * tig + 1) * 16 + rho + 8] = acc[3];
+    }
+    __syncwarp();
+    uint32_t old = 0;
+    if (lane == 0) {
+      __threadfence_block();
+      old = atomicAdd(cnt + slot, 1u);
+      __threadfence_block();
+    }
+    old = __shfl_sync(0xffffffffu, old, 0);
+    __syncwarp();
+    if (old + 1 != static_cast<uint32_t>(arrivals)) return;
+    // last arrival: lane l sums outputs l, l + 32, ... (col * 16 + row) over the warps, in warp order
+    const int64_t tile = blockIdx.x + static_cast<int64_t>(lt) * gridDim.x;
+    const bool bad = *abort_flag != 0u;
+    for (int idx = lane; idx < 16 * m; idx += 32) {
+      float v = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        v += rs[w * (kTileRows * 8) + idx];
+        rs[w * (kTileRows * 8) + idx] = 0.0f;
+      }
+      const int row = idx & 15, col = idx >> 4;
+      const int64_t r = tile * kTileRows + row;
+      if (r < N) y[static_cast<int64_t>(col) * N + r] = bad ? __int_as_float(0x7fc00000) : v * out_scale;
+    }
+    __threadfence_block();
+    __syncwarp();
+    if (lane == 0) {
+      cnt[slot] = 0u;
+      __threadfence_block();
+      uses[slot] = use + 1u;
+    }
+  };
+
+  // ---- consumer side ----
+  Cursor cons = {0, warp};
+  while (cons.c >= n_chunks) { cons.c -= n_chunks; ++cons.lt; }
   float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  for (int c = warp; c < n_chunks; c += kWarps) {
-    int g0, ng;
-    chunk_range(c, g0, ng);
-    // the next chunk of this warp is requested before this one is computed
-    const int cn = c + kWarps;
-    if (cn < n_chunks) {
-      int g0n, ngn;
-      chunk_range(cn, g0n, ngn);
-      load_chunk<META4>(nxt, crow0, crow1, srow0, srow1, zrow0, zrow1, g0n, ngn);
+  int lt_cur = cons.lt;
+  int slot = 0;
+  uint32_t phase = 0;
+  bool ok = true;
+  int n_done = 0;
+  for (int e = warp; e < total; e += kWarps) {
+    if (cons.lt != lt_cur) {
+      flush(lt_cur, acc);
+      acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+      lt_cur = cons.lt;
+    }
+    // every lane waits (the wait makes the TMA and cp.async data visible to it); the warp goes
+    // on only if all of them saw the chunk arrive
+    const bool got = mbar_wait_suspend(bars + slot, phase, abort_flag);
+    if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+    const uint8_t *box = ring + slot * kChunkBytes;
+    const int g0 = cons.c * kCG;
+    const int ng = KG - g0 < kCG ? KG - g0 : kCG;
+    const uint8_t *xb = xs_base + g0 * 128;
+    const uint32_t *sb = sum_base + g0 * 3;
+    uint4 sv0 = make_uint4(0, 0, 0, 0), sv1 = sv0;
+    uint2 zv0 = make_uint2(0, 0), zv1 = zv0;
+    int64_t r0 = 0, r1 = 0;
+    if (FULL) {
+      const uint8_t *ms = meta + slot * kMetaBytes;
+      sv0 = *reinterpret_cast<const uint4 *>(ms + rho * 16);
+      sv1 = *reinterpret_cast<const uint4 *>(ms + (rho + 8) * 16);
+      zv0 = *reinterpret_cast<const uint2 *>(ms + 256 + rho * 8);
+      zv1 = *reinterpret_cast<const uint2 *>(ms + 256 + (rho + 8) * 8);
+    } else {
+      const int64_t tile = blockIdx.x + static_cast<int64_t>(cons.lt) * gridDim.x;
+      r0 = tile * kTileRows + rho;
+      r1 = r0 + 8;
+      r0 = r0 < N ? r0 : N - 1;
+      r1 = r1 < N ? r1 : N - 1;
     }
 #pragma unroll
     for (int j = 0; j < kCG; ++j) {
-      if (j < ng) {
-        const int g = g0 + j;
-        uint32_t bx[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        float q[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        if (has_x) {
-          if (XS) {
-            const uint4 *xp = reinterpret_cast<const uint4 *>(xst + gid * xpitch + (g * 64 + tig * 16) * 2);
-            const uint4 lo = xp[0], hi = xp[1];
-            bx[0] = lo.x; bx[1] = lo.y; bx[2] = lo.z; bx[3] = lo.w;
-            bx[4] = hi.x; bx[5] = hi.y; bx[6] = hi.z; bx[7] = hi.w;
-          } else {
-            const uint4 *xp = reinterpret_cast<const uint4 *>(xrow + g * 64);
+      if (j < 4 || ng > 4) {
+        if (!FULL && j >= ng) continue;
+        float s0, s1;
+        uint32_t zw0, zw1;
+        if (FULL) {
+          const uint32_t h0 = word4(sv0, j >> 1), h1 = word4(sv1, j >> 1);
+          s0 = (j & 1) ? half_hi(h0) : half_lo(h0);
+          s1 = (j & 1) ? half_hi(h1) : half_lo(h1);
+          zw0 = j < 4 ? zv0.x : zv0.y;
+          zw1 = j < 4 ? zv1.x : zv1.y;
+        } else {
+          const int g = g0 + j;
+          s0 = f16_bits_to_f32(__ldg(scale + r0 * KG + g));
+          s1 = f16_bits_to_f32(__ldg(scale + r1 * KG + g));
+          zw0 = static_cast<uint32_t>(__ldg(zero + r0 * KG + g)) << (8 * (j & 3));
+          zw1 = static_cast<uint32_t>(__ldg(zero + r1 * KG + g)) << (8 * (j & 3));
+        }
+        const uint8_t *cw = box + off[j & 3] + (j >> 2) * kBoxBytes;
+        const uint2 w0 = *reinterpret_cast<const uint2 *>(cw);
+        const uint2 w1 = *reinterpret_cast<const uint2 *>(cw + 1024);
+        float p[4];
+        if (XS) {
+          // fp16 operands: for nibble pairs at bits 0-3 / 16-19 the pattern 0x6400 | q is
+          // 1024 + q, at bits 4-7 / 20-23 it is 1024 + 16 q (the staged x carries 1/16 there)
+          const uint4 *xp = reinterpret_cast<const uint4 *>(xb + j * 128);
+          const uint4 xl = xp[0], xh = xp[1];
+          const uint32_t bx[8] = {xl.x, xl.y, xl.z, xl.w, xh.x, xh.y, xh.z, xh.w};
+          // correction: -(1024 + z) * sum x + 960 * sum of odd-position x, from the split sums
+          const uint32_t bc = sb[j * 3];
+          const uint32_t sel = csel_base + csel_mul * (j & 3);
+          const uint32_t c0 = __byte_perm(zw0, 0x006380E4u, sel), c1 = __byte_perm(zw1, 0x006380E4u, sel);
+          const uint32_t ac[4] = {c0, c1, c0, c1};
+          mma_f16_16816_z(p, ac, bc, 0u);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t u0 = h ? w0.y : w0.x, u1 = h ? w1.y : w1.x;
+            const uint32_t t0 = u0 >> 8, t1 = u1 >> 8;
+            const uint32_t A0[4] = {lop_or<0x000F000Fu, 0x64006400u>(u0), lop_or<0x000F000Fu, 0x64006400u>(u1),
+                                    lop_or<0x00F000F0u, 0x64006400u>(u0), lop_or<0x00F000F0u, 0x64006400u>(u1)};
+            mma_f16_16816(p, A0, bx[4 * h + 0], bx[4 * h + 1]);
+            const uint32_t A1[4] = {lop_or<0x000F000Fu, 0x64006400u>(t0), lop_or<0x000F000Fu, 0x64006400u>(t1),
+                                    lop_or<0x00F000F0u, 0x64006400u>(t0), lop_or<0x00F000F0u, 0x64006400u>(t1)};
+            mma_f16_16816(p, A1, bx[4 * h + 2], bx[4 * h + 3]);
+          }
+        } else {
+          uint32_t bx[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) bx[i] = 0u;
+          if (has_x) {
+            const uint4 *xp = reinterpret_cast<const uint4 *>(xrow + (g0 + j) * 64);
             permute16(__ldg(xp), __ldg(xp + 1), bx);
           }
-        }
-        float p[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        const uint32_t w0[2] = {cur.a0[j].x, cur.a0[j].y}, w1[2] = {cur.a1[j].x, cur.a1[j].y};
+          float q[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          p[0] = p[1] = p[2] = p[3] = 0.0f;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t A0[4] = {nib_pair(w0[h]), nib_pair(w1[h]), nib_pair(w0[h] >> 4), nib_pair(w1[h] >> 4)};
-          mma_bf16_16816(p, A0, bx[4 * h + 0], bx[4 * h + 1]);
-          if (!XS) mma_bf16_16816(q, ones, bx[4 * h + 0], bx[4 * h + 1]);
-          const uint32_t A1[4] = {nib_pair(w0[h] >> 8), nib_pair(w1[h] >> 8), nib_pair(w0[h] >> 12),
-                                  nib_pair(w1[h] >> 12)};
-          mma_bf16_16816(p, A1, bx[4 * h + 2], bx[4 * h + 3]);
-          if (!XS) mma_bf16_16816(q, ones, bx[4 * h + 2], bx[4 * h + 3]);
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t u0 = h ? w0.y : w0.x, u1 = h ? w1.y : w1.x;
+            const uint32_t A0[4] = {nib_pair(u0), nib_pair(u1), nib_pair(u0 >> 4), nib_pair(u1 >> 4)};
+            mma_bf16_16816(p, A0, bx[4 * h + 0], bx[4 * h + 1]);
+            mma_bf16_16816(q, ones, bx[4 * h + 0], bx[4 * h + 1]);
+            const uint32_t A1[4] = {nib_pair(u0 >> 8), nib_pair(u1 >> 8), nib_pair(u0 >> 12), nib_pair(u1 >> 12)};
+            mma_bf16_16816(p, A1, bx[4 * h + 2], bx[4 * h + 3]);
+            mma_bf16_16816(q, ones, bx[4 * h + 2], bx[4 * h + 3]);
+          }
+          const float zc0 = 128.0f + static_cast<float>(__byte_perm(zw0, 0u, 0x4440u + (j & 3)));
+          const float zc1 = 128.0f + static_cast<float>(__byte_perm(zw1, 0u, 0x4440u + (j & 3)));
+          p[0] = fmaf(-zc0, q[0], p[0]);
+          p[1] = fmaf(-zc0, q[1], p[1]);
+          p[2] = fmaf(-zc1, q[2], p[2]);
+          p[3] = fmaf(-zc1, q[3], p[3]);
         }
-        if (XS) {
-          const float2 xs2 = *reinterpret_cast<const float2 *>(xsum + g * 8 + 2 * tig);
-          q[0] = xs2.x; q[1] = xs2.y; q[2] = xs2.x; q[3] = xs2.y;
-        }
-        const uint32_t sw0 = (j < 2 ? cur.s0.x : cur.s0.y) >> (16 * (j & 1));
-        const uint32_t sw1 = (j < 2 ? cur.s1.x : cur.s1.y) >> (16 * (j & 1));
-        const float sc0 = f16_bits_to_f32(static_cast<uint16_t>(sw0));
-        const float sc1 = f16_bits_to_f32(static_cast<uint16_t>(sw1));
-        const float zc0 = 128.0f + static_cast<float>((cur.z0 >> (8 * j)) & 0xFFu);
-        const float zc1 = 128.0f + static_cast<float>((cur.z1 >> (8 * j)) & 0xFFu);
-        // sum_k (q - z) x = sum_k (128 + q) x - (128 + z) sum_k x, in fp32
-        acc[0] = fmaf(sc0, fmaf(-zc0, q[0], p[0]), acc[0]);
-        acc[1] = fmaf(sc0, fmaf(-zc0, q[1], p[1]), acc[1]);
-        acc[2] = fmaf(sc1, fmaf(-zc1, q[2], p[2]), acc[2]);
-        acc[3] = fmaf(sc1, fmaf(-zc1, q[3], p[3]), acc[3]);
+        acc[0] = fmaf(s0, p[0], acc[0]);
+        acc[1] = fmaf(s0, p[1], acc[1]);
+        acc[2] = fmaf(s1, p[2], acc[2]);
+        acc[3] = fmaf(s1, p[3], acc[3]);
       }
     }
-    cur = nxt;
-  }
-  red[warp][gid][2 * tig] = acc[0];
-  red[warp][gid][2 * tig + 1] = acc[1];
-  red[warp][gid + 8][2 * tig] = acc[2];
-  red[warp][gid + 8][2 * tig + 1] = acc[3];
-  __syncthreads();
-  if (threadIdx.x < kTileRows * 8) {
-    const int row = threadIdx.x & 15, col = threadIdx.x >> 4;
-    const int64_t r = row0 + row;
-    if (col < m && r < N) {
-      float v = 0.0f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) v += red[w][row][col];
-      y[static_cast<int64_t>(col) * N + r] = v;
+    // every lane's reads of this slot have fed the MMAs above; refill it
+    __syncwarp();
+    ++n_done;
+    if (e + kStages * kWarps < total) {
+      issue(slot);
+      advance(prod, n_chunks);
+      ++n_issued;
     }
+    advance(cons, n_chunks);
+    if (++slot == kStages) { slot = 0; phase ^= 1u; }
+  }
+  if (ok && total > warp) flush(lt_cur, acc);
+  // a warp that gave up lets the copies it issued land before the CTA exits
+  for (; n_done < n_issued; ++n_done) {
+    mbar_wait_suspend(bars + slot, phase, abort_flag, false);
+    if (++slot == kStages) { slot = 0; phase ^= 1u; }
   }
 }
 
-template <bool META4, bool XS>
+template <bool FULL, bool XS>
 cq_status launch_gemv4(const cq_qweight &qw, const void *x, int m, float *y, cudaStream_t s) {
-  const int smem = kRedBytes + (XS ? static_cast<int>(xstage_bytes(m, qw.cols)) : 0);
-  cq_status st = cuda_check(cudaFuncSetAttribute(gemv4_kernel<META4, XS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 smem), "cq_dequant_gemv: shared memory attribute");
+  CUtensorMap tm;
+  cq_status st = code_tensor_map(&tm, qw.plane[2], qw.rows, qw.cols, kTileRows, "cq_dequant_gemv");
   if (st != CQ_OK) return st;
+  const int smem = static_cast<int>(gemv_smem(m, qw.cols, XS));
+  st = cuda_check(cudaFuncSetAttribute(gemv4_kernel<FULL, XS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                  "cq_dequant_gemv: shared memory attribute");
+  if (st != CQ_OK) return st;
+  const int64_t tiles = (qw.rows + kTileRows - 1) / kTileRows;
+  const int64_t grid = tiles < sm_count() ? tiles : sm_count();
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((qw.rows + kTileRows - 1) / kTileRows));
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kGemvThreads);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = s;
@@ -303,7 +599,7 @@ cq_status launch_gemv4(const cq_qweight &qw, const void *x, int m, float *y, cud
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_check(cudaLaunchKernelEx(&cfg, gemv4_kernel<META4, XS>, qw.plane[2], qw.scale, qw.zero,
+  return cuda_check(cudaLaunchKernelEx(&cfg, gemv4_kernel<FULL, XS>, tm, qw.scale, qw.zero,
                                        static_cast<const __nv_bfloat16 *>(x), m, qw.rows, qw.cols, y),
                     "cq_dequant_gemv");
 }
@@ -387,13 +683,13 @@ cq_status launch_gemv(const cq_qweight &qw, const void *x, cq_dtype xdt, int m, 
   if (K == 0) return cuda_check(cudaMemsetAsync(y, 0, sizeof(float) * m * N, s), "cq_dequant_gemv: zero y");
   const bool tc = qw.bits == nullptr && qw.residual == nullptr && xdt == CQ_BF16;
   if (tc) {
-    // 16-byte scale and 8-byte zero vectors need a row pitch of a multiple of 8 groups
     const int64_t KG = K >> 6;
-    // 8-byte scale and 4-byte zero vectors need a row pitch of a multiple of 4 groups
-    const bool meta4 = (KG % 4 == 0) && aligned8(qw.scale) && (reinterpret_cast<uintptr_t>(qw.zero) & 3u) == 0;
-    // small activation sets (decode) are staged once per CTA in shared memory
-    const bool xs = xstage_bytes(m, K) <= kXStageMax;
-    if (meta4) return xs ? launch_gemv4<true, true>(qw, x, m, y, s) : launch_gemv4<true, false>(qw, x, m, y, s);
+    // the per-chunk scale (8-byte) and zero (4-byte) copies need whole chunks of 4 groups
+    const bool full = (KG % 4 == 0) && aligned8(qw.scale) && (reinterpret_cast<uintptr_t>(qw.zero) & 3u) == 0;
+    // activations are staged once per CTA in shared memory when they fit
+    const bool xs = gemv_smem(m, K, true) <= kSmemCap;
+    if (gemv_smem(m, K, false) > kSmemCap) return fail(CQ_ERR_SHAPE, "cq_dequant_gemv: cols too large");
+    if (full) return xs ? launch_gemv4<true, true>(qw, x, m, y, s) : launch_gemv4<true, false>(qw, x, m, y, s);
     return xs ? launch_gemv4<false, true>(qw, x, m, y, s) : launch_gemv4<false, false>(qw, x, m, y, s);
   }
   const int64_t need = (N + 7) / 8;

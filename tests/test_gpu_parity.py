@@ -247,7 +247,10 @@ def test_gemv_config0_fp32_with_projected_residual():
     check_matmul(host(ops.gemv(qw0, x0)), y0, "cfg0 revoked")
 
 
-@pytest.mark.parametrize("rows,cols", [(256, 512), (16, 64), (47, 64 * 9), (300, 64 * 21), (1000, 4096)])
+# shapes: whole and ragged 4-group chunks and 16-row tiles; more tiles than the persistent
+# grid holds (5000 rows); activations too large to stage in shared memory (K = 16384, 12864)
+@pytest.mark.parametrize("rows,cols", [(256, 512), (16, 64), (47, 64 * 9), (300, 64 * 21), (1000, 4096),
+                                       (5000, 64 * 16), (48, 64 * 256), (40, 64 * 201)])
 @pytest.mark.parametrize("m", [1, 3, 8])
 def test_gemv_tensor_core_4bit(rows, cols, m):
     qw, x_d, y_ref, _ = _matmul_case(rows, cols, m, "bf16", seed=rows + m)
