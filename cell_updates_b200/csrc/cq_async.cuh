@@ -1,6 +1,6 @@
 // cq_async.cuh -- asynchronous-copy building blocks shared by the matmul kernels: mbarrier
 // waits with an iteration bound, TMA tiled loads, cp.async with mbarrier completion, and the
-// driver's tensor-map encoder. Every wait gives up after kSpinLimit polls: the caller raises
+// driver's tensor-map encoder. Every wait gives up after kSuspendLimit tries: the caller raises
 // its error flag, lets its own copies land and returns, so a lost arrival never hangs a GPU.
 #pragma once
 #include <cuda.h>
@@ -12,7 +12,6 @@
 
 namespace cq {
 
-constexpr uint32_t kSpinLimit = 1u << 22;   // try_wait polls before a wait gives up
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -40,21 +39,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity) {
   return ok != 0;
 }
 
-// bounded wait on the phase of the given parity; false on timeout or when another role gave up
-__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile uint32_t *abort_flag,
-                                          uint32_t *status, bool honour_abort = true) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(b, parity)) return true;
-    if ((i & 63) == 63) {
-      if (honour_abort && *abort_flag) return false;
-      __nanosleep(64);
-    }
-  }
-  *abort_flag = 1u;
-  if (status) atomicOr(status, 1u);
-  return false;
-}
-
 // try_wait that lets the hardware suspend the thread for up to hint_ns while the phase is open
 __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *b, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
@@ -66,18 +50,27 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *b, uint32_t parity,
   return ok != 0;
 }
 
-// bounded wait for consumers that mostly find the phase complete: suspends in hardware instead
-// of spinning; gives up after kSuspendLimit tries (about a second) or when another warp gave up
+// bounded wait on the phase of the given parity; false on timeout or when another role gave
+// up. A waiting thread is suspended in hardware (up to 1 us per try) instead of spinning, so
+// waiting warps leave the issue slots to the warps that have work; after kSuspendLimit tries
+// (about a second) the wait raises the abort flag and the status word.
 constexpr uint32_t kSuspendLimit = 1u << 20;
-__device__ __forceinline__ bool mbar_wait_suspend(uint64_t *b, uint32_t parity, volatile uint32_t *abort_flag,
-                                                  bool honour_abort = true) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile uint32_t *abort_flag,
+                                          uint32_t *status, bool honour_abort = true) {
   if (mbar_try_wait(b, parity)) return true;
   for (uint32_t i = 0; i < kSuspendLimit; ++i) {
     if (mbar_try_wait_hint(b, parity, 1000u)) return true;
     if (honour_abort && *abort_flag) return false;
   }
   *abort_flag = 1u;
+  if (status) atomicOr(status, 1u);
   return false;
+}
+
+// the same wait without a status word (the caller reports through its output)
+__device__ __forceinline__ bool mbar_wait_suspend(uint64_t *b, uint32_t parity, volatile uint32_t *abort_flag,
+                                                  bool honour_abort = true) {
+  return mbar_wait(b, parity, abort_flag, nullptr, honour_abort);
 }
 
 // 2-D tiled TMA load into this CTA's shared memory, completing on an mbarrier (no multicast)

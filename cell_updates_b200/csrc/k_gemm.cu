@@ -12,8 +12,10 @@
 // Structure (one CTA per SM, persistent; work = (128-row tile, group) items split evenly
 // over the CTAs in row-major order, so a CTA covers a contiguous K range of one or two tiles):
 //   warp 0      TMA producer: code blocks of 8 groups (two adjacent 128-byte-wide boxes per
-//               row, 128-byte swizzled: long DRAM runs and conflict-free shared reads), and per
-//               group the activations (m rows x 64 bf16, swizzled = the UMMA K-major layout)
+//               row, 128-byte swizzled: long DRAM runs and conflict-free shared reads)
+//   warp 18     TMA producer: per group the activations (m rows x 64 bf16, swizzled = the
+//               UMMA K-major layout); a separate warp, so code blocks are requested as soon as
+//               a buffer frees up, however far the activation ring runs ahead
 //   warp 1      MMA issuer: four tcgen05.mma (M=128, N=NT, K=16) per group into one of four
 //               tensor-memory accumulators; commits release the A and x stages and publish
 //   warps 2-9   dequantize: each thread turns half a row of the group's codes into bf16
@@ -29,23 +31,31 @@ namespace cq {
 namespace {
 
 constexpr int kTileM = 128;
-constexpr int kDeqWarps = 8;                       // two per row quarter: half a row each
+constexpr int kDeqWarps = 8;                       // two per TMEM lane quarter: half a row each
 constexpr int kEpiWarps = 8;                       // two per TMEM lane quarter: half the columns each
-constexpr int kThreads = 32 * (2 + kDeqWarps + kEpiWarps);
+constexpr int kThreads = 32 * (3 + kDeqWarps + kEpiWarps);
+constexpr int kXWarp = 2 + kDeqWarps + kEpiWarps;      // the last warp loads activations
 constexpr int kBlockGroups = 8;                    // groups per code block (two 128-byte boxes per row)
 constexpr uint32_t kCodeBox = kTileM * 128;        // one swizzled box: 128 rows x 4 groups
 constexpr uint32_t kCodeStage = 2 * kCodeBox;      // 32 KiB
-constexpr uint32_t kABytes = kTileM * 128;         // bf16 A tile: 128 rows x 64 columns
-constexpr int kCodeStages = 2, kAStages = 4, kXStages = 8, kAccBufs = 4;
+constexpr int kCodeStages = 4;                     // code blocks in flight
+constexpr int kG = 2;                              // groups per pipeline step
+constexpr int kSteps = 4;                          // A (tensor memory) and activation (shared) slots
+constexpr int kAccBufs = 2;                        // fp32 step accumulators in tensor memory
+constexpr uint32_t kACols = 32;                    // one group of A: 128 lanes x 64 bf16
 
 template <int NT>
 struct Cfg {
-  static constexpr uint32_t kXBytes = NT * 128;
-  static constexpr uint32_t kTmemCols = kAccBufs * NT < 32 ? 32 : kAccBufs * NT;
-  static constexpr int kBars = 2 * kCodeStages + 2 * kAStages + 2 * kXStages + 2 * kAccBufs + 1;
-  static constexpr uint32_t kSmem =
-      1024 + kCodeStages * kCodeStage + kAStages * kABytes + kXStages * kXBytes + kBars * 8 + 16;
+  static constexpr uint32_t kXBytes = NT * 128;                     // one group of activations
+  static constexpr uint32_t kAccCols = kAccBufs * kG * NT;
+  static constexpr uint32_t kACol0 = kAccCols;                     // A slots follow the accumulators
+  static constexpr uint32_t kCols = kAccCols + kSteps * kG * kACols;
+  static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
+  static_assert(kCols <= 512, "tensor memory holds 512 columns");
+  static constexpr int kBars = 2 * kCodeStages + 3 * kSteps + 2 * kAccBufs + 1;
+  static constexpr uint32_t kSmem = 1024 + kCodeStages * kCodeStage + kSteps * kG * kXBytes + kBars * 8 + 16;
 };
+
 // UMMA shared-memory descriptor: K-major operand in the 128-byte swizzled canonical layout
 // (8-row groups of 128-byte rows, 1024 bytes apart), sm_100 descriptor version 1.
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
@@ -71,6 +81,43 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint6
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
+
+// the same with A read from tensor memory (128 lanes = rows, two bf16 per 32-bit column, K-major)
+__device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// TS MMA with the B descriptor given as two 32-bit words and a compile-time accumulate flag:
+// the issuing thread shares its scheduler with busy warps, so each MMA costs it as few
+// instructions as possible
+template <bool kAccum>
+__device__ __forceinline__ void umma_ts_lean(uint32_t tmem_d, uint32_t tmem_a, uint32_t bdesc_lo, uint32_t bdesc_hi,
+                                             uint32_t idesc) {
+  if (kAccum)
+    asm volatile(
+        "{\n .reg .b64 bd;\n mov.b64 bd, {%2, %3};\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, 1;\n}\n" ::"r"(tmem_d),
+        "r"(tmem_a), "r"(bdesc_lo), "r"(bdesc_hi), "r"(idesc));
+  else
+    asm volatile(
+        "{\n .reg .b64 bd;\n mov.b64 bd, {%2, %3};\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, 0;\n}\n" ::"r"(tmem_d),
+        "r"(tmem_a), "r"(bdesc_lo), "r"(bdesc_hi), "r"(idesc));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(bar))
@@ -107,31 +154,38 @@ __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
   return d;
 }
 
-// the items of one CTA: (tile, group) pairs, grouped into code blocks of up to 8 groups
+// The work of one CTA: steps = (tile, pair of groups) in row-major order; a step covers
+// groups g, g + 1 of a tile (only g when it is the tile's last, odd group). Code blocks of
+// 8 groups = 4 steps; a block also ends at a tile end and at the end of the CTA's range.
 struct ItemWalk {
-  int64_t i;          // current item (tile * KG + g)
-  int tile, g;
+  int64_t i;          // current step (tile * P + pair)
+  int tile, p, g, ng; // tile, pair, first group, groups in this step (1 or 2)
   int block;          // index of the current code block
   int block_g0;       // first group of the current block
   bool block_start, block_end, tile_end;
 };
 
+__device__ __forceinline__ void walk_set_g(ItemWalk &w, int KG) {
+  w.g = 2 * w.p;
+  w.ng = KG - w.g < 2 ? KG - w.g : 2;
+}
+
 __device__ __forceinline__ void walk_init(ItemWalk &w, int64_t it_begin, int KG) {
+  const int P = (KG + 1) / 2;
   w.i = it_begin;
-  w.tile = static_cast<int>(it_begin / KG);
-  w.g = static_cast<int>(it_begin % KG);
+  w.tile = static_cast<int>(it_begin / P);
+  w.p = static_cast<int>(it_begin % P);
+  walk_set_g(w, KG);
   w.block = 0;
   w.block_g0 = w.g;
   w.block_start = true;
 }
 
-// flags of the current item, given the CTA's end
-// blocks end on multiples of 8 groups (and at tile and range ends), so every block after the
-// first one of a range starts on an 8-group boundary
+// flags of the current step, given the CTA's end
 __device__ __forceinline__ void walk_flags(ItemWalk &w, int64_t it_end, int KG) {
   const bool last = w.i + 1 >= it_end;
-  w.tile_end = (w.g == KG - 1) || last;
-  w.block_end = w.tile_end || (((w.g + 1) & (kBlockGroups - 1)) == 0);
+  w.tile_end = (w.g + w.ng == KG) || last;
+  w.block_end = w.tile_end || (((w.g + 2) & (kBlockGroups - 1)) == 0);
 }
 
 // first (tile, group) of the block after the current one (valid when it exists)
@@ -166,10 +220,11 @@ __device__ __forceinline__ void load_block_scales(const uint16_t *scale, int64_t
 __device__ __forceinline__ void walk_next(ItemWalk &w, int KG) {
   const bool new_block = w.block_end;
   ++w.i;
-  if (++w.g == KG) {
-    w.g = 0;
+  if (++w.p == (KG + 1) / 2) {
+    w.p = 0;
     ++w.tile;
   }
+  walk_set_g(w, KG);
   w.block_start = new_block;
   if (new_block) {
     ++w.block;
@@ -186,13 +241,13 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sC = smem;                                   // code blocks (1024-aligned, swizzled)
-  uint8_t *sA = sC + kCodeStages * kCodeStage;          // bf16 A tiles (1024-aligned)
-  uint8_t *sX = sA + kAStages * kABytes;                // activation tiles (1024-aligned)
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sX + kXStages * C::kXBytes);
+  uint8_t *sX = sC + kCodeStages * kCodeStage;          // activation tiles (1024-aligned)
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sX + kSteps * kG * C::kXBytes);
   uint64_t *c_full = bars, *c_empty = c_full + kCodeStages;
-  uint64_t *a_full = c_empty + kCodeStages, *a_empty = a_full + kAStages;
-  uint64_t *x_full = a_empty + kAStages, *x_empty = x_full + kXStages;
-  uint64_t *acc_full = x_empty + kXStages, *acc_empty = acc_full + kAccBufs;
+  // a step (two groups) has an A slot in tensor memory and an activation slot in shared memory,
+  // filled separately (a_full, x_full) and released together by one MMA commit (s_empty)
+  uint64_t *a_full = c_empty + kCodeStages, *x_full = a_full + kSteps, *s_empty = x_full + kSteps;
+  uint64_t *acc_full = s_empty + kSteps, *acc_empty = acc_full + kAccBufs;
   uint64_t *drain = acc_empty + kAccBufs;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile uint32_t *abort_flag = tmem_slot + 1;
@@ -207,13 +262,10 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
       mbar_init(c_full + i, 1);
       mbar_init(c_empty + i, kDeqWarps);
     }
-    for (int i = 0; i < kAStages; ++i) {
+    for (int i = 0; i < kSteps; ++i) {
       mbar_init(a_full + i, kDeqWarps);
-      mbar_init(a_empty + i, 1);
-    }
-    for (int i = 0; i < kXStages; ++i) {
       mbar_init(x_full + i, 1);
-      mbar_init(x_empty + i, 1);
+      mbar_init(s_empty + i, 1);
     }
     for (int i = 0; i < kAccBufs; ++i) {
       mbar_init(acc_full + i, 1);
@@ -234,52 +286,81 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- TMA producer: code blocks and activation tiles ----------------
+    // ---------------- TMA producer: code blocks ----------------
     if (lane == 0) {
       ItemWalk w;
       walk_init(w, it_begin, KG);
-      int code_issued = 0, x_issued = 0;
-      bool ok = true;
-      for (int li = 0; li < n_local && ok; ++li) {
+      int code_issued = 0;
+      for (int li = 0; li < n_local; ++li) {
         walk_flags(w, it_end, KG);
         if (w.block_start) {
           const int cs = w.block % kCodeStages;
-          if (!(ok = mbar_wait(c_empty + cs, ((w.block / kCodeStages) & 1) ^ 1, abort_flag, status))) break;
+          if (!mbar_wait(c_empty + cs, ((w.block / kCodeStages) & 1) ^ 1, abort_flag, status)) break;
           mbar_arrive_expect_tx(c_full + cs, kCodeStage);
           uint8_t *dst = sC + cs * kCodeStage;
           tma_load_2d(dst, &tm_codes, w.block_g0 * 32, w.tile * kTileM, c_full + cs);
           tma_load_2d(dst + kCodeBox, &tm_codes, w.block_g0 * 32 + 128, w.tile * kTileM, c_full + cs);
           code_issued = w.block + 1;
         }
-        const int xs = li % kXStages;
-        if (!(ok = mbar_wait(x_empty + xs, ((li / kXStages) & 1) ^ 1, abort_flag, status))) break;
-        mbar_arrive_expect_tx(x_full + xs, C::kXBytes);
-        tma_load_2d(sX + xs * C::kXBytes, &tm_x, w.g * 64, 0, x_full + xs);
-        x_issued = li + 1;
         walk_next(w, KG);
       }
       // every copy this thread started has landed before the CTA may exit
       for (int b = code_issued - kCodeStages > 0 ? code_issued - kCodeStages : 0; b < code_issued; ++b)
         mbar_wait(c_full + (b % kCodeStages), (b / kCodeStages) & 1, abort_flag, status, false);
-      for (int li = x_issued - kXStages > 0 ? x_issued - kXStages : 0; li < x_issued; ++li)
-        mbar_wait(x_full + (li % kXStages), (li / kXStages) & 1, abort_flag, status, false);
+    }
+  } else if (warp == kXWarp) {
+    // ---------------- TMA producer: the step's activation tiles ----------------
+    if (lane == 0) {
+      ItemWalk w;
+      walk_init(w, it_begin, KG);
+      int x_issued = 0;
+      for (int li = 0; li < n_local; ++li) {
+        const int st = li % kSteps;
+        if (!mbar_wait(s_empty + st, ((li / kSteps) & 1) ^ 1, abort_flag, status)) break;
+        uint8_t *dst = sX + st * kG * C::kXBytes;
+        mbar_arrive_expect_tx(x_full + st, w.ng * C::kXBytes);
+        tma_load_2d(dst, &tm_x, w.g * 64, 0, x_full + st);
+        if (w.ng > 1) tma_load_2d(dst + C::kXBytes, &tm_x, w.g * 64 + 64, 0, x_full + st);
+        x_issued = li + 1;
+        walk_flags(w, it_end, KG);
+        walk_next(w, KG);
+      }
+      for (int li = x_issued - kSteps > 0 ? x_issued - kSteps : 0; li < x_issued; ++li)
+        mbar_wait(x_full + (li % kSteps), (li / kSteps) & 1, abort_flag, status, false);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc<NT>();
+      // B descriptors differ only in the start-address field (bits 0-13, address >> 4), which
+      // no offset here carries out of: adding to the low word is enough
+      const uint64_t d0 = umma_desc_sw128(smem_u32(sX));
+      const uint32_t dlo0 = static_cast<uint32_t>(d0), dhi = static_cast<uint32_t>(d0 >> 32);
+      const int P = (KG + 1) / 2;
+      int p = static_cast<int>(it_begin % P);
       for (int li = 0; li < n_local; ++li) {
-        const int as = li % kAStages, xs = li % kXStages, b = li % kAccBufs;
-        if (!mbar_wait(a_full + as, (li / kAStages) & 1, abort_flag, status)) break;
-        if (!mbar_wait(x_full + xs, (li / kXStages) & 1, abort_flag, status)) break;
+        const int st = li % kSteps, b = li % kAccBufs;
+        const bool two = (KG & 1) == 0 || p != P - 1;
+        if (++p == P) p = 0;
+        if (!mbar_wait(a_full + st, (li / kSteps) & 1, abort_flag, status)) break;
+        if (!mbar_wait(x_full + st, (li / kSteps) & 1, abort_flag, status)) break;
         if (!mbar_wait(acc_empty + b, ((li / kAccBufs) & 1) ^ 1, abort_flag, status)) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + as * kABytes), b0 = smem_u32(sX + xs * C::kXBytes);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tmem + b * NT, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), idesc, kk > 0);
-        umma_commit(a_empty + as);
-        umma_commit(x_empty + xs);
+        const uint32_t ta = tmem + C::kACol0 + st * kG * kACols;
+        const uint32_t td = tmem + b * kG * NT;
+        const uint32_t blo = dlo0 + ((st * kG * C::kXBytes) >> 4);
+        umma_ts_lean<false>(td, ta, blo, dhi, idesc);
+        umma_ts_lean<true>(td, ta + 8, blo + 2, dhi, idesc);
+        umma_ts_lean<true>(td, ta + 16, blo + 4, dhi, idesc);
+        umma_ts_lean<true>(td, ta + 24, blo + 6, dhi, idesc);
+        if (two) {
+          constexpr uint32_t xo = C::kXBytes >> 4;
+          umma_ts_lean<false>(td + NT, ta + kACols, blo + xo, dhi, idesc);
+          umma_ts_lean<true>(td + NT, ta + kACols + 8, blo + xo + 2, dhi, idesc);
+          umma_ts_lean<true>(td + NT, ta + kACols + 16, blo + xo + 4, dhi, idesc);
+          umma_ts_lean<true>(td + NT, ta + kACols + 24, blo + xo + 6, dhi, idesc);
+        }
+        umma_commit(s_empty + st);
         umma_commit(acc_full + b);
       }
       // all issued MMAs have completed before tensor memory is released
@@ -287,10 +368,11 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
       mbar_wait(drain, 0, abort_flag, status, false);
     }
   } else if (warp < 2 + kDeqWarps) {
-    // ---------------- dequantize: half a row per thread ----------------
-    const int dw = warp - 2;
-    const int r = (dw & 3) * 32 + lane;          // tile row
-    const int half = dw >> 2;                     // columns 32*half .. 32*half+31 of the group
+    // ---------------- dequantize: half a row per thread, into tensor memory ----------------
+    // a warp may only touch TMEM lanes 32 * (warp % 4) .. + 31, so rows follow the warp index
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;               // tile row = TMEM lane
+    const int half = (warp - 2) >> 2;             // columns 32*half .. 32*half+31 of each group
     ItemWalk w;
     walk_init(w, it_begin, KG);
     auto clamp_row = [&](int tile) {
@@ -300,6 +382,7 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
     // zero points of the current block and, one block ahead, of the next one
     uint32_t zlo, zhi, nzlo = 0, nzhi = 0;
     load_block_zeros(zero, clamp_row(w.tile), KG, w.g, zlo, zhi);
+    const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
     for (int li = 0; li < n_local; ++li) {
       walk_flags(w, it_end, KG);
       const int cs = w.block % kCodeStages;
@@ -310,49 +393,54 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         }
         int nt, ng;
         walk_next_block(w, KG, nt, ng);
-        if (static_cast<int64_t>(nt) * KG + ng < it_end) load_block_zeros(zero, clamp_row(nt), KG, ng, nzlo, nzhi);
+        if (li + 1 < n_local) load_block_zeros(zero, clamp_row(nt), KG, ng, nzlo, nzhi);   // rows clamp: in bounds
         if (!mbar_wait(c_full + cs, (w.block / kCodeStages) & 1, abort_flag, status)) break;
       }
-      const int as = li % kAStages;
-      if (!mbar_wait(a_empty + as, ((li / kAStages) & 1) ^ 1, abort_flag, status)) break;
-      const int jz = w.g - w.block_g0;
-      const uint32_t z = ((jz < 4 ? zlo : zhi) >> (8 * (jz & 3))) & 0xFFu;
-      const uint32_t zz = 0x43004300u | z | (z << 16);      // (128 + z) in both halves
+      const int st = li % kSteps;
       // group j of the block sits in box j/4, 16-byte chunk (2*(j%4) + half) of the row, swizzled
-      const int j = w.g - w.block_g0;
-      const int chunk = ((j & 3) << 1) | half;
-      const uint4 cw = *reinterpret_cast<const uint4 *>(sC + cs * kCodeStage + (j >> 2) * kCodeBox + r * 128 +
-                                                        ((chunk ^ (r & 7)) << 4));
-      const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-      uint8_t *dst_row = sA + as * kABytes + r * 128;
+      uint32_t v[kG][16];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {       // A chunk 4*half + c = columns 8(4*half+c) .. +7
-        const uint32_t wd = words[c], w4 = wd >> 4;
-        uint4 v;
-        v.x = bf16x2_sub(nat_pair(wd, w4, 0x4400u), zz);
-        v.y = bf16x2_sub(nat_pair(wd, w4, 0x5511u), zz);
-        v.z = bf16x2_sub(nat_pair(wd, w4, 0x6622u), zz);
-        v.w = bf16x2_sub(nat_pair(wd, w4, 0x7733u), zz);
-        *reinterpret_cast<uint4 *>(dst_row + ((((half << 2) | c) ^ (r & 7)) << 4)) = v;
+      for (int jj = 0; jj < kG; ++jj) {
+        const int j = w.g - w.block_g0 + jj;
+        const uint32_t z = ((j < 4 ? zlo : zhi) >> (8 * (j & 3))) & 0xFFu;
+        const uint32_t zz = 0x43004300u | z | (z << 16);      // (128 + z) in both halves
+        const int chunk = ((j & 3) << 1) | half;
+        const uint4 cw = *reinterpret_cast<const uint4 *>(sC + cs * kCodeStage + ((j >> 2) & 1) * kCodeBox +
+                                                          r * 128 + ((chunk ^ (r & 7)) << 4));
+        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {       // columns 32*half + 8c .. +7, two per 32-bit TMEM column
+          const uint32_t wd = words[c], w4 = wd >> 4;
+          v[jj][4 * c + 0] = bf16x2_sub(nat_pair(wd, w4, 0x4400u), zz);
+          v[jj][4 * c + 1] = bf16x2_sub(nat_pair(wd, w4, 0x5511u), zz);
+          v[jj][4 * c + 2] = bf16x2_sub(nat_pair(wd, w4, 0x6622u), zz);
+          v[jj][4 * c + 3] = bf16x2_sub(nat_pair(wd, w4, 0x7733u), zz);
+        }
       }
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      // the code words are in registers: the block's last step releases its buffer now
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(a_full + as);
-        if (w.block_end) mbar_arrive(c_empty + cs);
-      }
+      if (lane == 0 && w.block_end) mbar_arrive(c_empty + cs);
+      if (!mbar_wait(s_empty + st, ((li / kSteps) & 1) ^ 1, abort_flag, status)) break;
+      tc_fence_after();
+      const uint32_t ta = tmem + tlane + C::kACol0 + st * kG * kACols + half * 16;
+      tmem_st16(ta, v[0]);
+      if (w.ng > 1) tmem_st16(ta + kACols, v[1]);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(a_full + st);
       walk_next(w, KG);
     }
-  } else {
+  } else if (warp < 2 + kDeqWarps + kEpiWarps) {
     // ---------------- epilogue: row r = TMEM lane, half of the columns ----------------
     const int ew = warp - 2 - kDeqWarps;
     const int quad = warp & 3;                 // this warp may read TMEM lanes 32*quad .. +31
     const int chalf = ew >> 2;                 // columns chalf*NT/2 .. +NT/2
     constexpr int NH = NT / 2;
     const int r = quad * 32 + lane;
-    float acc[NH];
+    float2 acc[NH / 2];                        // column pairs, updated with packed fp32x2 FMAs
 #pragma unroll
-    for (int c = 0; c < NH; ++c) acc[c] = 0.0f;
+    for (int c = 0; c < NH / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
     ItemWalk w;
     walk_init(w, it_begin, KG);
     auto clamp_row = [&](int tile) {
@@ -373,37 +461,48 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         }
         int nt, ng;
         walk_next_block(w, KG, nt, ng);
-        if (static_cast<int64_t>(nt) * KG + ng < it_end) load_block_scales(scale, clamp_row(nt), KG, ng, nsc);
+        if (li + 1 < n_local) load_block_scales(scale, clamp_row(nt), KG, ng, nsc);
       }
+      // a step's two scales share one word of the block's scale vector
       const int js = w.g - w.block_g0;
       const uint32_t sw = js < 2 ? sc[0] : js < 4 ? sc[1] : js < 6 ? sc[2] : sc[3];   // no local-memory indexing
-      const float sf = f16_bits_to_f32(static_cast<uint16_t>(sw >> (16 * (js & 1))));
+      const float sf0 = f16_bits_to_f32(static_cast<uint16_t>(sw & 0xFFFFu));
+      const float sf1 = w.ng > 1 ? f16_bits_to_f32(static_cast<uint16_t>(sw >> 16)) : 0.0f;
       if (!mbar_wait(acc_full + b, (li / kAccBufs) & 1, abort_flag, status)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + b * NT + chalf * NH;
-      uint32_t d[NH];
-      if constexpr (NH >= 16) {
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + b * kG * NT + chalf * NH;
 #pragma unroll
-        for (int c0 = 0; c0 < NH; c0 += 16) tmem_ld16(tbase + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
-      } else {
-        tmem_ld8(tbase, d);
+      for (int jj = 0; jj < kG; ++jj) {
+        if (jj < w.ng) {
+          uint32_t d[NH];
+          if constexpr (NH >= 16) {
+#pragma unroll
+            for (int c0 = 0; c0 < NH; c0 += 16)
+              tmem_ld16(tbase + jj * NT + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
+          } else {
+            tmem_ld8(tbase + jj * NT, d);
+          }
+          tmem_wait_ld();
+          const float sf = jj ? sf1 : sf0;
+          const float2 s2 = make_float2(sf, sf);
+#pragma unroll
+          for (int c = 0; c < NH / 2; ++c)
+            acc[c] = __ffma2_rn(s2, make_float2(__uint_as_float(d[2 * c]), __uint_as_float(d[2 * c + 1])), acc[c]);
+        }
       }
-      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty + b);
-#pragma unroll
-      for (int c = 0; c < NH; ++c) acc[c] = fmaf(sf, __uint_as_float(d[c]), acc[c]);
       if (w.tile_end) {
         if (row < N) {
 #pragma unroll
           for (int c = 0; c < NH; ++c) {
             const int col = chalf * NH + c;
-            if (col < m) atomicAdd(y + static_cast<int64_t>(col) * N + row, acc[c]);
+            if (col < m) atomicAdd(y + static_cast<int64_t>(col) * N + row, (c & 1) ? acc[c >> 1].y : acc[c >> 1].x);
           }
         }
 #pragma unroll
-        for (int c = 0; c < NH; ++c) acc[c] = 0.0f;
+        for (int c = 0; c < NH / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
       }
       walk_next(w, KG);
     }
@@ -438,7 +537,7 @@ cq_status launch_nt(const cq_qweight &qw, const void *x, int m, float *y, uint32
   }
   const int KG = static_cast<int>(K / kGroup);
   const int64_t tiles = (N + kTileM - 1) / kTileM;
-  const int64_t items = tiles * KG;
+  const int64_t items = tiles * ((KG + 1) / 2);          // steps of two groups
   const int64_t grid = items < sm_count() ? items : sm_count();
   cq_status st = cuda_check(cudaFuncSetAttribute(gemm4_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  static_cast<int>(C::kSmem)),
