@@ -121,9 +121,12 @@ constexpr int kSmemCap = 227 * 1024;
 static_assert(kOffSums % 16 == 0 && kOffRed % 16 == 0, "shared-memory carve-up must keep 16-byte alignment");
 
 // staged activations: m rows of K bf16 in fragment order, row pitch padded by 16 bytes so the
-// rows a warp reads fall in different banks; group sums [m][KG] as three words (six fp16)
+// rows a warp reads fall in different banks. Before them: per group the power-of-two factors
+// of the 8 batch columns [KG][8] f32, then the group sums [m][KG] as three words (six fp16)
 __host__ __device__ constexpr int64_t xstage_pitch(int64_t K) { return K * 2 + 16; }
-__host__ __device__ constexpr int64_t sums_bytes(int m, int64_t K) { return ((K / 64) * m * 12 + 15) & ~int64_t(15); }
+__host__ __device__ constexpr int64_t sums_bytes(int m, int64_t K) {
+  return (K / 64) * 32 + (((K / 64) * m * 12 + 15) & ~int64_t(15));
+}
 __host__ __device__ constexpr int64_t gemv_smem(int m, int64_t K, bool xs) {
   return 1024 + kOffSums + sums_bytes(m, K) + (xs ? m * xstage_pitch(K) : 0);
 }
@@ -179,7 +182,8 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
   uint32_t *cnt = reinterpret_cast<uint32_t *>(smem + kOffCnt);            // [kRedSlots] arrivals
   volatile uint32_t *uses = reinterpret_cast<volatile uint32_t *>(smem + kOffCnt + 16);   // reductions done
   volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + kOffCnt + 32);
-  uint32_t *sums = reinterpret_cast<uint32_t *>(smem + kOffSums);          // [m][KG][2]
+  float *fsc = reinterpret_cast<float *>(smem + kOffSums);                  // [KG][8] column factors
+  uint32_t *sums = reinterpret_cast<uint32_t *>(smem + kOffSums + KG * 32); // [m][KG][3]
   uint8_t *xst = smem + kOffSums + sums_bytes(m, K);
   const int64_t xpitch = xstage_pitch(K);
   const int total = n_local * n_chunks;                                      // chunks of this CTA
@@ -236,18 +240,17 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
   }
 
   pdl_wait();   // x may be the output of the previous kernel in the stream; y is written below
-  // Staged activations (XS): x' = x * 2^-e in fp16, e a power of two that puts max|x'| in
-  // [256, 512): every bf16 value down to max|x| * 2^-18 converts exactly, the fp16 group sums
-  // below stay finite, and y is scaled back by 2^e at the end (exact). Thread t owns the
-  // 16-element blocks t, t + 512, ... of the flattened [m][K/16]; four lanes make one group.
-  // Pass 1 stores the bf16 words in fragment order and the fp32 group sums (all elements,
-  // odd-position elements); pass 2 converts both in place once the maximum is known.
-  float out_scale = 1.0f;
+  // Staged activations (XS): per group and batch row, x' = x * 2^-e in fp16 with e the power
+  // of two that puts the group's max |x| in [256, 512): every bf16 value down to that max
+  // times 2^-18 converts exactly, the fp16 group sums below stay finite, and the factor 2^e
+  // (kept per group and column) multiplies the group's result. Thread t owns the 16-element
+  // blocks t, t + 512, ... of the flattened [m][K/16]; the four lanes of a group agree on e
+  // through two shuffles, so one pass and one barrier stage everything.
   if (XS) {
-    float *wmax = reinterpret_cast<float *>(smem + kOffCnt + 48);          // [1] block maximum
     const int bpr = KG * 4;                 // 16-element blocks per activation row
     const int nblk = m * bpr;
-    float amax = 0.0f;
+    for (int i = threadIdx.x; i < KG * 8; i += kGemvThreads)
+      if ((i & 7) >= m) fsc[i] = 0.0f;      // MMA columns past the batch are never stored
     for (int b0 = 0; b0 < nblk; b0 += kGemvThreads * 4) {
       uint4 v[4][2];
       int nn[4], kk[4];
@@ -259,6 +262,7 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
         for (int i = 1; i < 8; ++i) n += b >= i * bpr ? 1 : 0;      // m <= 8: no division
         nn[u] = n;
         kk[u] = b - n * bpr;
+        v[u][0] = v[u][1] = make_uint4(0, 0, 0, 0);
         if (b < nblk) {
           const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(n) * K + kk[u] * 16);
           v[u][0] = __ldg(src);
@@ -268,82 +272,49 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int b = b0 + u * kGemvThreads + threadIdx.x;
-        float se = 0.0f, so = 0.0f;
-        if (b < nblk) {
-          uint32_t f[8];
-          permute16(v[u][0], v[u][1], f);
-          uint4 *dst = reinterpret_cast<uint4 *>(xst + nn[u] * xpitch + kk[u] * 32);
-          dst[0] = make_uint4(f[0], f[1], f[2], f[3]);
-          dst[1] = make_uint4(f[4], f[5], f[6], f[7]);
-          const uint32_t w[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
-                                 v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+        const uint32_t w[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
+                               v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+        float se = 0.0f, so = 0.0f, amax = 0.0f;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
-            se += lo;
-            so += hi;
-            amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
-          }
+        for (int e = 0; e < 8; ++e) {
+          const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
+          se += lo;
+          so += hi;
+          amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
         }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
         float sx = se + so;
         sx += __shfl_xor_sync(0xffffffffu, sx, 1);
         sx += __shfl_xor_sync(0xffffffffu, sx, 2);
         so += __shfl_xor_sync(0xffffffffu, so, 1);
         so += __shfl_xor_sync(0xffffffffu, so, 2);
-        if (b < nblk && (threadIdx.x & 3) == 0) {
-          float *dst = reinterpret_cast<float *>(sums + (nn[u] * KG + (kk[u] >> 2)) * 3);
-          dst[0] = sx;
-          dst[1] = so;
+        int e = 0;
+        if (amax > 0.0f && amax <= 3.0e38f) {
+          e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 127 - 8;
+          e = e < -100 ? -100 : (e > 100 ? 100 : e);
         }
-      }
-    }
-    // block maximum (NaNs are skipped here; they reach y through the products)
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
-    if (threadIdx.x == 0) *wmax = 0.0f;
-    __syncthreads();
-    if (lane == 0) atomicMax(reinterpret_cast<int *>(wmax), __float_as_int(amax));   // amax >= 0: int order
-    __syncthreads();
-    const float gmax = *wmax;
-    int e = 0;
-    if (gmax > 0.0f && gmax <= 3.0e38f) {
-      e = static_cast<int>((__float_as_uint(gmax) >> 23) & 0xFFu) - 127 - 8;
-      e = e < -100 ? -100 : (e > 100 ? 100 : e);
-    }
-    const float in_scale = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
-    const float in_scale16 = in_scale * 0.0625f;
-    out_scale = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
-    for (int b0 = 0; b0 < nblk; b0 += kGemvThreads * 4) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int b = b0 + u * kGemvThreads + threadIdx.x;
+        const float in_scale = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+        const float in_scale16 = in_scale * 0.0625f;
         if (b < nblk) {
-          int n = 0;
+          uint32_t f[8];
+          permute16(v[u][0], v[u][1], f);
 #pragma unroll
-          for (int i = 1; i < 8; ++i) n += b >= i * bpr ? 1 : 0;
-          const int kb = b - n * bpr;
-          uint4 *dst = reinterpret_cast<uint4 *>(xst + n * xpitch + kb * 32);
-#pragma unroll
-          for (int hlf = 0; hlf < 2; ++hlf) {
-            uint4 q = dst[hlf];
-            uint32_t wv[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              // words 1 and 3 of each half feed codes that carry a factor 16 (see below)
-              const float sc = (i & 1) ? in_scale16 : in_scale;
-              const __half2 h2 = __floats2half2_rn(__uint_as_float(wv[i] << 16) * sc,
-                                                   __uint_as_float(wv[i] & 0xFFFF0000u) * sc);
-              wv[i] = *reinterpret_cast<const uint32_t *>(&h2);
-            }
-            dst[hlf] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          for (int i = 0; i < 8; ++i) {
+            // words 1, 3, 5, 7 feed codes that carry a factor 16 (see below)
+            const float sc = (i & 1) ? in_scale16 : in_scale;
+            const __half2 h2 = __floats2half2_rn(__uint_as_float(f[i] << 16) * sc,
+                                                 __uint_as_float(f[i] & 0xFFFF0000u) * sc);
+            f[i] = *reinterpret_cast<const uint32_t *>(&h2);
           }
+          uint4 *dst = reinterpret_cast<uint4 *>(xst + nn[u] * xpitch + kk[u] * 32);
+          dst[0] = make_uint4(f[0], f[1], f[2], f[3]);
+          dst[1] = make_uint4(f[4], f[5], f[6], f[7]);
           if ((threadIdx.x & 3) == 0) {
             // exact three-way fp16 splits of the scaled sums: hi + mid + lo == value
-            uint32_t *sw = sums + (n * KG + (kb >> 2)) * 3;
-            const float sx = reinterpret_cast<const float *>(sw)[0] * in_scale;
-            const float so = reinterpret_cast<const float *>(sw)[1] * in_scale;
+            const int g = kk[u] >> 2;
             uint16_t hx[3], ho[3];
-            float rx = sx, ro = so;
+            float rx = sx * in_scale, ro = so * in_scale;
 #pragma unroll
             for (int i = 0; i < 3; ++i) {
               const __half a = __float2half_rn(rx), c = __float2half_rn(ro);
@@ -352,9 +323,11 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
               rx -= __half2float(a);
               ro -= __half2float(c);
             }
+            uint32_t *sw = sums + (nn[u] * KG + g) * 3;
             sw[0] = hx[0] | (static_cast<uint32_t>(hx[1]) << 16);
             sw[1] = hx[2] | (static_cast<uint32_t>(ho[0]) << 16);
             sw[2] = ho[1] | (static_cast<uint32_t>(ho[2]) << 16);
+            fsc[g * 8 + nn[u]] = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
           }
         }
       }
@@ -371,6 +344,7 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
   const int xrow_s = has_x ? gid : 0;
   const uint8_t *xs_base = xst + xrow_s * xpitch + tig * 32;
   const uint32_t *sum_base = sums + xrow_s * KG * 3 + (tig < 2 ? tig : 2);
+  const float *fsc_lane = fsc + 2 * tig;
   // correction operand per lane (k = 2 tig, 2 tig + 1), fp16 halves: tig 0 (Z, Z), tig 1
   // (Z, 960), tig 2 (960, 960), tig 3 (0, 0), Z = -(1024 + z) = 0xE400 | z (byte j of the
   // zero word); constant bytes 4..7 = E4 80 63 00
@@ -381,7 +355,8 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
   const int arrivals = n_chunks < kWarps ? n_chunks : kWarps;
 
   // store this warp's partials of local tile lt; the last arrival reduces and writes y
-  auto flush = [&](int lt, const float acc[4]) {
+  auto flush = [&](int lt, const float2 acc01, const float2 acc23) {
+    const float acc[4] = {acc01.x, acc01.y, acc23.x, acc23.y};
     const int slot = lt % kRedSlots;
     const uint32_t use = static_cast<uint32_t>(lt / kRedSlots);
     // the slot's previous tile must be reduced (and its partials zeroed) first; lane 0 polls,
@@ -429,7 +404,7 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
       }
       const int row = idx & 15, col = idx >> 4;
       const int64_t r = tile * kTileRows + row;
-      if (r < N) y[static_cast<int64_t>(col) * N + r] = bad ? __int_as_float(0x7fc00000) : v * out_scale;
+      if (r < N) y[static_cast<int64_t>(col) * N + r] = bad ? __int_as_float(0x7fc00000) : v;
     }
     __threadfence_block();
     __syncwarp();
@@ -443,7 +418,7 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
   // ---- consumer side ----
   Cursor cons = {0, warp};
   while (cons.c >= n_chunks) { cons.c -= n_chunks; ++cons.lt; }
-  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  float2 acc01 = make_float2(0.0f, 0.0f), acc23 = acc01;   // (row rho | rho + 8) x (col 2 tig, 2 tig + 1)
   int lt_cur = cons.lt;
   int slot = 0;
   uint32_t phase = 0;
@@ -451,8 +426,8 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
   int n_done = 0;
   for (int e = warp; e < total; e += kWarps) {
     if (cons.lt != lt_cur) {
-      flush(lt_cur, acc);
-      acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+      flush(lt_cur, acc01, acc23);
+      acc01 = acc23 = make_float2(0.0f, 0.0f);
       lt_cur = cons.lt;
     }
     // every lane waits (the wait makes the TMA and cp.async data visible to it); the warp goes
@@ -464,6 +439,7 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
     const int ng = KG - g0 < kCG ? KG - g0 : kCG;
     const uint8_t *xb = xs_base + g0 * 128;
     const uint32_t *sb = sum_base + g0 * 3;
+    const float *fb = fsc_lane + g0 * 8;
     uint4 sv0 = make_uint4(0, 0, 0, 0), sv1 = sv0;
     uint2 zv0 = make_uint2(0, 0), zv1 = zv0;
     int64_t r0 = 0, r1 = 0;
@@ -553,10 +529,18 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
           p[2] = fmaf(-zc1, q[2], p[2]);
           p[3] = fmaf(-zc1, q[3], p[3]);
         }
-        acc[0] = fmaf(s0, p[0], acc[0]);
-        acc[1] = fmaf(s0, p[1], acc[1]);
-        acc[2] = fmaf(s1, p[2], acc[2]);
-        acc[3] = fmaf(s1, p[3], acc[3]);
+        if (XS) {
+          // scale times the activation factors of columns 2 tig, 2 tig + 1 of this group
+          const float2 fc = *reinterpret_cast<const float2 *>(fb + j * 8);
+          const float2 a01 = __fmul2_rn(make_float2(s0, s0), fc), a23 = __fmul2_rn(make_float2(s1, s1), fc);
+          acc01 = __ffma2_rn(a01, make_float2(p[0], p[1]), acc01);
+          acc23 = __ffma2_rn(a23, make_float2(p[2], p[3]), acc23);
+        } else {
+          acc01.x = fmaf(s0, p[0], acc01.x);
+          acc01.y = fmaf(s0, p[1], acc01.y);
+          acc23.x = fmaf(s1, p[2], acc23.x);
+          acc23.y = fmaf(s1, p[3], acc23.y);
+        }
       }
     }
     // every lane's reads of this slot have fed the MMAs above; refill it
@@ -570,7 +554,7 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
     advance(cons, n_chunks);
     if (++slot == kStages) { slot = 0; phase ^= 1u; }
   }
-  if (ok && total > warp) flush(lt_cur, acc);
+  if (ok && total > warp) flush(lt_cur, acc01, acc23);
   // a warp that gave up lets the copies it issued land before the CTA exits
   for (; n_done < n_issued; ++n_done) {
     mbar_wait_suspend(bars + slot, phase, abort_flag, false);
