@@ -212,6 +212,22 @@ class Workload:
         return tot
 
 
+def max_over_ranks(value, dist, device):
+    """The largest of the ranks' values, on every rank (identity without a process group):
+    multi-GPU times are the slowest rank's."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(bytes_per_rank_step, world, ms_per_step):
+    """Whole-job throughput in GB/s: every rank's bytes over the (max-over-ranks) step time."""
+    return bytes_per_rank_step * world / (ms_per_step * 1e-3) / 1e9
+
+
 def time_graph(torch, graph, reps, stream):
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -335,10 +351,7 @@ def run_gpu(args, rank, world, local_rank):
     for mk in marks:
         for (mi, k), (a, b) in mk.items():
             per_kernel[k] += a.elapsed_time(b)
-    if dist:
-        t = torch.tensor([t_step], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_step = float(t.item())
+    t_step = max_over_ranks(t_step, dist, device)
     checks = [int(m["mism"].item()) for m in wl.mats] + [int(m["mism0"].item()) for m in wl.mats] + \
              [int(m["status"].item()) for m in wl.mats]
     assert all(c == 0 for c in checks), f"hot-path results not clean: {checks}"
@@ -346,7 +359,7 @@ def run_gpu(args, rank, world, local_rank):
     bytes_step = wl.step_bytes()
     total_bytes = sum(bytes_step.values())
     n_w = wl.n_weights()
-    value = total_bytes * world / (t_step * 1e-3) / 1e9      # GB/s over all ranks
+    value = job_value(total_bytes, world, t_step)            # GB/s over all ranks
     comps = {}
     for k in KERNELS:
         t_k = per_kernel[k] / args.steps                  # ms per step for this kernel
@@ -365,11 +378,8 @@ def run_gpu(args, rank, world, local_rank):
 
     # end to end: pinned host inputs -> device, the step, results -> host
     e2e = run_e2e(torch, wl, g1, stream, args.steps)
-    if dist:
-        t = torch.tensor([e2e["ms_per_step"]], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e["ms_per_step"] = float(t.item())
-    e2e_value = total_bytes * world / (e2e["ms_per_step"] * 1e-3) / 1e9
+    e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], dist, device)
+    e2e_value = job_value(total_bytes, world, e2e["ms_per_step"])
 
     line = None
     if rank == 0:
