@@ -7,34 +7,78 @@
 // grids. Reading of the formula: see include/cq.h.
 //
 // Every fp32 operation is an explicit round-to-nearest intrinsic, so nothing is contracted.
-#include "cq_internal.cuh"
+#include "cq_async.cuh"
 
 namespace cq {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kWarps = 16;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kStages = 1;                       // the warp's tile buffer: refilled as soon as it is in registers
+constexpr int kTileGroups = 32;                  // one tile: 32 groups, one per lane
+constexpr int kBoxBytes = kTileGroups * 128;     // one box: 32 groups x 32 floats (128-byte rows)
+constexpr int kTileBytes = 2 * kBoxBytes;        // 8 KiB of fp32 weights
+constexpr int kSmem = 1024 + kWarps * kStages * kTileBytes + kWarps * kStages * 8 + 16;
 
 // One thread owns one group of 64 weights: the group's scale and zero point (two IEEE
-// divisions, a reciprocal) are paid once per 64 weights, the 256 bytes it loads are all in
-// flight at once, and min/max need no shuffles. Loads go through L1 (ld.global.nc), so the
-// second half of each 32-byte sector is an L1 hit for the next 16-byte load.
-__global__ void __launch_bounds__(kThreads)
-quantize_kernel(const float *__restrict__ w, int64_t G, const uint8_t *__restrict__ bits,
-                uint8_t *__restrict__ codes, uint16_t *__restrict__ scale,
+// divisions, a reciprocal) are paid once per 64 weights and min/max need no shuffles. The
+// weights reach shared memory through TMA: each warp owns a buffer for one tile of 32 groups,
+// two boxes of {32 floats, 32 groups} with the 128-byte swizzle, so a lane reads its own
+// group's 16-byte chunks without bank conflicts (chunk c of row r sits at c ^ (r & 7)). Once
+// the tile is in registers the warp requests its next tile, which streams in while it computes
+// (16 warps per SM: measured faster than fewer warps with deeper rings).
+__global__ void __launch_bounds__(kThreads, 1)
+quantize_kernel(const __grid_constant__ CUtensorMap tm_w, const float *__restrict__ w, int64_t G,
+                const uint8_t *__restrict__ bits, uint8_t *__restrict__ codes, uint16_t *__restrict__ scale,
                 uint8_t *__restrict__ zero, uint32_t *__restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint8_t *ring = smem + warp * kStages * kTileBytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kWarps * kStages * kTileBytes) + warp * kStages;
+  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + kWarps * kStages * kTileBytes +
+                                                                        kWarps * kStages * 8);
+  if (lane == 0) {
+    for (int i = 0; i < kStages; ++i) mbar_init(bars + i, 1);
+    mbar_init_fence();
+  }
+  if (threadIdx.x == 0) *abort_flag = 0u;
+  __syncthreads();
+
   uint32_t flags = 0;
-  const int64_t step = static_cast<int64_t>(gridDim.x) * kThreads;
-  // warp-uniform trip count (the exact path below votes across the warp)
-  const int64_t warp_first = static_cast<int64_t>(blockIdx.x) * kThreads + (threadIdx.x & ~31);
-  for (int64_t g0 = warp_first; g0 < G; g0 += step) {
-    const int64_t g = g0 + (threadIdx.x & 31);
+  const int64_t n_tiles = (G + kTileGroups - 1) / kTileGroups;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarps;
+  const int64_t t_first = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+  auto issue = [&](int slot, int64_t tile) {
+    uint64_t *bar = bars + slot;
+    uint8_t *dst = ring + slot * kTileBytes;
+    mbar_arrive_expect_tx(bar, kTileBytes);
+    tma_load_2d(dst, &tm_w, 0, static_cast<int>(tile * kTileGroups), bar);
+    tma_load_2d(dst + kBoxBytes, &tm_w, 32, static_cast<int>(tile * kTileGroups), bar);
+  };
+  int n_issued = 0, n_done = 0;
+  if (lane == 0)
+    for (int64_t t = t_first; n_issued < kStages && t < n_tiles; t += stride, ++n_issued) issue(n_issued, t);
+  n_issued = __shfl_sync(0xffffffffu, n_issued, 0);
+  int slot = 0;
+  uint32_t phase = 0;
+  for (int64_t tile = t_first; tile < n_tiles; tile += stride) {
+    const bool got = mbar_wait(bars + slot, phase, abort_flag, nullptr);
+    if (!__all_sync(0xffffffffu, got)) {
+      flags |= CQ_QSTATUS_TIMEOUT;
+      break;
+    }
+    const int64_t g = tile * kTileGroups + lane;
     const bool valid = g < G;
     float v[64];
-    const float4 *p = reinterpret_cast<const float4 *>(w + (valid ? g : 0) * kGroup);
+    const uint8_t *row = ring + slot * kTileBytes + lane * 128;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float4 t = __ldg(p + i);
-      v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float4 t4 = *reinterpret_cast<const float4 *>(row + h * kBoxBytes + ((c ^ (lane & 7)) << 4));
+        v[32 * h + 4 * c] = t4.x; v[32 * h + 4 * c + 1] = t4.y; v[32 * h + 4 * c + 2] = t4.z; v[32 * h + 4 * c + 3] = t4.w;
+      }
     }
     // NaN-propagating min/max: a NaN or an infinity shows up as a non-finite extreme
     float lo = v[0], hi = v[0];
@@ -43,6 +87,17 @@ quantize_kernel(const float *__restrict__ w, int64_t G, const uint8_t *__restric
       asm("min.NaN.f32 %0, %0, %1;\n" : "+f"(lo) : "f"(v[j]));
       asm("max.NaN.f32 %0, %0, %1;\n" : "+f"(hi) : "f"(v[j]));
     }
+    // every lane's words of this slot are in registers (min/max consumed them): refill it
+    __syncwarp();
+    ++n_done;
+    {
+      const int64_t next = tile + static_cast<int64_t>(kStages) * stride;
+      if (next < n_tiles) {
+        if (lane == 0) issue(slot, next);
+        ++n_issued;
+      }
+    }
+    if (++slot == kStages) { slot = 0; phase ^= 1u; }
     const bool finite = isfinite(lo) && isfinite(hi);
     const int b = (bits && valid) ? static_cast<int>(__ldg(bits + g)) : 4;
     const bool width_good = width_ok(b);
@@ -59,40 +114,50 @@ quantize_kernel(const float *__restrict__ w, int64_t G, const uint8_t *__restric
     }
     const float rc = __frcp_rn(sf);
     const int z = clamp_code(rne_quotient(-lo, sf, rc), L);
-    // t_j = rne(RN32(w_j / s)) through the division-free filter: with qt = RN32(w_j * rc),
-    // |RN32(w_j / s) - qt| < |qt| * 2^-21, so |qt - rint(qt)| + |qt| * 2^-20 < 0.4999 decides
-    // the rounding; the rest (near a half-way point, huge, non-finite) is redone with the
-    // IEEE division in a branch of its own
-    uint64_t need_exact = 0;
+    // t_j = rne(RN32(w_j / s)) through a division-free certificate. With rc = RN(1/s) and
+    // qt = RN32(w_j * rc): qt = (w/s)(1 + d1)(1 + d2) and RN32(w/s) = (w/s)(1 + d3), |d_i| <= 2^-24,
+    // so |RN32(w_j / s) - qt| <= 1.5 * 2^-23 |w/s| < 2^-22 |qt|. If RN(|qt| 2^-22 + |qt - t|) is
+    // below 0.5 - 2^-20 (t = rint(qt); qt - t is exact), RN32(w_j / s) is within 0.5 of t and
+    // rounds to it. Otherwise (near a half-way point, huge, non-finite: ~1e-5 of the weights) the
+    // thread redoes its whole group with the IEEE division.
+    bool need_exact = false;
 #pragma unroll
-    for (int j = 0; j < 64; ++j) {
-      const float qt = __fmul_rn(v[j], rc);
-      const float t = rintf(qt);
-      need_exact |= static_cast<uint64_t>(!(__fmaf_rn(fabsf(qt), 0x1p-20f, fabsf(__fsub_rn(qt, t))) < 0.4999f)) << j;
-      v[j] = t;                                 // v now holds the rounded quotients
+    for (int j = 0; j < 64; j += 2) {
+      const float2 qt = __fmul2_rn(make_float2(v[j], v[j + 1]), make_float2(rc, rc));
+      const float2 t = make_float2(rintf(qt.x), rintf(qt.y));
+      const float2 d = __fadd2_rn(qt, make_float2(-t.x, -t.y));
+      const float2 m = __ffma2_rn(make_float2(fabsf(qt.x), fabsf(qt.y)), make_float2(0x1p-22f, 0x1p-22f),
+                                  make_float2(fabsf(d.x), fabsf(d.y)));
+      need_exact |= !(m.x < 0.5f - 0x1p-20f) || !(m.y < 0.5f - 0x1p-20f);
+      v[j] = t.x;                               // v now holds the rounded quotients
+      v[j + 1] = t.y;
     }
-    if (__any_sync(0xffffffffu, need_exact != 0)) {
-      // rare: re-read the weights and divide
-#pragma unroll 1
-      for (int j = 0; j < 64; ++j)
-        if ((need_exact >> j) & 1u) v[j] = rintf(__fdiv_rn(__ldg(w + (valid ? g : 0) * kGroup + j), sf));
+    if (__any_sync(0xffffffffu, need_exact)) {
+      // rare: re-read the group and divide every weight
+      if (need_exact) {
+        const float *wg = w + (valid ? g : 0) * kGroup;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) v[j] = rintf(__fdiv_rn(__ldg(wg + j), sf));   // unrolled: v stays in registers
+      }
     }
     const bool bad = !width_good || !finite || overflow;
     if (valid) {
       if (bad) flags |= !width_good ? CQ_QSTATUS_BADBITS : (!finite ? CQ_QSTATUS_NONFINITE : CQ_QSTATUS_RANGE);
-      const float zf = static_cast<float>(z), Lf = static_cast<float>(L);
+      // clamp(t + z, 0, L) in the float domain, offset by 2^23 so the integer sits in the low
+      // mantissa bits: t + (2^23 + z) is exact whenever the clamp does not bind, and when it
+      // does the rounded sum is still on the same side of the clamp interval
+      const float kb = 8388608.0f + static_cast<float>(z), kl = 8388608.0f + static_cast<float>(L);
       uint4 *dst = reinterpret_cast<uint4 *>(codes + g * kGroup);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t wd[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          uint32_t word = 0;
+          uint32_t e4[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float q = fminf(fmaxf(__fadd_rn(v[16 * c + 4 * k + e], zf), 0.0f), Lf);
-            word |= static_cast<uint32_t>(static_cast<int>(q)) << (8 * e);
-          }
+          for (int e = 0; e < 4; ++e)
+            e4[e] = __float_as_uint(fminf(fmaxf(__fadd_rn(v[16 * c + 4 * k + e], kb), 8388608.0f), kl));
+          const uint32_t word = __byte_perm(__byte_perm(e4[0], e4[1], 0x0040), __byte_perm(e4[2], e4[3], 0x0040), 0x5410);
           wd[k] = bad ? 0u : word;
         }
         __stcs(dst + c, make_uint4(wd[0], wd[1], wd[2], wd[3]));
@@ -101,8 +166,13 @@ quantize_kernel(const float *__restrict__ w, int64_t G, const uint8_t *__restric
       zero[g] = bad ? 0 : static_cast<uint8_t>(z);
     }
   }
+  // a warp that gave up lets the copies it issued land before the CTA exits
+  for (; n_done < n_issued; ++n_done) {
+    mbar_wait(bars + slot, phase, abort_flag, nullptr, false);
+    if (++slot == kStages) { slot = 0; phase ^= 1u; }
+  }
   flags = __reduce_or_sync(0xffffffffu, flags);
-  if ((threadIdx.x & 31) == 0 && flags && status) atomicOr(status, flags);
+  if (lane == 0 && flags && status) atomicOr(status, flags);
 }
 
 }  // namespace
@@ -114,10 +184,26 @@ cq_status launch_quantize(const float *w, int64_t G, const uint8_t *bits, uint8_
     if (st != CQ_OK) return st;
   }
   if (G == 0) return CQ_OK;
-  const int64_t need = (G + kThreads - 1) / kThreads;
-  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  auto encode = encode_fn();
+  if (!encode) return fail(CQ_ERR_CUDA, "cq_quantize: cuTensorMapEncodeTiled unavailable");
+  if (G > (int64_t(1) << 31) - kTileGroups) return fail(CQ_ERR_RANGE, "cq_quantize: more than 2^31 groups");
+  CUtensorMap tm;
+  cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(G)};
+  cuuint64_t strides[1] = {64 * sizeof(float)};
+  cuuint32_t box[2] = {32, kTileGroups};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = encode(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(w), dims, strides, box, es,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CQ_ERR_CUDA, "cq_quantize: weight tensor map (%d)", static_cast<int>(r));
+  cq_status st = cuda_check(cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem),
+                            "cq_quantize: shared memory attribute");
+  if (st != CQ_OK) return st;
+  const int64_t tiles = (G + kTileGroups - 1) / kTileGroups;
+  const int64_t need = (tiles + kWarps - 1) / kWarps;
+  const int64_t cap = sm_count();
   const int blocks = static_cast<int>(need < cap ? need : cap);
-  quantize_kernel<<<blocks, kThreads, 0, s>>>(w, G, bits, codes, scale, zero, status);
+  quantize_kernel<<<blocks, kThreads, kSmem, s>>>(tm, w, G, bits, codes, scale, zero, status);
   return launch_check("cq_quantize");
 }
 

@@ -67,6 +67,7 @@ typedef enum { CQ_F32 = 0, CQ_BF16 = 1 } cq_dtype;
 #define CQ_QSTATUS_NONFINITE 1u /* a group held a NaN or infinity: written as s=+0, z=0, q=0 */
 #define CQ_QSTATUS_RANGE 2u     /* a group's scale overflowed fp16: written as s=+0, z=0, q=0 */
 #define CQ_QSTATUS_BADBITS 4u   /* bits[g] not in {1,2,4,8}: written as s=+0, z=0, q=0        */
+#define CQ_QSTATUS_TIMEOUT 8u   /* an internal wait gave up (never expected): outputs incomplete */
 
 /*
  * A quantized weight matrix ([VBQ] bit-packed per-group widths, [CF] frozen codes + scales).
