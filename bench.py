@@ -292,7 +292,60 @@ def isolated_components(torch, cq, ops, device, peaks, stream):
     out["l2_bytes"] = L2
     del g, layers
     torch.cuda.empty_cache()
+    out["cellfill_stack"] = cellfill_stack_verify(torch, cq, ops, synth_module(), device, peaks, stream)
     return out
+
+
+def synth_module():
+    from cell_updates_b200 import synth
+    return synth
+
+
+def cellfill_stack_verify(torch, cq, ops, synth, device, peaks, stream):
+    """The CellFill configuration at its own size: a 28-layer 1.7B-shaped stack
+    (1,526,726,656 weights, frozen 4-bit codes, bf16 residuals ~N(0,(0.3 s)^2)) built on the
+    device by the counter-based generator; project, verify with the residual, verify without it
+    (revocation), each over the whole stack in one call. Rates in weights/s and GB/s."""
+    n = 28 * (4 * 2048 * 2048 + 2 * 2048 * 6144 + 6144 * 2048)
+    G = n // GROUP
+    plane = torch.empty(n // 2, dtype=torch.uint8, device=device)
+    scale = torch.empty(G, dtype=torch.int16, device=device)
+    zero = torch.empty(G, dtype=torch.uint8, device=device)
+    r = torch.empty(n, dtype=torch.bfloat16, device=device)
+    with torch.cuda.stream(stream):
+        cq.cqs_code_words(plane.view(torch.int64), 3, 0, stream)
+        cq.cqs_scales(scale, 3, 0, stream)
+        cq.cqs_zeros(zero, 3, 0, stream)
+        cq.cqs_residual_bf16(r, scale, 3, 0, float(synth.ih4_multiplier(0.3)), stream)
+    torch.cuda.synchronize()
+    ncl = torch.zeros(1, dtype=torch.int64, device=device)
+    mism = torch.zeros(1, dtype=torch.int64, device=device)
+    first = torch.zeros(1, dtype=torch.int64, device=device)
+    qw_r = cq.QWeight(1, n, [None, None, plane, None], scale, zero, residual=r)
+    qw_0 = cq.QWeight(1, n, [None, None, plane, None], scale, zero)
+    res = {"weights": n}
+    calls = {"project": lambda: cq.cq_project_residual(r, scale, ncl, stream),
+             "verify": lambda: cq.cq_requant_verify(qw_r, 0, n, mism, first, None, stream),
+             "revoke_verify": lambda: cq.cq_requant_verify(qw_0, 0, n, mism, first, None, stream)}
+    per_w = {"project": 4.0 + 2.0 / GROUP, "verify": 2.5 + 3.0 / GROUP, "revoke_verify": 0.5 + 3.0 / GROUP}
+    for name, fn in calls.items():
+        with torch.cuda.stream(stream):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+        g.replay()
+        ms = time_graph(torch, g, 10, stream)
+        if name != "project":
+            assert int(mism.item()) == 0, f"{name}: {int(mism.item())} mismatches"
+        res[name] = {"ms": ms, "weights_per_s": n / (ms * 1e-3), "GBps": n * per_w[name] / (ms * 1e-3) / 1e9,
+                     "frac_hbm": n * per_w[name] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        del g
+    del plane, scale, zero, r, qw_r, qw_0
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_gpu(args, rank, world, local_rank):
@@ -405,6 +458,7 @@ def run_gpu(args, rank, world, local_rank):
         if iso:
             line["isolated"] = iso
             line["tokens_per_s"] = iso["decode_32_layers"]["tokens_per_s"]
+            line["requant_verify_weights_per_s_cellfill_stack"] = iso["cellfill_stack"]["verify"]["weights_per_s"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_sample_rows)
     if dist:

@@ -290,6 +290,80 @@ __global__ void __launch_bounds__(kThreads) verify4_kernel(VerifyArgs a) {
   if (first != INT64_MAX) atomicMin(a.first_bad, static_cast<unsigned long long>(first));
 }
 
+// Revocation (no residual) of fixed-4 weights moves only 0.55 bytes per weight, so a lane
+// keeps four 32-weight units in flight: a warp reads 4 x 512 contiguous bytes of codes (plus
+// their scales and zeros) before it computes, and the grid needs 4x fewer warps for the same
+// bytes in flight. The certificate is that of verify4_kernel without a residual.
+constexpr int kRevokeUnroll = 4;
+
+__global__ void __launch_bounds__(kThreads) revoke4_kernel(VerifyArgs a) {
+  const int lane = threadIdx.x & 31;
+  uint32_t count = 0;
+  int64_t first = INT64_MAX;
+  const int64_t n32 = a.n_units >> 2;            // units of 32 weights
+  const int64_t warp_id = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
+  const int64_t step = static_cast<int64_t>(gridDim.x) * (kThreads / 32) * 32 * kRevokeUnroll;
+  for (int64_t base = warp_id * 32 * kRevokeUnroll; base < n32; base += step) {
+    uint4 cw[kRevokeUnroll];
+    uint32_t sbits[kRevokeUnroll], zv[kRevokeUnroll];
+#pragma unroll
+    for (int k = 0; k < kRevokeUnroll; ++k) {
+      const int64_t u = base + 32 * k + lane;
+      cw[k] = make_uint4(0, 0, 0, 0);
+      sbits[k] = 0x3C00u;                        // 1.0 for lanes past the end (never counted)
+      zv[k] = 0;
+      if (u < n32) {
+        const int64_t i0 = a.first_w + 32 * u;
+        cw[k] = __ldcs(reinterpret_cast<const uint4 *>(a.plane[2] + (i0 >> 1)));
+        sbits[k] = __ldg(a.scale + (i0 >> 6));
+        zv[k] = __ldg(a.zero + (i0 >> 6));
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kRevokeUnroll; ++k) {
+      const int64_t u = base + 32 * k + lane;
+      const bool valid = u < n32;
+      const int64_t i0 = a.first_w + 32 * u;
+      const int64_t g = i0 >> 6;
+      const float sf = f16_bits_to_f32(static_cast<uint16_t>(sbits[k]));
+      const int z = static_cast<int>(zv[k]);
+      const float rc = __frcp_rn(sf);
+      // |RN32(s*k * rc) - k| <= |k| * |s * rc - 1| (1 + 2^-24), |k| <= max(qor - z, z)
+      uint32_t qor = cw[k].x | cw[k].y | cw[k].z | cw[k].w;
+      qor = (qor | (qor >> 4)) & 0x0F0F0F0Fu;
+      qor |= qor >> 16;
+      qor = (qor | (qor >> 8)) & 0xFu;
+      const float kmax = static_cast<float>(max(static_cast<int>(qor) - z, z));
+      const float eps = fabsf(__fmaf_rn(sf, rc, -1.0f));
+      const float m = __fmul_rn(__fmul_rn(kmax, eps), 1.0f + 0x1p-22f);   // NaN when s is 0, inf or NaN
+      uint32_t bad = 0;
+      if (valid && !(m < 0.49951171875f)) {
+        // the exact definition, weight by weight (rare path)
+#pragma unroll 1
+        for (int j = 0; j < 32; ++j) {
+          const int64_t i = i0 + j;
+          const int q = static_cast<int>((__ldg(a.plane[2] + (i >> 1)) >> (4 * (i & 1))) & 0xFu);
+          if (!exact_match<false>(q, z, 15, sf, 0.0f)) bad |= 1u << j;
+        }
+      }
+      if (__ballot_sync(0xffffffffu, bad != 0)) {
+        count += __popc(bad);
+        if (bad) {
+          const int64_t fi = i0 + (__ffs(bad) - 1);
+          first = fi < first ? fi : first;
+        }
+        if (a.flags && bad) {
+          const int64_t gl = g - (a.first_w >> 6);
+          atomicOr(a.flags + (gl >> 5), 1u << (gl & 31));
+        }
+      }
+    }
+  }
+  count = __reduce_add_sync(0xffffffffu, count);
+  if (lane == 0 && count) atomicAdd(a.mism, static_cast<unsigned long long>(count));
+  if (first != INT64_MAX) atomicMin(a.first_bad, static_cast<unsigned long long>(first));
+}
+
 template <bool VAR>
 void dispatch(int rk, VerifyArgs a, int blocks, cudaStream_t s) {
   switch (rk) {
@@ -301,7 +375,7 @@ void dispatch(int rk, VerifyArgs a, int blocks, cudaStream_t s) {
 
 void dispatch4(int rk, VerifyArgs a, int blocks, cudaStream_t s) {
   switch (rk) {
-    case kNoR: verify4_kernel<kNoR><<<blocks, kThreads, 0, s>>>(a); break;
+    case kNoR: revoke4_kernel<<<(blocks + kRevokeUnroll - 1) / kRevokeUnroll, kThreads, 0, s>>>(a); break;
     case kF32: verify4_kernel<kF32><<<blocks, kThreads, 0, s>>>(a); break;
     default: verify4_kernel<kBF16><<<blocks, kThreads, 0, s>>>(a); break;
   }
