@@ -31,7 +31,6 @@ sys.path.insert(0, ROOT)
 
 GROUP = 64
 SHAPES = [(4096, 4096), (11008, 4096), (4096, 11008)]       # rows (out) x cols (in)
-LAYER_MIX = [4, 2, 1]       # per layer of a 7B-shaped decoder: q,k,v,o | gate,up | down
 N_LAYERS = 32
 GEMM_M = 64
 METRIC = "dequant-GEMV weight GB/s & tokens/s vs HBM peak; requant-verify weights/s"
@@ -243,37 +242,55 @@ def isolated_components(torch, cq, ops, device, peaks, stream):
     """Cold-L2 component rates: GEMV (rotating > 2x L2), the 32-layer decode proxy, verify."""
     out = {}
     L2 = torch.cuda.get_device_properties(device).L2_cache_size
-    # 32-layer 7B-shaped decode: distinct weights per layer (3.54 GB), one graph per token
+    # 32-layer 7B-shaped decode: distinct weights per layer (3.54 GB), one graph per token. Per
+    # layer: q, k, v (4096x4096, one fused launch: they read the same x), o, gate and up
+    # (11008x4096, one fused launch), down (4096x11008); the unfused variant launches all seven.
     base = []
     for (N, K) in SHAPES:
         w = torch.randn(N, K, device=device) * 0.02
         qw, _, _ = ops.quantize_and_pack(w)
         base.append(qw)
         del w
-    layers = []
-    for l in range(N_LAYERS):
-        for qw, mult in zip(base, LAYER_MIX):
-            for _ in range(mult):
-                layers.append(cq.QWeight(qw.rows, qw.cols, [None, None, qw.planes[2].clone(), None],
-                                         qw.scale.clone(), qw.zero.clone()))
+
+    def clone(q):
+        return cq.QWeight(q.rows, q.cols, [None, None, q.planes[2].clone(), None], q.scale.clone(), q.zero.clone())
+
+    stack = [{"qkv": [clone(base[0]) for _ in range(3)], "o": clone(base[0]),
+              "gu": [clone(base[1]) for _ in range(2)], "down": clone(base[2])} for _ in range(N_LAYERS)]
+    layers = [q for L in stack for q in L["qkv"] + [L["o"]] + L["gu"] + [L["down"]]]
     xs = {K: torch.randn(1, K, device=device).to(torch.bfloat16) for (_, K) in SHAPES}
     ys = {N: torch.empty(1, N, device=device) for (N, _) in SHAPES}
+    y4 = [torch.empty(1, 4096, device=device) for _ in range(3)]
+    y11 = [torch.empty(1, 11008, device=device) for _ in range(2)]
     token_bytes = sum(q.rows * q.cols // 2 + 3 * q.rows * q.cols // GROUP for q in layers)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        for q in layers:     # warm-up outside capture
-            cq.cq_dequant_gemv(q, xs[q.cols], ys[q.rows], stream)
-        torch.cuda.synchronize()
-        with torch.cuda.graph(g, stream=stream):
-            for q in layers:
-                cq.cq_dequant_gemv(q, xs[q.cols], ys[q.rows], stream)
-    for _ in range(3):
-        g.replay()
-    t_ms = time_graph(torch, g, 20, stream)
-    out["decode_32_layers"] = {"tokens_per_s": 1e3 / t_ms, "ms_per_token": t_ms, "weight_bytes_per_token": token_bytes,
-                               "GBps": token_bytes / t_ms / 1e6, "frac_hbm": token_bytes / t_ms / 1e6 / peaks["hbm_gbs"],
-                               "ceiling_tokens_per_s": peaks["hbm_gbs"] * 1e9 / token_bytes,
-                               "launches_per_token": len(layers)}
+
+    def token(fused):
+        for L in stack:
+            if fused:
+                cq.cq_dequant_gemv_multi(L["qkv"], xs[4096], y4, stream)
+                cq.cq_dequant_gemv(L["o"], xs[4096], y4[0], stream)
+                cq.cq_dequant_gemv_multi(L["gu"], xs[4096], y11, stream)
+                cq.cq_dequant_gemv(L["down"], xs[11008], y4[1], stream)
+            else:
+                for q in L["qkv"] + [L["o"]] + L["gu"] + [L["down"]]:
+                    cq.cq_dequant_gemv(q, xs[q.cols], ys[q.rows], stream)
+
+    for fused in (True, False):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            token(fused)     # warm-up outside capture
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                token(fused)
+        for _ in range(3):
+            g.replay()
+        t_ms = time_graph(torch, g, 20, stream)
+        key = "decode_32_layers" if fused else "decode_32_layers_unfused"
+        out[key] = {"tokens_per_s": 1e3 / t_ms, "ms_per_token": t_ms, "weight_bytes_per_token": token_bytes,
+                    "GBps": token_bytes / t_ms / 1e6, "frac_hbm": token_bytes / t_ms / 1e6 / peaks["hbm_gbs"],
+                    "ceiling_tokens_per_s": peaks["hbm_gbs"] * 1e9 / token_bytes,
+                    "launches_per_token": N_LAYERS * (4 if fused else 7)}
+        del g
     # per shape, the same pool (rotation over 32 copies > 2 x L2)
     per = {}
     for si, (N, K) in enumerate(SHAPES):
@@ -290,7 +307,7 @@ def isolated_components(torch, cq, ops, device, peaks, stream):
         del g1
     out["gemv_m1_cold"] = per
     out["l2_bytes"] = L2
-    del g, layers
+    del layers, stack
     torch.cuda.empty_cache()
     out["cellfill_stack"] = cellfill_stack_verify(torch, cq, ops, synth_module(), device, peaks, stream)
     return out

@@ -22,7 +22,7 @@ QSTATUS_NONFINITE, QSTATUS_RANGE, QSTATUS_BADBITS = 1, 2, 4
 
 # every symbol include/cq.h declares
 EXPORTS = ["cq_quantize", "cq_varbits_index", "cq_pack_varbits", "cq_unpack_varbits",
-           "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemm",
+           "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemv_multi", "cq_dequant_gemm",
            "cq_dequant_gemm_static", "cq_gemm_workspace", "cq_last_error", "cq_status_string"]
 SYNTH_EXPORTS = ["cqs_normal_f32", "cqs_code_words", "cqs_scales", "cqs_zeros", "cqs_residual_bf16"]
 
@@ -58,6 +58,7 @@ def lib():
         L.cq_project_residual.argtypes = [p, i32, p, i64, p, p]
         L.cq_requant_verify.argtypes = [p, i64, i64, p, p, p, p]
         L.cq_dequant_gemv.argtypes = [p, p, i32, i32, p, p]
+        L.cq_dequant_gemv_multi.argtypes = [p, i32, p, i32, i32, p, p]
         L.cq_dequant_gemm.argtypes = [p, p, i32, i32, p, p, C.c_size_t, p]
         L.cq_dequant_gemm_static.argtypes = [p, p, i32, i32, p, p]
         L.cq_gemm_workspace.argtypes = [i64, i64, i32]
@@ -66,8 +67,8 @@ def lib():
         L.cq_status_string.argtypes = [i32]
         L.cq_status_string.restype = C.c_char_p
         for name in ("cq_quantize", "cq_varbits_index", "cq_pack_varbits", "cq_unpack_varbits",
-                     "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemm",
-                     "cq_dequant_gemm_static"):
+                     "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemv_multi",
+                     "cq_dequant_gemm", "cq_dequant_gemm_static"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -185,6 +186,16 @@ def cq_dequant_gemv(qw, x, y, stream=None):
     m = x.shape[0] if x.dim() == 2 else 1
     _check(lib().cq_dequant_gemv(C.byref(s), _ptr(x), _dtype_code(x), m, _ptr(y), _stream(stream)),
            "cq_dequant_gemv")
+
+
+def cq_dequant_gemv_multi(qws, x, ys, stream=None):
+    """Several matrices with the same cols against one x (see include/cq.h)."""
+    structs = [q.struct() for q in qws]
+    arr = (C.POINTER(cq_qweight) * len(structs))(*[C.pointer(st) for st in structs])
+    yarr = (C.c_void_p * len(ys))(*[_ptr(y) for y in ys])
+    m = x.shape[0] if x.dim() == 2 else 1
+    _check(lib().cq_dequant_gemv_multi(C.cast(arr, C.c_void_p), len(structs), _ptr(x), _dtype_code(x), m,
+                                       C.cast(yarr, C.c_void_p), _stream(stream)), "cq_dequant_gemv_multi")
 
 
 def cq_gemm_workspace(rows, cols, m):

@@ -194,6 +194,23 @@ cq_status cq_dequant_gemv(const cq_qweight *qw, const void *x, cq_dtype x_dtype,
   return launch_gemv(*qw, x, x_dtype, m, y, reinterpret_cast<cudaStream_t>(stream));
 }
 
+cq_status cq_dequant_gemv_multi(const cq_qweight *const *qws, int count, const void *x, cq_dtype x_dtype, int m,
+                                float *const *ys, cq_stream_t stream) {
+  const char *fn = "cq_dequant_gemv_multi";
+  if (count < 0) return fail(CQ_ERR_ARG, "%s: negative count", fn);
+  if (count == 0) return CQ_OK;
+  if (!qws || !ys) return fail(CQ_ERR_ARG, "%s: NULL matrix or output list", fn);
+  for (int i = 0; i < count; ++i) {
+    if (!qws[i]) return fail(CQ_ERR_ARG, "%s: matrix %d is NULL", fn, i);
+    cq_status st = check_matmul(qws[i], x, x_dtype, m, ys[i], 8, fn);
+    if (st != CQ_OK) return st;
+    if (qws[i]->cols != qws[0]->cols)
+      return fail(CQ_ERR_SHAPE, "%s: matrix %d has %lld cols, matrix 0 has %lld", fn, i,
+                  (long long)qws[i]->cols, (long long)qws[0]->cols);
+  }
+  return launch_gemv_multi(qws, count, x, x_dtype, m, ys, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t cq_gemm_workspace(int64_t rows, int64_t cols, int m) {
   if (rows <= 0 || cols <= 0 || m < 16) return 0;
   return gemm_tc_workspace(rows, cols, m);

@@ -35,6 +35,8 @@ cq_status launch_verify(const cq_qweight &qw, int64_t first_w, int64_t n_w, uint
                         int64_t *first_bad, uint32_t *flags, cudaStream_t s);
 cq_status launch_gemv(const cq_qweight &qw, const void *x, cq_dtype xdt, int m, float *y,
                       cudaStream_t s);
+cq_status launch_gemv_multi(const cq_qweight *const *qws, int count, const void *x, cq_dtype xdt, int m,
+                            float *const *ys, cudaStream_t s);
 cq_status launch_gemm_tc(const cq_qweight &qw, const void *x, int m, float *y, void *ws,
                          size_t ws_bytes, cudaStream_t s);
 size_t gemm_tc_workspace(int64_t rows, int64_t cols, int m);

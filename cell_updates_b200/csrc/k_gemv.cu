@@ -158,17 +158,39 @@ __device__ __forceinline__ void advance(Cursor &cu, int n_chunks) {
   }
 }
 
+// Matrices that share the activations (q, k and v of a decoder layer; gate and up) run as
+// one launch: their 16-row tiles are numbered one after the other (segment s owns the tiles
+// tile0[s] .. tile0[s+1]-1) and every CTA deals with the concatenated sequence.
+constexpr int kMaxSegs = 4;
+struct GemvSegs {
+  CUtensorMap tm[kMaxSegs];                 // the code plane of each matrix
+  const uint16_t *scale[kMaxSegs];
+  const uint8_t *zero[kMaxSegs];
+  float *y[kMaxSegs];
+  int64_t rows[kMaxSegs];
+  int64_t tile0[kMaxSegs + 1];              // tile0[count] = all tiles; unused entries = INT64_MAX
+};
+
+__device__ __forceinline__ int seg_of(const GemvSegs &sg, int64_t tile) {
+  return (tile >= sg.tile0[1]) + (tile >= sg.tile0[2]) + (tile >= sg.tile0[3]);
+}
+__device__ __forceinline__ const CUtensorMap *seg_map(const GemvSegs &sg, int s) {
+  return s == 0 ? &sg.tm[0] : s == 1 ? &sg.tm[1] : s == 2 ? &sg.tm[2] : &sg.tm[3];
+}
+template <typename T, int kN>
+__device__ __forceinline__ T seg_pick(const T (&a)[kN], int s) {
+  return s == 0 ? a[0] : s == 1 ? a[1] : s == 2 ? a[2] : a[3];
+}
+
 template <bool FULL, bool XS>
 __global__ void __launch_bounds__(kGemvThreads, 1)
-gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__restrict__ scale,
-             const uint8_t *__restrict__ zero, const __nv_bfloat16 *__restrict__ x, int m, int64_t N,
-             int64_t K, float *__restrict__ y) {
+gemv4_kernel(const __grid_constant__ GemvSegs segs, const __nv_bfloat16 *__restrict__ x, int m, int64_t K) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   pdl_launch_dependents();
   const int KG = static_cast<int>(K >> 6);
   const int n_chunks = (KG + kCG - 1) / kCG;
-  const int64_t n_tiles = (N + kTileRows - 1) / kTileRows;
+  const int64_t n_tiles = segs.tile0[kMaxSegs];
   const int n_local = static_cast<int>((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gid = lane >> 2, tig = lane & 3;
@@ -204,17 +226,21 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
   Cursor prod = {0, warp};       // chunk number `warp` of the stream may lie beyond the first tile
   while (prod.c >= n_chunks) { prod.c -= n_chunks; ++prod.lt; }
   int prod_lt = -1, prod_y = 0;
-  const uint16_t *ps = scale;
-  const uint8_t *pz = zero;
+  const uint16_t *ps = segs.scale[0];
+  const uint8_t *pz = segs.zero[0];
+  const CUtensorMap *ptm = &segs.tm[0];
   auto issue = [&](int slot) {
     if (prod.lt != prod_lt) {
       prod_lt = prod.lt;
       const int64_t tile = blockIdx.x + static_cast<int64_t>(prod_lt) * gridDim.x;
-      int64_t row = tile * kTileRows + prow;
-      row = row < N ? row : N - 1;
-      ps = scale + row * KG + phalf * 4;
-      pz = zero + row * KG + phalf * 4;
-      prod_y = static_cast<int>(tile * kTileRows);
+      const int sg = seg_of(segs, tile);
+      const int64_t lrow0 = (tile - seg_pick(segs.tile0, sg)) * kTileRows, nrows = seg_pick(segs.rows, sg);
+      int64_t row = lrow0 + prow;
+      row = row < nrows ? row : nrows - 1;
+      ps = seg_pick(segs.scale, sg) + row * KG + phalf * 4;
+      pz = seg_pick(segs.zero, sg) + row * KG + phalf * 4;
+      ptm = seg_map(segs, sg);
+      prod_y = static_cast<int>(lrow0);
     }
     uint64_t *bar = bars + slot;
     const int g0 = prod.c * kCG;
@@ -229,8 +255,8 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
     if (lane == 0) {
       uint8_t *dst = ring + slot * kChunkBytes;
       mbar_arrive_expect_tx(bar, second ? kChunkBytes : kBoxBytes);
-      tma_load_2d(dst, &tm_codes, prod.c * 256, prod_y, bar);
-      if (second) tma_load_2d(dst + kBoxBytes, &tm_codes, prod.c * 256 + 128, prod_y, bar);
+      tma_load_2d(dst, ptm, prod.c * 256, prod_y, bar);
+      if (second) tma_load_2d(dst + kBoxBytes, ptm, prod.c * 256 + 128, prod_y, bar);
     }
   };
   int n_issued = 0;
@@ -394,6 +420,9 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
     if (old + 1 != static_cast<uint32_t>(arrivals)) return;
     // last arrival: lane l sums outputs l, l + 32, ... (col * 16 + row) over the warps, in warp order
     const int64_t tile = blockIdx.x + static_cast<int64_t>(lt) * gridDim.x;
+    const int sg = seg_of(segs, tile);
+    const int64_t lrow0 = (tile - seg_pick(segs.tile0, sg)) * kTileRows, N = seg_pick(segs.rows, sg);
+    float *y = seg_pick(segs.y, sg);
     const bool bad = *abort_flag != 0u;
     for (int idx = lane; idx < 16 * m; idx += 32) {
       float v = 0.0f;
@@ -403,7 +432,7 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
         rs[w * (kTileRows * 8) + idx] = 0.0f;
       }
       const int row = idx & 15, col = idx >> 4;
-      const int64_t r = tile * kTileRows + row;
+      const int64_t r = lrow0 + row;
       if (r < N) y[static_cast<int64_t>(col) * N + r] = bad ? __int_as_float(0x7fc00000) : v;
     }
     __threadfence_block();
@@ -443,6 +472,8 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
     uint4 sv0 = make_uint4(0, 0, 0, 0), sv1 = sv0;
     uint2 zv0 = make_uint2(0, 0), zv1 = zv0;
     int64_t r0 = 0, r1 = 0;
+    const uint16_t *scale = segs.scale[0];
+    const uint8_t *zero = segs.zero[0];
     if (FULL) {
       const uint8_t *ms = meta + slot * kMetaBytes;
       sv0 = *reinterpret_cast<const uint4 *>(ms + rho * 16);
@@ -451,7 +482,11 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
       zv1 = *reinterpret_cast<const uint2 *>(ms + 256 + (rho + 8) * 8);
     } else {
       const int64_t tile = blockIdx.x + static_cast<int64_t>(cons.lt) * gridDim.x;
-      r0 = tile * kTileRows + rho;
+      const int sg = seg_of(segs, tile);
+      const int64_t N = seg_pick(segs.rows, sg);
+      scale = seg_pick(segs.scale, sg);
+      zero = seg_pick(segs.zero, sg);
+      r0 = (tile - seg_pick(segs.tile0, sg)) * kTileRows + rho;
       r1 = r0 + 8;
       r0 = r0 < N ? r0 : N - 1;
       r1 = r1 < N ? r1 : N - 1;
@@ -563,15 +598,12 @@ gemv4_kernel(const __grid_constant__ CUtensorMap tm_codes, const uint16_t *__res
 }
 
 template <bool FULL, bool XS>
-cq_status launch_gemv4(const cq_qweight &qw, const void *x, int m, float *y, cudaStream_t s) {
-  CUtensorMap tm;
-  cq_status st = code_tensor_map(&tm, qw.plane[2], qw.rows, qw.cols, kTileRows, "cq_dequant_gemv");
+cq_status launch_gemv4(const GemvSegs &segs, const void *x, int m, int64_t K, cudaStream_t s) {
+  const int smem = static_cast<int>(gemv_smem(m, K, XS));
+  cq_status st = cuda_check(cudaFuncSetAttribute(gemv4_kernel<FULL, XS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 smem), "cq_dequant_gemv: shared memory attribute");
   if (st != CQ_OK) return st;
-  const int smem = static_cast<int>(gemv_smem(m, qw.cols, XS));
-  st = cuda_check(cudaFuncSetAttribute(gemv4_kernel<FULL, XS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
-                  "cq_dequant_gemv: shared memory attribute");
-  if (st != CQ_OK) return st;
-  const int64_t tiles = (qw.rows + kTileRows - 1) / kTileRows;
+  const int64_t tiles = segs.tile0[kMaxSegs];
   const int64_t grid = tiles < sm_count() ? tiles : sm_count();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -583,9 +615,42 @@ cq_status launch_gemv4(const cq_qweight &qw, const void *x, int m, float *y, cud
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_check(cudaLaunchKernelEx(&cfg, gemv4_kernel<FULL, XS>, tm, qw.scale, qw.zero,
-                                       static_cast<const __nv_bfloat16 *>(x), m, qw.rows, qw.cols, y),
+  return cuda_check(cudaLaunchKernelEx(&cfg, gemv4_kernel<FULL, XS>, segs, static_cast<const __nv_bfloat16 *>(x), m, K),
                     "cq_dequant_gemv");
+}
+
+// the tensor-core path for up to kMaxSegs fixed-4 matrices with the same cols and bf16 x
+cq_status launch_gemv4_segs(const cq_qweight *const *qws, int count, const void *x, int m, float *const *ys,
+                            cudaStream_t s) {
+  const int64_t K = qws[0]->cols, KG = K >> 6;
+  GemvSegs segs;
+  memset(&segs, 0, sizeof(segs));
+  bool full = KG % 4 == 0;
+  int64_t t = 0;
+  for (int i = 0; i < kMaxSegs; ++i) {
+    if (i < count) {
+      const cq_qweight &qw = *qws[i];
+      cq_status st = code_tensor_map(&segs.tm[i], qw.plane[2], qw.rows, qw.cols, kTileRows, "cq_dequant_gemv");
+      if (st != CQ_OK) return st;
+      segs.scale[i] = qw.scale;
+      segs.zero[i] = qw.zero;
+      segs.y[i] = ys[i];
+      segs.rows[i] = qw.rows;
+      segs.tile0[i] = t;
+      t += (qw.rows + kTileRows - 1) / kTileRows;
+      // the per-chunk scale (8-byte) and zero (4-byte) copies need aligned rows of whole 4-group runs
+      full = full && aligned8(qw.scale) && (reinterpret_cast<uintptr_t>(qw.zero) & 3u) == 0;
+    } else {
+      segs.tile0[i] = INT64_MAX;
+    }
+  }
+  segs.tile0[kMaxSegs] = t;
+  if (count < kMaxSegs) segs.tile0[count] = t;
+  // activations are staged once per CTA in shared memory when they fit
+  const bool xs = gemv_smem(m, K, true) <= kSmemCap;
+  if (gemv_smem(m, K, false) > kSmemCap) return fail(CQ_ERR_SHAPE, "cq_dequant_gemv: cols too large");
+  if (full) return xs ? launch_gemv4<true, true>(segs, x, m, K, s) : launch_gemv4<true, false>(segs, x, m, K, s);
+  return xs ? launch_gemv4<false, true>(segs, x, m, K, s) : launch_gemv4<false, false>(segs, x, m, K, s);
 }
 
 // ------------------------------------------------------------------------------------
@@ -667,14 +732,8 @@ cq_status launch_gemv(const cq_qweight &qw, const void *x, cq_dtype xdt, int m, 
   if (K == 0) return cuda_check(cudaMemsetAsync(y, 0, sizeof(float) * m * N, s), "cq_dequant_gemv: zero y");
   const bool tc = qw.bits == nullptr && qw.residual == nullptr && xdt == CQ_BF16;
   if (tc) {
-    const int64_t KG = K >> 6;
-    // the per-chunk scale (8-byte) and zero (4-byte) copies need whole chunks of 4 groups
-    const bool full = (KG % 4 == 0) && aligned8(qw.scale) && (reinterpret_cast<uintptr_t>(qw.zero) & 3u) == 0;
-    // activations are staged once per CTA in shared memory when they fit
-    const bool xs = gemv_smem(m, K, true) <= kSmemCap;
-    if (gemv_smem(m, K, false) > kSmemCap) return fail(CQ_ERR_SHAPE, "cq_dequant_gemv: cols too large");
-    if (full) return xs ? launch_gemv4<true, true>(qw, x, m, y, s) : launch_gemv4<true, false>(qw, x, m, y, s);
-    return xs ? launch_gemv4<false, true>(qw, x, m, y, s) : launch_gemv4<false, false>(qw, x, m, y, s);
+    const cq_qweight *one = &qw;
+    return launch_gemv4_segs(&one, 1, x, m, &y, s);
   }
   const int64_t need = (N + 7) / 8;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
@@ -690,6 +749,31 @@ cq_status launch_gemv(const cq_qweight &qw, const void *x, cq_dtype xdt, int m, 
     else launch_generic<false, 2>(qw, x, m, y, blocks, s);
   }
   return launch_check("cq_dequant_gemv");
+}
+
+bool gemv_tc_eligible(const cq_qweight &qw, cq_dtype xdt) {
+  return qw.bits == nullptr && qw.residual == nullptr && xdt == CQ_BF16 && qw.rows > 0 && qw.cols > 0;
+}
+
+cq_status launch_gemv_multi(const cq_qweight *const *qws, int count, const void *x, cq_dtype xdt, int m,
+                            float *const *ys, cudaStream_t s) {
+  // runs of up to kMaxSegs tensor-core-eligible matrices become one launch; anything else goes
+  // through the single-matrix path
+  int i = 0;
+  while (i < count) {
+    if (!gemv_tc_eligible(*qws[i], xdt)) {
+      cq_status st = launch_gemv(*qws[i], x, xdt, m, ys[i], s);
+      if (st != CQ_OK) return st;
+      ++i;
+      continue;
+    }
+    int j = i + 1;
+    while (j < count && j - i < kMaxSegs && gemv_tc_eligible(*qws[j], xdt)) ++j;
+    cq_status st = launch_gemv4_segs(qws + i, j - i, x, m, ys + i, s);
+    if (st != CQ_OK) return st;
+    i = j;
+  }
+  return CQ_OK;
 }
 
 }  // namespace cq

@@ -90,6 +90,12 @@ def gemv(qw, x, stream=None):
     return y
 
 
+def gemv_multi(qws, x, stream=None):
+    ys = [torch.empty((x.shape[0], q.rows), dtype=torch.float32, device=x.device) for q in qws]
+    cq.cq_dequant_gemv_multi(qws, x, ys, stream)
+    return ys
+
+
 def gemm(qw, x, workspace=None, stream=None):
     m = x.shape[0]
     y = torch.empty((m, qw.rows), dtype=torch.float32, device=x.device)

@@ -161,6 +161,21 @@ cq_status cq_dequant_gemv(const cq_qweight *qw, const void *x, cq_dtype x_dtype,
                           float *y, cq_stream_t stream);
 
 /*
+ * cq_dequant_gemv_multi -- cq_dequant_gemv for several matrices that read the same x (the q, k
+ * and v projections of a decoder layer, or its gate and up projections) in as few launches as
+ * possible: consecutive runs of up to four fixed-4 matrices with bf16 x and no residual become
+ * one tensor-core launch whose 16-row tiles cover all of them; any other matrix runs as in
+ * cq_dequant_gemv. qws: count pointers to matrices that all have the same cols; x: [m, cols];
+ * ys[i]: [m, qws[i]->rows] fp32, overwritten. Each output is the same contraction as
+ * cq_dequant_gemv computes (same tolerance; the order of the fp32 partial sums can differ).
+ * Validation is that of cq_dequant_gemv for every matrix, plus CQ_ERR_SHAPE for unequal cols.
+ * The pages have no counterpart to the grouping: it serves decode, where one token runs many
+ * small GEMVs and launch latency rivals the weight stream.
+ */
+cq_status cq_dequant_gemv_multi(const cq_qweight *const *qws, int count, const void *x, cq_dtype x_dtype,
+                                int m, float *const *ys, cq_stream_t stream);
+
+/*
  * cq_dequant_gemm -- the same contraction for a batch, 1 <= m <= 256. Fixed-4 weights with
  * bf16 x, no residual and m >= 16 run on the sm_100a tcgen05 tensor cores with accumulators
  * in tensor memory; m < 16 goes to the GEMV kernels, as do other formats (in slices of 8).

@@ -62,6 +62,15 @@ def test_host_validation_rejects_bad_arguments():
     assert L.cq_dequant_gemv(C.byref(qw), p, 1, 1, p, None) == 1
     assert "offset" in cq.cq_last_error()
     assert L.cq_gemm_workspace(8192, 28672, 8) == 0
+    qw.bits = None
+    other = cq.cq_qweight()
+    other.rows, other.cols, other.scale, other.zero = 4, 128, 16, 16
+    other.plane[2] = 16
+    qws = (C.POINTER(cq.cq_qweight) * 2)(C.pointer(qw), C.pointer(other))
+    ys = (C.c_void_p * 2)(16, 16)
+    assert L.cq_dequant_gemv_multi(C.cast(qws, C.c_void_p), 2, p, 1, 1, C.cast(ys, C.c_void_p), None) == 2  # unequal cols
+    assert L.cq_dequant_gemv_multi(None, 2, p, 1, 1, C.cast(ys, C.c_void_p), None) == 1                    # NULL list
+    assert L.cq_dequant_gemv_multi(None, 0, p, 1, 1, None, None) == 0                                      # nothing to do
 
 
 def test_missing_library_fails_loudly(monkeypatch):

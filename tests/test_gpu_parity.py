@@ -257,6 +257,26 @@ def test_gemv_tensor_core_4bit(rows, cols, m):
     check_matmul(host(ops.gemv(qw, x_d)), y_ref, f"{rows}x{cols} m={m}")
 
 
+# several matrices sharing x in one launch: ragged tiles in every segment, more than four
+# matrices (two launches), and a variable-width matrix in the list (single-matrix path)
+@pytest.mark.parametrize("m", [1, 3, 8])
+def test_gemv_multi_segments(m):
+    cols = 64 * 21
+    specs = [(300, None), (47, None), (64, "vbq"), (1000, None), (16, None), (129, None)]
+    x = synth.activations(m, cols, seed=91 + m, dtype="bf16")
+    qws, refs = [], []
+    for i, (rows, kind) in enumerate(specs):
+        w = synth.normal_weights(rows, cols, seed=70 + i)
+        bits = synth.vbq_bits(rows * cols // 64, seed=80 + i) if kind else None
+        qw, _, _, oc = _quantize_both(w, bits)
+        planes, off = _oracle_qw(oc[0], oc[1], oc[2], bits)
+        qws.append(qw)
+        refs.append(co.dequant_matmul_f64(planes, oc[1], oc[2], rows, cols, x, "bf16", bits, off))
+    ys = ops.gemv_multi(qws, bf16_dev(x))
+    for i, (qw, y_ref) in enumerate(zip(qws, refs)):
+        check_matmul(host(ys[i]), y_ref, f"multi[{i}] {qw.rows}x{qw.cols} m={m}")
+
+
 @pytest.mark.parametrize("m", [1, 8])
 def test_gemv_varbits(m):
     G = 512 * 1024 // 64
