@@ -39,9 +39,9 @@ constexpr int kBlockGroups = 8;                    // groups per code block (two
 constexpr uint32_t kCodeBox = kTileM * 128;        // one swizzled box: 128 rows x 4 groups
 constexpr uint32_t kCodeStage = 2 * kCodeBox;      // 32 KiB
 constexpr int kCodeStages = 4;                     // code blocks in flight
-constexpr int kG = 2;                              // groups per pipeline step
-constexpr int kSteps = 4;                          // A (tensor memory) and activation (shared) slots
-constexpr int kAccBufs = 2;                        // fp32 step accumulators in tensor memory
+constexpr int kG = 4;                              // groups per pipeline step
+constexpr int kSteps = 2;                          // A (tensor memory) and activation (shared) slots
+constexpr int kAccBufs = 1;                        // fp32 step accumulator in tensor memory (released as soon as read)
 constexpr uint32_t kACols = 32;                    // one group of A: 128 lanes x 64 bf16
 
 template <int NT>
@@ -166,12 +166,13 @@ struct ItemWalk {
 };
 
 __device__ __forceinline__ void walk_set_g(ItemWalk &w, int KG) {
-  w.g = 2 * w.p;
-  w.ng = KG - w.g < 2 ? KG - w.g : 2;
+  w.g = kG * w.p;
+  w.ng = KG - w.g < kG ? KG - w.g : kG;
 }
+__device__ __forceinline__ int n_steps(int KG) { return (KG + kG - 1) / kG; }
 
 __device__ __forceinline__ void walk_init(ItemWalk &w, int64_t it_begin, int KG) {
-  const int P = (KG + 1) / 2;
+  const int P = n_steps(KG);
   w.i = it_begin;
   w.tile = static_cast<int>(it_begin / P);
   w.p = static_cast<int>(it_begin % P);
@@ -185,7 +186,7 @@ __device__ __forceinline__ void walk_init(ItemWalk &w, int64_t it_begin, int KG)
 __device__ __forceinline__ void walk_flags(ItemWalk &w, int64_t it_end, int KG) {
   const bool last = w.i + 1 >= it_end;
   w.tile_end = (w.g + w.ng == KG) || last;
-  w.block_end = w.tile_end || (((w.g + 2) & (kBlockGroups - 1)) == 0);
+  w.block_end = w.tile_end || (((w.g + kG) & (kBlockGroups - 1)) == 0);
 }
 
 // first (tile, group) of the block after the current one (valid when it exists)
@@ -220,7 +221,7 @@ __device__ __forceinline__ void load_block_scales(const uint16_t *scale, int64_t
 __device__ __forceinline__ void walk_next(ItemWalk &w, int KG) {
   const bool new_block = w.block_end;
   ++w.i;
-  if (++w.p == (KG + 1) / 2) {
+  if (++w.p == n_steps(KG)) {
     w.p = 0;
     ++w.tile;
   }
@@ -244,7 +245,7 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
   uint8_t *sX = sC + kCodeStages * kCodeStage;          // activation tiles (1024-aligned)
   uint64_t *bars = reinterpret_cast<uint64_t *>(sX + kSteps * kG * C::kXBytes);
   uint64_t *c_full = bars, *c_empty = c_full + kCodeStages;
-  // a step (two groups) has an A slot in tensor memory and an activation slot in shared memory,
+  // a step (kG groups) has an A slot in tensor memory and an activation slot in shared memory,
   // filled separately (a_full, x_full) and released together by one MMA commit (s_empty)
   uint64_t *a_full = c_empty + kCodeStages, *x_full = a_full + kSteps, *s_empty = x_full + kSteps;
   uint64_t *acc_full = s_empty + kSteps, *acc_empty = acc_full + kAccBufs;
@@ -319,8 +320,7 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         if (!mbar_wait(s_empty + st, ((li / kSteps) & 1) ^ 1, abort_flag, status)) break;
         uint8_t *dst = sX + st * kG * C::kXBytes;
         mbar_arrive_expect_tx(x_full + st, w.ng * C::kXBytes);
-        tma_load_2d(dst, &tm_x, w.g * 64, 0, x_full + st);
-        if (w.ng > 1) tma_load_2d(dst + C::kXBytes, &tm_x, w.g * 64 + 64, 0, x_full + st);
+        for (int jj = 0; jj < w.ng; ++jj) tma_load_2d(dst + jj * C::kXBytes, &tm_x, (w.g + jj) * 64, 0, x_full + st);
         x_issued = li + 1;
         walk_flags(w, it_end, KG);
         walk_next(w, KG);
@@ -336,11 +336,11 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
       // no offset here carries out of: adding to the low word is enough
       const uint64_t d0 = umma_desc_sw128(smem_u32(sX));
       const uint32_t dlo0 = static_cast<uint32_t>(d0), dhi = static_cast<uint32_t>(d0 >> 32);
-      const int P = (KG + 1) / 2;
+      const int P = n_steps(KG);
       int p = static_cast<int>(it_begin % P);
       for (int li = 0; li < n_local; ++li) {
         const int st = li % kSteps, b = li % kAccBufs;
-        const bool two = (KG & 1) == 0 || p != P - 1;
+        const int ng = KG - kG * p < kG ? KG - kG * p : kG;
         if (++p == P) p = 0;
         if (!mbar_wait(a_full + st, (li / kSteps) & 1, abort_flag, status)) break;
         if (!mbar_wait(x_full + st, (li / kSteps) & 1, abort_flag, status)) break;
@@ -349,16 +349,15 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         const uint32_t ta = tmem + C::kACol0 + st * kG * kACols;
         const uint32_t td = tmem + b * kG * NT;
         const uint32_t blo = dlo0 + ((st * kG * C::kXBytes) >> 4);
-        umma_ts_lean<false>(td, ta, blo, dhi, idesc);
-        umma_ts_lean<true>(td, ta + 8, blo + 2, dhi, idesc);
-        umma_ts_lean<true>(td, ta + 16, blo + 4, dhi, idesc);
-        umma_ts_lean<true>(td, ta + 24, blo + 6, dhi, idesc);
-        if (two) {
-          constexpr uint32_t xo = C::kXBytes >> 4;
-          umma_ts_lean<false>(td + NT, ta + kACols, blo + xo, dhi, idesc);
-          umma_ts_lean<true>(td + NT, ta + kACols + 8, blo + xo + 2, dhi, idesc);
-          umma_ts_lean<true>(td + NT, ta + kACols + 16, blo + xo + 4, dhi, idesc);
-          umma_ts_lean<true>(td + NT, ta + kACols + 24, blo + xo + 6, dhi, idesc);
+#pragma unroll
+        for (int jj = 0; jj < kG; ++jj) {
+          if (jj < ng) {
+            const uint32_t tdj = td + jj * NT, taj = ta + jj * kACols, bj = blo + jj * (C::kXBytes >> 4);
+            umma_ts_lean<false>(tdj, taj, bj, dhi, idesc);
+            umma_ts_lean<true>(tdj, taj + 8, bj + 2, dhi, idesc);
+            umma_ts_lean<true>(tdj, taj + 16, bj + 4, dhi, idesc);
+            umma_ts_lean<true>(tdj, taj + 24, bj + 6, dhi, idesc);
+          }
         }
         umma_commit(s_empty + st);
         umma_commit(acc_full + b);
@@ -423,8 +422,9 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
       if (!mbar_wait(s_empty + st, ((li / kSteps) & 1) ^ 1, abort_flag, status)) break;
       tc_fence_after();
       const uint32_t ta = tmem + tlane + C::kACol0 + st * kG * kACols + half * 16;
-      tmem_st16(ta, v[0]);
-      if (w.ng > 1) tmem_st16(ta + kACols, v[1]);
+#pragma unroll
+      for (int jj = 0; jj < kG; ++jj)
+        if (jj < w.ng) tmem_st16(ta + jj * kACols, v[jj]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -463,11 +463,15 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         walk_next_block(w, KG, nt, ng);
         if (li + 1 < n_local) load_block_scales(scale, clamp_row(nt), KG, ng, nsc);
       }
-      // a step's two scales share one word of the block's scale vector
+      // the step's scales: groups js .. js + kG - 1 of the block's scale vector (two per word)
       const int js = w.g - w.block_g0;
-      const uint32_t sw = js < 2 ? sc[0] : js < 4 ? sc[1] : js < 6 ? sc[2] : sc[3];   // no local-memory indexing
-      const float sf0 = f16_bits_to_f32(static_cast<uint16_t>(sw & 0xFFFFu));
-      const float sf1 = w.ng > 1 ? f16_bits_to_f32(static_cast<uint16_t>(sw >> 16)) : 0.0f;
+      float sfs[kG];
+#pragma unroll
+      for (int jj = 0; jj < kG; ++jj) {
+        const int q = js + jj;
+        const uint32_t sw = q < 2 ? sc[0] : q < 4 ? sc[1] : q < 6 ? sc[2] : sc[3];   // no local-memory indexing
+        sfs[jj] = jj < w.ng ? f16_bits_to_f32(static_cast<uint16_t>((q & 1) ? (sw >> 16) : (sw & 0xFFFFu))) : 0.0f;
+      }
       if (!mbar_wait(acc_full + b, (li / kAccBufs) & 1, abort_flag, status)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + b * kG * NT + chalf * NH;
@@ -483,7 +487,7 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
             tmem_ld8(tbase + jj * NT, d);
           }
           tmem_wait_ld();
-          const float sf = jj ? sf1 : sf0;
+          const float sf = sfs[jj];
           const float2 s2 = make_float2(sf, sf);
 #pragma unroll
           for (int c = 0; c < NH / 2; ++c)
@@ -537,7 +541,7 @@ cq_status launch_nt(const cq_qweight &qw, const void *x, int m, float *y, uint32
   }
   const int KG = static_cast<int>(K / kGroup);
   const int64_t tiles = (N + kTileM - 1) / kTileM;
-  const int64_t items = tiles * ((KG + 1) / 2);          // steps of two groups
+  const int64_t items = tiles * ((KG + kG - 1) / kG);     // steps of kG groups
   const int64_t grid = items < sm_count() ? items : sm_count();
   cq_status st = cuda_check(cudaFuncSetAttribute(gemm4_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  static_cast<int>(C::kSmem)),
