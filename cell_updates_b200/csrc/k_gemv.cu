@@ -214,7 +214,9 @@ gemv4_kernel(const __grid_constant__ GemvSegs segs, const __nv_bfloat16 *__restr
     for (int i = 0; i < kStages; ++i) mbar_init(bars + i, FULL ? 33u : 1u);
     mbar_init_fence();
   }
-  for (int i = threadIdx.x; i < kRedSlots * kRedFloats; i += kGemvThreads) red[i] = 0.0f;
+  // the reduction slots need zeros only where a warp never writes: tiles with fewer chunks than warps
+  if (n_chunks < kWarps)
+    for (int i = threadIdx.x; i < kRedSlots * kRedFloats; i += kGemvThreads) red[i] = 0.0f;
   if (threadIdx.x < kRedSlots) { cnt[threadIdx.x] = 0u; uses[threadIdx.x] = 0u; }
   if (threadIdx.x == 0) *abort_flag = 0u;
   __syncthreads();

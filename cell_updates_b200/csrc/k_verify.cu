@@ -292,8 +292,7 @@ __global__ void __launch_bounds__(kThreads) verify4_kernel(VerifyArgs a) {
 
 // Revocation (no residual) of fixed-4 weights moves only 0.55 bytes per weight, so a lane
 // keeps four 32-weight units in flight: a warp reads 4 x 512 contiguous bytes of codes (plus
-// their scales and zeros) before it computes, and the grid needs 4x fewer warps for the same
-// bytes in flight. The certificate is that of verify4_kernel without a residual.
+// their scales and zeros) before it computes, which quadruples the bytes in flight per SM. The certificate is that of verify4_kernel without a residual.
 constexpr int kRevokeUnroll = 4;
 
 __global__ void __launch_bounds__(kThreads) revoke4_kernel(VerifyArgs a) {
@@ -375,7 +374,7 @@ void dispatch(int rk, VerifyArgs a, int blocks, cudaStream_t s) {
 
 void dispatch4(int rk, VerifyArgs a, int blocks, cudaStream_t s) {
   switch (rk) {
-    case kNoR: revoke4_kernel<<<(blocks + kRevokeUnroll - 1) / kRevokeUnroll, kThreads, 0, s>>>(a); break;
+    case kNoR: revoke4_kernel<<<blocks, kThreads, 0, s>>>(a); break;
     case kF32: verify4_kernel<kF32><<<blocks, kThreads, 0, s>>>(a); break;
     default: verify4_kernel<kBF16><<<blocks, kThreads, 0, s>>>(a); break;
   }
