@@ -63,7 +63,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile
     if (honour_abort && *abort_flag) return false;
   }
   *abort_flag = 1u;
-  if (status) atomicOr(status, 1u);
+  if (status) {
+    // the status word may be cleared by the kernel this grid overlaps (programmatic dependent
+    // launch): report only once that kernel has finished (no-op for an ordinary launch)
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    atomicOr(status, 1u);
+  }
   return false;
 }
 
@@ -72,6 +77,10 @@ __device__ __forceinline__ bool mbar_wait_suspend(uint64_t *b, uint32_t parity, 
                                                   bool honour_abort = true) {
   return mbar_wait(b, parity, abort_flag, nullptr, honour_abort);
 }
+
+// programmatic dependent launch: wait for the preceding grid's results / let the next grid start
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::); }
 
 // 2-D tiled TMA load into this CTA's shared memory, completing on an mbarrier (no multicast)
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {

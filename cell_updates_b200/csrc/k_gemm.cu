@@ -5,55 +5,82 @@
 // low-bit weights. Here the batch is large enough (m >= 16) for a real dense contraction:
 //     y[i, n] = sum_g s[n, g] * sum_{k in g} (q[n, k] - z[n, g]) * x[i, k]
 //
-// Exactness: q - z (|q - z| <= 15 for 4-bit codes) and x are exact bf16 operands, the tensor
-// core forms exact products and accumulates one group (64 columns) in fp32 in tensor memory;
-// the epilogue multiplies that group sum by the fp32 scale and accumulates in registers.
+// Operands. Every weight is dequantized once, to fp16: A[n, k] = RN16(s * (q - z)). q - z is
+// exact, and the exact product has at most 15 significant bits, so its one rounding is a
+// relative error below 2^-11; |s| <= 4096 keeps |A| <= 61440 < 65504. The activations are
+// copied to fp16 by a preparation kernel with one power of two per batch row,
+// x16[i, k] = x[i, k] * 2^-e_i, chosen so that max_k |x16[i, k]| lies in [2^14, 2^15): a bf16
+// value keeps all of its 8 significant bits, nothing overflows, and only values below 2^-28
+// of the row's largest become fp16 subnormals. Products are exact in fp32 and the tensor
+// cores accumulate a whole K range of a tile in fp32 in tensor memory; the epilogue writes
+// y += acc * 2^e_i once per range. A group whose scale is above 4096 in magnitude (or not
+// finite) or whose zero point is above 15 is left out of A (written as zeros) and added in
+// fp32 by the epilogue warps, which are otherwise idle while a range accumulates.
 //
-// Structure (one CTA per SM, persistent; work = (128-row tile, group) items split evenly
-// over the CTAs in row-major order, so a CTA covers a contiguous K range of one or two tiles):
-//   warp 0      TMA producer: code blocks of 8 groups (two adjacent 128-byte-wide boxes per
-//               row, 128-byte swizzled: long DRAM runs and conflict-free shared reads)
-//   warp 18     TMA producer: per group the activations (m rows x 64 bf16, swizzled = the
-//               UMMA K-major layout); a separate warp, so code blocks are requested as soon as
-//               a buffer frees up, however far the activation ring runs ahead
-//   warp 1      MMA issuer: four tcgen05.mma (M=128, N=NT, K=16) per group into one of four
-//               tensor-memory accumulators; commits release the A and x stages and publish
-//   warps 2-9   dequantize: each thread turns half a row of the group's codes into bf16
-//               (q - z) in the 128-byte swizzled K-major layout the MMA descriptor expects
-//   warps 10-17 epilogue: tcgen05.ld the group's fp32 sums (one row and half the columns per
-//               thread), acc += s * sum; at the end of a tile (or of the CTA's range) add to y
-// y is zeroed first; tiles split between two CTAs are combined with fp32 atomics.
-// Every barrier wait is bounded: on timeout the CTA raises a status flag, drains what it
-// issued, frees its tensor memory and returns.
+// Structure (one CTA per SM, persistent; work = (128-row tile, step of four groups) items
+// split evenly over the CTAs in row-major order, so a CTA covers a contiguous K range of one
+// or a few tiles; a maximal run of one tile's steps in one CTA is a "segment"):
+//   warps 10-13 loaders and epilogue: copy each step's codes (128 rows x 128 bytes, eight
+//               lanes per row, so every warp instruction reads four whole 128-byte lines) and
+//               the rows' scales and zero points with cp.async into an 8-stage ring, seven
+//               steps ahead; cp.async completion arrives on the stage's barrier. At a
+//               segment's end they tcgen05.ld their rows of the accumulator, scale and add to y
+//               with atomics (segments of one tile in two CTAs combine there). Per-thread
+//               copies keep many short row runs in flight: DRAM serves this 128-row pattern
+//               about twice as fast as 128-row TMA boxes of the same bytes.
+//   warps 2-9   dequantize: thread (row, half) turns its half row of a group into fp16
+//               s * (q - z) and stores it to tensor memory (its lane = its row)
+//   warp 0      TMA producer: per step the fp16 activations (m rows x 64 per group, 128-byte
+//               swizzled = the UMMA K-major layout), double-buffered
+//   warp 1      MMA issuer: per group four tcgen05.mma (M=128, N=NT, K=16), A from tensor
+//               memory and B from shared memory, into the segment's accumulator (two
+//               accumulators alternate between segments)
+// A step's A operand is stored to tensor memory only once the previous step's MMAs have
+// completed (the dequantization arithmetic still overlaps them): stores into other columns of
+// the same lanes while MMAs that read A from tensor memory were in flight gave wrong sums on
+// this part for N = 16 and 32.
+// The preparation kernel also zeroes y and the status word. Every barrier wait is bounded: on
+// timeout the CTA raises a status flag, drains what it issued, frees its tensor memory and
+// returns.
 #include "cq_async.cuh"
 
 namespace cq {
 namespace {
 
 constexpr int kTileM = 128;
+constexpr int kXWarp = 0;                          // TMA producer of the activation tiles
+constexpr int kMmaWarp = 1;
+constexpr int kDeqWarp0 = 2;
 constexpr int kDeqWarps = 8;                       // two per TMEM lane quarter: half a row each
-constexpr int kEpiWarps = 8;                       // two per TMEM lane quarter: half the columns each
-constexpr int kThreads = 32 * (3 + kDeqWarps + kEpiWarps);
-constexpr int kXWarp = 2 + kDeqWarps + kEpiWarps;      // the last warp loads activations
-constexpr int kBlockGroups = 8;                    // groups per code block (two 128-byte boxes per row)
-constexpr uint32_t kCodeBox = kTileM * 128;        // one swizzled box: 128 rows x 4 groups
-constexpr uint32_t kCodeStage = 2 * kCodeBox;      // 32 KiB
-constexpr int kCodeStages = 4;                     // code blocks in flight
+constexpr int kEpiWarp0 = kDeqWarp0 + kDeqWarps;
+constexpr int kEpiWarps = 4;                       // one per TMEM lane quarter
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr int kG = 4;                              // groups per pipeline step
 constexpr int kSteps = 2;                          // A (tensor memory) and activation (shared) slots
-constexpr int kAccBufs = 1;                        // fp32 step accumulator in tensor memory (released as soon as read)
-constexpr uint32_t kACols = 32;                    // one group of A: 128 lanes x 64 bf16
+constexpr int kAccBufs = 2;                        // fp32 segment accumulators in tensor memory
+constexpr int kRing = 8;                           // code / metadata stages loaded ahead
+constexpr uint32_t kCodeStepBytes = kTileM * 128;           // 128 rows x 4 groups x 32 B, swizzled
+constexpr uint32_t kScaleOff = kCodeStepBytes;              // 128 rows x 4 scales
+constexpr uint32_t kZeroOff = kScaleOff + kTileM * 8;       // 128 rows x 4 zero points
+constexpr uint32_t kStageBytes = kZeroOff + kTileM * 4;
+constexpr int kFlagSlots = 8;                      // per-segment masks of rows with slow groups
+constexpr uint32_t kACols = 32;                    // one group of A: 128 lanes x 64 fp16
+constexpr uint32_t kMaxFastScale = 0x6C00u;        // 4096 in fp16 bits
+constexpr uint32_t kMaxFastZero = 15u;
+constexpr int kPrepThreads = 256;
 
 template <int NT>
 struct Cfg {
   static constexpr uint32_t kXBytes = NT * 128;                     // one group of activations
-  static constexpr uint32_t kAccCols = kAccBufs * kG * NT;
+  static constexpr uint32_t kAccCols = kAccBufs * NT;
   static constexpr uint32_t kACol0 = kAccCols;                     // A slots follow the accumulators
   static constexpr uint32_t kCols = kAccCols + kSteps * kG * kACols;
   static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
   static_assert(kCols <= 512, "tensor memory holds 512 columns");
-  static constexpr int kBars = 2 * kCodeStages + 3 * kSteps + 2 * kAccBufs + 1;
-  static constexpr uint32_t kSmem = 1024 + kCodeStages * kCodeStage + kSteps * kG * kXBytes + kBars * 8 + 16;
+  static constexpr int kBars = 2 * kRing + 3 * kSteps + 2 * kAccBufs + kFlagSlots + 1;
+  static constexpr uint32_t kSmem =
+      1024 + kRing * kStageBytes + kSteps * kG * kXBytes + kBars * 8 + kFlagSlots * 16 + NT * 4 + 16;
+  static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
 // UMMA shared-memory descriptor: K-major operand in the 128-byte swizzled canonical layout
@@ -67,33 +94,15 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
   return d;
 }
 
-// instruction descriptor: D fp32, A and B bf16, both K-major, M = 128, N = NT
+// instruction descriptor: D fp32, A and B fp16 (format 0), both K-major, M = 128, N = NT
 template <int NT>
 __device__ __forceinline__ constexpr uint32_t umma_idesc() {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(NT >> 3) << 17) |
-         (static_cast<uint32_t>(kTileM >> 4) << 24);
+  return (1u << 4) | (static_cast<uint32_t>(NT >> 3) << 17) | (static_cast<uint32_t>(kTileM >> 4) << 24);
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-
-// the same with A read from tensor memory (128 lanes = rows, two bf16 per 32-bit column, K-major)
-__device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-
-// TS MMA with the B descriptor given as two 32-bit words and a compile-time accumulate flag:
-// the issuing thread shares its scheduler with busy warps, so each MMA costs it as few
-// instructions as possible
+// TS MMA (A from tensor memory: 128 lanes = rows, two fp16 per 32-bit column, K-major) with the
+// B descriptor given as two 32-bit words and a compile-time accumulate flag: the issuing thread
+// shares its scheduler with busy warps, so each MMA costs it as few instructions as possible
 template <bool kAccum>
 __device__ __forceinline__ void umma_ts_lean(uint32_t tmem_d, uint32_t tmem_a, uint32_t bdesc_lo, uint32_t bdesc_hi,
                                              uint32_t idesc) {
@@ -127,141 +136,195 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t *r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t *r) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
-}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
-// (128 + q) pairs in natural column order from one word of 8 nibbles: pair j = columns 2j, 2j+1
-__device__ __forceinline__ uint32_t nat_pair(uint32_t w, uint32_t w4, uint32_t sel) {
-  uint32_t t = __byte_perm(w, w4, sel), out;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(out) : "r"(t), "r"(0x000F000Fu), "r"(0x43004300u));
-  return out;
+// a wait for a whole warp: every lane polls, and the warp leaves together and agrees on the
+// outcome -- the tcgen05.ld / tcgen05.st that follow are .sync.aligned, which a warp whose
+// lanes left the wait at different times would execute diverged
+__device__ __forceinline__ bool warp_wait(uint64_t *b, uint32_t parity, volatile uint32_t *abort_flag,
+                                          uint32_t *status) {
+  const bool ok = mbar_wait(b, parity, abort_flag, status);
+  return __all_sync(0xFFFFFFFFu, ok);
 }
 
-__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+// named barrier of the epilogue warps only
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(32 * kEpiWarps) : "memory"); }
+
+// ---- fp16 dequantization --------------------------------------------------------------------
+// (w & mask) | 0x64006400: a nibble at bits 0-3 (16-19) gives the fp16 1024 + q, a nibble at
+// bits 4-7 (20-23) gives 1024 + 16 q, in the low (high) half
+__device__ __forceinline__ uint32_t nib_f16(uint32_t w, uint32_t mask) {
+  uint32_t out;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(out) : "r"(w), "r"(mask), "r"(0x64006400u));
+  return out;
+}
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("sub.rn.bf16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
 
-// The work of one CTA: steps = (tile, pair of groups) in row-major order; a step covers
-// groups g, g + 1 of a tile (only g when it is the tile's last, odd group). Code blocks of
-// 8 groups = 4 steps; a block also ends at a tile end and at the end of the CTA's range.
-struct ItemWalk {
-  int64_t i;          // current step (tile * P + pair)
-  int tile, p, g, ng; // tile, pair, first group, groups in this step (1 or 2)
-  int block;          // index of the current code block
-  int block_g0;       // first group of the current block
-  bool block_start, block_end, tile_end;
+// Eight codes of one row (K positions 8t .. 8t+7, the first in the low nibble) -> four 32-bit
+// tensor-memory columns holding the fp16 pairs (0,4), (1,5), (2,6), (3,7) of s * (q - z); the
+// preparation kernel stores the activations in the same order. zz1 = (1024 + z) in both
+// halves, nzz16 = -(64 + z), s2 = s in both halves. The subtractions are exact: (1024 + q) -
+// (1024 + z) directly, and (1024 + 16 q) / 16 - (64 + z) in one FMA whose product is exact.
+__device__ __forceinline__ void deq_word(uint32_t wd, uint32_t zz1, uint32_t nzz16, uint32_t s2, uint32_t *out) {
+  const uint32_t w8 = wd >> 8;
+  out[0] = h2_mul(h2_sub(nib_f16(wd, 0x000F000Fu), zz1), s2);
+  out[1] = h2_mul(h2_fma(nib_f16(wd, 0x00F000F0u), 0x2C002C00u, nzz16), s2);
+  out[2] = h2_mul(h2_sub(nib_f16(w8, 0x000F000Fu), zz1), s2);
+  out[3] = h2_mul(h2_fma(nib_f16(w8, 0x00F000F0u), 0x2C002C00u, nzz16), s2);
+}
+
+// groups the tensor cores take: |s| <= 4096 (finite) and z <= 15
+__device__ __forceinline__ bool slow_group(uint32_t sbits, uint32_t z) {
+  return (sbits & 0x7FFFu) > kMaxFastScale || z > kMaxFastZero;
+}
+
+// 16-byte copy into shared memory that bypasses L1, and the wait for all of a thread's copies
+__device__ __forceinline__ void cp_async_16cg(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
+// The work of one CTA: steps = (tile, kG groups) in row-major order; step p of a tile covers
+// groups kG*p .. kG*p + kG - 1 (the tensor-core path takes K a multiple of 4 groups).
+struct Walk {
+  int64_t i;    // current step (tile * P + p)
+  int tile, p;  // tile, step within the tile
 };
-
-__device__ __forceinline__ void walk_set_g(ItemWalk &w, int KG) {
-  w.g = kG * w.p;
-  w.ng = KG - w.g < kG ? KG - w.g : kG;
+__device__ __forceinline__ void walk_init(Walk &w, int64_t i, int P) {
+  w.i = i;
+  w.tile = static_cast<int>(i / P);
+  w.p = static_cast<int>(i % P);
 }
-__device__ __forceinline__ int n_steps(int KG) { return (KG + kG - 1) / kG; }
-
-__device__ __forceinline__ void walk_init(ItemWalk &w, int64_t it_begin, int KG) {
-  const int P = n_steps(KG);
-  w.i = it_begin;
-  w.tile = static_cast<int>(it_begin / P);
-  w.p = static_cast<int>(it_begin % P);
-  walk_set_g(w, KG);
-  w.block = 0;
-  w.block_g0 = w.g;
-  w.block_start = true;
-}
-
-// flags of the current step, given the CTA's end
-__device__ __forceinline__ void walk_flags(ItemWalk &w, int64_t it_end, int KG) {
-  const bool last = w.i + 1 >= it_end;
-  w.tile_end = (w.g + w.ng == KG) || last;
-  w.block_end = w.tile_end || (((w.g + kG) & (kBlockGroups - 1)) == 0);
-}
-
-// first (tile, group) of the block after the current one (valid when it exists)
-__device__ __forceinline__ void walk_next_block(const ItemWalk &w, int KG, int &tile, int &g) {
-  const int g_end = (w.block_g0 | (kBlockGroups - 1)) + 1;     // next multiple of 8
-  if (g_end >= KG) {
-    tile = w.tile + 1;
-    g = 0;
-  } else {
-    tile = w.tile;
-    g = g_end;
-  }
-}
-
-// the (up to) 8 per-group bytes / halves of one row for the block starting at group g
-__device__ __forceinline__ void load_block_zeros(const uint8_t *zero, int64_t row, int KG, int g, uint32_t &lo,
-                                                 uint32_t &hi) {
-  uint32_t v[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) v[j] = (g + j < KG && ((g + j) & ~7) == (g & ~7)) ? __ldg(zero + row * KG + g + j) : 0u;
-  lo = v[0] | (v[1] << 8) | (v[2] << 16) | (v[3] << 24);
-  hi = v[4] | (v[5] << 8) | (v[6] << 16) | (v[7] << 24);
-}
-__device__ __forceinline__ void load_block_scales(const uint16_t *scale, int64_t row, int KG, int g, uint32_t (&s)[4]) {
-  uint32_t v[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) v[j] = (g + j < KG && ((g + j) & ~7) == (g & ~7)) ? __ldg(scale + row * KG + g + j) : 0u;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) s[j] = v[2 * j] | (v[2 * j + 1] << 16);
-}
-
-__device__ __forceinline__ void walk_next(ItemWalk &w, int KG) {
-  const bool new_block = w.block_end;
+__device__ __forceinline__ void walk_next(Walk &w, int P) {
   ++w.i;
-  if (++w.p == n_steps(KG)) {
+  if (++w.p == P) {
     w.p = 0;
     ++w.tile;
   }
-  walk_set_g(w, KG);
-  w.block_start = new_block;
-  if (new_block) {
-    ++w.block;
-    w.block_g0 = w.g;
-  }
+}
+// the step ends a segment: the tile's last step or the CTA's last
+__device__ __forceinline__ bool walk_seg_end(const Walk &w, int P, int64_t it_end) {
+  return w.p + 1 == P || w.i + 1 == it_end;
 }
 
+// ---- the activation preparation kernel --------------------------------------------------------
+// grid (splits, m): every CTA of batch row i finds max_k |x[i, k]| (the row is read by each of
+// the row's CTAs; the repeats hit L2), then converts its share of the row to fp16 scaled by
+// 2^-e_i in the dequantizer's pair order, and zeroes its share of y[i, :]. xmul[i] = 2^e_i.
+__global__ void __launch_bounds__(kPrepThreads)
+gemm_prep_kernel(const uint16_t *__restrict__ x, int64_t K, uint16_t *__restrict__ x16, float *__restrict__ xmul,
+                 float *__restrict__ y, int64_t N, uint32_t *__restrict__ status) {
+  pdl_launch_dependents();     // the GEMM may set up (barriers, tensor memory, code loads) meanwhile
+  __shared__ uint32_t red[kPrepThreads / 32];
+  const int64_t i = blockIdx.y;
+  const uint4 *xr = reinterpret_cast<const uint4 *>(x + i * K);
+  const int64_t n8 = K / 8;
+  uint32_t mx = 0;             // non-negative bf16 values order like their bit patterns (NaN above inf)
+  for (int64_t c = threadIdx.x; c < n8; c += kPrepThreads) {
+    const uint4 v = __ldg(xr + c);
+    const uint32_t a = v.x & 0x7FFF7FFFu, b = v.y & 0x7FFF7FFFu, d = v.z & 0x7FFF7FFFu, e = v.w & 0x7FFF7FFFu;
+    mx = max(mx, max(max(a & 0xFFFFu, a >> 16), max(b & 0xFFFFu, b >> 16)));
+    mx = max(mx, max(max(d & 0xFFFFu, d >> 16), max(e & 0xFFFFu, e >> 16)));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  mx = red[0];
+#pragma unroll
+  for (int k = 1; k < kPrepThreads / 32; ++k) mx = max(mx, red[k]);
+  // e_i: max * 2^-e_i in [2^14, 2^15); 0 for an all-zero or non-finite row
+  int e = 0;
+  if (mx != 0u && mx < 0x7F80u) {
+    int fe;
+    frexpf(bf16_bits_to_f32(static_cast<uint16_t>(mx)), &fe);   // max = f * 2^fe, f in [0.5, 1)
+    e = fe - 15;
+  }
+  // 2^-e as two normal floats (|e| <= 147 does not fit one)
+  const int ea = -e / 2, eb = -e - ea;
+  const float fa = __int_as_float((ea + 127) << 23), fb = __int_as_float((eb + 127) << 23);
+  if (blockIdx.x == 0 && threadIdx.x == 0) xmul[i] = ldexpf(1.0f, e);
+  if (status && i == 0 && blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
+  // this CTA's share of the 8-element chunks
+  const int64_t c0 = n8 * blockIdx.x / gridDim.x, c1 = n8 * (blockIdx.x + 1) / gridDim.x;
+  uint4 *xo = reinterpret_cast<uint4 *>(x16 + i * K);
+  for (int64_t c = c0 + threadIdx.x; c < c1; c += kPrepThreads) {
+    const uint4 v = __ldg(xr + c);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f[2 * j] = __fmul_rn(__fmul_rn(__uint_as_float(wv[j] << 16), fa), fb);
+      f[2 * j + 1] = __fmul_rn(__fmul_rn(__uint_as_float(wv[j] & 0xFFFF0000u), fa), fb);
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __half2 h = __floats2half2_rn(f[j], f[j + 4]);      // pair (j, j + 4)
+      o[j] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    xo[c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  const int64_t n0 = N * blockIdx.x / gridDim.x, n1 = N * (blockIdx.x + 1) / gridDim.x;
+  for (int64_t n = n0 + threadIdx.x; n < n1; n += kPrepThreads) y[i * N + n] = 0.0f;
+}
+
+// ---- the GEMM kernel ----------------------------------------------------------------------------
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
-                const uint16_t *__restrict__ scale, const uint8_t *__restrict__ zero, float *__restrict__ y,
-                int m, int64_t N, int KG, int64_t n_items, uint32_t *__restrict__ status) {
+gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restrict__ plane,
+                const uint16_t *__restrict__ scale, const uint8_t *__restrict__ zero,
+                const uint16_t *__restrict__ xb, const float *__restrict__ xmul, float *__restrict__ y, int m,
+                int64_t N, int64_t K, int KG, int64_t n_items, uint32_t *__restrict__ status) {
   using C = Cfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sC = smem;                                   // code blocks (1024-aligned, swizzled)
-  uint8_t *sX = sC + kCodeStages * kCodeStage;          // activation tiles (1024-aligned)
+  uint8_t *sR = smem;                                   // code / metadata ring filled by the loader warps
+  uint8_t *sX = sR + kRing * kStageBytes;               // activation tiles (1024-aligned, swizzled)
   uint64_t *bars = reinterpret_cast<uint64_t *>(sX + kSteps * kG * C::kXBytes);
-  uint64_t *c_full = bars, *c_empty = c_full + kCodeStages;
   // a step (kG groups) has an A slot in tensor memory and an activation slot in shared memory,
   // filled separately (a_full, x_full) and released together by one MMA commit (s_empty)
-  uint64_t *a_full = c_empty + kCodeStages, *x_full = a_full + kSteps, *s_empty = x_full + kSteps;
+  uint64_t *r_full = bars, *r_empty = r_full + kRing;   // ring stages: copies landed / stage read
+  uint64_t *a_full = r_empty + kRing, *x_full = a_full + kSteps, *s_empty = x_full + kSteps;
   uint64_t *acc_full = s_empty + kSteps, *acc_empty = acc_full + kAccBufs;
-  uint64_t *drain = acc_empty + kAccBufs;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  uint64_t *seg_done = acc_empty + kAccBufs;            // dequantizers finished a segment's masks
+  uint64_t *drain = seg_done + kFlagSlots;
+  uint32_t *seg_mask = reinterpret_cast<uint32_t *>(drain + 1);   // [kFlagSlots][4 lane quarters]
+  float *s_xmul = reinterpret_cast<float *>(seg_mask + kFlagSlots * 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(s_xmul + NT);
   volatile uint32_t *abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t it_begin = static_cast<int64_t>(blockIdx.x) * n_items / gridDim.x;
   const int64_t it_end = static_cast<int64_t>(blockIdx.x + 1) * n_items / gridDim.x;
   const int n_local = static_cast<int>(it_end - it_begin);
+  const int P = KG / kG;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kCodeStages; ++i) {
-      mbar_init(c_full + i, 1);
-      mbar_init(c_empty + i, kDeqWarps);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(r_full + i, 32 * kEpiWarps);     // one cp.async arrival per loader thread
+      mbar_init(r_empty + i, kDeqWarps);
     }
     for (int i = 0; i < kSteps; ++i) {
       mbar_init(a_full + i, kDeqWarps);
@@ -272,11 +335,13 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
       mbar_init(acc_full + i, 1);
       mbar_init(acc_empty + i, kEpiWarps);
     }
+    for (int i = 0; i < kFlagSlots; ++i) mbar_init(seg_done + i, kDeqWarps);
+    for (int i = 0; i < kFlagSlots * 4; ++i) seg_mask[i] = 0u;
     mbar_init(drain, 1);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_slot)),
                  "r"(C::kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
@@ -286,49 +351,26 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ---------------- TMA producer: code blocks ----------------
-    if (lane == 0) {
-      ItemWalk w;
-      walk_init(w, it_begin, KG);
-      int code_issued = 0;
-      for (int li = 0; li < n_local; ++li) {
-        walk_flags(w, it_end, KG);
-        if (w.block_start) {
-          const int cs = w.block % kCodeStages;
-          if (!mbar_wait(c_empty + cs, ((w.block / kCodeStages) & 1) ^ 1, abort_flag, status)) break;
-          mbar_arrive_expect_tx(c_full + cs, kCodeStage);
-          uint8_t *dst = sC + cs * kCodeStage;
-          tma_load_2d(dst, &tm_codes, w.block_g0 * 32, w.tile * kTileM, c_full + cs);
-          tma_load_2d(dst + kCodeBox, &tm_codes, w.block_g0 * 32 + 128, w.tile * kTileM, c_full + cs);
-          code_issued = w.block + 1;
-        }
-        walk_next(w, KG);
-      }
-      // every copy this thread started has landed before the CTA may exit
-      for (int b = code_issued - kCodeStages > 0 ? code_issued - kCodeStages : 0; b < code_issued; ++b)
-        mbar_wait(c_full + (b % kCodeStages), (b / kCodeStages) & 1, abort_flag, status, false);
-    }
-  } else if (warp == kXWarp) {
+  if (warp == kXWarp) {
     // ---------------- TMA producer: the step's activation tiles ----------------
     if (lane == 0) {
-      ItemWalk w;
-      walk_init(w, it_begin, KG);
+      pdl_wait();                 // the fp16 activations come from the preparation kernel
+      Walk w;
+      walk_init(w, it_begin, P);
       int x_issued = 0;
       for (int li = 0; li < n_local; ++li) {
         const int st = li % kSteps;
         if (!mbar_wait(s_empty + st, ((li / kSteps) & 1) ^ 1, abort_flag, status)) break;
         uint8_t *dst = sX + st * kG * C::kXBytes;
-        mbar_arrive_expect_tx(x_full + st, w.ng * C::kXBytes);
-        for (int jj = 0; jj < w.ng; ++jj) tma_load_2d(dst + jj * C::kXBytes, &tm_x, (w.g + jj) * 64, 0, x_full + st);
+        mbar_arrive_expect_tx(x_full + st, kG * C::kXBytes);
+        for (int jj = 0; jj < kG; ++jj) tma_load_2d(dst + jj * C::kXBytes, &tm_x, (kG * w.p + jj) * 64, 0, x_full + st);
         x_issued = li + 1;
-        walk_flags(w, it_end, KG);
-        walk_next(w, KG);
+        walk_next(w, P);
       }
       for (int li = x_issued - kSteps > 0 ? x_issued - kSteps : 0; li < x_issued; ++li)
         mbar_wait(x_full + (li % kSteps), (li / kSteps) & 1, abort_flag, status, false);
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc<NT>();
@@ -336,183 +378,210 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
       // no offset here carries out of: adding to the low word is enough
       const uint64_t d0 = umma_desc_sw128(smem_u32(sX));
       const uint32_t dlo0 = static_cast<uint32_t>(d0), dhi = static_cast<uint32_t>(d0 >> 32);
-      const int P = n_steps(KG);
-      int p = static_cast<int>(it_begin % P);
+      Walk w;
+      walk_init(w, it_begin, P);
+      int seg = 0;
+      bool first = true;          // the next step opens a segment
       for (int li = 0; li < n_local; ++li) {
-        const int st = li % kSteps, b = li % kAccBufs;
-        const int ng = KG - kG * p < kG ? KG - kG * p : kG;
-        if (++p == P) p = 0;
+        const int st = li % kSteps, b = seg % kAccBufs;
+        const bool seg_end = walk_seg_end(w, P, it_end);
+        if (first && !mbar_wait(acc_empty + b, ((seg / kAccBufs) & 1) ^ 1, abort_flag, status)) break;
         if (!mbar_wait(a_full + st, (li / kSteps) & 1, abort_flag, status)) break;
         if (!mbar_wait(x_full + st, (li / kSteps) & 1, abort_flag, status)) break;
-        if (!mbar_wait(acc_empty + b, ((li / kAccBufs) & 1) ^ 1, abort_flag, status)) break;
         tc_fence_after();
         const uint32_t ta = tmem + C::kACol0 + st * kG * kACols;
-        const uint32_t td = tmem + b * kG * NT;
+        const uint32_t td = tmem + b * NT;
         const uint32_t blo = dlo0 + ((st * kG * C::kXBytes) >> 4);
+        if (first) umma_ts_lean<false>(td, ta, blo, dhi, idesc);
+        else umma_ts_lean<true>(td, ta, blo, dhi, idesc);
+        umma_ts_lean<true>(td, ta + 8, blo + 2, dhi, idesc);
+        umma_ts_lean<true>(td, ta + 16, blo + 4, dhi, idesc);
+        umma_ts_lean<true>(td, ta + 24, blo + 6, dhi, idesc);
 #pragma unroll
-        for (int jj = 0; jj < kG; ++jj) {
-          if (jj < ng) {
-            const uint32_t tdj = td + jj * NT, taj = ta + jj * kACols, bj = blo + jj * (C::kXBytes >> 4);
-            umma_ts_lean<false>(tdj, taj, bj, dhi, idesc);
-            umma_ts_lean<true>(tdj, taj + 8, bj + 2, dhi, idesc);
-            umma_ts_lean<true>(tdj, taj + 16, bj + 4, dhi, idesc);
-            umma_ts_lean<true>(tdj, taj + 24, bj + 6, dhi, idesc);
-          }
+        for (int jj = 1; jj < kG; ++jj) {
+          const uint32_t taj = ta + jj * kACols, bj = blo + jj * (C::kXBytes >> 4);
+          umma_ts_lean<true>(td, taj, bj, dhi, idesc);
+          umma_ts_lean<true>(td, taj + 8, bj + 2, dhi, idesc);
+          umma_ts_lean<true>(td, taj + 16, bj + 4, dhi, idesc);
+          umma_ts_lean<true>(td, taj + 24, bj + 6, dhi, idesc);
         }
         umma_commit(s_empty + st);
-        umma_commit(acc_full + b);
+        if (seg_end) {
+          umma_commit(acc_full + b);
+          ++seg;
+        }
+        first = seg_end;
+        walk_next(w, P);
       }
       // all issued MMAs have completed before tensor memory is released
       umma_commit(drain);
       mbar_wait(drain, 0, abort_flag, status, false);
     }
-  } else if (warp < 2 + kDeqWarps) {
+  } else if (warp < kEpiWarp0) {
     // ---------------- dequantize: half a row per thread, into tensor memory ----------------
     // a warp may only touch TMEM lanes 32 * (warp % 4) .. + 31, so rows follow the warp index
     const int quad = warp & 3;
     const int r = quad * 32 + lane;               // tile row = TMEM lane
-    const int half = (warp - 2) >> 2;             // columns 32*half .. 32*half+31 of each group
-    ItemWalk w;
-    walk_init(w, it_begin, KG);
-    auto clamp_row = [&](int tile) {
-      const int64_t row = static_cast<int64_t>(tile) * kTileM + r;
-      return row < N ? row : N - 1;
-    };
-    // zero points of the current block and, one block ahead, of the next one
-    uint32_t zlo, zhi, nzlo = 0, nzhi = 0;
-    load_block_zeros(zero, clamp_row(w.tile), KG, w.g, zlo, zhi);
+    const int half = (warp - kDeqWarp0) >> 2;     // columns 32*half .. 32*half+31 of each group
+    Walk w;
+    walk_init(w, it_begin, P);
     const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
+    int seg = 0;
+    bool slow = false;                            // this row has a slow group in the segment
     for (int li = 0; li < n_local; ++li) {
-      walk_flags(w, it_end, KG);
-      const int cs = w.block % kCodeStages;
-      if (w.block_start) {
-        if (li > 0) {
-          zlo = nzlo;
-          zhi = nzhi;
-        }
-        int nt, ng;
-        walk_next_block(w, KG, nt, ng);
-        if (li + 1 < n_local) load_block_zeros(zero, clamp_row(nt), KG, ng, nzlo, nzhi);   // rows clamp: in bounds
-        if (!mbar_wait(c_full + cs, (w.block / kCodeStages) & 1, abort_flag, status)) break;
-      }
-      const int st = li % kSteps;
-      // group j of the block sits in box j/4, 16-byte chunk (2*(j%4) + half) of the row, swizzled
+      const int st = li % kSteps, rs = li % kRing;
+      if (!warp_wait(r_full + rs, (li / kRing) & 1, abort_flag, status)) break;
+      const uint8_t *sb = sR + rs * kStageBytes;
+      const uint2 sm = *reinterpret_cast<const uint2 *>(sb + kScaleOff + r * 8);
+      const uint32_t zw = *reinterpret_cast<const uint32_t *>(sb + kZeroOff + r * 4);
       uint32_t v[kG][16];
 #pragma unroll
       for (int jj = 0; jj < kG; ++jj) {
-        const int j = w.g - w.block_g0 + jj;
-        const uint32_t z = ((j < 4 ? zlo : zhi) >> (8 * (j & 3))) & 0xFFu;
-        const uint32_t zz = 0x43004300u | z | (z << 16);      // (128 + z) in both halves
-        const int chunk = ((j & 3) << 1) | half;
-        const uint4 cw = *reinterpret_cast<const uint4 *>(sC + cs * kCodeStage + ((j >> 2) & 1) * kCodeBox +
-                                                          r * 128 + ((chunk ^ (r & 7)) << 4));
-        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {       // columns 32*half + 8c .. +7, two per 32-bit TMEM column
-          const uint32_t wd = words[c], w4 = wd >> 4;
-          v[jj][4 * c + 0] = bf16x2_sub(nat_pair(wd, w4, 0x4400u), zz);
-          v[jj][4 * c + 1] = bf16x2_sub(nat_pair(wd, w4, 0x5511u), zz);
-          v[jj][4 * c + 2] = bf16x2_sub(nat_pair(wd, w4, 0x6622u), zz);
-          v[jj][4 * c + 3] = bf16x2_sub(nat_pair(wd, w4, 0x7733u), zz);
-        }
+        const uint32_t z = (zw >> (8 * jj)) & 0xFFu;
+        const uint32_t sbits = ((jj < 2 ? sm.x : sm.y) >> (16 * (jj & 1))) & 0xFFFFu;
+        const bool sl = slow_group(sbits, z);
+        slow |= sl;
+        const uint32_t zc = sl ? 0u : z;
+        const uint32_t zz1 = 0x64006400u | zc | (zc << 16);
+        const uint32_t nzz16 = 0xD400D400u | (zc << 4) | (zc << 20);
+        const uint32_t s2 = sl ? 0u : (sbits | (sbits << 16));
+        // 16-byte chunk (2 jj + half) of row r, swizzled by the row's low three bits
+        const uint4 cw = *reinterpret_cast<const uint4 *>(sb + r * 128 + ((((jj << 1) | half) ^ (r & 7)) << 4));
+        deq_word(cw.x, zz1, nzz16, s2, &v[jj][0]);
+        deq_word(cw.y, zz1, nzz16, s2, &v[jj][4]);
+        deq_word(cw.z, zz1, nzz16, s2, &v[jj][8]);
+        deq_word(cw.w, zz1, nzz16, s2, &v[jj][12]);
       }
-      // the code words are in registers: the block's last step releases its buffer now
       __syncwarp();
-      if (lane == 0 && w.block_end) mbar_arrive(c_empty + cs);
-      if (!mbar_wait(s_empty + st, ((li / kSteps) & 1) ^ 1, abort_flag, status)) break;
+      if (lane == 0) mbar_arrive(r_empty + rs);   // the stage is in registers
+      // A is stored only while no MMA is in flight: the previous step's commit covers them all
+      if (li > 0 && !warp_wait(s_empty + (li - 1) % kSteps, ((li - 1) / kSteps) & 1, abort_flag, status)) break;
       tc_fence_after();
       const uint32_t ta = tmem + tlane + C::kACol0 + st * kG * kACols + half * 16;
 #pragma unroll
-      for (int jj = 0; jj < kG; ++jj)
-        if (jj < w.ng) tmem_st16(ta + jj * kACols, v[jj]);
+      for (int jj = 0; jj < kG; ++jj) tmem_st16(ta + jj * kACols, v[jj]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(a_full + st);
-      walk_next(w, KG);
+      if (walk_seg_end(w, P, it_end)) {
+        // rows whose slow groups the epilogue adds; then the segment's mask is complete
+        const uint32_t bal = __ballot_sync(0xFFFFFFFFu, slow);
+        const int slot = seg % kFlagSlots;
+        if (lane == 0) {
+          if (bal) atomicOr(seg_mask + slot * 4 + quad, bal);
+          mbar_arrive(seg_done + slot);
+        }
+        slow = false;
+        ++seg;
+      }
+      walk_next(w, P);
     }
-  } else if (warp < 2 + kDeqWarps + kEpiWarps) {
-    // ---------------- epilogue: row r = TMEM lane, half of the columns ----------------
-    const int ew = warp - 2 - kDeqWarps;
+  } else {
+    // ---------------- epilogue: one row per thread, all NT columns ----------------
     const int quad = warp & 3;                 // this warp may read TMEM lanes 32*quad .. +31
-    const int chalf = ew >> 2;                 // columns chalf*NT/2 .. +NT/2
-    constexpr int NH = NT / 2;
     const int r = quad * 32 + lane;
-    float2 acc[NH / 2];                        // column pairs, updated with packed fp32x2 FMAs
+    const int et = threadIdx.x - 32 * kEpiWarp0;
+    // loader: step la's copies into ring stage la % kRing, once the dequantizers have read the
+    // step that used it before; lane l of a warp copies 16-byte chunk l % 8 of four rows per
+    // instruction, each thread also the four scales and zero points of row et
+    const int64_t row_bytes = K / 2;
+    Walk wl;
+    walk_init(wl, it_begin, P);
+    int la = 0;
+    bool ok = true;
+    auto load_until = [&](int target) {
+      const int lim = target < n_local ? target : n_local;
+      while (ok && la < lim) {
+        const int rs = la % kRing;
+        if (!warp_wait(r_empty + rs, ((la / kRing) & 1) ^ 1, abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        uint8_t *sb = sR + rs * kStageBytes;
+        const int g = kG * wl.p;
+        const int64_t row0 = static_cast<int64_t>(wl.tile) * kTileM;
 #pragma unroll
-    for (int c = 0; c < NH / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
-    ItemWalk w;
-    walk_init(w, it_begin, KG);
-    auto clamp_row = [&](int tile) {
-      const int64_t row = static_cast<int64_t>(tile) * kTileM + r;
-      return row < N ? row : N - 1;
+        for (int k = 0; k < 8; ++k) {
+          const int rr = ((et >> 5) * 8 + k) * 4 + (lane >> 3), c = lane & 7;
+          int64_t row = row0 + rr;
+          row = row < N ? row : N - 1;            // rows past the end: any valid row, result unused
+          cp_async_16cg(sb + rr * 128 + ((c ^ (rr & 7)) << 4), plane + row * row_bytes + g * 32 + c * 16);
+        }
+        {
+          int64_t row = row0 + et;
+          row = row < N ? row : N - 1;
+          cp_async_8(sb + kScaleOff + et * 8, scale + row * KG + g);
+          cp_async_4(sb + kZeroOff + et * 4, zero + row * KG + g);
+        }
+        cp_async_arrive_noinc(r_full + rs);
+        walk_next(wl, P);
+        ++la;
+      }
     };
-    // scales of the current block and, one block ahead, of the next one
-    uint32_t sc[4], nsc[4] = {0, 0, 0, 0};
-    load_block_scales(scale, clamp_row(w.tile), KG, w.g, sc);
-    for (int li = 0; li < n_local; ++li) {
-      walk_flags(w, it_end, KG);
-      const int b = li % kAccBufs;
-      const int64_t row = static_cast<int64_t>(w.tile) * kTileM + r;
-      if (w.block_start) {
-        if (li > 0) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) sc[j] = nsc[j];
-        }
-        int nt, ng;
-        walk_next_block(w, KG, nt, ng);
-        if (li + 1 < n_local) load_block_scales(scale, clamp_row(nt), KG, ng, nsc);
-      }
-      // the step's scales: groups js .. js + kG - 1 of the block's scale vector (two per word)
-      const int js = w.g - w.block_g0;
-      float sfs[kG];
-#pragma unroll
-      for (int jj = 0; jj < kG; ++jj) {
-        const int q = js + jj;
-        const uint32_t sw = q < 2 ? sc[0] : q < 4 ? sc[1] : q < 6 ? sc[2] : sc[3];   // no local-memory indexing
-        sfs[jj] = jj < w.ng ? f16_bits_to_f32(static_cast<uint16_t>((q & 1) ? (sw >> 16) : (sw & 0xFFFFu))) : 0.0f;
-      }
-      if (!mbar_wait(acc_full + b, (li / kAccBufs) & 1, abort_flag, status)) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + b * kG * NT + chalf * NH;
-#pragma unroll
-      for (int jj = 0; jj < kG; ++jj) {
-        if (jj < w.ng) {
-          uint32_t d[NH];
-          if constexpr (NH >= 16) {
-#pragma unroll
-            for (int c0 = 0; c0 < NH; c0 += 16)
-              tmem_ld16(tbase + jj * NT + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
-          } else {
-            tmem_ld8(tbase + jj * NT, d);
+    load_until(kRing);                         // fill the ring before anything else
+    pdl_wait();                                // xmul and the zeroed y come from the preparation kernel
+    if (et < NT) s_xmul[et] = et < m ? xmul[et] : 0.0f;
+    epi_sync();
+    Walk w;
+    walk_init(w, it_begin, P);
+    int seg = 0, ga = kG * w.p;
+    bool open = true;                          // the next step opens a segment
+    for (int li = 0; li < n_local && ok; ++li) {
+      load_until(li + kRing);                  // refill the stage the dequantizers freed
+      if (open) ga = kG * w.p;
+      const bool seg_end = walk_seg_end(w, P, it_end);
+      open = seg_end;
+      if (seg_end) {
+        const int b = seg % kAccBufs, slot = seg % kFlagSlots;
+        const int gb = kG * w.p + kG;
+        const int64_t row = static_cast<int64_t>(w.tile) * kTileM + r;
+        if (!warp_wait(seg_done + slot, (seg / kFlagSlots) & 1, abort_flag, status)) break;
+        const uint32_t mask = seg_mask[slot * 4 + quad];
+        __syncwarp();
+        if (lane == 0) seg_mask[slot * 4 + quad] = 0u;
+        if (((mask >> lane) & 1u) && row < N) {
+          // groups the tensor cores did not take: s * sum_k (q - z) x in fp32, straight to y
+          for (int g = ga; g < gb; ++g) {
+            const uint32_t sbits = scale[row * KG + g], z = zero[row * KG + g];
+            if (!slow_group(sbits, z)) continue;
+            const float sf = f16_bits_to_f32(static_cast<uint16_t>(sbits));
+            const uint8_t *cp = plane + row * (K / 2) + g * 32;
+            for (int i = 0; i < m; ++i) {
+              const uint16_t *xg = xb + i * K + g * 64;
+              float acc = 0.0f;
+              for (int k = 0; k < 64; ++k) {
+                const int q = (cp[k >> 1] >> ((k & 1) * 4)) & 15;
+                acc = fmaf(static_cast<float>(q - static_cast<int>(z)), bf16_bits_to_f32(xg[k]), acc);
+              }
+              atomicAdd(y + static_cast<int64_t>(i) * N + row, __fmul_rn(acc, sf));
+            }
           }
-          tmem_wait_ld();
-          const float sf = sfs[jj];
-          const float2 s2 = make_float2(sf, sf);
-#pragma unroll
-          for (int c = 0; c < NH / 2; ++c)
-            acc[c] = __ffma2_rn(s2, make_float2(__uint_as_float(d[2 * c]), __uint_as_float(d[2 * c + 1])), acc[c]);
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty + b);
-      if (w.tile_end) {
+        __syncwarp();
+        if (!warp_wait(acc_full + b, (seg / kAccBufs) & 1, abort_flag, status)) break;
+        tc_fence_after();
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + b * NT;
+        uint32_t dv[NT];
+#pragma unroll
+        for (int c0 = 0; c0 < NT; c0 += 16) tmem_ld16(tbase + c0, dv + c0);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty + b);   // the accumulator is in registers
         if (row < N) {
 #pragma unroll
-          for (int c = 0; c < NH; ++c) {
-            const int col = chalf * NH + c;
-            if (col < m) atomicAdd(y + static_cast<int64_t>(col) * N + row, (c & 1) ? acc[c >> 1].y : acc[c >> 1].x);
-          }
+          for (int c = 0; c < NT; ++c)
+            if (c < m) atomicAdd(y + static_cast<int64_t>(c) * N + row, __fmul_rn(__uint_as_float(dv[c]), s_xmul[c]));
         }
-#pragma unroll
-        for (int c = 0; c < NH / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
+        ++seg;
       }
-      walk_next(w, KG);
+      walk_next(w, P);
     }
+    cp_async_wait_all();                       // no copy may land after the CTA has exited
   }
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(C::kTmemCols));
   }
@@ -520,63 +589,96 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
 
 // ---- host side ---------------------------------------------------------------------------
 
+// workspace: [0, 16) status word, [16, 16 + 4 * 64) xmul, [512, ...) fp16 activations of a
+// batch slice of at most 64 rows
+constexpr size_t kWsXmul = 16, kWsX16 = 512;
+constexpr int kSliceRows = 64;
+
 template <int NT>
-cq_status launch_nt(const cq_qweight &qw, const void *x, int m, float *y, uint32_t *status, cudaStream_t s) {
+cq_status launch_nt(const cq_qweight &qw, const void *x, int m, float *y, uint8_t *ws, bool clear_status,
+                    cudaStream_t s) {
   using C = Cfg<NT>;
   auto encode = encode_fn();
   if (!encode) return fail(CQ_ERR_CUDA, "cq_dequant_gemm: cuTensorMapEncodeTiled unavailable");
   const int64_t N = qw.rows, K = qw.cols;
-  CUtensorMap tm_codes, tm_x;
-  cq_status cs = code_tensor_map(&tm_codes, qw.plane[2], N, K, kTileM, "cq_dequant_gemm");
-  if (cs != CQ_OK) return cs;
+  uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+  float *xmul = reinterpret_cast<float *>(ws + kWsXmul);
+  uint16_t *x16 = reinterpret_cast<uint16_t *>(ws + kWsX16);
+  CUtensorMap tm_x;
   {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(m)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * 2)};
     cuuint32_t box[2] = {64, NT};
     cuuint32_t es[2] = {1, 1};
-    CUresult r = encode(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box, es,
+    CUresult r = encode(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, dims, strides, box, es,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(CQ_ERR_CUDA, "cq_dequant_gemm: activation tensor map (%d)", (int)r);
   }
+  // 1. the activation preparation (fp16 copy, y and status cleared)
+  {
+    const int64_t want = (2 * static_cast<int64_t>(sm_count()) + m - 1) / m;
+    const int64_t splits = want < 1 ? 1 : want > 64 ? 64 : want;
+    gemm_prep_kernel<<<dim3(static_cast<unsigned>(splits), static_cast<unsigned>(m)), kPrepThreads, 0, s>>>(
+        static_cast<const uint16_t *>(x), K, x16, xmul, y, N, clear_status ? status : nullptr);
+    cq_status st = launch_check("cq_dequant_gemm: preparation");
+    if (st != CQ_OK) return st;
+  }
+  // 2. the GEMM, allowed to start while the preparation runs (it waits for it where it must)
   const int KG = static_cast<int>(K / kGroup);
   const int64_t tiles = (N + kTileM - 1) / kTileM;
-  const int64_t items = tiles * ((KG + kG - 1) / kG);     // steps of kG groups
+  const int64_t items = tiles * (KG / kG);                // steps of kG groups
   const int64_t grid = items < sm_count() ? items : sm_count();
   cq_status st = cuda_check(cudaFuncSetAttribute(gemm4_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  static_cast<int>(C::kSmem)),
                             "cq_dequant_gemm: shared memory attribute");
   if (st != CQ_OK) return st;
-  gemm4_tc_kernel<NT><<<static_cast<unsigned>(grid), kThreads, C::kSmem, s>>>(tm_codes, tm_x, qw.scale, qw.zero, y,
-                                                                              m, N, KG, items, status);
-  return launch_check("cq_dequant_gemm");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_check(cudaLaunchKernelEx(&cfg, gemm4_tc_kernel<NT>, tm_x, static_cast<const uint8_t *>(qw.plane[2]),
+                                       qw.scale, qw.zero, static_cast<const uint16_t *>(x),
+                                       static_cast<const float *>(xmul), y, m, N, K, KG, items, status),
+                    "cq_dequant_gemm");
 }
 
 }  // namespace
 
+// fixed-4 weights without a residual, bf16 x, m >= 16, K a multiple of 4 groups, and the
+// alignments the per-thread copies need (16-byte codes, 8-byte scales, 4-byte zero points)
 bool gemm_tc_eligible(const cq_qweight &qw, cq_dtype xdt, int m) {
-  return qw.bits == nullptr && qw.residual == nullptr && xdt == CQ_BF16 && m >= 16 && qw.rows > 0 && qw.cols > 0;
+  return qw.bits == nullptr && qw.residual == nullptr && xdt == CQ_BF16 && m >= 16 && qw.rows > 0 && qw.cols > 0 &&
+         (qw.cols / kGroup) % kG == 0 && aligned16(qw.plane[2]) && aligned8(qw.scale) &&
+         (reinterpret_cast<uintptr_t>(qw.zero) & 3u) == 0;
 }
 
-// the workspace holds the kernel's status word (non-zero if a wait timed out)
-size_t gemm_tc_workspace(int64_t, int64_t, int) { return 16; }
+// the status word, the per-row powers of two and the fp16 activations of one batch slice
+size_t gemm_tc_workspace(int64_t, int64_t cols, int m) {
+  const int64_t rows = m < kSliceRows ? m : kSliceRows;
+  return kWsX16 + static_cast<size_t>(rows) * static_cast<size_t>(cols) * 2;
+}
 
 cq_status launch_gemm_tc(const cq_qweight &qw, const void *x, int m, float *y, void *ws, size_t, cudaStream_t s) {
   const int64_t N = qw.rows;
-  uint32_t *status = static_cast<uint32_t *>(ws);
-  cq_status st = cuda_check(cudaMemsetAsync(status, 0, sizeof(uint32_t), s), "cq_dequant_gemm: clear status");
-  if (st != CQ_OK) return st;
-  st = cuda_check(cudaMemsetAsync(y, 0, sizeof(float) * static_cast<size_t>(m) * N, s), "cq_dequant_gemm: zero y");
-  if (st != CQ_OK) return st;
-  // the batch in slices of at most 64 columns (the epilogue keeps one fp32 sum per column
-  // in registers; 64 of them fit without spilling)
-  for (int i0 = 0; i0 < m; i0 += 64) {
-    const int mi = m - i0 < 64 ? m - i0 : 64;
+  if (!aligned16(x)) return fail(CQ_ERR_ALIGN, "cq_dequant_gemm: x must be 16-byte aligned");
+  // the batch in slices of at most 64 rows (the MMA's N); slices run in stream order, so each
+  // preparation overwrites the previous slice's fp16 activations only after that GEMM ended
+  for (int i0 = 0; i0 < m; i0 += kSliceRows) {
+    const int mi = m - i0 < kSliceRows ? m - i0 : kSliceRows;
     const void *xi = static_cast<const uint16_t *>(x) + static_cast<int64_t>(i0) * qw.cols;
     float *yi = y + static_cast<int64_t>(i0) * N;
-    if (mi <= 16) st = launch_nt<16>(qw, xi, mi, yi, status, s);
-    else if (mi <= 32) st = launch_nt<32>(qw, xi, mi, yi, status, s);
-    else st = launch_nt<64>(qw, xi, mi, yi, status, s);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    cq_status st;
+    if (mi <= 16) st = launch_nt<16>(qw, xi, mi, yi, w8, i0 == 0, s);
+    else if (mi <= 32) st = launch_nt<32>(qw, xi, mi, yi, w8, i0 == 0, s);
+    else st = launch_nt<64>(qw, xi, mi, yi, w8, i0 == 0, s);
     if (st != CQ_OK) return st;
   }
   return CQ_OK;
@@ -594,7 +696,7 @@ cq_status launch_gemm_tc(const cq_qweight &qw, const void *x, int m, float *y, v
 namespace cq {
 namespace {
 
-constexpr size_t kStaticScratchBytes = 4096;
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;   // the fp16 activations of a 64-row slice, K <= 65532
 __device__ __align__(256) unsigned char g_gemm_scratch[kStaticScratchBytes];
 
 constexpr int kMaxScratchDevices = 64;

@@ -74,9 +74,6 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
   return out;   // (w & 0x000F000F) | 0x43004300
 }
 
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::); }
-
 // ---- the kernel -------------------------------------------------------------------------------
 // Persistent CTAs of 16 warps, one per SM; CTA b owns the 16-row tiles b, b + G, b + 2G, ...
 // Each tile is cut into chunks of 4 groups (16 rows x 128 bytes), and the CTA's chunks, tile

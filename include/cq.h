@@ -179,8 +179,13 @@ cq_status cq_dequant_gemv_multi(const cq_qweight *const *qws, int count, const v
  * cq_dequant_gemm -- the same contraction for a batch, 1 <= m <= 256. Fixed-4 weights with
  * bf16 x, no residual and m >= 16 run on the sm_100a tcgen05 tensor cores with accumulators
  * in tensor memory; m < 16 goes to the GEMV kernels, as do other formats (in slices of 8).
+ * On the tensor cores each weight s * (q - z) is rounded once to fp16 (relative error below
+ * 2^-11) and x is copied to fp16 with an exact power of two per row; groups with |s| > 4096,
+ * a non-finite s or z > 15 are summed in fp32 instead (slowly). x must be 16-byte aligned
+ * there (CQ_ERR_ALIGN otherwise).
  * workspace: caller-owned device scratch of at least cq_gemm_workspace(rows, cols, m) bytes
- * (may be NULL when that is 0), 16-byte aligned. y: [m, rows] fp32, overwritten.
+ * (may be NULL when that is 0), 16-byte aligned; it holds the fp16 copy of x and a status
+ * word (first 4 bytes, non-zero if an internal wait gave up). y: [m, rows] fp32, overwritten.
  */
 cq_status cq_dequant_gemm(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m,
                           float *y, void *workspace, size_t workspace_bytes, cq_stream_t stream);
@@ -192,9 +197,10 @@ cq_status cq_dequant_gemm(const cq_qweight *qw, const void *x, cq_dtype x_dtype,
  * plug-in that is handed device buffers by a host framework that owns all device memory, or a
  * serving loop with a fixed memory budget where an allocation could block on the device or
  * fail at the worst moment. The pages have no counterpart to this call.
- * Its scratch is a 4096-byte array inside the library that every GPU which loads the library
+ * Its scratch is an 8 MiB array inside the library that every GPU which loads the library
  * keeps until the process exits. A shape that would need more scratch than that is refused
- * with CQ_ERR_RANGE (no shape does today: the GEMM needs 16 bytes). The first call on a device
+ * with CQ_ERR_RANGE: the tensor-core GEMM needs 512 + 2 * min(m, 64) * cols bytes, so with
+ * m >= 64 cols may be at most 65532. The first call on a device
  * looks up the array's device address with that device current; make that first call before
  * any stream capture. All calls share the array and the call clears what must start at zero,
  * but calls that overlap on the GPU (other streams, other threads) race on it.

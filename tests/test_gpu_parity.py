@@ -293,6 +293,41 @@ def test_gemm_tensor_core(rows, cols, m):
     check_matmul(host(ops.gemm(qw, x_d)), y_ref, f"gemm {rows}x{cols} m={m}")
 
 
+def test_gemm_slow_groups_and_activation_range():
+    """Groups the fp16 tensor-core operand cannot hold (|s| > 4096, z > 15) are summed by the
+    epilogue in fp32; batch rows of very small, very large and zero activations go through the
+    per-row power of two. Checked per (batch row, row subset) so no scale hides another."""
+    rows, cols, m = 300, 64 * 24, 40
+    KG = cols // 64
+    w = synth.normal_weights(rows, cols, seed=31)
+    codes, scale, zero, _ = co.quantize(w)
+    rng = np.random.default_rng(32)
+    slow_rows = np.sort(rng.choice(rows, 37, replace=False))
+    scale2, zero2 = scale.copy(), zero.copy()
+    big = np.array([5000.0, 60000.0, 4100.0], np.float16).view(np.uint16)
+    for n, r in enumerate(slow_rows):
+        g = r * KG + rng.integers(0, KG)
+        if n % 3 == 2:
+            zero2[g] = 200                               # zero point beyond the 4-bit range
+        else:
+            scale2[g] = big[n % 3]
+    planes = co.pack(codes)
+    x = synth.activations(m, cols, seed=33, dtype="f32")
+    x[0] *= 1e-30
+    x[1] *= 1e30
+    x[2] = 0.0
+    x[3, ::7] *= 1e6                                     # a row with a few large outliers
+    xb = synth.f32_to_bf16_bits(x).reshape(m, cols)
+    y_ref = co.dequant_matmul_f64(planes, scale2, zero2, rows, cols, xb, "bf16")
+    qw = cq.QWeight(rows, cols, [None, None, dev(planes[2]), None], u16_dev(scale2), dev(zero2))
+    y = host(ops.gemm(qw, bf16_dev(xb)))
+    assert np.array_equal(y[2], np.zeros(rows, np.float32))
+    fast_rows = np.setdiff1d(np.arange(rows), slow_rows)
+    for i in [0, 1, 3, 4, m - 1]:
+        for sub, name in ((slow_rows, "slow"), (fast_rows, "fast")):
+            check_matmul(y[i, sub], y_ref[i, sub], f"batch row {i}, {name} rows")
+
+
 def test_gemm_small_batch_uses_gemv_slices():
     qw, x_d, y_ref, _ = _matmul_case(300, 64 * 21, 12, "bf16", seed=12)
     check_matmul(host(ops.gemm(qw, x_d)), y_ref, "gemm m=12")
