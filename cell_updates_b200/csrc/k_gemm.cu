@@ -20,7 +20,7 @@
 // Structure (one CTA per SM, persistent; work = (128-row tile, step of four groups) items
 // split evenly over the CTAs in row-major order, so a CTA covers a contiguous K range of one
 // or a few tiles; a maximal run of one tile's steps in one CTA is a "segment"):
-//   warps 10-13 loaders and epilogue: copy each step's codes (128 rows x 128 bytes, eight
+//   warps 10-13 epilogue, and warps 10-12 loaders: copy each step's codes (128 rows x 128 bytes, eight
 //               lanes per row, so every warp instruction reads four whole 128-byte lines) and
 //               the rows' scales and zero points with cp.async into an 8-stage ring, seven
 //               steps ahead; cp.async completion arrives on the stage's barrier. At a
@@ -28,7 +28,7 @@
 //               with atomics (segments of one tile in two CTAs combine there). Per-thread
 //               copies keep many short row runs in flight: DRAM serves this 128-row pattern
 //               about twice as fast as 128-row TMA boxes of the same bytes.
-//   warps 2-9   dequantize: thread (row, half) turns its half row of a group into fp16
+//   warps 2-9   dequantize: thread (row, part) turns half a row of a group into fp16
 //               s * (q - z) and stores it to tensor memory (its lane = its row)
 //   warp 0      TMA producer: per step the fp16 activations (m rows x 64 per group, 128-byte
 //               swizzled = the UMMA K-major layout), double-buffered
@@ -51,9 +51,11 @@ constexpr int kTileM = 128;
 constexpr int kXWarp = 0;                          // TMA producer of the activation tiles
 constexpr int kMmaWarp = 1;
 constexpr int kDeqWarp0 = 2;
-constexpr int kDeqWarps = 8;                       // two per TMEM lane quarter: half a row each
+constexpr int kRowParts = 2;                       // dequantizers per row, each 64 / kRowParts columns of a group
+constexpr int kDeqWarps = 4 * kRowParts;           // kRowParts per TMEM lane quarter
 constexpr int kEpiWarp0 = kDeqWarp0 + kDeqWarps;
 constexpr int kEpiWarps = 4;                       // one per TMEM lane quarter
+constexpr int kLoadWarps = 3;                      // epilogue warps that also load (not warp 13)
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr int kG = 4;                              // groups per pipeline step
 constexpr int kSteps = 2;                          // A (tensor memory) and activation (shared) slots
@@ -118,13 +120,18 @@ __device__ __forceinline__ void umma_ts_lean(uint32_t tmem_d, uint32_t tmem_a, u
         "r"(tmem_a), "r"(bdesc_lo), "r"(bdesc_hi), "r"(idesc));
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+[[maybe_unused]] __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
           taddr),
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
       "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+[[maybe_unused]] __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
@@ -323,7 +330,7 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kRing; ++i) {
-      mbar_init(r_full + i, 32 * kEpiWarps);     // one cp.async arrival per loader thread
+      mbar_init(r_full + i, 32 * kLoadWarps);   // one cp.async arrival per loader thread
       mbar_init(r_empty + i, kDeqWarps);
     }
     for (int i = 0; i < kSteps; ++i) {
@@ -418,11 +425,12 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
       mbar_wait(drain, 0, abort_flag, status, false);
     }
   } else if (warp < kEpiWarp0) {
-    // ---------------- dequantize: half a row per thread, into tensor memory ----------------
+    // ---------------- dequantize: a part of a row per thread, into tensor memory ----------------
     // a warp may only touch TMEM lanes 32 * (warp % 4) .. + 31, so rows follow the warp index
+    constexpr int kW = 8 / kRowParts;             // code words per group and thread (4 columns each)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;               // tile row = TMEM lane
-    const int half = (warp - kDeqWarp0) >> 2;     // columns 32*half .. 32*half+31 of each group
+    const int part = (warp - kDeqWarp0) >> 2;     // columns (64 / kRowParts) * part .. of each group
     Walk w;
     walk_init(w, it_begin, P);
     const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
@@ -434,7 +442,7 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
       const uint8_t *sb = sR + rs * kStageBytes;
       const uint2 sm = *reinterpret_cast<const uint2 *>(sb + kScaleOff + r * 8);
       const uint32_t zw = *reinterpret_cast<const uint32_t *>(sb + kZeroOff + r * 4);
-      uint32_t v[kG][16];
+      uint32_t v[kG][4 * kW];
 #pragma unroll
       for (int jj = 0; jj < kG; ++jj) {
         const uint32_t z = (zw >> (8 * jj)) & 0xFFu;
@@ -445,21 +453,33 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
         const uint32_t zz1 = 0x64006400u | zc | (zc << 16);
         const uint32_t nzz16 = 0xD400D400u | (zc << 4) | (zc << 20);
         const uint32_t s2 = sl ? 0u : (sbits | (sbits << 16));
-        // 16-byte chunk (2 jj + half) of row r, swizzled by the row's low three bits
-        const uint4 cw = *reinterpret_cast<const uint4 *>(sb + r * 128 + ((((jj << 1) | half) ^ (r & 7)) << 4));
-        deq_word(cw.x, zz1, nzz16, s2, &v[jj][0]);
-        deq_word(cw.y, zz1, nzz16, s2, &v[jj][4]);
-        deq_word(cw.z, zz1, nzz16, s2, &v[jj][8]);
-        deq_word(cw.w, zz1, nzz16, s2, &v[jj][12]);
+        // bytes 32 jj + 4 kW part .. of row r: 16-byte chunk (32 jj + 4 kW part) / 16, swizzled by
+        // the row's low three bits
+        const int byte0 = jj * 32 + 4 * kW * part;
+        const uint8_t *cp = sb + r * 128 + ((((byte0 >> 4) ^ (r & 7))) << 4) + (byte0 & 15);
+        if constexpr (kW == 4) {
+          const uint4 cw = *reinterpret_cast<const uint4 *>(cp);
+          deq_word(cw.x, zz1, nzz16, s2, &v[jj][0]);
+          deq_word(cw.y, zz1, nzz16, s2, &v[jj][4]);
+          deq_word(cw.z, zz1, nzz16, s2, &v[jj][8]);
+          deq_word(cw.w, zz1, nzz16, s2, &v[jj][12]);
+        } else {
+          const uint2 cw = *reinterpret_cast<const uint2 *>(cp);
+          deq_word(cw.x, zz1, nzz16, s2, &v[jj][0]);
+          deq_word(cw.y, zz1, nzz16, s2, &v[jj][4]);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(r_empty + rs);   // the stage is in registers
       // A is stored only while no MMA is in flight: the previous step's commit covers them all
       if (li > 0 && !warp_wait(s_empty + (li - 1) % kSteps, ((li - 1) / kSteps) & 1, abort_flag, status)) break;
       tc_fence_after();
-      const uint32_t ta = tmem + tlane + C::kACol0 + st * kG * kACols + half * 16;
+      const uint32_t ta = tmem + tlane + C::kACol0 + st * kG * kACols + part * 4 * kW;
 #pragma unroll
-      for (int jj = 0; jj < kG; ++jj) tmem_st16(ta + jj * kACols, v[jj]);
+      for (int jj = 0; jj < kG; ++jj) {
+        if constexpr (kW == 4) tmem_st16(ta + jj * kACols, v[jj]);
+        else tmem_st8(ta + jj * kACols, v[jj]);
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -484,13 +504,18 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
     const int et = threadIdx.x - 32 * kEpiWarp0;
     // loader: step la's copies into ring stage la % kRing, once the dequantizers have read the
     // step that used it before; lane l of a warp copies 16-byte chunk l % 8 of four rows per
-    // instruction, each thread also the four scales and zero points of row et
+    // instruction, and the four scales and zero points of one or two rows
     const int64_t row_bytes = K / 2;
     Walk wl;
     walk_init(wl, it_begin, P);
     int la = 0;
     bool ok = true;
+    // the warp on the MMA issuer's scheduler (warp % 4 == 1) does not load: it would slow the
+    // dequantizers that share that scheduler, which already lose issue slots to the MMA issuer
+    const bool loader = (warp & 3) != kMmaWarp;
+    const int lw = (warp & 3) == 0 ? 2 : (warp & 3) - 2;   // warps 10, 11, 12 -> 0, 1, 2
     auto load_until = [&](int target) {
+      if (!loader) return;
       const int lim = target < n_local ? target : n_local;
       while (ok && la < lim) {
         const int rs = la % kRing;
@@ -502,17 +527,19 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
         const int g = kG * wl.p;
         const int64_t row0 = static_cast<int64_t>(wl.tile) * kTileM;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int rr = ((et >> 5) * 8 + k) * 4 + (lane >> 3), c = lane & 7;
+        for (int k = 0; k < (32 + kLoadWarps - 1) / kLoadWarps; ++k) {
+          const int rg = lw + kLoadWarps * k;     // group of four rows
+          if (rg >= 32) break;
+          const int rr = rg * 4 + (lane >> 3), c = lane & 7;
           int64_t row = row0 + rr;
           row = row < N ? row : N - 1;            // rows past the end: any valid row, result unused
           cp_async_16cg(sb + rr * 128 + ((c ^ (rr & 7)) << 4), plane + row * row_bytes + g * 32 + c * 16);
         }
-        {
-          int64_t row = row0 + et;
+        for (int t = lw * 32 + lane; t < kTileM; t += 32 * kLoadWarps) {
+          int64_t row = row0 + t;
           row = row < N ? row : N - 1;
-          cp_async_8(sb + kScaleOff + et * 8, scale + row * KG + g);
-          cp_async_4(sb + kZeroOff + et * 4, zero + row * KG + g);
+          cp_async_8(sb + kScaleOff + t * 8, scale + row * KG + g);
+          cp_async_4(sb + kZeroOff + t * 4, zero + row * KG + g);
         }
         cp_async_arrive_noinc(r_full + rs);
         walk_next(wl, P);
@@ -562,18 +589,23 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
         if (!warp_wait(acc_full + b, (seg / kAccBufs) & 1, abort_flag, status)) break;
         tc_fence_after();
         const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + b * NT;
-        uint32_t dv[NT];
+        constexpr int kChunk = NT < 32 ? NT : 32;   // columns per load (registers are scarce)
 #pragma unroll
-        for (int c0 = 0; c0 < NT; c0 += 16) tmem_ld16(tbase + c0, dv + c0);
-        tmem_wait_ld();
+        for (int c0 = 0; c0 < NT; c0 += kChunk) {
+          uint32_t dv[kChunk];
+#pragma unroll
+          for (int c1 = 0; c1 < kChunk; c1 += 16) tmem_ld16(tbase + c0 + c1, dv + c1);
+          tmem_wait_ld();
+          if (row < N) {
+#pragma unroll
+            for (int c = 0; c < kChunk; ++c)
+              if (c0 + c < m)
+                atomicAdd(y + static_cast<int64_t>(c0 + c) * N + row, __fmul_rn(__uint_as_float(dv[c]), s_xmul[c0 + c]));
+          }
+        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty + b);   // the accumulator is in registers
-        if (row < N) {
-#pragma unroll
-          for (int c = 0; c < NT; ++c)
-            if (c < m) atomicAdd(y + static_cast<int64_t>(c) * N + row, __fmul_rn(__uint_as_float(dv[c]), s_xmul[c]));
-        }
+        if (lane == 0) mbar_arrive(acc_empty + b);   // the accumulator has been read
         ++seg;
       }
       walk_next(w, P);
