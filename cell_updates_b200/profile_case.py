@@ -29,7 +29,7 @@ def main():
     qw, codes, _ = ops.quantize_and_pack(w)
     x = torch.randn(m, K, device=dev).to(torch.bfloat16)
     y = torch.empty(m, N, device=dev)
-    ws = torch.empty(64, dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(16, cq.cq_gemm_workspace(N, K, m)), dtype=torch.uint8, device=dev)
     r = (torch.randn(N * K, device=dev) * 1e-3).to(torch.bfloat16)
     mism = torch.empty(1, dtype=torch.int64, device=dev)
     first = torch.empty(1, dtype=torch.int64, device=dev)
