@@ -30,6 +30,7 @@ def lib():
         L.oq_quantize_group.argtypes = [p, i32, p, p, p]; L.oq_quantize_group.restype = C.c_uint32
         L.oq_quantize.argtypes = [p, i64, i64, p, p, p, p, p, i32]; L.oq_quantize.restype = i32
         L.oq_varbits_index.argtypes = [p, i64, p, p]; L.oq_varbits_index.restype = i32
+        L.oq_rrq_stage.argtypes = [p, i64, i64, i32, p, p, p]; L.oq_rrq_stage.restype = C.c_uint32
         L.oq_pack.argtypes = [p, i64, p, p, p, p, p, p]; L.oq_pack.restype = i32
         L.oq_unpack.argtypes = [p, p, p, p, i64, p, p, p]; L.oq_unpack.restype = i32
         L.oq_project_f32.argtypes = [p, p, i64, p]; L.oq_project_f32.restype = i32
@@ -104,6 +105,30 @@ def quantize(w, bits=None, nthreads=None):
     _check(lib().oq_quantize(_ptr(w), rows, cols, _ptr(bits), _ptr(codes), _ptr(scale), _ptr(zero),
                              _ptr(st), nthreads or default_threads()), "oq_quantize")
     return codes, scale, zero, int(st[0])
+
+
+def rrq_stage(r, b=2):
+    """One RRQ stage (see oq_rrq_stage): r float32 [rows, cols] -> (codes u8 [rows*cols],
+    scale u16 [G], zero u8 [G], status, new residual float32 [rows, cols])."""
+    r = np.array(r, dtype=np.float32, order="C", copy=True)
+    rows, cols = r.shape
+    G = rows * (cols // 64)
+    codes = np.zeros(rows * cols, np.uint8)
+    scale = np.zeros(G, np.uint16)
+    zero = np.zeros(G, np.uint8)
+    st = lib().oq_rrq_stage(_ptr(r), rows, cols, int(b), _ptr(codes), _ptr(scale), _ptr(zero))
+    return codes, scale, zero, int(st), r
+
+
+def rrq_build(w, stages, b=2):
+    """The RRQ package: `stages` stages of width b from w -> list of (codes, scale, zero,
+    status) and the final residual."""
+    out = []
+    r = np.asarray(w, np.float32)
+    for _ in range(stages):
+        codes, scale, zero, st, r = rrq_stage(r, b)
+        out.append((codes, scale, zero, st))
+    return out, r
 
 
 def quantize_group(w64, b):

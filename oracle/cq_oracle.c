@@ -493,6 +493,42 @@ int oq_quantize(const float *w, int64_t rows, int64_t cols, const uint8_t *bits,
 }
 
 /* ------------------------------------------------------------------------------
+ * One stage of Recurrent Residual Quantization.
+ * [RRQ] the listing page thelatestinai.com/papers/2512.18934, "Recurrent Residual
+ * Quantization" abstract: the weights become a low-bit base plus a sequence of quantized
+ * residual corrections; from a 2-bit round-to-nearest base, 2-bit round-to-nearest
+ * residuals are added one after another to reach 4, 6 and 8 bits, without calibration.
+ * Reading: each stage quantizes the running residual with the group quantizer above at
+ * one width b for every group, then the residual becomes what that stage does not
+ * represent:
+ *     r_i <- RN32(r_i - RN32(s * (q_i - z)))
+ * with the stored s, z and q of the stage (s*(q-z) is exact: 11 + 8 significant bits fit
+ * in 24).  A group the quantizer flags (s = +0, z = 0, q = 0) keeps its residual.  The
+ * first stage is run on the weights themselves, so its codes are the 2-bit base; after
+ * stage j the model of the weights is the sum of the stages' s*(q-z).
+ * r: rows x cols fp32, replaced in place.  Returns the OR of the groups' status bits.
+ * ---------------------------------------------------------------------------- */
+uint32_t oq_rrq_stage(float *r, int64_t rows, int64_t cols, int b, uint8_t *codes, uint16_t *scale,
+                      uint8_t *zero)
+{
+    if (rows < 0 || cols < 0 || cols % GROUP) return OQ_ST_BADBITS;
+    int64_t G = rows * (cols / GROUP);
+    uint32_t st = 0;
+    for (int64_t g = 0; g < G; g++) {
+        float *rg = r + g * GROUP;
+        uint8_t *qg = codes + g * GROUP;
+        st |= oq_quantize_group(rg, b, qg, scale + g, zero + g);
+        float sf = oq_f16_to_f32(scale[g]);
+        float z = (float)zero[g];
+        for (int i = 0; i < GROUP; i++) {
+            float deq = sf * ((float)qg[i] - z);       /* exact */
+            rg[i] = rg[i] - deq;                        /* one rounding */
+        }
+    }
+    return st;
+}
+
+/* ------------------------------------------------------------------------------
  * Dequantize-and-multiply reference ([VBQ]: fused dequantize-and-multiply for decode):
  *   y[m, n] = sum_k (s_g * (q[n,k] - z_g) + r[n,k]) * x[m, k]
  * evaluated in binary64: s*(q-z) and every product of binary32/bfloat16 values are

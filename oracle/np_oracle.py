@@ -15,6 +15,9 @@ Sources (cited by page title and section):
         and scales, residual confined to its rounding cell, exact re-quantization,
         revocation by dropping the residual, bounded drift.
   [SLQ] page 2 listing, SLQ abstract: asymmetric quantization.
+  [RRQ] page 2 listing (thelatestinai.com/papers/2512.18934), "Recurrent Residual
+        Quantization" abstract: a 2-bit round-to-nearest base and 2-bit round-to-nearest
+        residual corrections stacked to 4, 6 and 8 bits.
 """
 import numpy as np
 
@@ -115,6 +118,26 @@ def quantize(w, bits=None):
     scale = np.where(bad, np.uint16(0), s16.view(np.uint16)).astype(np.uint16)
     zero = np.where(bad, 0, z).astype(np.uint8)
     return codes, scale, zero, status
+
+
+def rrq_stage(r, b=2):
+    """[RRQ] one stage: quantize the running residual at width b for every group, then
+    r <- RN32(r - s*(q - z)) with the stored s, z, q (s*(q - z) is exact in binary32;
+    a flagged group, s = +0, keeps its residual). Returns (codes, scale, zero, status, r')."""
+    r = np.asarray(r, np.float32)
+    rows, cols = r.shape
+    G = rows * (cols // GROUP)
+    codes, scale, zero, status = quantize(r, np.full(G, b, np.uint8))
+    sf = _f16_to_f32(scale)
+    deq = sf[:, None] * (codes.reshape(G, GROUP).astype(np.float32) - zero.astype(np.float32)[:, None])
+    with np.errstate(invalid="ignore"):
+        r_new = _rrq_residual(r.reshape(G, GROUP), deq).astype(np.float32).reshape(rows, cols)
+    return codes, scale, zero, status, r_new
+
+
+def _rrq_residual(r, deq):
+    """what the stage does not represent: RN32(r - s*(q - z))"""
+    return r - deq
 
 
 # ---- packed storage ([VBQ]: per-group widths stored bit-packed) ----------------------

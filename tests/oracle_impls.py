@@ -41,6 +41,9 @@ class COracle:
         mask = ((flags[np.arange(G) // 32] >> (np.arange(G) % 32).astype(np.uint32)) & 1).astype(bool)
         return m, fb, mask
 
+    def rrq_stage(self, r, b=2):
+        return co.rrq_stage(r, b)
+
     def dequant_matmul_f64(self, planes, scale, zero, rows, cols, x, x_dtype="f32", bits=None,
                            r=None, r_dtype="f32"):
         off = None if bits is None else co.varbits_index(bits)[0]
@@ -71,6 +74,9 @@ class NpOracle:
 
     def verify(self, planes, scale, zero, bits=None, r=None, r_dtype="f32"):
         return no.verify(planes, scale, zero, bits, r, r_dtype)
+
+    def rrq_stage(self, r, b=2):
+        return no.rrq_stage(r, b)
 
     def dequant_matmul_f64(self, planes, scale, zero, rows, cols, x, x_dtype="f32", bits=None,
                            r=None, r_dtype="f32"):

@@ -406,4 +406,87 @@ def pin_matmul(impl, seed=61):
                        rtol=1e-12, atol=1e-15)
 
 
+# ---- RRQ: recurrent residual quantization ---------------------------------------------
+# [RRQ] page 2 listing, "Recurrent Residual Quantization" abstract: a 2-bit round-to-nearest
+# base plus 2-bit round-to-nearest residual corrections, stacked to 4, 6 and 8 bits.
+
+def _rrq_stages(impl, w, n):
+    out, r = [], np.asarray(w, np.float32)
+    for _ in range(n):
+        codes, scale, zero, st, r_new = impl.rrq_stage(r, 2)
+        out.append((r, codes, scale, zero, st, r_new))
+        r = r_new
+    return out
+
+
+def pin_rrq_residual_inside_half_step(impl, seed=71):
+    """Round-to-nearest leaves every weight within half a grid step of its level: for a
+    group whose values straddle zero (so the zero point is not clamped),
+    |r'| <= s/2 + L |range/L - s| <= s (1/2 + 3 * 2^-11) for the fp16-rounded s. Each
+    stage must therefore shrink the residual to about s/2 of that stage."""
+    rng = np.random.default_rng(seed)
+    w = (rng.standard_t(5, (32, 512)) * 0.02).astype(np.float32)
+    for j, (r, codes, scale, zero, st, r_new) in enumerate(_rrq_stages(impl, w, 4)):
+        assert st == 0
+        R = r.reshape(-1, GROUP).astype(np.float64)
+        Rn = r_new.reshape(-1, GROUP).astype(np.float64)
+        sf = np.asarray(scale, np.uint16).view(np.float16).astype(np.float64)
+        straddle = (R.min(axis=1) <= 0) & (R.max(axis=1) >= 0)
+        assert straddle.mean() > 0.9, f"stage {j}: test data should straddle zero"
+        lim = sf * (0.5 + 3 * 2.0 ** -11) * (1 + 2.0 ** -20)
+        worst = (np.abs(Rn).max(axis=1) / lim)[straddle].max()
+        assert worst <= 1.0, f"stage {j}: residual {worst:.4f} of the half-step bound"
+
+
+def pin_rrq_telescopes(impl, seed=73):
+    """The stages' dequantized values plus the final residual give back the weights up to
+    one binary32 rounding per stage: |w - sum_j s_j(q_j - z_j) - r_J| <= sum_j 2^-24 |r_j|
+    elementwise (each stage's subtraction is rounded once; the product is exact)."""
+    rng = np.random.default_rng(seed)
+    w = (rng.standard_normal((16, 256)) * 0.05).astype(np.float32)
+    stages = _rrq_stages(impl, w, 4)
+    total = np.zeros(w.size, np.float64)
+    bound = np.zeros(w.size, np.float64)
+    for r, codes, scale, zero, st, r_new in stages:
+        G = codes.size // GROUP
+        sf = np.asarray(scale, np.uint16).view(np.float16).astype(np.float64)
+        total += (sf[:, None] * (codes.reshape(G, GROUP).astype(np.float64) -
+                                 np.asarray(zero, np.float64)[:, None])).ravel()
+        bound += 2.0 ** -24 * np.abs(r_new.astype(np.float64).ravel())
+    r_last = stages[-1][5].astype(np.float64).ravel()
+    err = np.abs(w.astype(np.float64).ravel() - total - r_last)
+    assert (err <= bound * (1 + 1e-9) + 1e-300).all(), f"max excess {np.max(err - bound):.3e}"
+    # and the package converges: four 2-bit stages at least 3^3 times finer than the base
+    assert np.abs(r_last).max() * 27 <= np.abs(stages[0][5]).max()
+
+
+def pin_rrq_on_grid_is_exact(impl):
+    """Weights already on a 2-bit grid: the base reproduces them, the residual is exactly
+    zero, and the next stage sees a constant group (floored scale 2^-14, zero 0, codes 0)."""
+    s = np.float32(2.0 ** -4)
+    levels = np.array([-1, 0, 1, 2], np.float32) * s        # z = 1: codes 0..3
+    w = np.tile(levels, 16).reshape(1, GROUP).astype(np.float32)
+    codes, scale, zero, st, r = impl.rrq_stage(w, 2)
+    assert st == 0 and int(scale[0]) == 0x2C00 and int(zero[0]) == 1
+    assert np.array_equal(codes, np.tile(np.array([0, 1, 2, 3], np.uint8), 16))
+    assert np.array_equal(r, np.zeros_like(w))
+    codes1, scale1, zero1, st1, r1 = impl.rrq_stage(r, 2)
+    assert int(scale1[0]) == 0x0400 and int(zero1[0]) == 0 and not codes1.any()
+    assert np.array_equal(r1, r)
+
+
+def pin_rrq_base_is_the_2bit_quantizer(impl, seed=75):
+    """The first stage is the group quantizer at 2 bits (pinned above), and a flagged group
+    (a NaN) keeps its residual unchanged."""
+    rng = np.random.default_rng(seed)
+    w = (rng.standard_normal((4, 256)) * 0.03).astype(np.float32)
+    w[2, 70] = np.nan
+    codes, scale, zero, st, r = impl.rrq_stage(w, 2)
+    qc, qs, qz, qst = impl.quantize(w, np.full(w.size // GROUP, 2, np.uint8))
+    assert np.array_equal(codes, qc) and np.array_equal(scale, qs) and np.array_equal(zero, qz)
+    assert st == qst == 1
+    g = (2 * 256 + 70) // GROUP
+    assert np.array_equal(r.reshape(-1, GROUP)[g].view(np.uint32), w.reshape(-1, GROUP)[g].view(np.uint32))
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
