@@ -29,6 +29,7 @@ LIBCQ_UNITS = {
     "k_verify.cu": EXACT,
     "k_gemv.cu": [],
     "k_gemm.cu": [],
+    "k_rrq.cu": [],
 }
 SYNTH_UNITS = {"synth.cu": EXACT}
 

@@ -23,7 +23,8 @@ QSTATUS_NONFINITE, QSTATUS_RANGE, QSTATUS_BADBITS = 1, 2, 4
 # every symbol include/cq.h declares
 EXPORTS = ["cq_quantize", "cq_varbits_index", "cq_pack_varbits", "cq_unpack_varbits",
            "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemv_multi", "cq_dequant_gemm",
-           "cq_dequant_gemm_static", "cq_gemm_workspace", "cq_last_error", "cq_status_string"]
+           "cq_dequant_gemm_static", "cq_gemm_workspace", "cq_last_error", "cq_status_string", "cq_rrq_stage",
+           "cq_dequant_gemv_stages"]
 SYNTH_EXPORTS = ["cqs_normal_f32", "cqs_code_words", "cqs_scales", "cqs_zeros", "cqs_residual_bf16"]
 
 
@@ -61,6 +62,8 @@ def lib():
         L.cq_dequant_gemv_multi.argtypes = [p, i32, p, i32, i32, p, p]
         L.cq_dequant_gemm.argtypes = [p, p, i32, i32, p, p, C.c_size_t, p]
         L.cq_dequant_gemm_static.argtypes = [p, p, i32, i32, p, p]
+        L.cq_rrq_stage.argtypes = [p, i64, i64, i32, p, p, p, p, p]
+        L.cq_dequant_gemv_stages.argtypes = [p, i32, p, i32, i32, p, p]
         L.cq_gemm_workspace.argtypes = [i64, i64, i32]
         L.cq_gemm_workspace.restype = C.c_size_t
         L.cq_last_error.restype = C.c_char_p
@@ -68,7 +71,7 @@ def lib():
         L.cq_status_string.restype = C.c_char_p
         for name in ("cq_quantize", "cq_varbits_index", "cq_pack_varbits", "cq_unpack_varbits",
                      "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemv_multi",
-                     "cq_dequant_gemm", "cq_dequant_gemm_static"):
+                     "cq_dequant_gemm", "cq_dequant_gemm_static", "cq_rrq_stage", "cq_dequant_gemv_stages"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -196,6 +199,22 @@ def cq_dequant_gemv_multi(qws, x, ys, stream=None):
     m = x.shape[0] if x.dim() == 2 else 1
     _check(lib().cq_dequant_gemv_multi(C.cast(arr, C.c_void_p), len(structs), _ptr(x), _dtype_code(x), m,
                                        C.cast(yarr, C.c_void_p), _stream(stream)), "cq_dequant_gemv_multi")
+
+
+def cq_rrq_stage(r, bits, codes, scale, zero, status_word=None, stream=None):
+    """One recurrent-residual stage: quantize r at one width, replace r by what it misses."""
+    rows, cols = r.shape
+    _check(lib().cq_rrq_stage(_ptr(r), rows, cols, int(bits), _ptr(codes), _ptr(scale), _ptr(zero),
+                              _ptr(status_word), _stream(stream)), "cq_rrq_stage")
+
+
+def cq_dequant_gemv_stages(stages, x, y, stream=None):
+    """y = (sum of the stages' dequantized weights) x (see include/cq.h)."""
+    structs = [q.struct() for q in stages]
+    arr = (C.POINTER(cq_qweight) * len(structs))(*[C.pointer(st) for st in structs])
+    m = x.shape[0] if x.dim() == 2 else 1
+    _check(lib().cq_dequant_gemv_stages(C.cast(arr, C.c_void_p), len(structs), _ptr(x), _dtype_code(x), m, _ptr(y),
+                                        _stream(stream)), "cq_dequant_gemv_stages")
 
 
 def cq_gemm_workspace(rows, cols, m):

@@ -43,6 +43,8 @@ int sm_count() {
 
 namespace {
 
+static bool width_ok_host(int b) { return b == 1 || b == 2 || b == 4 || b == 8; }
+
 cq_status check_shape(int64_t rows, int64_t cols, const char *fn) {
   if (rows < 0 || cols < 0) return fail(CQ_ERR_SHAPE, "%s: negative shape %lld x %lld", fn, (long long)rows, (long long)cols);
   if (cols % kGroup) return fail(CQ_ERR_SHAPE, "%s: cols=%lld is not a multiple of 64", fn, (long long)cols);
@@ -113,6 +115,21 @@ cq_status cq_quantize(const float *w, int64_t rows, int64_t cols, const uint8_t 
     if (!aligned16(codes)) return fail(CQ_ERR_ALIGN, "%s: codes is not 16-byte aligned", fn);
   }
   return launch_quantize(w, G, bits, codes, scale, zero, status_word, reinterpret_cast<cudaStream_t>(stream));
+}
+
+cq_status cq_rrq_stage(float *r, int64_t rows, int64_t cols, int bits, uint8_t *codes, uint16_t *scale, uint8_t *zero,
+                       uint32_t *status_word, cq_stream_t stream) {
+  const char *fn = "cq_rrq_stage";
+  cq_status st = check_shape(rows, cols, fn);
+  if (st != CQ_OK) return st;
+  if (!width_ok_host(bits)) return fail(CQ_ERR_BITS, "%s: width %d is not 1, 2, 4 or 8", fn, bits);
+  const int64_t G = rows * (cols / kGroup);
+  if (G > 0) {
+    if (!r || !codes || !scale || !zero) return fail(CQ_ERR_ARG, "%s: NULL buffer", fn);
+    if (!aligned16(r)) return fail(CQ_ERR_ALIGN, "%s: r is not 16-byte aligned", fn);
+    if (!aligned16(codes)) return fail(CQ_ERR_ALIGN, "%s: codes is not 16-byte aligned", fn);
+  }
+  return launch_rrq_stage(r, G, bits, codes, scale, zero, status_word, reinterpret_cast<cudaStream_t>(stream));
 }
 
 cq_status cq_varbits_index(const uint8_t *bits, int64_t n_groups, uint32_t *offset, uint64_t *plane_bytes,
@@ -209,6 +226,24 @@ cq_status cq_dequant_gemv_multi(const cq_qweight *const *qws, int count, const v
                   (long long)qws[i]->cols, (long long)qws[0]->cols);
   }
   return launch_gemv_multi(qws, count, x, x_dtype, m, ys, reinterpret_cast<cudaStream_t>(stream));
+}
+
+cq_status cq_dequant_gemv_stages(const cq_qweight *const *stages, int count, const void *x, cq_dtype x_dtype, int m,
+                                 float *y, cq_stream_t stream) {
+  const char *fn = "cq_dequant_gemv_stages";
+  if (count < 1 || count > kMaxRrqStages)
+    return fail(CQ_ERR_ARG, "%s: %d stages, 1 to %d supported", fn, count, kMaxRrqStages);
+  if (!stages) return fail(CQ_ERR_ARG, "%s: NULL stage list", fn);
+  for (int j = 0; j < count; ++j) {
+    if (!stages[j]) return fail(CQ_ERR_ARG, "%s: stage %d is NULL", fn, j);
+    cq_status st = check_matmul(stages[j], x, x_dtype, m, y, 8, fn);
+    if (st != CQ_OK) return st;
+    if (stages[j]->rows != stages[0]->rows || stages[j]->cols != stages[0]->cols)
+      return fail(CQ_ERR_SHAPE, "%s: stage %d is %lldx%lld, stage 0 is %lldx%lld", fn, j, (long long)stages[j]->rows,
+                  (long long)stages[j]->cols, (long long)stages[0]->rows, (long long)stages[0]->cols);
+    if (stages[j]->residual) return fail(CQ_ERR_UNSUPPORTED, "%s: stage %d has a residual", fn, j);
+  }
+  return launch_gemv_stages(stages, count, x, x_dtype, m, y, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t cq_gemm_workspace(int64_t rows, int64_t cols, int m) {

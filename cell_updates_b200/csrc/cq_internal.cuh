@@ -40,6 +40,11 @@ cq_status launch_gemv_multi(const cq_qweight *const *qws, int count, const void 
 cq_status launch_gemm_tc(const cq_qweight &qw, const void *x, int m, float *y, void *ws,
                          size_t ws_bytes, cudaStream_t s);
 size_t gemm_tc_workspace(int64_t rows, int64_t cols, int m);
+cq_status launch_rrq_stage(float *r, int64_t G, int b, uint8_t *codes, uint16_t *scale, uint8_t *zero,
+                           uint32_t *status, cudaStream_t s);
+constexpr int kMaxRrqStages = 8;
+cq_status launch_gemv_stages(const cq_qweight *const *stages, int count, const void *x, cq_dtype xdt, int m,
+                             float *y, cudaStream_t s);
 bool gemm_tc_eligible(const cq_qweight &qw, cq_dtype xdt, int m);
 
 // ---- device-side helpers -------------------------------------------------------------

@@ -27,9 +27,17 @@ constexpr int kSmem = 1024 + kWarps * kStages * kTileBytes + kWarps * kStages * 
 // group's 16-byte chunks without bank conflicts (chunk c of row r sits at c ^ (r & 7)). Once
 // the tile is in registers the warp requests its next tile, which streams in while it computes
 // (16 warps per SM: measured faster than fewer warps with deeper rings).
+//
+// With kResid (one stage of recurrent residual quantization, [RRQ] the 2512.18934 listing
+// page, "Recurrent Residual Quantization" abstract: 2-bit round-to-nearest residual
+// corrections stacked on a 2-bit base) the thread then re-reads its group (L2-resident: the
+// tile was just loaded) and writes back, in place, what the stage does not represent:
+// r <- RN32(r - s (q - z)), the product exact; a flagged group keeps its values. w is then
+// read and written by the same thread only, reads first, so it carries no __restrict__.
+template <bool kResid>
 __global__ void __launch_bounds__(kThreads, 1)
-quantize_kernel(const __grid_constant__ CUtensorMap tm_w, const float *__restrict__ w, int64_t G,
-                const uint8_t *__restrict__ bits, uint8_t *__restrict__ codes, uint16_t *__restrict__ scale,
+quantize_kernel(const __grid_constant__ CUtensorMap tm_w, float *w, int64_t G, const uint8_t *__restrict__ bits,
+                int uniform_b, uint8_t *__restrict__ codes, uint16_t *__restrict__ scale,
                 uint8_t *__restrict__ zero, uint32_t *__restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -99,7 +107,7 @@ quantize_kernel(const __grid_constant__ CUtensorMap tm_w, const float *__restric
     }
     if (++slot == kStages) { slot = 0; phase ^= 1u; }
     const bool finite = isfinite(lo) && isfinite(hi);
-    const int b = (bits && valid) ? static_cast<int>(__ldg(bits + g)) : 4;
+    const int b = (bits && valid) ? static_cast<int>(__ldg(bits + g)) : uniform_b;
     const bool width_good = width_ok(b);
     const int L = width_good ? (1 << b) - 1 : 15;
     // s = RN_fp16(RN32(RN32(wmax - wmin) / L)), floored at the smallest normal fp16
@@ -137,7 +145,7 @@ quantize_kernel(const __grid_constant__ CUtensorMap tm_w, const float *__restric
       if (need_exact) {
         const float *wg = w + (valid ? g : 0) * kGroup;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) v[j] = rintf(__fdiv_rn(__ldg(wg + j), sf));   // unrolled: v stays in registers
+        for (int j = 0; j < 64; ++j) v[j] = rintf(__fdiv_rn(wg[j], sf));   // unrolled: v stays in registers
       }
     }
     const bool bad = !width_good || !finite || overflow;
@@ -155,12 +163,24 @@ quantize_kernel(const __grid_constant__ CUtensorMap tm_w, const float *__restric
         for (int k = 0; k < 4; ++k) {
           uint32_t e4[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            e4[e] = __float_as_uint(fminf(fmaxf(__fadd_rn(v[16 * c + 4 * k + e], kb), 8388608.0f), kl));
+          for (int e = 0; e < 4; ++e) {
+            const float cl = fminf(fmaxf(__fadd_rn(v[16 * c + 4 * k + e], kb), 8388608.0f), kl);
+            e4[e] = __float_as_uint(cl);
+            if (kResid) v[16 * c + 4 * k + e] = __fsub_rn(cl, kb);   // q - z, exact (both in [2^23, 2^24))
+          }
           const uint32_t word = __byte_perm(__byte_perm(e4[0], e4[1], 0x0040), __byte_perm(e4[2], e4[3], 0x0040), 0x5410);
           wd[k] = bad ? 0u : word;
         }
         __stcs(dst + c, make_uint4(wd[0], wd[1], wd[2], wd[3]));
+      }
+      if (kResid && !bad) {
+        float4 *rg = reinterpret_cast<float4 *>(w + g * kGroup);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float4 o = rg[c];
+          __stcs(rg + c, make_float4(__fsub_rn(o.x, __fmul_rn(sf, v[4 * c])), __fsub_rn(o.y, __fmul_rn(sf, v[4 * c + 1])),
+                                     __fsub_rn(o.z, __fmul_rn(sf, v[4 * c + 2])), __fsub_rn(o.w, __fmul_rn(sf, v[4 * c + 3]))));
+        }
       }
       scale[g] = bad ? 0 : s16;
       zero[g] = bad ? 0 : static_cast<uint8_t>(z);
@@ -175,18 +195,17 @@ quantize_kernel(const __grid_constant__ CUtensorMap tm_w, const float *__restric
   if (lane == 0 && flags && status) atomicOr(status, flags);
 }
 
-}  // namespace
-
-cq_status launch_quantize(const float *w, int64_t G, const uint8_t *bits, uint8_t *codes,
-                          uint16_t *scale, uint8_t *zero, uint32_t *status, cudaStream_t s) {
+template <bool kResid>
+cq_status launch_quantize_impl(float *w, int64_t G, const uint8_t *bits, int uniform_b, uint8_t *codes,
+                               uint16_t *scale, uint8_t *zero, uint32_t *status, cudaStream_t s, const char *who) {
   if (status) {
-    cq_status st = cuda_check(cudaMemsetAsync(status, 0, sizeof(uint32_t), s), "cq_quantize: clear status");
+    cq_status st = cuda_check(cudaMemsetAsync(status, 0, sizeof(uint32_t), s), who);
     if (st != CQ_OK) return st;
   }
   if (G == 0) return CQ_OK;
   auto encode = encode_fn();
-  if (!encode) return fail(CQ_ERR_CUDA, "cq_quantize: cuTensorMapEncodeTiled unavailable");
-  if (G > (int64_t(1) << 31) - kTileGroups) return fail(CQ_ERR_RANGE, "cq_quantize: more than 2^31 groups");
+  if (!encode) return fail(CQ_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable", who);
+  if (G > (int64_t(1) << 31) - kTileGroups) return fail(CQ_ERR_RANGE, "%s: more than 2^31 groups", who);
   CUtensorMap tm;
   cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(G)};
   cuuint64_t strides[1] = {64 * sizeof(float)};
@@ -195,16 +214,30 @@ cq_status launch_quantize(const float *w, int64_t G, const uint8_t *bits, uint8_
   CUresult r = encode(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(w), dims, strides, box, es,
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(CQ_ERR_CUDA, "cq_quantize: weight tensor map (%d)", static_cast<int>(r));
-  cq_status st = cuda_check(cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem),
-                            "cq_quantize: shared memory attribute");
+  if (r != CUDA_SUCCESS) return fail(CQ_ERR_CUDA, "%s: weight tensor map (%d)", who, static_cast<int>(r));
+  cq_status st = cuda_check(cudaFuncSetAttribute(quantize_kernel<kResid>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kSmem),
+                            who);
   if (st != CQ_OK) return st;
   const int64_t tiles = (G + kTileGroups - 1) / kTileGroups;
   const int64_t need = (tiles + kWarps - 1) / kWarps;
   const int64_t cap = sm_count();
   const int blocks = static_cast<int>(need < cap ? need : cap);
-  quantize_kernel<<<blocks, kThreads, kSmem, s>>>(tm, w, G, bits, codes, scale, zero, status);
-  return launch_check("cq_quantize");
+  quantize_kernel<kResid><<<blocks, kThreads, kSmem, s>>>(tm, w, G, bits, uniform_b, codes, scale, zero, status);
+  return launch_check(who);
+}
+
+}  // namespace
+
+cq_status launch_quantize(const float *w, int64_t G, const uint8_t *bits, uint8_t *codes,
+                          uint16_t *scale, uint8_t *zero, uint32_t *status, cudaStream_t s) {
+  // the plain quantizer only reads w
+  return launch_quantize_impl<false>(const_cast<float *>(w), G, bits, 4, codes, scale, zero, status, s, "cq_quantize");
+}
+
+cq_status launch_rrq_stage(float *r, int64_t G, int b, uint8_t *codes, uint16_t *scale, uint8_t *zero,
+                           uint32_t *status, cudaStream_t s) {
+  return launch_quantize_impl<true>(r, G, nullptr, b, codes, scale, zero, status, s, "cq_rrq_stage");
 }
 
 }  // namespace cq

@@ -104,3 +104,31 @@ def gemm(qw, x, workspace=None, stream=None):
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     cq.cq_dequant_gemm(qw, x, y, workspace if need else None, stream)
     return y
+
+
+def rrq_build(w, n_stages, bits=2, stream=None):
+    """Recurrent residual quantization of fp32 w [rows, cols] (left unchanged): n_stages
+    stages of width `bits`, each packed -> (list of QWeight, statuses, final residual)."""
+    rows, cols = w.shape
+    G = rows * cols // GROUP
+    dev = w.device
+    r = w.clone()
+    width = torch.full((G,), bits, dtype=torch.uint8, device=dev)
+    offset, pb = varbits_index(width, stream)
+    stages, statuses = [], []
+    for _ in range(n_stages):
+        codes = empty_u8(rows * cols, dev)
+        scale = torch.empty(G, dtype=torch.int16, device=dev)
+        zero = empty_u8(G, dev)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        cq.cq_rrq_stage(r, bits, codes, scale, zero, status, stream)
+        planes = pack(codes, rows, cols, width, offset, pb, stream)
+        stages.append(cq.QWeight(rows, cols, planes, scale, zero, width, offset))
+        statuses.append(status)
+    return stages, statuses, r
+
+
+def gemv_stages(stages, x, stream=None):
+    y = torch.empty((x.shape[0], stages[0].rows), dtype=torch.float32, device=x.device)
+    cq.cq_dequant_gemv_stages(stages, x, y, stream)
+    return y

@@ -102,6 +102,33 @@ cq_status cq_quantize(const float *w, int64_t rows, int64_t cols, const uint8_t 
                       cq_stream_t stream);
 
 /*
+ * cq_rrq_stage -- one stage of Recurrent Residual Quantization ([RRQ] the listing page
+ * thelatestinai.com/papers/2512.18934, "Recurrent Residual Quantization" abstract: a 2-bit
+ * round-to-nearest base plus 2-bit round-to-nearest residual corrections stacked to 4, 6 and
+ * 8 bits, so one artifact holds several precisions). The running residual r ([rows, cols]
+ * fp32, 16-byte aligned; the weights themselves for the first stage) is quantized exactly as
+ * cq_quantize does with one width `bits` (1, 2, 4 or 8) for every group, then replaced in
+ * place by what the stage does not represent: r <- RN32(r - s*(q - z)) with the stored s, z
+ * and codes (the product is exact); a flagged group keeps its r. codes/scale/zero/status_word
+ * as for cq_quantize. Calling it J+1 times (bits = 2) on the same buffer yields the stages of a
+ * 2(J+1)-bit model; pack each stage with cq_pack_varbits (a width map of `bits`).
+ * Errors: CQ_ERR_SHAPE (cols % 64), CQ_ERR_BITS (width), CQ_ERR_ARG (NULL), CQ_ERR_ALIGN.
+ */
+cq_status cq_rrq_stage(float *r, int64_t rows, int64_t cols, int bits, uint8_t *codes, uint16_t *scale,
+                       uint8_t *zero, uint32_t *status_word, cq_stream_t stream);
+
+/*
+ * cq_dequant_gemv_stages -- the multiply over an RRQ stage stack ([RRQ] as above): y[m, rows]
+ * (fp32, overwritten) = sum over k of (sum over stages j of s_j (q_j - z_j)) * x[m, k], for
+ * 1 <= count <= 8 stages of the same shape, each fixed-4 or with a per-group width map, none
+ * with a residual (CQ_ERR_UNSUPPORTED), 1 <= m <= 8, x fp32 or bf16 (16-byte aligned). The
+ * stage sum of a weight is formed in fp32 before the product; fp32 accumulation.
+ * Errors: CQ_ERR_ARG (count, NULL, m, dtype), CQ_ERR_SHAPE (unequal shapes), CQ_ERR_ALIGN.
+ */
+cq_status cq_dequant_gemv_stages(const cq_qweight *const *stages, int count, const void *x, cq_dtype x_dtype,
+                                 int m, float *y, cq_stream_t stream);
+
+/*
  * cq_varbits_index -- [VBQ] codes stored bit-packed at their group widths: builds offset[G] (byte
  * offsets as in cq_qweight) and plane_bytes[4] (device, uint64: bytes needed by each plane).
  * bits: [G]. Device-side, widths outside {1,2,4,8} count as width 0 (offset 0, no bytes);

@@ -71,6 +71,18 @@ def test_host_validation_rejects_bad_arguments():
     assert L.cq_dequant_gemv_multi(C.cast(qws, C.c_void_p), 2, p, 1, 1, C.cast(ys, C.c_void_p), None) == 2  # unequal cols
     assert L.cq_dequant_gemv_multi(None, 2, p, 1, 1, C.cast(ys, C.c_void_p), None) == 1                    # NULL list
     assert L.cq_dequant_gemv_multi(None, 0, p, 1, 1, None, None) == 0                                      # nothing to do
+    # recurrent residual quantization
+    assert L.cq_rrq_stage(p, 4, 64, 3, p, p, p, None, None) == 3             # width 3
+    assert L.cq_rrq_stage(p, 4, 96, 2, p, p, p, None, None) == 2             # cols % 64
+    assert L.cq_rrq_stage(C.c_void_p(8), 4, 64, 2, p, p, p, None, None) == 4  # misaligned r
+    assert L.cq_rrq_stage(None, 4, 64, 2, p, p, p, None, None) == 1          # NULL r
+    assert L.cq_dequant_gemv_stages(C.cast(qws, C.c_void_p), 0, p, 1, 1, p, None) == 1   # no stages
+    assert L.cq_dequant_gemv_stages(C.cast(qws, C.c_void_p), 9, p, 1, 1, p, None) == 1   # too many
+    assert L.cq_dequant_gemv_stages(C.cast(qws, C.c_void_p), 2, p, 1, 1, p, None) == 2   # unequal shapes
+    qw.residual = 16
+    one = (C.POINTER(cq.cq_qweight) * 1)(C.pointer(qw))
+    assert L.cq_dequant_gemv_stages(C.cast(one, C.c_void_p), 1, p, 1, 1, p, None) == 8   # residual
+    qw.residual = None
 
 
 def test_missing_library_fails_loudly(monkeypatch):
