@@ -315,6 +315,45 @@ def isolated_components(torch, cq, ops, device, peaks, stream):
     del layers, stack
     torch.cuda.empty_cache()
     out["cellfill_stack"] = cellfill_stack_verify(torch, cq, ops, synth_module(), device, peaks, stream)
+    out["rrq"] = rrq_components(torch, cq, ops, device, peaks, stream)
+    return out
+
+
+def rrq_components(torch, cq, ops, device, peaks, stream):
+    """Recurrent residual quantization on the config's 11008x4096 shape (4 two-bit stages =
+    the 8-bit model): one stage (quantize the fp32 residual, write codes, scales, zero points
+    and the new residual: 9 + 3/64 B per weight), and the stage-stack GEMV at m=1 over 1, 2
+    and 4 stages (per stage 0.25 B codes + 3/64 B scale/zero + 5/64 B width map and offset)."""
+    N, K = 11008, 4096
+    G = N * K // GROUP
+    w = torch.randn(N, K, device=device) * 0.02
+    stages, _, _ = ops.rrq_build(w, 4)
+    r = w.clone()
+    codes = torch.empty(N * K, dtype=torch.uint8, device=device)
+    sc = torch.empty(G, dtype=torch.int16, device=device)
+    zr = torch.empty(G, dtype=torch.uint8, device=device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        cq.cq_rrq_stage(r, 2, codes, sc, zr, None, stream)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            cq.cq_rrq_stage(r, 2, codes, sc, zr, None, stream)
+    t = time_graph(torch, g, 10, stream)
+    b = N * K * 9 + G * 3
+    out = {"shape": f"{N}x{K}", "stage": {"us": t * 1e3, "GBps": b / t / 1e6, "frac_hbm": b / t / 1e6 / peaks["hbm_gbs"]}}
+    x = torch.randn(1, K, device=device).to(torch.bfloat16)
+    y = torch.empty(1, N, device=device)
+    for n in (1, 2, 4):
+        gs = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(gs, stream=stream):
+                cq.cq_dequant_gemv_stages(stages[:n], x, y, stream)
+        t = time_graph(torch, gs, 10, stream)
+        b = n * (N * K // 4 + G * 8)
+        out[f"gemv_m1_{n}_stages"] = {"us": t * 1e3, "GBps": b / t / 1e6, "frac_hbm": b / t / 1e6 / peaks["hbm_gbs"]}
+        del gs
+    del stages, w, r, g
+    torch.cuda.empty_cache()
     return out
 
 
