@@ -9,8 +9,9 @@ configuration (three weight matrices 4096x4096, 11008x4096, 4096x11008, drawn as
     -> requant-verify without it (revocation) -> dequant-GEMV at batch 1 (decode)
     -> dequant-GEMM at batch 64
 
-for each matrix.  The step is captured once as a CUDA graph and replayed; per-kernel
-durations come from event-record nodes inside the same graph (the timed region).
+for each matrix (each row runs over the three matrices before the next row starts).  K steps
+are captured as one CUDA graph and replayed for the timed region; per-row durations come from a
+second K-step graph with an event pair around each row's three launches, replayed after it.
 Printed: one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cq|reference]
@@ -174,36 +175,29 @@ class Workload:
         torch.cuda.synchronize()
 
     def step(self, stream, marks=None):
-        """Enqueue one step. marks[(matrix, kernel)] = (start, end) external events: recorded
-        inside a graph capture they become event nodes that time each launch on replay."""
+        """Enqueue one step: each row of the path over the three matrices, then the next row
+        (every matrix keeps its own order quantize -> pack -> project -> verify -> revoke ->
+        GEMV -> GEMM). marks[kernel] = (start, end) external events around a row's three
+        launches: recorded inside a graph capture they become event nodes that time the row on
+        replay (one pair per row keeps their own cost out of the launches they time)."""
         cq = self.cq
-        for mi, m in enumerate(self.mats):
-            qw = m["qw"]
-            def mark(name, which):
-                if marks is not None:
-                    marks[(mi, name)][which].record(stream)
-            mark("quantize", 0)
-            cq.cq_quantize(m["w"], None, m["codes"], qw.scale, qw.zero, m["status"], stream)
-            mark("quantize", 1)
-            mark("pack", 0)
-            cq.cq_pack_varbits(m["codes"], m["n"] // GROUP, None, None, qw.planes, stream)
-            mark("pack", 1)
-            mark("project", 0)
-            cq.cq_project_residual(m["r"], qw.scale, m["nclamp"], stream)
-            mark("project", 1)
-            qwr = qw.with_residual(m["r"])
-            mark("verify", 0)
-            cq.cq_requant_verify(qwr, 0, m["n"], m["mism"], m["first"], None, stream)
-            mark("verify", 1)
-            mark("revoke_verify", 0)
-            cq.cq_requant_verify(qw, 0, m["n"], m["mism0"], m["first0"], None, stream)
-            mark("revoke_verify", 1)
-            mark("gemv", 0)
-            cq.cq_dequant_gemv(qw, m["x"], m["y"], stream)
-            mark("gemv", 1)
-            mark("gemm", 0)
-            cq.cq_dequant_gemm(qw, m["X"], m["Y"], m["ws"], stream)
-            mark("gemm", 1)
+
+        def row(name, fn):
+            if marks is not None:
+                marks[name][0].record(stream)
+            for m in self.mats:
+                fn(m, m["qw"])
+            if marks is not None:
+                marks[name][1].record(stream)
+
+        row("quantize", lambda m, qw: cq.cq_quantize(m["w"], None, m["codes"], qw.scale, qw.zero, m["status"], stream))
+        row("pack", lambda m, qw: cq.cq_pack_varbits(m["codes"], m["n"] // GROUP, None, None, qw.planes, stream))
+        row("project", lambda m, qw: cq.cq_project_residual(m["r"], qw.scale, m["nclamp"], stream))
+        row("verify", lambda m, qw: cq.cq_requant_verify(qw.with_residual(m["r"]), 0, m["n"], m["mism"], m["first"],
+                                                         None, stream))
+        row("revoke_verify", lambda m, qw: cq.cq_requant_verify(qw, 0, m["n"], m["mism0"], m["first0"], None, stream))
+        row("gemv", lambda m, qw: cq.cq_dequant_gemv(qw, m["x"], m["y"], stream))
+        row("gemm", lambda m, qw: cq.cq_dequant_gemm(qw, m["X"], m["Y"], m["ws"], stream))
 
     def n_weights(self):
         return sum(m["n"] for m in self.mats)
@@ -424,9 +418,9 @@ def run_gpu(args, rank, world, local_rank):
     wl = Workload(torch, cq, ops, synth, device, seed_base=1 + 100000 * rank)
     stream = torch.cuda.Stream(device)
     # eager run, then a one-step graph for the warm-up, a K-step graph for the timed region,
-    # and a second K-step graph whose launches are each bracketed by their own event pair: it
-    # is replayed after the timed region for the per-kernel breakdown only (event nodes between
-    # the launches add time of their own, so they stay out of the headline)
+    # and a second K-step graph with an event pair around each row's three launches: it is
+    # replayed after the timed region for the per-row breakdown only (event nodes add time of
+    # their own, so they stay out of the headline)
     with torch.cuda.stream(stream):
         wl.step(stream)
     torch.cuda.synchronize()
@@ -435,9 +429,9 @@ def run_gpu(args, rank, world, local_rank):
         with torch.cuda.graph(g1, stream=stream):
             wl.step(stream)
     launches_per_step = count_kernel_nodes(g1)
-    marks = [{(mi, k): (torch.cuda.Event(enable_timing=True, external=True),
-                        torch.cuda.Event(enable_timing=True, external=True))
-              for mi in range(len(wl.mats)) for k in KERNELS} for _ in range(args.steps)]
+    marks = [{k: (torch.cuda.Event(enable_timing=True, external=True),
+                  torch.cuda.Event(enable_timing=True, external=True))
+              for k in KERNELS} for _ in range(args.steps)]
     gK = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         with torch.cuda.graph(gK, stream=stream):
@@ -468,7 +462,7 @@ def run_gpu(args, rank, world, local_rank):
         dist.barrier()
     clk = clocks.stop()
     t_step = start.elapsed_time(end) / args.steps
-    # the per-kernel breakdown: the same K steps with an event pair around every launch
+    # the per-row breakdown: the same K steps with an event pair around each row
     with torch.cuda.stream(stream):
         start.record(stream)
         gM.replay()
@@ -477,7 +471,7 @@ def run_gpu(args, rank, world, local_rank):
     t_marked = start.elapsed_time(end) / args.steps
     per_kernel = {k: 0.0 for k in KERNELS}           # ms summed over every launch
     for mk in marks:
-        for (mi, k), (a, b) in mk.items():
+        for k, (a, b) in mk.items():
             per_kernel[k] += a.elapsed_time(b)
     t_step = max_over_ranks(t_step, dist, device)
     checks = [int(m["mism"].item()) for m in wl.mats] + [int(m["mism0"].item()) for m in wl.mats] + \
