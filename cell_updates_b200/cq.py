@@ -24,7 +24,7 @@ QSTATUS_NONFINITE, QSTATUS_RANGE, QSTATUS_BADBITS = 1, 2, 4
 EXPORTS = ["cq_quantize", "cq_varbits_index", "cq_pack_varbits", "cq_unpack_varbits",
            "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemv_multi", "cq_dequant_gemm",
            "cq_dequant_gemm_static", "cq_gemm_workspace", "cq_last_error", "cq_status_string", "cq_rrq_stage",
-           "cq_dequant_gemv_stages"]
+           "cq_dequant_gemv_stages", "cq_requant_verify_pair"]
 SYNTH_EXPORTS = ["cqs_normal_f32", "cqs_code_words", "cqs_scales", "cqs_zeros", "cqs_residual_bf16"]
 
 
@@ -63,6 +63,7 @@ def lib():
         L.cq_dequant_gemm.argtypes = [p, p, i32, i32, p, p, C.c_size_t, p]
         L.cq_dequant_gemm_static.argtypes = [p, p, i32, i32, p, p]
         L.cq_rrq_stage.argtypes = [p, i64, i64, i32, p, p, p, p, p]
+        L.cq_requant_verify_pair.argtypes = [p, i64, i64, p, p, p, p, p, p]
         L.cq_dequant_gemv_stages.argtypes = [p, i32, p, i32, i32, p, p]
         L.cq_gemm_workspace.argtypes = [i64, i64, i32]
         L.cq_gemm_workspace.restype = C.c_size_t
@@ -71,7 +72,8 @@ def lib():
         L.cq_status_string.restype = C.c_char_p
         for name in ("cq_quantize", "cq_varbits_index", "cq_pack_varbits", "cq_unpack_varbits",
                      "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemv_multi",
-                     "cq_dequant_gemm", "cq_dequant_gemm_static", "cq_rrq_stage", "cq_dequant_gemv_stages"):
+                     "cq_dequant_gemm", "cq_dequant_gemm_static", "cq_rrq_stage", "cq_dequant_gemv_stages",
+                     "cq_requant_verify_pair"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -199,6 +201,13 @@ def cq_dequant_gemv_multi(qws, x, ys, stream=None):
     m = x.shape[0] if x.dim() == 2 else 1
     _check(lib().cq_dequant_gemv_multi(C.cast(arr, C.c_void_p), len(structs), _ptr(x), _dtype_code(x), m,
                                        C.cast(yarr, C.c_void_p), _stream(stream)), "cq_dequant_gemv_multi")
+
+
+def cq_requant_verify_pair(qw, first_w, n_w, mism, first_bad, mism0, first0, group_flags=None, stream=None):
+    """Verify with the residual and without it (revocation) in one pass (see include/cq.h)."""
+    s = qw.struct()
+    _check(lib().cq_requant_verify_pair(C.byref(s), first_w, n_w, _ptr(mism), _ptr(first_bad), _ptr(mism0),
+                                        _ptr(first0), _ptr(group_flags), _stream(stream)), "cq_requant_verify_pair")
 
 
 def cq_rrq_stage(r, bits, codes, scale, zero, status_word=None, stream=None):

@@ -193,6 +193,23 @@ cq_status cq_requant_verify(const cq_qweight *qw, int64_t first_w, int64_t n_w, 
   return launch_verify(*qw, first_w, n_w, mismatches, first_bad, group_flags, reinterpret_cast<cudaStream_t>(stream));
 }
 
+cq_status cq_requant_verify_pair(const cq_qweight *qw, int64_t first_w, int64_t n_w, uint64_t *mismatches,
+                                 int64_t *first_bad, uint64_t *revoke_mismatches, int64_t *revoke_first_bad,
+                                 uint32_t *group_flags, cq_stream_t stream) {
+  const char *fn = "cq_requant_verify_pair";
+  cq_status st = check_qweight(qw, fn, true);
+  if (st != CQ_OK) return st;
+  if (!qw->residual && qw->rows * qw->cols) return fail(CQ_ERR_ARG, "%s: the pair needs a residual", fn);
+  if (!mismatches || !first_bad || !revoke_mismatches || !revoke_first_bad)
+    return fail(CQ_ERR_ARG, "%s: a result pointer is NULL", fn);
+  const int64_t total = qw->rows * qw->cols;
+  if (first_w < 0 || n_w < 0 || first_w % kGroup || n_w % kGroup || first_w > total || n_w > total - first_w)
+    return fail(CQ_ERR_SHAPE, "%s: chunk [%lld, +%lld) is not whole groups inside the %lld weights", fn,
+                (long long)first_w, (long long)n_w, (long long)total);
+  return launch_verify_pair(*qw, first_w, n_w, mismatches, first_bad, revoke_mismatches, revoke_first_bad, group_flags,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
 static cq_status check_matmul(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m, float *y,
                               int max_m, const char *fn) {
   cq_status st = check_qweight(qw, fn, false);

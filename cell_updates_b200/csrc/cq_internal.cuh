@@ -33,6 +33,8 @@ cq_status launch_project(void *r, cq_dtype dt, const uint16_t *scale, int64_t n,
                          uint64_t *n_clamped, cudaStream_t s);
 cq_status launch_verify(const cq_qweight &qw, int64_t first_w, int64_t n_w, uint64_t *mism,
                         int64_t *first_bad, uint32_t *flags, cudaStream_t s);
+cq_status launch_verify_pair(const cq_qweight &qw, int64_t first_w, int64_t n_w, uint64_t *mism, int64_t *first_bad,
+                             uint64_t *mism0, int64_t *first0, uint32_t *flags, cudaStream_t s);
 cq_status launch_gemv(const cq_qweight &qw, const void *x, cq_dtype xdt, int m, float *y,
                       cudaStream_t s);
 cq_status launch_gemv_multi(const cq_qweight *const *qws, int count, const void *x, cq_dtype xdt, int m,

@@ -18,7 +18,7 @@
 // lane's b bytes of its group (per-group widths), plus 16 bytes of bf16 residual or 32
 // of fp32. Mismatch counts are warp-aggregated; the smallest index and the per-group
 // flags are only touched when a warp sees a mismatch.
-#include "cq_internal.cuh"
+#include "cq_async.cuh"
 
 namespace cq {
 namespace {
@@ -37,7 +37,22 @@ struct VerifyArgs {
   unsigned long long *mism;
   unsigned long long *first_bad;   // int64 in the ABI; -1 is the all-ones pattern
   uint32_t *flags;
+  unsigned long long *mism0;       // pair mode: the same check without the residual (revocation)
+  unsigned long long *first0;
 };
+
+// the results start at 0 mismatches and first index -1; one thread, then the verify grid
+// (launched as its programmatic dependent) may start
+__global__ void verify_clear_kernel(unsigned long long *mism, unsigned long long *first,
+                                    unsigned long long *mism0, unsigned long long *first0) {
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    *mism = 0ull;
+    *first = ~0ull;
+    if (mism0) *mism0 = 0ull;
+    if (first0) *first0 = ~0ull;
+  }
+}
 
 enum RKind { kNoR = 0, kF32 = 1, kBF16 = 2 };
 
@@ -75,6 +90,7 @@ __device__ __forceinline__ bool exact_match(int q, int z, int L, float sf, float
 
 template <bool VAR, int RK>
 __global__ void __launch_bounds__(kThreads) verify_kernel(VerifyArgs a) {
+  pdl_wait();                                    // inputs and cleared results from earlier work
   const int lane = threadIdx.x & 31;
   uint32_t count = 0;
   int64_t first = INT64_MAX;
@@ -180,18 +196,21 @@ __device__ __forceinline__ float max_nan_abs(float m, float d) {
 // -(2^23 + q) as a float, for a nibble q already in the low bits
 __device__ __forceinline__ float neg_magic_code(uint32_t bits) { return __uint_as_float(0xCB000000u | bits); }
 
-template <int RK>
+// kPair: the same pass also checks the artifact without the residual (revocation) from the
+// codes and metadata already in registers; its certificate is that of the no-residual case
+template <int RK, bool kPair>
 __global__ void __launch_bounds__(kThreads) verify4_kernel(VerifyArgs a) {
+  pdl_wait();                                    // inputs and cleared results from earlier work
   const int lane = threadIdx.x & 31;
-  uint32_t count = 0;
-  int64_t first = INT64_MAX;
+  uint32_t count = 0, count0 = 0;
+  int64_t first = INT64_MAX, first0 = INT64_MAX;
   const int64_t n32 = a.n_units >> 2;            // units of 32 weights
   const int64_t step = static_cast<int64_t>(gridDim.x) * kThreads;
   const int64_t base_u = blockIdx.x * static_cast<int64_t>(kThreads) + (threadIdx.x & ~31);
   for (int64_t u0 = base_u; u0 < n32; u0 += step) {
     const int64_t u = u0 + lane;
     const bool valid = u < n32;
-    uint32_t bad = 0;
+    uint32_t bad = 0, bad0 = 0;
     int64_t i0 = 0;
     int64_t g = 0;
     if (valid) {
@@ -270,6 +289,29 @@ __global__ void __launch_bounds__(kThreads) verify4_kernel(VerifyArgs a) {
           if (!exact_match<RK != kNoR>(q, z, 15, sf, r)) bad |= 1u << j;
         }
       }
+      if (kPair) {
+        uint32_t qor = words[0] | words[1] | words[2] | words[3];
+        qor = (qor | (qor >> 4)) & 0x0F0F0F0Fu;
+        qor |= qor >> 16;
+        qor = (qor | (qor >> 8)) & 0xFu;
+        const float kmax = static_cast<float>(max(static_cast<int>(qor) - z, z));
+        const float m0 = __fmul_rn(__fmul_rn(kmax, fabsf(__fmaf_rn(sf, rc, -1.0f))), 1.0f + 0x1p-22f);
+        if (!(m0 < 0.49951171875f)) {
+#pragma unroll 1
+          for (int j = 0; j < 32; ++j) {
+            const int64_t i = i0 + j;
+            const int q = static_cast<int>((__ldg(a.plane[2] + (i >> 1)) >> (4 * (i & 1))) & 0xFu);
+            if (!exact_match<false>(q, z, 15, sf, 0.0f)) bad0 |= 1u << j;
+          }
+        }
+      }
+    }
+    if (kPair && __ballot_sync(0xffffffffu, bad0 != 0)) {
+      count0 += __popc(bad0);
+      if (bad0) {
+        const int64_t fi = i0 + (__ffs(bad0) - 1);
+        first0 = fi < first0 ? fi : first0;
+      }
     }
     const uint32_t any = __ballot_sync(0xffffffffu, bad != 0);
     if (any) {
@@ -288,6 +330,11 @@ __global__ void __launch_bounds__(kThreads) verify4_kernel(VerifyArgs a) {
   count = __reduce_add_sync(0xffffffffu, count);
   if (lane == 0 && count) atomicAdd(a.mism, static_cast<unsigned long long>(count));
   if (first != INT64_MAX) atomicMin(a.first_bad, static_cast<unsigned long long>(first));
+  if (kPair) {
+    count0 = __reduce_add_sync(0xffffffffu, count0);
+    if (lane == 0 && count0) atomicAdd(a.mism0, static_cast<unsigned long long>(count0));
+    if (first0 != INT64_MAX) atomicMin(a.first0, static_cast<unsigned long long>(first0));
+  }
 }
 
 // Revocation (no residual) of fixed-4 weights moves only 0.55 bytes per weight, so a lane
@@ -296,6 +343,7 @@ __global__ void __launch_bounds__(kThreads) verify4_kernel(VerifyArgs a) {
 constexpr int kRevokeUnroll = 4;
 
 __global__ void __launch_bounds__(kThreads) revoke4_kernel(VerifyArgs a) {
+  pdl_wait();                                    // inputs and cleared results from earlier work
   const int lane = threadIdx.x & 31;
   uint32_t count = 0;
   int64_t first = INT64_MAX;
@@ -363,38 +411,58 @@ __global__ void __launch_bounds__(kThreads) revoke4_kernel(VerifyArgs a) {
   if (first != INT64_MAX) atomicMin(a.first_bad, static_cast<unsigned long long>(first));
 }
 
+// the verify grids are programmatic dependents of the clearing kernel: their CTAs may be
+// scheduled while it runs, and wait (griddepcontrol.wait) before touching memory
+template <typename Kern>
+cudaError_t launch_pdl(Kern kern, int blocks, const VerifyArgs &a, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
 template <bool VAR>
-void dispatch(int rk, VerifyArgs a, int blocks, cudaStream_t s) {
+cudaError_t dispatch(int rk, const VerifyArgs &a, int blocks, cudaStream_t s) {
   switch (rk) {
-    case kNoR: verify_kernel<VAR, kNoR><<<blocks, kThreads, 0, s>>>(a); break;
-    case kF32: verify_kernel<VAR, kF32><<<blocks, kThreads, 0, s>>>(a); break;
-    default: verify_kernel<VAR, kBF16><<<blocks, kThreads, 0, s>>>(a); break;
+    case kNoR: return launch_pdl(verify_kernel<VAR, kNoR>, blocks, a, s);
+    case kF32: return launch_pdl(verify_kernel<VAR, kF32>, blocks, a, s);
+    default: return launch_pdl(verify_kernel<VAR, kBF16>, blocks, a, s);
   }
 }
 
-void dispatch4(int rk, VerifyArgs a, int blocks, cudaStream_t s) {
+cudaError_t dispatch4(int rk, bool pair, const VerifyArgs &a, int blocks, cudaStream_t s) {
+  if (pair) return rk == kF32 ? launch_pdl(verify4_kernel<kF32, true>, blocks, a, s)
+                              : launch_pdl(verify4_kernel<kBF16, true>, blocks, a, s);
   switch (rk) {
-    case kNoR: revoke4_kernel<<<blocks, kThreads, 0, s>>>(a); break;
-    case kF32: verify4_kernel<kF32><<<blocks, kThreads, 0, s>>>(a); break;
-    default: verify4_kernel<kBF16><<<blocks, kThreads, 0, s>>>(a); break;
+    case kNoR: return launch_pdl(revoke4_kernel, blocks, a, s);
+    case kF32: return launch_pdl(verify4_kernel<kF32, false>, blocks, a, s);
+    default: return launch_pdl(verify4_kernel<kBF16, false>, blocks, a, s);
   }
 }
 
-}  // namespace
-
-cq_status launch_verify(const cq_qweight &qw, int64_t first_w, int64_t n_w, uint64_t *mism,
-                        int64_t *first_bad, uint32_t *flags, cudaStream_t s) {
-  cq_status st = cuda_check(cudaMemsetAsync(mism, 0, sizeof(uint64_t), s), "cq_requant_verify: clear count");
-  if (st != CQ_OK) return st;
-  st = cuda_check(cudaMemsetAsync(first_bad, 0xFF, sizeof(int64_t), s), "cq_requant_verify: clear first");
-  if (st != CQ_OK) return st;
+// clear the results (flags by memset, then the counters by one small kernel) and launch the
+// verify grid; pair = fixed-4 with a residual, checked with it and without it in one pass
+cq_status launch_verify_impl(const cq_qweight &qw, int64_t first_w, int64_t n_w, uint64_t *mism, int64_t *first_bad,
+                             uint64_t *mism0, int64_t *first0, uint32_t *flags, bool pair, cudaStream_t s,
+                             const char *who) {
   const int64_t n_groups = n_w / kGroup;
   if (flags) {
-    st = cuda_check(cudaMemsetAsync(flags, 0, static_cast<size_t>((n_groups + 31) / 32) * 4, s),
-                    "cq_requant_verify: clear flags");
+    cq_status st = cuda_check(cudaMemsetAsync(flags, 0, static_cast<size_t>((n_groups + 31) / 32) * 4, s), who);
     if (st != CQ_OK) return st;
   }
-  if (n_w == 0) return CQ_OK;
+  verify_clear_kernel<<<1, 32, 0, s>>>(reinterpret_cast<unsigned long long *>(mism),
+                                       reinterpret_cast<unsigned long long *>(first_bad),
+                                       reinterpret_cast<unsigned long long *>(mism0),
+                                       reinterpret_cast<unsigned long long *>(first0));
+  cq_status st = launch_check(who);
+  if (st != CQ_OK || n_w == 0) return st;
   VerifyArgs a;
   a.bits = qw.bits;
   a.offset = qw.offset;
@@ -407,18 +475,44 @@ cq_status launch_verify(const cq_qweight &qw, int64_t first_w, int64_t n_w, uint
   a.mism = reinterpret_cast<unsigned long long *>(mism);
   a.first_bad = reinterpret_cast<unsigned long long *>(first_bad);
   a.flags = flags;
+  a.mism0 = reinterpret_cast<unsigned long long *>(mism0);
+  a.first0 = reinterpret_cast<unsigned long long *>(first0);
   const int rk = qw.residual == nullptr ? kNoR : (qw.residual_dtype == CQ_BF16 ? kBF16 : kF32);
   const int64_t need = (a.n_units + kThreads - 1) / kThreads;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const int blocks = static_cast<int>(need < cap ? need : cap);
+  cudaError_t e;
   if (qw.bits) {
-    dispatch<true>(rk, a, blocks, s);
+    e = dispatch<true>(rk, a, blocks, s);
   } else {
     // 32 weights per lane; n_w is a multiple of 64
     const int64_t need4 = (a.n_units / 4 + kThreads - 1) / kThreads;
-    dispatch4(rk, a, static_cast<int>(need4 < cap ? need4 : cap), s);
+    e = dispatch4(rk, pair, a, static_cast<int>(need4 < cap ? need4 : cap), s);
   }
-  return launch_check("cq_requant_verify");
+  st = cuda_check(e, who);
+  if (st != CQ_OK) return st;
+  return launch_check(who);
+}
+
+}  // namespace
+
+cq_status launch_verify(const cq_qweight &qw, int64_t first_w, int64_t n_w, uint64_t *mism,
+                        int64_t *first_bad, uint32_t *flags, cudaStream_t s) {
+  return launch_verify_impl(qw, first_w, n_w, mism, first_bad, nullptr, nullptr, flags, false, s,
+                            "cq_requant_verify");
+}
+
+cq_status launch_verify_pair(const cq_qweight &qw, int64_t first_w, int64_t n_w, uint64_t *mism, int64_t *first_bad,
+                             uint64_t *mism0, int64_t *first0, uint32_t *flags, cudaStream_t s) {
+  const char *who = "cq_requant_verify_pair";
+  if (qw.bits == nullptr)
+    return launch_verify_impl(qw, first_w, n_w, mism, first_bad, mism0, first0, flags, true, s, who);
+  // per-group widths: the two checks as two passes
+  cq_status st = launch_verify_impl(qw, first_w, n_w, mism, first_bad, nullptr, nullptr, flags, false, s, who);
+  if (st != CQ_OK) return st;
+  cq_qweight q0 = qw;
+  q0.residual = nullptr;
+  return launch_verify_impl(q0, first_w, n_w, mism0, first0, nullptr, nullptr, nullptr, false, s, who);
 }
 
 }  // namespace cq

@@ -84,6 +84,19 @@ def verify(qw, first_w=0, n_w=None, flags=False, stream=None):
     return mism, first, gf
 
 
+def verify_pair(qw, first_w=0, n_w=None, flags=False, stream=None):
+    """-> (mismatches, first_bad, revoke_mismatches, revoke_first_bad, group_flags or None)."""
+    dev = qw.scale.device
+    if n_w is None:
+        n_w = qw.rows * qw.cols - first_w
+    out = [torch.empty(1, dtype=torch.int64, device=dev) for _ in range(4)]
+    gf = None
+    if flags:
+        gf = torch.empty(max(1, (n_w // GROUP + 31) // 32), dtype=torch.int32, device=dev)
+    cq.cq_requant_verify_pair(qw, first_w, n_w, out[0], out[1], out[2], out[3], gf, stream)
+    return out[0], out[1], out[2], out[3], gf
+
+
 def gemv(qw, x, stream=None):
     y = torch.empty((x.shape[0], qw.rows), dtype=torch.float32, device=x.device)
     cq.cq_dequant_gemv(qw, x, y, stream)

@@ -177,6 +177,19 @@ cq_status cq_requant_verify(const cq_qweight *qw, int64_t first_w, int64_t n_w,
                             cq_stream_t stream);
 
 /*
+ * cq_requant_verify_pair -- both [CF] guarantees in one pass over a fixed-4 artifact with a
+ * residual: the served weights s(q-z)+r re-quantize to the codes (mismatches, first_bad, and
+ * group_flags if not NULL, exactly as cq_requant_verify with the residual), and dropping the
+ * residual revokes the update (revoke_mismatches, revoke_first_bad, exactly as
+ * cq_requant_verify with residual = NULL). The codes and metadata are read once. Per-group-width
+ * artifacts are checked in two passes with the same results. qw->residual must be set
+ * (CQ_ERR_ARG); other arguments and errors as for cq_requant_verify.
+ */
+cq_status cq_requant_verify_pair(const cq_qweight *qw, int64_t first_w, int64_t n_w, uint64_t *mismatches,
+                                 int64_t *first_bad, uint64_t *revoke_mismatches, int64_t *revoke_first_bad,
+                                 uint32_t *group_flags, cq_stream_t stream);
+
+/*
  * cq_dequant_gemv -- [VBQ] fused dequantize-and-multiply for decode:
  *     y[i, n] = sum_k (s*(q-z) + r)[n, k] * x[i, k],   i < m, 1 <= m <= 8,
  * products accumulated in fp32. x: [m, cols] of x_dtype (16-byte aligned); y: [m, rows] fp32.

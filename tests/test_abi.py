@@ -71,6 +71,11 @@ def test_host_validation_rejects_bad_arguments():
     assert L.cq_dequant_gemv_multi(C.cast(qws, C.c_void_p), 2, p, 1, 1, C.cast(ys, C.c_void_p), None) == 2  # unequal cols
     assert L.cq_dequant_gemv_multi(None, 2, p, 1, 1, C.cast(ys, C.c_void_p), None) == 1                    # NULL list
     assert L.cq_dequant_gemv_multi(None, 0, p, 1, 1, None, None) == 0                                      # nothing to do
+    assert L.cq_requant_verify_pair(C.byref(qw), 0, 256, p, p, p, p, None, None) == 1   # no residual
+    qw.residual = 16
+    assert L.cq_requant_verify_pair(C.byref(qw), 0, 256, p, p, None, p, None, None) == 1  # NULL result
+    assert L.cq_requant_verify_pair(C.byref(qw), 32, 64, p, p, p, p, None, None) == 2    # not whole groups
+    qw.residual = None
     # recurrent residual quantization
     assert L.cq_rrq_stage(p, 4, 64, 3, p, p, p, None, None) == 3             # width 3
     assert L.cq_rrq_stage(p, 4, 96, 2, p, p, p, None, None) == 2             # cols % 64

@@ -220,6 +220,60 @@ def test_verify_boundary_and_corrupt_scales():
     assert m > 0
 
 
+def _pair_both(qw_r, planes, scale, zero, bits, off, r, r_dtype, first_w=0, n_w=None):
+    """cq_requant_verify_pair against the oracle's two checks (with r, and with r dropped)"""
+    total = qw_r.rows * qw_r.cols
+    if n_w is None:
+        n_w = total - first_w
+    m_d, f_d, m0_d, f0_d, g_d = ops.verify_pair(qw_r, first_w, n_w, flags=True)
+    torch.cuda.synchronize()
+    m, f, flags = co.verify(planes, scale, zero, bits, off, r, r_dtype, first_w, n_w, want_flags=True)
+    m0, f0, _ = co.verify(planes, scale, zero, bits, off, None, "f32", first_w, n_w, want_flags=True)
+    assert (int(host(m_d)[0]), int(host(f_d)[0])) == (m, f)
+    assert (int(host(m0_d)[0]), int(host(f0_d)[0])) == (m0, f0)
+    assert np.array_equal(host(g_d, np.uint32)[:flags.size], flags)
+    return m, m0
+
+
+@pytest.mark.parametrize("varbits", [False, True])
+def test_verify_pair(varbits):
+    """both CellFill checks in one call: with the residual and after dropping it"""
+    rows, cols = 300, 64 * 21
+    w = synth.normal_weights(rows, cols, seed=40)
+    w[7, 100] = np.nan                                    # a flagged group: both checks mismatch there
+    G = rows * cols // 64
+    bits = synth.vbq_bits(G, seed=41) if varbits else None
+    codes, scale, zero, _ = co.quantize(w, bits)
+    planes, off = _oracle_qw(codes, scale, zero, bits)
+    qw, _, _, _ = _quantize_both(w, bits)
+    r = synth.uniform_residual_f32(scale, seed=42)
+    m, m0 = _pair_both(qw.with_residual(dev(r)), planes, scale, zero, bits, off, r, "f32")
+    assert m > 64 and m0 == 64
+    rp, _ = co.project_f32(r, scale)
+    m, m0 = _pair_both(qw.with_residual(dev(rp)), planes, scale, zero, bits, off, rp, "f32")
+    assert m0 == 64                                       # only the flagged group fails revocation
+    rb = synth.normal_residual_bf16(scale, seed=43, rel_sigma=0.3)
+    _pair_both(qw.with_residual(bf16_dev(rb)), planes, scale, zero, bits, off, rb, "bf16")
+    rbp, _ = co.project_bf16(rb, scale)
+    for first, n in [(0, 64 * 100), (64 * 100, 64 * 37), (64 * 1000, w.size - 64 * 1000)]:
+        _pair_both(qw.with_residual(bf16_dev(rbp)), planes, scale, zero, bits, off, rbp, "bf16", first, n)
+
+
+def test_verify_pair_corrupt_scales():
+    """zero, infinite, NaN and negative scales, residuals on and across the cell edges"""
+    rng = np.random.default_rng(44)
+    G = 4096 + 17
+    codes = rng.integers(0, 16, G * 64).astype(np.uint8)
+    zero = rng.integers(0, 16, G).astype(np.uint8)
+    scale = rng.integers(0x0001, 0x7C00, G).astype(np.uint16)
+    scale[:4] = [0x0000, 0x7C00, 0x7E00, 0xBC00]
+    planes = co.pack(codes)
+    r = _residual_cases(scale, 45)
+    qw = cq.QWeight(G, 64, [None, None, dev(planes[2]), None], u16_dev(scale), dev(zero))
+    m, m0 = _pair_both(qw.with_residual(dev(r)), planes, scale, zero, None, None, r, "f32")
+    assert m > 0 and m0 > 0
+
+
 # ---- matmuls ------------------------------------------------------------------------------------
 
 def _matmul_case(rows, cols, m, x_dtype, bits=None, r=None, seed=0):
