@@ -5,8 +5,8 @@ configuration (three weight matrices 4096x4096, 11008x4096, 4096x11008, drawn as
 0.02 * Student-t(5) with 0.1% of entries x10):
 
     quantize (fp32 -> 4-bit codes, fp16 scales, u8 zeros)   -> pack into the 4-bit plane
-    -> project a bf16 residual ~ N(0, (0.3 s)^2) into the cells -> requant-verify with it
-    -> requant-verify without it (revocation) -> dequant-GEMV at batch 1 (decode)
+    -> project a bf16 residual ~ N(0, (0.3 s)^2) into the cells -> requant-verify with it and
+    without it (revocation), both in one pass -> dequant-GEMV at batch 1 (decode)
     -> dequant-GEMM at batch 64
 
 for each matrix (each row runs over the three matrices before the next row starts).  K steps
@@ -58,14 +58,14 @@ def kernel_bytes(n):
         "quantize": 4 * n + n + meta,                 # read fp32 W, write u8 codes + meta
         "pack": n + n // 2,                           # read codes, write nibbles
         "project": 2 * n + 2 * n + 2 * G,             # read + write bf16 r, read scales
-        "verify": n // 2 + meta + 2 * n,              # codes + meta + bf16 r
-        "revoke_verify": n // 2 + meta,               # codes + meta
+        # both checks (with r, and with r dropped) in one pass: codes + meta + bf16 r
+        "verify_pair": n // 2 + meta + 2 * n,
         "gemv": n // 2 + meta,                        # weights (x, y negligible)
         "gemm": n // 2 + meta,
     }
 
 
-KERNELS = ["quantize", "pack", "project", "verify", "revoke_verify", "gemv", "gemm"]
+KERNELS = ["quantize", "pack", "project", "verify_pair", "gemv", "gemm"]
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
 # the kernel's launches in one step of this workload (mean over the three matrices), taken with
@@ -176,7 +176,7 @@ class Workload:
 
     def step(self, stream, marks=None):
         """Enqueue one step: each row of the path over the three matrices, then the next row
-        (every matrix keeps its own order quantize -> pack -> project -> verify -> revoke ->
+        (every matrix keeps its own order quantize -> pack -> project -> verify pair ->
         GEMV -> GEMM). marks[kernel] = (start, end) external events around a row's three
         launches: recorded inside a graph capture they become event nodes that time the row on
         replay (one pair per row keeps their own cost out of the launches they time)."""
@@ -193,9 +193,9 @@ class Workload:
         row("quantize", lambda m, qw: cq.cq_quantize(m["w"], None, m["codes"], qw.scale, qw.zero, m["status"], stream))
         row("pack", lambda m, qw: cq.cq_pack_varbits(m["codes"], m["n"] // GROUP, None, None, qw.planes, stream))
         row("project", lambda m, qw: cq.cq_project_residual(m["r"], qw.scale, m["nclamp"], stream))
-        row("verify", lambda m, qw: cq.cq_requant_verify(qw.with_residual(m["r"]), 0, m["n"], m["mism"], m["first"],
-                                                         None, stream))
-        row("revoke_verify", lambda m, qw: cq.cq_requant_verify(qw, 0, m["n"], m["mism0"], m["first0"], None, stream))
+        row("verify_pair", lambda m, qw: cq.cq_requant_verify_pair(qw.with_residual(m["r"]), 0, m["n"], m["mism"],
+                                                                   m["first"], m["mism0"], m["first0"], None,
+                                                                   stream))
         row("gemv", lambda m, qw: cq.cq_dequant_gemv(qw, m["x"], m["y"], stream))
         row("gemm", lambda m, qw: cq.cq_dequant_gemm(qw, m["X"], m["Y"], m["ws"], stream))
 
@@ -376,13 +376,17 @@ def cellfill_stack_verify(torch, cq, ops, synth, device, peaks, stream):
     ncl = torch.zeros(1, dtype=torch.int64, device=device)
     mism = torch.zeros(1, dtype=torch.int64, device=device)
     first = torch.zeros(1, dtype=torch.int64, device=device)
+    mism0 = torch.zeros(1, dtype=torch.int64, device=device)
+    first0 = torch.zeros(1, dtype=torch.int64, device=device)
     qw_r = cq.QWeight(1, n, [None, None, plane, None], scale, zero, residual=r)
     qw_0 = cq.QWeight(1, n, [None, None, plane, None], scale, zero)
     res = {"weights": n}
     calls = {"project": lambda: cq.cq_project_residual(r, scale, ncl, stream),
              "verify": lambda: cq.cq_requant_verify(qw_r, 0, n, mism, first, None, stream),
-             "revoke_verify": lambda: cq.cq_requant_verify(qw_0, 0, n, mism, first, None, stream)}
-    per_w = {"project": 4.0 + 2.0 / GROUP, "verify": 2.5 + 3.0 / GROUP, "revoke_verify": 0.5 + 3.0 / GROUP}
+             "revoke_verify": lambda: cq.cq_requant_verify(qw_0, 0, n, mism, first, None, stream),
+             "verify_pair": lambda: cq.cq_requant_verify_pair(qw_r, 0, n, mism, first, mism0, first0, None, stream)}
+    per_w = {"project": 4.0 + 2.0 / GROUP, "verify": 2.5 + 3.0 / GROUP, "revoke_verify": 0.5 + 3.0 / GROUP,
+             "verify_pair": 2.5 + 3.0 / GROUP}
     for name, fn in calls.items():
         with torch.cuda.stream(stream):
             fn()
@@ -395,6 +399,8 @@ def cellfill_stack_verify(torch, cq, ops, synth, device, peaks, stream):
         ms = time_graph(torch, g, 10, stream)
         if name != "project":
             assert int(mism.item()) == 0, f"{name}: {int(mism.item())} mismatches"
+        if name == "verify_pair":
+            assert int(mism0.item()) == 0, f"{name}: {int(mism0.item())} revocation mismatches"
         res[name] = {"ms": ms, "weights_per_s": n / (ms * 1e-3), "GBps": n * per_w[name] / (ms * 1e-3) / 1e9,
                      "frac_hbm": n * per_w[name] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
         del g
@@ -514,8 +520,8 @@ def run_gpu(args, rank, world, local_rank):
                        "residual": "bf16", "l2": "inputs larger than L2 (377 MB fp32 weights per step)",
                        "parallelism": f"replicas x{world}", "step": "+".join(KERNELS)},
             "roofline": roofline,
-            "requant_verify_weights_per_s": n_w / (per_kernel["verify"] / args.steps * 1e-3),
-            "revoke_verify_weights_per_s": n_w / (per_kernel["revoke_verify"] / args.steps * 1e-3),
+            # weights checked per second by the pass that checks both (with r, and revoked)
+            "requant_verify_weights_per_s": n_w / (per_kernel["verify_pair"] / args.steps * 1e-3),
             "dequant_gemv_GBps_in_step": comps["gemv"]["GBps"],
             "components": comps,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
