@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <utility>
 
 #include "cq_internal.cuh"
 
@@ -81,6 +82,36 @@ __device__ __forceinline__ bool mbar_wait_suspend(uint64_t *b, uint32_t parity, 
 // programmatic dependent launch: wait for the preceding grid's results / let the next grid start
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::); }
+
+// launch `kern` as the programmatic dependent of the kernel before it in the stream: its CTAs
+// may be scheduled while that kernel finishes; the kernel must execute pdl_wait() before it
+// touches global memory that earlier work reads or writes
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// result words set to zero by one thread (either may be NULL) before the kernel that
+// accumulates into them, which is launched as this kernel's programmatic dependent (one copy
+// per translation unit)
+static __global__ void clear_results_kernel(uint32_t *w32, unsigned long long *w64) {
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    if (w32) *w32 = 0u;
+    if (w64) *w64 = 0ull;
+  }
+}
 
 // 2-D tiled TMA load into this CTA's shared memory, completing on an mbarrier (no multicast)
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {

@@ -8,7 +8,7 @@
 // Work unit: eight lanes per group, one lane per eight consecutive codes. Lane `sub` of a
 // group of width b owns exactly b bytes of the plane (8 codes * b bits), so packing and
 // unpacking are single stores/loads of 1, 2, 4 or 8 bytes with no read-modify-write.
-#include "cq_internal.cuh"
+#include "cq_async.cuh"
 
 namespace cq {
 namespace {
@@ -120,6 +120,7 @@ __device__ __forceinline__ uint32_t pack8codes(uint32_t lo, uint32_t hi) {
 
 __global__ void __launch_bounds__(kThreads)
 pack4_kernel(const uint8_t *__restrict__ codes, int64_t n32, uint8_t *__restrict__ plane) {
+  pdl_wait();                     // the codes come from earlier work
   const int64_t step = static_cast<int64_t>(gridDim.x) * kThreads;
   for (int64_t u = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; u < n32; u += 2 * step) {
     const int64_t u2 = u + step;
@@ -326,7 +327,10 @@ cq_status launch_pack(const uint8_t *codes, int64_t G, const uint8_t *bits, cons
   if (G == 0) return CQ_OK;
   if (!bits) {
     const int64_t n32 = G * 2;
-    pack4_kernel<<<grid_for((n32 + 1) / 2), kThreads, 0, s>>>(codes, n32, plane[2]);
+    cq_status st = cuda_check(launch_pdl(pack4_kernel, dim3(grid_for((n32 + 1) / 2)), dim3(kThreads), 0, s, codes, n32,
+                                         plane[2]),
+                              "cq_pack_varbits");
+    if (st != CQ_OK) return st;
     return launch_check("cq_pack_varbits");
   }
   Planes P{{plane[0], plane[1], plane[2], plane[3]}};

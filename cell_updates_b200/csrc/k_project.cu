@@ -10,7 +10,7 @@
 //
 // Layout: one lane per eight residuals (one 16-byte load for bf16, two for fp32); eight
 // lanes share a group scale. Streaming, in place.
-#include "cq_internal.cuh"
+#include "cq_async.cuh"
 
 namespace cq {
 namespace {
@@ -41,6 +41,7 @@ template <bool BF16>
 __global__ void __launch_bounds__(kThreads)
 project_kernel(void *__restrict__ rv, const uint16_t *__restrict__ scale, int64_t n_units,
                unsigned long long *__restrict__ n_clamped) {
+  pdl_wait();                     // r, the scales and the cleared count come from earlier work
   uint32_t changed = 0;
   const int64_t step = static_cast<int64_t>(gridDim.x) * kThreads;
   for (int64_t u0 = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; u0 < n_units; u0 += kUnroll * step) {
@@ -110,7 +111,8 @@ project_kernel(void *__restrict__ rv, const uint16_t *__restrict__ scale, int64_
 cq_status launch_project(void *r, cq_dtype dt, const uint16_t *scale, int64_t n, uint64_t *n_clamped,
                          cudaStream_t s) {
   if (n_clamped) {
-    cq_status st = cuda_check(cudaMemsetAsync(n_clamped, 0, sizeof(uint64_t), s), "cq_project_residual: clear count");
+    clear_results_kernel<<<1, 32, 0, s>>>(nullptr, reinterpret_cast<unsigned long long *>(n_clamped));
+    cq_status st = launch_check("cq_project_residual: clear count");
     if (st != CQ_OK) return st;
   }
   if (n == 0) return CQ_OK;
@@ -119,10 +121,12 @@ cq_status launch_project(void *r, cq_dtype dt, const uint16_t *scale, int64_t n,
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const int blocks = static_cast<int>(need < cap ? need : cap);
   auto *cnt = reinterpret_cast<unsigned long long *>(n_clamped);
-  if (dt == CQ_BF16)
-    project_kernel<true><<<blocks, kThreads, 0, s>>>(r, scale, units, cnt);
-  else
-    project_kernel<false><<<blocks, kThreads, 0, s>>>(r, scale, units, cnt);
+  const cudaError_t e = dt == CQ_BF16 ? launch_pdl(project_kernel<true>, dim3(blocks), dim3(kThreads), 0, s, r, scale,
+                                                   units, cnt)
+                                      : launch_pdl(project_kernel<false>, dim3(blocks), dim3(kThreads), 0, s, r, scale,
+                                                   units, cnt);
+  cq_status st = cuda_check(e, "cq_project_residual");
+  if (st != CQ_OK) return st;
   return launch_check("cq_project_residual");
 }
 

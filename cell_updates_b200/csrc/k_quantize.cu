@@ -52,6 +52,7 @@ quantize_kernel(const __grid_constant__ CUtensorMap tm_w, float *w, int64_t G, c
   }
   if (threadIdx.x == 0) *abort_flag = 0u;
   __syncthreads();
+  pdl_wait();                     // w, the cleared status word and the outputs' earlier readers
 
   uint32_t flags = 0;
   const int64_t n_tiles = (G + kTileGroups - 1) / kTileGroups;
@@ -199,7 +200,8 @@ template <bool kResid>
 cq_status launch_quantize_impl(float *w, int64_t G, const uint8_t *bits, int uniform_b, uint8_t *codes,
                                uint16_t *scale, uint8_t *zero, uint32_t *status, cudaStream_t s, const char *who) {
   if (status) {
-    cq_status st = cuda_check(cudaMemsetAsync(status, 0, sizeof(uint32_t), s), who);
+    clear_results_kernel<<<1, 32, 0, s>>>(status, nullptr);
+    cq_status st = launch_check(who);
     if (st != CQ_OK) return st;
   }
   if (G == 0) return CQ_OK;
@@ -223,7 +225,10 @@ cq_status launch_quantize_impl(float *w, int64_t G, const uint8_t *bits, int uni
   const int64_t need = (tiles + kWarps - 1) / kWarps;
   const int64_t cap = sm_count();
   const int blocks = static_cast<int>(need < cap ? need : cap);
-  quantize_kernel<kResid><<<blocks, kThreads, kSmem, s>>>(tm, w, G, bits, uniform_b, codes, scale, zero, status);
+  st = cuda_check(launch_pdl(quantize_kernel<kResid>, dim3(blocks), dim3(kThreads), kSmem, s, tm, w, G, bits, uniform_b,
+                             codes, scale, zero, status),
+                  who);
+  if (st != CQ_OK) return st;
   return launch_check(who);
 }
 
