@@ -3,8 +3,9 @@
     python -m cell_updates_b200.profile_case <kernel> [--reps 3]
 
 kernels: gemv (16384x16384, m=1), gemv8 (same, m=8), gemm (8192x28672, m=64), quantize,
-pack, project, verify (projected bf16 residual), revoke (no residual) -- the last five on
-8192x16384.
+pack, project, verify (projected bf16 residual), revoke (no residual), pair (both checks),
+rrq (one 2-bit residual stage), stages (the stage-stack GEMV, 4 two-bit stages, m=1) -- all
+but the first three on 8192x16384.
 Each is preceded by the set-up launches (random weights, quantize, pack); capture the
 measured kernel with `ncu -k regex:<name> -s <set-up launches + warm-up> -c 1`.
 """
@@ -35,8 +36,13 @@ def main():
     first = torch.empty(1, dtype=torch.int64, device=dev)
     scale, zero = qw.scale, qw.zero
     st = torch.zeros(1, dtype=torch.int32, device=dev)
-    if a.kernel == "verify":
+    if a.kernel in ("verify", "pair"):
         cq.cq_project_residual(r, scale, None)     # a residual inside its cells, as after an update
+    stages = None
+    if a.kernel == "stages":
+        stages, _, _ = ops.rrq_build(w, 4)
+    if a.kernel == "rrq":
+        rr = w.clone()
     if a.kernel in ("gemv", "gemv8", "gemm"):
         del w, r                                   # keep the device footprint small under the profiler
         torch.cuda.empty_cache()
@@ -56,6 +62,14 @@ def main():
             cq.cq_requant_verify(qw.with_residual(r), 0, N * K, mism, first)
         elif a.kernel == "revoke":
             cq.cq_requant_verify(qw, 0, N * K, mism, first)
+        elif a.kernel == "pair":
+            m0 = torch.empty(1, dtype=torch.int64, device=dev)
+            f0 = torch.empty(1, dtype=torch.int64, device=dev)
+            cq.cq_requant_verify_pair(qw.with_residual(r), 0, N * K, mism, first, m0, f0)
+        elif a.kernel == "rrq":
+            cq.cq_rrq_stage(rr, 2, codes, scale, zero, st)
+        elif a.kernel == "stages":
+            cq.cq_dequant_gemv_stages(stages, x, y)
         else:
             raise SystemExit(f"unknown kernel {a.kernel}")
     torch.cuda.synchronize()
