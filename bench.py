@@ -310,6 +310,67 @@ def isolated_components(torch, cq, ops, device, peaks, stream):
     torch.cuda.empty_cache()
     out["cellfill_stack"] = cellfill_stack_verify(torch, cq, ops, synth_module(), device, peaks, stream)
     out["rrq"] = rrq_components(torch, cq, ops, device, peaks, stream)
+    out["vbq"] = vbq_components(torch, cq, ops, synth_module(), device, peaks, stream)
+    return out
+
+
+def vbq_components(torch, cq, ops, synth, device, peaks, stream):
+    """Per-group widths on the 2048x8192 shape of the VBQ configuration (widths drawn from
+    {1, 2, 4, 8} with probabilities .69/.15/.12/.04, mean 1.79 bits): quantize with the width map
+    (4 B read + 1 B code + 3/64 B scale/zero + 1/64 B width per weight), the offset index (1 B
+    read, 4 B written per group), pack (1 B code + 5/64 B index read, the planes written),
+    unpack (the reverse), and the GEMV at m = 1 and m = 8 (planes + 3/64 B scale/zero + 5/64 B
+    width/offset per weight). One matrix is 5.9 MB packed, far below L2, so every figure comes
+    from a pool of copies run back to back in one graph (32 for the GEMV, 187 MB; 8 for the
+    others), which also shows the grouped launch escaping launch latency."""
+    N, K = 2048, 8192
+    G = N * K // GROUP
+    bits = torch.from_numpy(synth.vbq_bits(G, seed=2)).to(device)
+    offset, pb = ops.varbits_index(bits, stream)
+    plane_bytes = sum(pb)
+    out = {"shape": f"{N}x{K}", "mean_bits": plane_bytes * 8 / (N * K), "plane_bytes": plane_bytes}
+
+    def timed(fn, n_in_pool, bytes_one):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            fn()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+        g.replay()
+        t = time_graph(torch, g, 10, stream) / n_in_pool
+        del g
+        return {"us": t * 1e3, "GBps": bytes_one / t / 1e6, "frac_hbm": bytes_one / t / 1e6 / peaks["hbm_gbs"]}
+
+    ws = [torch.randn(N, K, device=device) * 0.02 for _ in range(8)]
+    qs = [ops.quantize_and_pack(w, bits, stream) for w in ws]
+    codes_out = [torch.empty(N * K, dtype=torch.uint8, device=device) for _ in range(8)]
+    sc = torch.empty(G, dtype=torch.int16, device=device)
+    zr = torch.empty(G, dtype=torch.uint8, device=device)
+    off2 = torch.empty(G, dtype=torch.int32, device=device)
+    pb2 = torch.empty(4, dtype=torch.int64, device=device)
+    out["quantize"] = timed(lambda: [cq.cq_quantize(w, bits, c, sc, zr, None, stream) for w, c in zip(ws, codes_out)],
+                            8, N * K * 5 + G * 4)
+    out["index"] = timed(lambda: [cq.cq_varbits_index(bits, off2, pb2, stream) for _ in range(8)], 8, G * 5)
+    out["pack"] = timed(lambda: [cq.cq_pack_varbits(c, G, bits, offset, q.planes, stream)
+                                 for (q, c, _), _ in zip(qs, range(8))], 8, N * K + G * 5 + plane_bytes)
+    out["unpack"] = timed(lambda: [cq.cq_unpack_varbits(q, c, stream) for (q, _, _), c in zip(qs, codes_out)],
+                          8, N * K + G * 5 + plane_bytes)
+    del ws
+    torch.cuda.empty_cache()
+    # 32 packed copies for the GEMV pool
+    pool = [q for q, _, _ in qs]
+    while len(pool) < 32:
+        q = pool[len(pool) % 8]
+        pool.append(cq.QWeight(N, K, [p.clone() if p is not None else None for p in q.planes], q.scale.clone(),
+                               q.zero.clone(), q.bits, q.offset))
+    gemv_bytes = plane_bytes + G * 8
+    for m in (1, 8):
+        x = torch.randn(m, K, device=device).to(torch.bfloat16)
+        y = torch.empty(m, N, device=device)
+        out[f"gemv_m{m}"] = timed(lambda: [cq.cq_dequant_gemv(q, x, y, stream) for q in pool], len(pool), gemv_bytes)
+    del pool, qs, codes_out
+    torch.cuda.empty_cache()
     return out
 
 
@@ -317,7 +378,8 @@ def rrq_components(torch, cq, ops, device, peaks, stream):
     """Recurrent residual quantization on the config's 11008x4096 shape (4 two-bit stages =
     the 8-bit model): one stage (quantize the fp32 residual, write codes, scales, zero points
     and the new residual: 9 + 3/64 B per weight), and the stage-stack GEMV at m=1 over 1, 2
-    and 4 stages (per stage 0.25 B codes + 3/64 B scale/zero + 5/64 B width map and offset)."""
+    and 4 stages (per stage 0.25 B codes + 3/64 B scale/zero + 5/64 B width map and offset), at
+    m = 1 and m = 8, rotating over three stacks so the weights come from HBM."""
     N, K = 11008, 4096
     G = N * K // GROUP
     w = torch.randn(N, K, device=device) * 0.02
@@ -335,18 +397,27 @@ def rrq_components(torch, cq, ops, device, peaks, stream):
     t = time_graph(torch, g, 10, stream)
     b = N * K * 9 + G * 3
     out = {"shape": f"{N}x{K}", "stage": {"us": t * 1e3, "GBps": b / t / 1e6, "frac_hbm": b / t / 1e6 / peaks["hbm_gbs"]}}
-    x = torch.randn(1, K, device=device).to(torch.bfloat16)
-    y = torch.empty(1, N, device=device)
-    for n in (1, 2, 4):
-        gs = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(stream):
-            with torch.cuda.graph(gs, stream=stream):
-                cq.cq_dequant_gemv_stages(stages[:n], x, y, stream)
-        t = time_graph(torch, gs, 10, stream)
-        b = n * (N * K // 4 + G * 8)
-        out[f"gemv_m1_{n}_stages"] = {"us": t * 1e3, "GBps": b / t / 1e6, "frac_hbm": b / t / 1e6 / peaks["hbm_gbs"]}
-        del gs
-    del stages, w, r, g
+    # the stage-stack GEMV over a pool of stacks larger than L2 (3 x 4 stages x 17 MB)
+    pool = [stages] + [ops.rrq_build(w * (1.0 + 0.01 * i), 4)[0] for i in (1, 2)]
+    for m in (1, 8):
+        x = torch.randn(m, K, device=device).to(torch.bfloat16)
+        y = torch.empty(m, N, device=device)
+        for n in (1, 2, 4):
+            gs = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                for st in pool:
+                    cq.cq_dequant_gemv_stages(st[:n], x, y, stream)
+                torch.cuda.synchronize()
+                with torch.cuda.graph(gs, stream=stream):
+                    for st in pool:
+                        cq.cq_dequant_gemv_stages(st[:n], x, y, stream)
+            gs.replay()
+            t = time_graph(torch, gs, 10, stream) / len(pool)
+            b = n * (N * K // 4 + G * 8)
+            out[f"gemv_m{m}_{n}_stages"] = {"us": t * 1e3, "GBps": b / t / 1e6,
+                                            "frac_hbm": b / t / 1e6 / peaks["hbm_gbs"]}
+            del gs
+    del stages, pool, w, r, g
     torch.cuda.empty_cache()
     return out
 

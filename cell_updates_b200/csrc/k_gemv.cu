@@ -17,9 +17,9 @@
 //    sum, so the kernel may pair any code with any activation as long as both operands
 //    use the same order: each lane feeds the MMA with the 16 codes it loaded contiguously
 //    (one 8-byte load per row and group) and permutes its 16 activations to match (PRMT).
-//  * gemv_generic: any format (per-group widths), fp32 or bf16 x, optional residual; one
-//    warp per row, fp32 CUDA-core math. Used for the small fp32-activation cases and for
-//    residual-carrying weights.
+//  * gemv_generic: any format (per-group widths), fp32 or bf16 x, with a residual; one warp
+//    per row, fp32 CUDA-core math. Used for residual-carrying weights only: without a residual,
+//    per-group widths and fp32 activations go to the tensor-core kernel of k_rrq.cu.
 #include "cq_async.cuh"
 
 namespace cq {
@@ -734,17 +734,21 @@ cq_status launch_gemv(const cq_qweight &qw, const void *x, cq_dtype xdt, int m, 
     const cq_qweight *one = &qw;
     return launch_gemv4_segs(&one, 1, x, m, &y, s);
   }
+  // per-group widths, or fp32 activations, without a residual: the tensor-core kernel over a
+  // list of one stage (k_rrq.cu)
+  if (qw.residual == nullptr) {
+    const cq_qweight *one = &qw;
+    return launch_gemv_stages(&one, 1, x, xdt, m, y, s);
+  }
   const int64_t need = (N + 7) / 8;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const int blocks = static_cast<int>(need < cap ? need : cap);
-  const int rk = qw.residual == nullptr ? 0 : (qw.residual_dtype == CQ_BF16 ? 2 : 1);
+  const bool rf32 = qw.residual_dtype != CQ_BF16;
   if (xdt == CQ_BF16) {
-    if (rk == 0) launch_generic<true, 0>(qw, x, m, y, blocks, s);
-    else if (rk == 1) launch_generic<true, 1>(qw, x, m, y, blocks, s);
+    if (rf32) launch_generic<true, 1>(qw, x, m, y, blocks, s);
     else launch_generic<true, 2>(qw, x, m, y, blocks, s);
   } else {
-    if (rk == 0) launch_generic<false, 0>(qw, x, m, y, blocks, s);
-    else if (rk == 1) launch_generic<false, 1>(qw, x, m, y, blocks, s);
+    if (rf32) launch_generic<false, 1>(qw, x, m, y, blocks, s);
     else launch_generic<false, 2>(qw, x, m, y, blocks, s);
   }
   return launch_check("cq_dequant_gemv");

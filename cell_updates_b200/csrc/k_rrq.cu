@@ -1,24 +1,40 @@
-// k_rrq.cu -- recurrent residual quantization: the multiply over a stack of stages.
+// k_rrq.cu -- dequantize-and-multiply over per-group-width weights and over stacks of stages.
 //
-// [RRQ] the listing page thelatestinai.com/papers/2512.18934, "Recurrent Residual
-// Quantization" abstract: the weights are a low-bit base plus a sequence of quantized residual
-// corrections (2-bit round-to-nearest stages stacked to 4, 6 and 8 bits), so one artifact
-// serves several precisions; a model of 2(J+1) bits uses the first J+1 stages. The stages
-// themselves come from cq_rrq_stage (the group quantizer with an in-place residual update,
-// k_quantize.cu); here
-//     y[i, n] = sum_k (sum_j s_j[n, g] * (q_j[n, k] - z_j[n, g])) * x[i, k]
-// over any stage list of one shape, each stage fixed-4 or per-group width.
+// [VBQ] "In-Cell Learning: Language Models That Update Their Own Weights in Sequence Without
+// Changing the File They Ship", abstract: per-group bit-widths in bit-packed storage, served by a
+// fused dequantize-and-multiply kernel for memory-bound decode. [RRQ] the listing page
+// thelatestinai.com/papers/2512.18934, "Recurrent Residual Quantization" abstract: the weights
+// are a low-bit base plus a sequence of quantized residual corrections (2-bit round-to-nearest
+// stages stacked to 4, 6 and 8 bits), so one artifact serves several precisions; a model of
+// 2(J+1) bits uses the first J+1 stages (made by cq_rrq_stage, k_quantize.cu). One kernel serves
+// both: for a list of stages of one shape, each fixed-4 or with a per-group width map,
+//     y[i, n] = sum_j sum_g s_j[n, g] * sum_{k in g} (q_j[n, k] - z_j[n, g]) * x[i, k]
+// (a single VBQ matrix is a list of one stage).
 //
-// Per 16 columns the stage sum of each weight is formed in fp32 first (s * (q - z), the
-// product exact), then multiplied with the batch rows of x, so x is read once per column and
-// batch row whatever the number of stages. fp32 accumulation, a warp reduction per row.
+// Tensor cores, mma.sync m16n8k16 (bf16 operands, fp32 accumulation): a warp takes 16 rows of one
+// group at a time; A is the 16 x 64 block of q - z, B the group's 64 activations of up to 8
+// batch rows. q - z is an integer in [-255, 255], exact in bf16, so every product is exact; the
+// group's four MMAs start from zero and the group result is scaled by s (fp32) and added to the
+// running sums, so the only rounding is fp32 accumulation (fp32 activations enter as two bf16
+// parts, hi + lo, which leaves |x - hi - lo| <= 2^-17 |x|). The contraction over k is a sum, so
+// codes and activations may be paired in any order both operands share: lane (gid, tig) feeds the
+// 16 codes 16 tig .. 16 tig + 15 of rows gid and gid + 8, as the pairs (t, t + 8), and loads the
+// matching 16 activations of batch row gid.
+//
+// For widths 1, 2 and 4 the bf16 pair (128 + q_t, 128 + q_{t+8}) comes from the packed bytes
+// with one shift and one LOP3 whatever the width (the width only sets the shift step and the
+// mask), and one bf16x2 subtraction of 128 + z gives q - z; so rows of different widths in one
+// warp run the same instructions. 8-bit groups (128 + q is not exact in bf16 past q = 127) go
+// through fp32: (2^23 + q) - (2^23 + z), exact, then packed to bf16.
 #include "cq_internal.cuh"
 
 namespace cq {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kPerLaunch = 4;         // stages per launch (their metadata lives in registers)
+constexpr int kWarps = 16;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kTileRows = 16;
+constexpr int kPerLaunch = 4;         // stages per launch (their pointers live in the parameter space)
 
 struct StageSet {
   const uint8_t *bits[kPerLaunch];
@@ -27,6 +43,329 @@ struct StageSet {
   const uint16_t *scale[kPerLaunch];
   const uint8_t *zero[kPerLaunch];
 };
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 v) { return *reinterpret_cast<const uint32_t *>(&v); }
+
+// (w & mask) | magic in one LOP3
+__device__ __forceinline__ uint32_t and_or(uint32_t w, uint32_t mask, uint32_t magic) {
+  uint32_t out;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(out) : "r"(w), "r"(mask), "r"(magic));
+  return out;
+}
+
+// where a group's bytes are: width (0 for a width outside {1, 2, 4, 8}) and raw byte offset
+struct RowMeta {
+  int b;
+  uint32_t off;
+};
+// what the MMA step needs of one row and group: the lane's packed code bytes, width, scale, zero
+struct RowCodes {
+  uint4 w;
+  float s;
+  uint32_t z;
+  int b;
+};
+
+__device__ __forceinline__ RowMeta load_meta(const StageSet &ss, int j, int64_t gabs) {
+  RowMeta m;
+  if (ss.bits[j]) {
+    const int b = __ldg(ss.bits[j] + gabs);
+    m.b = width_ok(b) ? b : 0;
+    m.off = __ldg(ss.offset[j] + gabs);
+  } else {
+    m.b = 4;
+    m.off = static_cast<uint32_t>(gabs) * 32u;   // unused: the fixed-4 address is formed from gabs
+  }
+  return m;
+}
+
+// the lane's share of the group's packed bytes: for b <= 4 the aligned 8-byte word at byte
+// (2 b tig) & ~7 of the group (in w.x, w.y), for b = 8 the 16 bytes at 16 tig
+__device__ __forceinline__ RowCodes load_codes(const StageSet &ss, int j, int64_t gabs, const RowMeta &m, int tig) {
+  RowCodes c;
+  c.b = m.b;
+  c.w = make_uint4(0u, 0u, 0u, 0u);
+  if (m.b) {
+    const uint8_t *src;
+    if (ss.bits[j]) {
+      // offsets are multiples of 8 b by construction; the mask keeps a damaged map aligned
+      src = ss.plane[j][width_slot(m.b)] + (m.off & ~static_cast<uint32_t>(8 * m.b - 1));
+    } else {
+      src = ss.plane[j][2] + gabs * 32;
+    }
+    if (m.b == 8) {
+      c.w = __ldg(reinterpret_cast<const uint4 *>(src + 16 * tig));
+    } else {
+      const uint2 v = __ldg(reinterpret_cast<const uint2 *>(src + ((2 * m.b * tig) & ~7)));
+      c.w.x = v.x;
+      c.w.y = v.y;
+    }
+  }
+  c.s = f16_bits_to_f32(__ldg(ss.scale[j] + gabs));
+  c.z = __ldg(ss.zero[j] + gabs);
+  return c;
+}
+
+// The A-operand share of one row: codes 16 tig .. 16 tig + 15 of the group, as eight bf16 pairs
+// (q_t - z, q_{t+8} - z). Width 0 (outside {1, 2, 4, 8}) gives zeros.
+__device__ __forceinline__ void row_operand(const RowCodes &c, int tig, uint32_t (&r)[8]) {
+  const int b = c.b;
+  if (b == 1 || b == 2 || b == 4) {
+    uint32_t v0, v1;
+    if (b == 4) {                       // codes 0-3 | 8-11 and 4-7 | 12-15 as 16-bit halves
+      v0 = __byte_perm(c.w.x, c.w.y, 0x5410);
+      v1 = __byte_perm(c.w.x, c.w.y, 0x7632);
+    } else if (b == 2) {                // bytes 4 tig .. 4 tig + 3: codes 0-7 | 8-15
+      v0 = v1 = (tig & 1) ? c.w.y : c.w.x;
+    } else {                            // bytes 2 tig, 2 tig + 1 moved to bits 0-7 and 16-23
+      const uint32_t u = (tig >> 1) ? c.w.y : c.w.x;
+      const uint32_t o = 2u * (tig & 1);
+      v0 = v1 = __byte_perm(u, 0u, 0x4040u | o | ((o + 1u) << 8));
+    }
+    const uint32_t mask = (b == 4 ? 0x000F000Fu : (b == 2 ? 0x00030003u : 0x00010001u));
+    const uint32_t adj = b == 4 ? 16u : 0u;     // codes 4-7 of a 4-bit group restart at bit 0 of v1
+    const uint32_t zz = (0x4300u | c.z) * 0x00010001u;   // bf16 (128 + z) twice
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const uint32_t sh = t < 4 ? static_cast<uint32_t>(t * b) : static_cast<uint32_t>(t * b) - adj;
+      const uint32_t p = and_or((t < 4 ? v0 : v1) >> sh, mask, 0x43004300u);   // 128 + q, exact
+      r[t] = bf2_bits(__hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&p),
+                              *reinterpret_cast<const __nv_bfloat162 *>(&zz)));
+    }
+  } else if (b == 8) {
+    const float zf = 8388608.0f + static_cast<float>(c.z);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const uint32_t sel = 0x7440u | static_cast<uint32_t>(t & 3);   // [byte t & 3, 0, 0, 0x4B]
+      const float f0 = __uint_as_float(__byte_perm(t < 4 ? c.w.x : c.w.y, 0x4B000000u, sel)) - zf;
+      const float f1 = __uint_as_float(__byte_perm(t < 4 ? c.w.z : c.w.w, 0x4B000000u, sel)) - zf;
+      r[t] = bf2_bits(__floats2bfloat162_rn(f0, f1));
+    }
+  } else {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) r[t] = 0u;
+  }
+}
+
+// the same for a width B known to the whole warp: constant shifts and masks
+template <int B>
+__device__ __forceinline__ void row_operand_w(const RowCodes &c, int tig, uint32_t (&r)[8]) {
+  uint32_t v0, v1;
+  if (B == 4) {
+    v0 = __byte_perm(c.w.x, c.w.y, 0x5410);
+    v1 = __byte_perm(c.w.x, c.w.y, 0x7632);
+  } else if (B == 2) {
+    v0 = v1 = (tig & 1) ? c.w.y : c.w.x;
+  } else {
+    const uint32_t u = (tig >> 1) ? c.w.y : c.w.x;
+    v0 = v1 = __byte_perm(u, 0u, (tig & 1) ? 0x4342u : 0x4140u);
+  }
+  constexpr uint32_t kMask = B == 4 ? 0x000F000Fu : (B == 2 ? 0x00030003u : 0x00010001u);
+  const uint32_t zz = (0x4300u | c.z) * 0x00010001u;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const int sh = B == 4 ? 4 * (t & 3) : t * B;
+    const uint32_t p = and_or((t < 4 ? v0 : v1) >> sh, kMask, 0x43004300u);
+    r[t] = bf2_bits(__hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&p),
+                            *reinterpret_cast<const __nv_bfloat162 *>(&zz)));
+  }
+}
+
+// both rows' operands: one specialised path when every lane of the warp holds the same width
+// in both rows (a stage of one width, or a uniform run of a width map), else the generic one
+__device__ __forceinline__ void rows_operand(const RowCodes &cl, const RowCodes &ch, int tig, uint32_t (&alo)[8],
+                                             uint32_t (&ahi)[8]) {
+  const int b0 = __shfl_sync(0xffffffffu, cl.b, 0);
+  const bool uni = __all_sync(0xffffffffu, cl.b == b0 && ch.b == b0);
+  if (uni && b0 == 2) {
+    row_operand_w<2>(cl, tig, alo);
+    row_operand_w<2>(ch, tig, ahi);
+  } else if (uni && b0 == 4) {
+    row_operand_w<4>(cl, tig, alo);
+    row_operand_w<4>(ch, tig, ahi);
+  } else if (uni && b0 == 1) {
+    row_operand_w<1>(cl, tig, alo);
+    row_operand_w<1>(ch, tig, ahi);
+  } else {
+    row_operand(cl, tig, alo);
+    row_operand(ch, tig, ahi);
+  }
+}
+
+// batch row gid's activations 16 tig .. 16 tig + 15 of group g (zeros past the batch)
+template <bool XF32>
+struct XFrag {
+  uint4 v[XF32 ? 4 : 2];
+};
+template <bool XF32>
+__device__ __forceinline__ XFrag<XF32> load_x(const void *x, int64_t xi, bool has_x) {
+  XFrag<XF32> f;
+#pragma unroll
+  for (int i = 0; i < (XF32 ? 4 : 2); ++i) f.v[i] = make_uint4(0u, 0u, 0u, 0u);
+  if (has_x) {
+    const uint4 *p = XF32 ? reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + xi)
+                          : reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(x) + xi);
+#pragma unroll
+    for (int i = 0; i < (XF32 ? 4 : 2); ++i) f.v[i] = __ldg(p + i);
+  }
+  return f;
+}
+
+// B operand from the fragment, as pairs (t, t + 8): register 2 c feeds MMA c's b0 (codes 2c,
+// 2c + 8), register 2 c + 1 its b1 (codes 2c + 1, 2c + 9); fp32 activations as hi + lo parts
+template <bool XF32>
+__device__ __forceinline__ void b_operand(const XFrag<XF32> &f, uint32_t (&bh)[8], uint32_t (&bl)[8]) {
+  if (XF32) {
+    float xv[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      xv[4 * i] = __uint_as_float(f.v[i].x);
+      xv[4 * i + 1] = __uint_as_float(f.v[i].y);
+      xv[4 * i + 2] = __uint_as_float(f.v[i].z);
+      xv[4 * i + 3] = __uint_as_float(f.v[i].w);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float a = xv[2 * c + h], b = xv[2 * c + h + 8];
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(a, b);
+        bh[2 * c + h] = bf2_bits(hi);
+        bl[2 * c + h] = bf2_bits(__floats2bfloat162_rn(a - __low2float(hi), b - __high2float(hi)));
+      }
+    }
+  } else {
+    const uint32_t lw[4] = {f.v[0].x, f.v[0].y, f.v[0].z, f.v[0].w};
+    const uint32_t hw[4] = {f.v[1].x, f.v[1].y, f.v[1].z, f.v[1].w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      bh[2 * c] = __byte_perm(lw[c], hw[c], 0x5410);
+      bh[2 * c + 1] = __byte_perm(lw[c], hw[c], 0x7632);
+      bl[2 * c] = bl[2 * c + 1] = 0u;
+    }
+  }
+}
+
+// CTA = one 16-row tile at a time (grid-stride); its warps split the tile's groups into
+// contiguous runs and meet in shared memory, where the partial sums are added in warp order
+// (deterministic, no atomics). A warp walks its (stage, group) items as a software pipeline:
+// the widths and offsets of item i + 2 and the code bytes, scales, zero points and activations
+// of item i + 1 are in flight while item i is multiplied, so the offset -> code dependence of
+// the packed format costs no round trip of its own.
+template <bool XF32>
+__global__ void __launch_bounds__(kThreads, 1)
+gemv_vb_kernel(const __grid_constant__ StageSet ss, int count, const void *__restrict__ x, int m, int64_t N,
+               int64_t K, float *__restrict__ y, bool accumulate) {
+  __shared__ float red[kWarps][kTileRows * 8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int64_t KG = K >> 6;
+  const int64_t ga = KG * warp / kWarps;
+  const int L = static_cast<int>(KG * (warp + 1) / kWarps - ga);
+  const int n_items = L * count;
+  const bool has_x = gid < m;
+  const int64_t xrow = static_cast<int64_t>(has_x ? gid : 0) * K + 16 * tig;
+  const int64_t n_tiles = (N + kTileRows - 1) / kTileRows;
+  for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+    const int64_t r0 = tile * kTileRows;
+    const int64_t glo = (r0 + gid < N ? r0 + gid : N - 1) * KG + ga;
+    const int64_t ghi = (r0 + gid + 8 < N ? r0 + gid + 8 : N - 1) * KG + ga;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};     // (row gid | gid + 8) x (batch 2 tig, 2 tig + 1)
+    // item i = (stage j, group ga + g), g fastest; three cursors walk the sequence
+    RowMeta ml1 = {}, mh1 = {}, ml2 = {}, mh2 = {};
+    RowCodes cl = {}, ch = {};
+    XFrag<XF32> xf = {};
+    int j1 = 0, g1 = 0;        // item i + 1
+    int j2 = 0, g2 = 0;        // item i + 2
+    auto step = [&](int &j, int &g) {
+      if (++g == L) { g = 0; ++j; }
+    };
+    if (n_items > 0) {
+      ml1 = load_meta(ss, 0, glo);
+      mh1 = load_meta(ss, 0, ghi);
+      step(j1, g1);
+      step(j2, g2);
+      step(j2, g2);
+      if (n_items > 1) {
+        ml2 = load_meta(ss, j1, glo + g1);
+        mh2 = load_meta(ss, j1, ghi + g1);
+      }
+      cl = load_codes(ss, 0, glo, ml1, tig);
+      ch = load_codes(ss, 0, ghi, mh1, tig);
+      xf = load_x<XF32>(x, xrow + ga * 64, has_x);
+    }
+#pragma unroll 2
+    for (int i = 0; i < n_items; ++i) {
+      // prefetch: widths/offsets of item i + 2, codes and activations of item i + 1
+      RowMeta ml3 = ml2, mh3 = mh2;
+      if (i + 2 < n_items) {
+        ml3 = load_meta(ss, j2, glo + g2);
+        mh3 = load_meta(ss, j2, ghi + g2);
+      }
+      RowCodes cl2 = cl, ch2 = ch;
+      XFrag<XF32> xf2 = xf;
+      if (i + 1 < n_items) {
+        cl2 = load_codes(ss, j1, glo + g1, ml2, tig);
+        ch2 = load_codes(ss, j1, ghi + g1, mh2, tig);
+        xf2 = load_x<XF32>(x, xrow + (ga + g1) * 64, has_x);
+      }
+      step(j1, g1);
+      step(j2, g2);
+      // item i
+      uint32_t bh[8], bl[8], alo[8], ahi[8];
+      b_operand<XF32>(xf, bh, bl);
+      rows_operand(cl, ch, tig, alo, ahi);
+      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t a[4] = {alo[2 * c], ahi[2 * c], alo[2 * c + 1], ahi[2 * c + 1]};
+        mma_bf16(d, a, bh[2 * c], bh[2 * c + 1]);
+        if (XF32) mma_bf16(d, a, bl[2 * c], bl[2 * c + 1]);
+      }
+      acc[0] = fmaf(cl.s, d[0], acc[0]);
+      acc[1] = fmaf(cl.s, d[1], acc[1]);
+      acc[2] = fmaf(ch.s, d[2], acc[2]);
+      acc[3] = fmaf(ch.s, d[3], acc[3]);
+      ml2 = ml3;
+      mh2 = mh3;
+      cl = cl2;
+      ch = ch2;
+      xf = xf2;
+    }
+    float *rw = red[warp];
+    rw[gid * 8 + 2 * tig] = acc[0];
+    rw[gid * 8 + 2 * tig + 1] = acc[1];
+    rw[(gid + 8) * 8 + 2 * tig] = acc[2];
+    rw[(gid + 8) * 8 + 2 * tig + 1] = acc[3];
+    __syncthreads();
+    if (threadIdx.x < kTileRows * 8) {
+      const int row = threadIdx.x >> 3, col = threadIdx.x & 7;
+      float v = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) v += red[w][threadIdx.x];
+      if (col < m && r0 + row < N) {
+        float *yp = y + static_cast<int64_t>(col) * N + r0 + row;
+        *yp = accumulate ? *yp + v : v;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ---- a warp per output row, a lane per group: the batch-1 path ----------------------------
+// Lane l owns group 32 p + l of the row in pass p, so the warp's metadata and code reads are
+// coalesced whatever the widths. The lane reads each stage's width, offset, scale and zero point
+// once, then walks the group in four chunks of 16 columns: per chunk it sums the 16 weights over
+// the stages in fp32 (s * (q - z), the product exact) and multiplies them with the chunk of every
+// batch row of x (x stays in L1), so one batch row costs one FMA per weight and stage.
+constexpr int kLaneThreads = 256;
 
 template <bool XBF16>
 __device__ __forceinline__ void load_x16(const void *x, int64_t idx, float (&xv)[16]) {
@@ -55,48 +394,61 @@ __device__ __forceinline__ void load_x16(const void *x, int64_t idx, float (&xv)
   }
 }
 
-// codes 16 c .. 16 c + 15 of one group of width b (LSB-first bit string at src) -> q[16]; the
+// codes 16 c .. 16 c + 15 of one group of width b (LSB-first bit string at src) -> the fp32
+// bit patterns of 2^23 + q (one shift and one LOP3 each, no integer-to-float conversion); the
 // chunk is 2b bytes at byte 2bc, aligned to its size
 __device__ __forceinline__ void load_codes16(const uint8_t *src, int b, int c, uint32_t (&q)[16]) {
   if (b == 2) {
     const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(src + 4 * c));
 #pragma unroll
-    for (int t = 0; t < 16; ++t) q[t] = (w >> (2 * t)) & 3u;
+    for (int t = 0; t < 16; ++t) q[t] = and_or(w >> (2 * t), 3u, 0x4B000000u);
   } else if (b == 4) {
     const uint2 w = __ldg(reinterpret_cast<const uint2 *>(src + 8 * c));
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
-      q[t] = (w.x >> (4 * t)) & 15u;
-      q[8 + t] = (w.y >> (4 * t)) & 15u;
+      q[t] = and_or(w.x >> (4 * t), 15u, 0x4B000000u);
+      q[8 + t] = and_or(w.y >> (4 * t), 15u, 0x4B000000u);
     }
   } else if (b == 1) {
     const uint32_t w = __ldg(reinterpret_cast<const uint16_t *>(src + 2 * c));
 #pragma unroll
-    for (int t = 0; t < 16; ++t) q[t] = (w >> t) & 1u;
+    for (int t = 0; t < 16; ++t) q[t] = and_or(w >> t, 1u, 0x4B000000u);
   } else {
     const uint4 w = __ldg(reinterpret_cast<const uint4 *>(src + 16 * c));
     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int t = 0; t < 16; ++t) q[t] = (ww[t >> 2] >> (8 * (t & 3))) & 255u;
+    for (int t = 0; t < 16; ++t) q[t] = __byte_perm(ww[t >> 2], 0x4B000000u, 0x7440u | (t & 3));
   }
 }
 
-// A warp per output row (grid-stride); lane l owns group 32 p + l in pass p, so the warp's
-// code reads cover 32 consecutive groups. The lane reads each stage's width, offset, scale and
-// zero point of its group once, then walks the group in four chunks of 16 columns: for each
-// chunk it sums the 16 weights over the stages in fp32 and multiplies them with the chunk of
-// every batch row of x (x stays in L1).
-template <bool XBF16, int M>
-__global__ void __launch_bounds__(kThreads)
-gemv_stages_kernel(const __grid_constant__ StageSet ss, int count, const void *__restrict__ x, int m, int64_t N,
-                   int64_t K, float *__restrict__ y, bool accumulate) {
+// Batch 1: a warp per output row (grid-stride); lane l owns group 32 p + l in pass p, so the
+// warp's metadata and code reads cover 32 consecutive groups. The lane reads each stage's width,
+// offset, scale and zero point of its group once, then walks the group in four chunks of 16
+// columns: per chunk it sums the 16 weights over the stages in fp32 (s * (q - z), the product
+// exact) and multiplies them with the 16 activations. The activations are staged once per CTA
+// in shared memory (XS), one group of 64 per row of `pitch` bytes: the pitch is 16 bytes longer
+// than the group, so the 16-byte reads of the 32 lanes (one group each) fall in all 32 banks;
+// when x is too long to stage, lanes read it from L1 with a 128-byte stride.
+__host__ __device__ constexpr int lane_pitch(bool xbf16) { return xbf16 ? 144 : 272; }
+
+template <bool XBF16, bool XS>
+__global__ void __launch_bounds__(kLaneThreads)
+gemv_lane_kernel(const __grid_constant__ StageSet ss, int count, const void *__restrict__ x, int64_t N, int64_t K,
+                 float *__restrict__ y, bool accumulate) {
+  extern __shared__ __align__(16) uint8_t xs[];
+  constexpr int kPitch = lane_pitch(XBF16);
   const int lane = threadIdx.x & 31;
   const int64_t KG = K >> 6;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
-  for (int64_t n = blockIdx.x * static_cast<int64_t>(kThreads / 32) + (threadIdx.x >> 5); n < N; n += warps) {
-    float acc[M];
-#pragma unroll
-    for (int i = 0; i < M; ++i) acc[i] = 0.0f;
+  if (XS) {
+    constexpr int kUnits = XBF16 ? 8 : 16;           // 16-byte units per group of x
+    const uint4 *src = static_cast<const uint4 *>(x);
+    for (int64_t u = threadIdx.x; u < KG * kUnits; u += kLaneThreads)
+      *reinterpret_cast<uint4 *>(xs + (u / kUnits) * kPitch + (u % kUnits) * 16) = __ldg(src + u);
+    __syncthreads();
+  }
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (kLaneThreads / 32);
+  for (int64_t n = blockIdx.x * static_cast<int64_t>(kLaneThreads / 32) + (threadIdx.x >> 5); n < N; n += warps) {
+    float acc = 0.0f;
     for (int64_t gk = lane; gk < KG; gk += 32) {
       const int64_t g = n * KG + gk;
       const uint8_t *src[kPerLaunch];
@@ -108,14 +460,15 @@ gemv_stages_kernel(const __grid_constant__ StageSet ss, int count, const void *_
           int b = 4;
           if (ss.bits[j]) {
             b = __ldg(ss.bits[j] + g);
-            const int slot = b == 1 ? 0 : b == 2 ? 1 : b == 4 ? 2 : 3;
-            src[j] = ss.plane[j][slot] + __ldg(ss.offset[j] + g);
+            const int bb = width_ok(b) ? b : 1;
+            // offsets are multiples of 8 b by construction; the mask keeps a damaged map aligned
+            src[j] = ss.plane[j][width_slot(bb)] + (__ldg(ss.offset[j] + g) & ~static_cast<uint32_t>(8 * bb - 1));
           } else {
             src[j] = ss.plane[j][2] + g * 32;
           }
           bv[j] = width_ok(b) ? b : 0;             // a bad width in a map contributes nothing
           sv[j] = f16_bits_to_f32(__ldg(ss.scale[j] + g));
-          zv[j] = static_cast<float>(__ldg(ss.zero[j] + g));
+          zv[j] = 8388608.0f + static_cast<float>(__ldg(ss.zero[j] + g));   // 2^23 + z
         }
       }
 #pragma unroll 1
@@ -129,37 +482,60 @@ gemv_stages_kernel(const __grid_constant__ StageSet ss, int count, const void *_
             uint32_t q[16];
             load_codes16(src[j], bv[j], c, q);
 #pragma unroll
-            for (int t = 0; t < 16; ++t) wsum[t] = fmaf(sv[j], __fsub_rn(static_cast<float>(q[t]), zv[j]), wsum[t]);
+            for (int t = 0; t < 16; ++t) wsum[t] = fmaf(sv[j], __fsub_rn(__uint_as_float(q[t]), zv[j]), wsum[t]);
           }
         }
+        float xv[16];
+        if (XS) {
+          const uint8_t *p = xs + gk * kPitch + c * (XBF16 ? 32 : 64);
+          if (XBF16) {
 #pragma unroll
-        for (int i = 0; i < M; ++i) {
-          if (i < m) {
-            float xv[16];
-            load_x16<XBF16>(x, i * K + gk * 64 + 16 * c, xv);
+            for (int h = 0; h < 2; ++h) {
+              const uint4 u = *reinterpret_cast<const uint4 *>(p + 16 * h);
+              const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int t = 0; t < 16; ++t) acc[i] = fmaf(wsum[t], xv[t], acc[i]);
+              for (int e = 0; e < 4; ++e) {
+                xv[8 * h + 2 * e] = __uint_as_float(w[e] << 16);
+                xv[8 * h + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float4 f = *reinterpret_cast<const float4 *>(p + 16 * h);
+              xv[4 * h] = f.x; xv[4 * h + 1] = f.y; xv[4 * h + 2] = f.z; xv[4 * h + 3] = f.w;
+            }
           }
+        } else {
+          load_x16<XBF16>(x, gk * 64 + 16 * c, xv);
         }
+#pragma unroll
+        for (int t = 0; t < 16; ++t) acc = fmaf(wsum[t], xv[t], acc);
       }
     }
 #pragma unroll
-    for (int i = 0; i < M; ++i) {
-      float v = acc[i];
-#pragma unroll
-      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0 && i < m) y[i * N + n] = accumulate ? y[i * N + n] + v : v;
-    }
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) y[n] = accumulate ? y[n] + acc : acc;
   }
 }
 
 template <bool XBF16>
-cq_status launch_m(const StageSet &ss, int count, const void *x, int m, int64_t N, int64_t K, float *y, bool acc,
-                   int blocks, cudaStream_t s) {
-  if (m == 1) gemv_stages_kernel<XBF16, 1><<<blocks, kThreads, 0, s>>>(ss, count, x, m, N, K, y, acc);
-  else if (m <= 4) gemv_stages_kernel<XBF16, 4><<<blocks, kThreads, 0, s>>>(ss, count, x, m, N, K, y, acc);
-  else gemv_stages_kernel<XBF16, 8><<<blocks, kThreads, 0, s>>>(ss, count, x, m, N, K, y, acc);
-  return launch_check("cq_dequant_gemv_stages");
+cq_status launch_lane(const StageSet &ss, int count, const void *x, int64_t N, int64_t K, float *y, bool acc,
+                      cudaStream_t s) {
+  const int64_t smem = (K >> 6) * lane_pitch(XBF16);
+  const bool xs = smem <= 160 * 1024;
+  const int64_t need = (N + 7) / 8, cap = static_cast<int64_t>(sm_count()) * 3;
+  const int blocks = static_cast<int>(need < cap ? need : cap);
+  if (xs) {
+    cq_status st = cuda_check(cudaFuncSetAttribute(gemv_lane_kernel<XBF16, true>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
+                              "cq_dequant_gemv: shared memory attribute");
+    if (st != CQ_OK) return st;
+    gemv_lane_kernel<XBF16, true><<<blocks, kLaneThreads, static_cast<size_t>(smem), s>>>(ss, count, x, N, K, y, acc);
+  } else {
+    gemv_lane_kernel<XBF16, false><<<blocks, kLaneThreads, 0, s>>>(ss, count, x, N, K, y, acc);
+  }
+  return launch_check("cq_dequant_gemv (batch 1, per-group widths / stages)");
 }
 
 }  // namespace
@@ -168,10 +544,10 @@ cq_status launch_gemv_stages(const cq_qweight *const *stages, int count, const v
                              float *y, cudaStream_t s) {
   const int64_t N = stages[0]->rows, K = stages[0]->cols;
   if (N == 0) return CQ_OK;
-  if (K == 0) return cuda_check(cudaMemsetAsync(y, 0, sizeof(float) * m * N, s), "cq_dequant_gemv_stages: zero y");
-  const int64_t need = (N + kThreads / 32 - 1) / (kThreads / 32);
-  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
-  const int blocks = static_cast<int>(need < cap ? need : cap);
+  if (K == 0) return cuda_check(cudaMemsetAsync(y, 0, sizeof(float) * m * N, s), "cq_dequant_gemv: zero y");
+  const int64_t tiles = (N + kTileRows - 1) / kTileRows;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+  const int blocks = static_cast<int>(tiles < cap ? tiles : cap);
   // up to kPerLaunch stages per launch; later launches add to y in stream order
   for (int j0 = 0; j0 < count; j0 += kPerLaunch) {
     const int cnt = count - j0 < kPerLaunch ? count - j0 : kPerLaunch;
@@ -184,8 +560,19 @@ cq_status launch_gemv_stages(const cq_qweight *const *stages, int count, const v
       ss.scale[j] = q.scale;
       ss.zero[j] = q.zero;
     }
-    cq_status st = xdt == CQ_BF16 ? launch_m<true>(ss, cnt, x, m, N, K, y, j0 > 0, blocks, s)
-                                  : launch_m<false>(ss, cnt, x, m, N, K, y, j0 > 0, blocks, s);
+    // batch 1 over a stack of stages: the lane-per-group kernel (measured faster there); any
+    // other batch, and a single matrix of per-group widths, the tensor-core kernel
+    if (m == 1 && count >= 2) {
+      cq_status st = xdt == CQ_BF16 ? launch_lane<true>(ss, cnt, x, N, K, y, j0 > 0, s)
+                                    : launch_lane<false>(ss, cnt, x, N, K, y, j0 > 0, s);
+      if (st != CQ_OK) return st;
+      continue;
+    }
+    if (xdt == CQ_BF16)
+      gemv_vb_kernel<false><<<blocks, kThreads, 0, s>>>(ss, cnt, x, m, N, K, y, j0 > 0);
+    else
+      gemv_vb_kernel<true><<<blocks, kThreads, 0, s>>>(ss, cnt, x, m, N, K, y, j0 > 0);
+    cq_status st = launch_check("cq_dequant_gemv (per-group widths / stages)");
     if (st != CQ_OK) return st;
   }
   return CQ_OK;

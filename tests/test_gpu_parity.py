@@ -339,6 +339,25 @@ def test_gemv_varbits(m):
     check_matmul(host(ops.gemv(qw, x_d)), y_ref, f"vbq m={m}")
 
 
+# the per-group-width kernel: ragged 16-row tiles, group runs that do not split evenly over the
+# CTA's warps (fewer groups than warps, too), fp32 activations (two bf16 parts), and width maps
+# of one width only (8-bit groups take their own operand path)
+@pytest.mark.parametrize("rows,cols,m,x_dtype,only", [(47, 64 * 9, 3, "f32", None), (300, 64 * 21, 8, "bf16", None),
+                                                      (16, 64, 1, "bf16", None), (1000, 4096, 1, "f32", None),
+                                                      (129, 64 * 37, 5, "bf16", 8), (64, 64 * 40, 8, "f32", 8),
+                                                      (200, 64 * 16, 2, "bf16", 1), (33, 64 * 5, 7, "bf16", 2)])
+def test_gemv_varbits_shapes(rows, cols, m, x_dtype, only):
+    G = rows * cols // 64
+    bits = np.full(G, only, np.uint8) if only else synth.vbq_bits(G, seed=rows + cols)
+    qw, x_d, y_ref, _ = _matmul_case(rows, cols, m, x_dtype, bits=bits, seed=rows + m)
+    check_matmul(host(ops.gemv(qw, x_d)), y_ref, f"vbq {rows}x{cols} m={m} {x_dtype} only={only}")
+
+
+def test_gemv_fixed4_fp32_activations():
+    qw, x_d, y_ref, _ = _matmul_case(300, 64 * 21, 6, "f32", seed=17)
+    check_matmul(host(ops.gemv(qw, x_d)), y_ref, "fixed-4 f32 x")
+
+
 @pytest.mark.parametrize("rows,cols,m", [(384, 64 * 40, 16), (384, 64 * 40, 64), (200, 64 * 7, 17),
                                          (1000, 4096, 33), (128, 64, 100), (2500, 2048, 256),
                                          (4096, 4096, 64)])

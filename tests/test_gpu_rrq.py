@@ -91,6 +91,16 @@ def test_rrq_gemv_stages(rows, cols, n_stages, m, x_dtype):
     check_matmul(y, matmul(x, x_dtype), f"rrq {rows}x{cols} stages={n_stages} m={m} {x_dtype}")
 
 
+def test_rrq_gemv_stages_long_rows():
+    """fp32 activations too long to stage in shared memory at batch 1 (read from L1 instead)."""
+    rows, cols = 24, 64 * 640
+    w = synth.normal_weights(rows, cols, seed=21)
+    stages, _, _ = ops.rrq_build(dev(w), 2)
+    matmul = _oracle_stack(w, 2)
+    x = synth.activations(1, cols, seed=22, dtype="f32")
+    check_matmul(host(ops.gemv_stages(stages, dev(x))), matmul(x, "f32"), "rrq long rows f32")
+
+
 def test_rrq_more_stages_approach_the_weights():
     """The stack's product approaches the unquantized weights' product stage by stage
     (each 2-bit stage shrinks the residual about threefold)."""
