@@ -32,6 +32,7 @@ def varbits_index(bits, stream=None):
     offset = torch.empty(bits.numel(), dtype=torch.int32, device=dev)
     pb = torch.empty(4, dtype=torch.int64, device=dev)
     cq.cq_varbits_index(bits, offset, pb, stream)
+    (stream if stream is not None else torch.cuda.current_stream()).synchronize()   # pb is read below
     return offset, [int(v) for v in pb.cpu()]
 
 
