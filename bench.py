@@ -378,8 +378,9 @@ def rrq_components(torch, cq, ops, device, peaks, stream):
     """Recurrent residual quantization on the config's 11008x4096 shape (4 two-bit stages =
     the 8-bit model): one stage (quantize the fp32 residual, write codes, scales, zero points
     and the new residual: 9 + 3/64 B per weight), and the stage-stack GEMV at m=1 over 1, 2
-    and 4 stages (per stage 0.25 B codes + 3/64 B scale/zero + 5/64 B width map and offset), at
-    m = 1 and m = 8, rotating over three stacks so the weights come from HBM."""
+    and 4 stages (per stage 0.25 B codes + 3/64 B scale/zero; the stages share one 5/64 B width
+    map and offset index), at m = 1 and m = 8, rotating over three stacks so the weights come
+    from HBM."""
     N, K = 11008, 4096
     G = N * K // GROUP
     w = torch.randn(N, K, device=device) * 0.02
@@ -413,7 +414,7 @@ def rrq_components(torch, cq, ops, device, peaks, stream):
                         cq.cq_dequant_gemv_stages(st[:n], x, y, stream)
             gs.replay()
             t = time_graph(torch, gs, 10, stream) / len(pool)
-            b = n * (N * K // 4 + G * 8)
+            b = n * (N * K // 4 + G * 3) + G * 5        # the stages share one width map and index
             out[f"gemv_m{m}_{n}_stages"] = {"us": t * 1e3, "GBps": b / t / 1e6,
                                             "frac_hbm": b / t / 1e6 / peaks["hbm_gbs"]}
             del gs

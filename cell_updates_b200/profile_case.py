@@ -4,8 +4,9 @@
 
 kernels: gemv (16384x16384, m=1), gemv8 (same, m=8), gemm (8192x28672, m=64), quantize,
 pack, project, verify (projected bf16 residual), revoke (no residual), pair (both checks),
-rrq (one 2-bit residual stage), stages (the stage-stack GEMV, 4 two-bit stages, m=1) -- all
-but the first three on 8192x16384.
+rrq (one 2-bit residual stage), stages / stages8 (the stage-stack GEMV over 4 two-bit stages,
+m=1 / m=8), vbq / vbq8 (the GEMV of a matrix of per-group widths drawn as in the VBQ
+configuration, m=1 / m=8) -- all but the first three on 8192x16384.
 Each is preceded by the set-up launches (random weights, quantize, pack); capture the
 measured kernel with `ncu -k regex:<name> -s <set-up launches + warm-up> -c 1`.
 """
@@ -13,7 +14,7 @@ import argparse
 
 import torch
 
-from . import build, cq, ops
+from . import build, cq, ops, synth
 
 
 def main():
@@ -24,10 +25,13 @@ def main():
     build.build()
     dev = torch.device("cuda")
     torch.manual_seed(0)
-    N, K, m = {"gemv": (16384, 16384, 1), "gemv8": (16384, 16384, 8), "gemm": (8192, 28672, 64)}.get(
-        a.kernel, (8192, 16384, 1))
+    N, K, m = {"gemv": (16384, 16384, 1), "gemv8": (16384, 16384, 8), "gemm": (8192, 28672, 64),
+               "stages8": (8192, 16384, 8), "vbq8": (8192, 16384, 8)}.get(a.kernel, (8192, 16384, 1))
     w = torch.randn(N, K, device=dev) * 0.02
-    qw, codes, _ = ops.quantize_and_pack(w)
+    bits = None
+    if a.kernel in ("vbq", "vbq8"):
+        bits = torch.from_numpy(synth.vbq_bits(N * K // 64, seed=2)).to(dev)
+    qw, codes, _ = ops.quantize_and_pack(w, bits)
     x = torch.randn(m, K, device=dev).to(torch.bfloat16)
     y = torch.empty(m, N, device=dev)
     ws = torch.empty(max(16, cq.cq_gemm_workspace(N, K, m)), dtype=torch.uint8, device=dev)
@@ -39,16 +43,16 @@ def main():
     if a.kernel in ("verify", "pair"):
         cq.cq_project_residual(r, scale, None)     # a residual inside its cells, as after an update
     stages = None
-    if a.kernel == "stages":
+    if a.kernel in ("stages", "stages8"):
         stages, _, _ = ops.rrq_build(w, 4)
     if a.kernel == "rrq":
         rr = w.clone()
-    if a.kernel in ("gemv", "gemv8", "gemm"):
+    if a.kernel in ("gemv", "gemv8", "gemm", "vbq", "vbq8"):
         del w, r                                   # keep the device footprint small under the profiler
         torch.cuda.empty_cache()
     torch.cuda.synchronize()
     for _ in range(a.reps):
-        if a.kernel in ("gemv", "gemv8"):
+        if a.kernel in ("gemv", "gemv8", "vbq", "vbq8"):
             cq.cq_dequant_gemv(qw, x, y)
         elif a.kernel == "gemm":
             cq.cq_dequant_gemm(qw, x, y, ws)
@@ -68,7 +72,7 @@ def main():
             cq.cq_requant_verify_pair(qw.with_residual(r), 0, N * K, mism, first, m0, f0)
         elif a.kernel == "rrq":
             cq.cq_rrq_stage(rr, 2, codes, scale, zero, st)
-        elif a.kernel == "stages":
+        elif a.kernel in ("stages", "stages8"):
             cq.cq_dequant_gemv_stages(stages, x, y)
         else:
             raise SystemExit(f"unknown kernel {a.kernel}")
