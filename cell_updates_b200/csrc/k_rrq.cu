@@ -359,182 +359,187 @@ gemv_vb_kernel(const __grid_constant__ StageSet ss, int count, const void *__res
   }
 }
 
-// ---- a warp per output row, a lane per group: the batch-1 path ----------------------------
-// Lane l owns group 32 p + l of the row in pass p, so the warp's metadata and code reads are
-// coalesced whatever the widths. The lane reads each stage's width, offset, scale and zero point
-// once, then walks the group in four chunks of 16 columns: per chunk it sums the 16 weights over
-// the stages in fp32 (s * (q - z), the product exact) and multiplies them with the chunk of every
-// batch row of x (x stays in L1), so one batch row costs one FMA per weight and stage.
-constexpr int kLaneThreads = 256;
+// ---- batch 1, one matrix of per-group widths: width-sorted passes --------------------------
+// A warp per row. Within a row the groups of one width are consecutive in that width's plane,
+// so the warp first lists the row's groups by width (one coalesced read of the width map per
+// 32 groups, a ballot per width, ranks by popcount) in shared memory, then runs one pass per
+// width in which lane i takes the i-th group of that width: the whole warp decodes one width
+// with constant shifts (no divergence), and the code reads of a pass are contiguous in the
+// plane. Per weight: the code as the bit pattern of 2^23 + q (shift, LOP3), minus 2^23 + z
+// (exact), times x (fp32, staged once per CTA with the padded pitch of the lane kernel), summed
+// per group in fp32 and scaled by s.
+constexpr int kVbqWarps = 8;
+constexpr int kVbqThreads = 32 * kVbqWarps;
+constexpr int kVbqMaxGroups = 1024;        // per row (K <= 65536); longer rows use the tensor-core kernel
+constexpr int kVbqPitch = 272;             // fp32 x: 256 bytes per group + 16
+
+__host__ __device__ constexpr int64_t vbq_smem(int64_t KG) {
+  return KG * kVbqPitch + static_cast<int64_t>(kVbqWarps) * kVbqMaxGroups * 2;
+}
+
+// the 8 B bytes of one group of width B
+template <int B>
+struct GroupCodes {
+  uint32_t w[2 * B];
+};
+template <int B>
+__device__ __forceinline__ GroupCodes<B> load_group(const uint8_t *src) {
+  GroupCodes<B> gc;
+  if (B == 1) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2 *>(src));
+    gc.w[0] = v.x;
+    gc.w[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < B / 2; ++i) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(src) + i);
+      gc.w[4 * i] = v.x; gc.w[4 * i + 1] = v.y; gc.w[4 * i + 2] = v.z; gc.w[4 * i + 3] = v.w;
+    }
+  }
+  return gc;
+}
+
+// sum over the group of (q - z) * x, fp32 (q - z exact from the 2^23 + q bit pattern)
+template <int B>
+__device__ __forceinline__ float group_dot(const GroupCodes<B> &gc, uint32_t z, const uint8_t *xg) {
+  const float zc = 8388608.0f + static_cast<float>(z);
+  constexpr int kPer = 32 / B;                         // codes per word
+  float d = 0.0f;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {                       // 4 codes per 16-byte x read
+    const float4 xv = *reinterpret_cast<const float4 *>(xg + 16 * c);
+    const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int t = 4 * c + e;
+      const uint32_t word = gc.w[t / kPer];
+      const int sh = (t % kPer) * B;
+      const uint32_t bitsq = B == 8 ? __byte_perm(word, 0x4B000000u, 0x7440u | (t % 4))
+                                    : and_or(word >> sh, (1u << B) - 1u, 0x4B000000u);
+      d = fmaf(__fsub_rn(__uint_as_float(bitsq), zc), xa[e], d);
+    }
+  }
+  return d;
+}
+
+// One width pass of a row: lane i takes list entries i, i + 32, ... (the row's groups of width
+// B, or with list == nullptr every group of a fixed-4 stage) two at a time, both groups' loads
+// issued before either product.
+template <int B>
+__device__ __forceinline__ float width_pass(const uint16_t *list, int cnt, int lane, int64_t g0, const uint8_t *pl,
+                                           const uint32_t *offset, const uint16_t *scale, const uint8_t *zero,
+                                           const uint8_t *xs) {
+  float acc = 0.0f;
+  for (int i = lane; i < cnt; i += 64) {
+    const bool two = i + 32 < cnt;
+    const int ga = list ? list[i] : i;
+    const int gb = two ? (list ? list[i + 32] : i + 32) : ga;
+    const uint8_t *sa, *sb;
+    if (offset) {
+      // offsets are multiples of 8 B by construction; the mask keeps a damaged map aligned
+      sa = pl + (__ldg(offset + g0 + ga) & ~static_cast<uint32_t>(8 * B - 1));
+      sb = pl + (__ldg(offset + g0 + gb) & ~static_cast<uint32_t>(8 * B - 1));
+    } else {
+      sa = pl + (g0 + ga) * 32;
+      sb = pl + (g0 + gb) * 32;
+    }
+    const uint32_t za = __ldg(zero + g0 + ga), zb = __ldg(zero + g0 + gb);
+    const float fa = f16_bits_to_f32(__ldg(scale + g0 + ga)), fb = f16_bits_to_f32(__ldg(scale + g0 + gb));
+    const GroupCodes<B> ca = load_group<B>(sa);
+    const GroupCodes<B> cb = load_group<B>(sb);
+    acc = fmaf(fa, group_dot<B>(ca, za, xs + static_cast<int64_t>(ga) * kVbqPitch), acc);
+    if (two) acc = fmaf(fb, group_dot<B>(cb, zb, xs + static_cast<int64_t>(gb) * kVbqPitch), acc);
+  }
+  return acc;
+}
 
 template <bool XBF16>
-__device__ __forceinline__ void load_x16(const void *x, int64_t idx, float (&xv)[16]) {
-  if (XBF16) {
-    const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(x) + idx);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint4 u = __ldg(p + h);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        xv[8 * h + 2 * e] = __uint_as_float(w[e] << 16);
-        xv[8 * h + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-      }
-    }
-  } else {
-    const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(x) + idx);
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const float4 f = __ldg(p + h);
-      xv[4 * h] = f.x;
-      xv[4 * h + 1] = f.y;
-      xv[4 * h + 2] = f.z;
-      xv[4 * h + 3] = f.w;
-    }
-  }
-}
-
-// codes 16 c .. 16 c + 15 of one group of width b (LSB-first bit string at src) -> the fp32
-// bit patterns of 2^23 + q (one shift and one LOP3 each, no integer-to-float conversion); the
-// chunk is 2b bytes at byte 2bc, aligned to its size
-__device__ __forceinline__ void load_codes16(const uint8_t *src, int b, int c, uint32_t (&q)[16]) {
-  if (b == 2) {
-    const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(src + 4 * c));
-#pragma unroll
-    for (int t = 0; t < 16; ++t) q[t] = and_or(w >> (2 * t), 3u, 0x4B000000u);
-  } else if (b == 4) {
-    const uint2 w = __ldg(reinterpret_cast<const uint2 *>(src + 8 * c));
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      q[t] = and_or(w.x >> (4 * t), 15u, 0x4B000000u);
-      q[8 + t] = and_or(w.y >> (4 * t), 15u, 0x4B000000u);
-    }
-  } else if (b == 1) {
-    const uint32_t w = __ldg(reinterpret_cast<const uint16_t *>(src + 2 * c));
-#pragma unroll
-    for (int t = 0; t < 16; ++t) q[t] = and_or(w >> t, 1u, 0x4B000000u);
-  } else {
-    const uint4 w = __ldg(reinterpret_cast<const uint4 *>(src + 16 * c));
-    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int t = 0; t < 16; ++t) q[t] = __byte_perm(ww[t >> 2], 0x4B000000u, 0x7440u | (t & 3));
-  }
-}
-
-// Batch 1: a warp per output row (grid-stride); lane l owns group 32 p + l in pass p, so the
-// warp's metadata and code reads cover 32 consecutive groups. The lane reads each stage's width,
-// offset, scale and zero point of its group once, then walks the group in four chunks of 16
-// columns: per chunk it sums the 16 weights over the stages in fp32 (s * (q - z), the product
-// exact) and multiplies them with the 16 activations. The activations are staged once per CTA
-// in shared memory (XS), one group of 64 per row of `pitch` bytes: the pitch is 16 bytes longer
-// than the group, so the 16-byte reads of the 32 lanes (one group each) fall in all 32 banks;
-// when x is too long to stage, lanes read it from L1 with a 128-byte stride.
-__host__ __device__ constexpr int lane_pitch(bool xbf16) { return xbf16 ? 144 : 272; }
-
-template <bool XBF16, bool XS>
-__global__ void __launch_bounds__(kLaneThreads)
-gemv_lane_kernel(const __grid_constant__ StageSet ss, int count, const void *__restrict__ x, int64_t N, int64_t K,
+__global__ void __launch_bounds__(kVbqThreads, 2)
+gemv_vbq1_kernel(const __grid_constant__ StageSet ss, int count, const void *__restrict__ x, int64_t N, int64_t K,
                  float *__restrict__ y, bool accumulate) {
   extern __shared__ __align__(16) uint8_t xs[];
-  constexpr int kPitch = lane_pitch(XBF16);
-  const int lane = threadIdx.x & 31;
-  const int64_t KG = K >> 6;
-  if (XS) {
-    constexpr int kUnits = XBF16 ? 8 : 16;           // 16-byte units per group of x
-    const uint4 *src = static_cast<const uint4 *>(x);
-    for (int64_t u = threadIdx.x; u < KG * kUnits; u += kLaneThreads)
-      *reinterpret_cast<uint4 *>(xs + (u / kUnits) * kPitch + (u % kUnits) * 16) = __ldg(src + u);
-    __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int KG = static_cast<int>(K >> 6);
+  // stage x as fp32, one group per kVbqPitch bytes
+  for (int64_t u = threadIdx.x; u < static_cast<int64_t>(KG) * 16; u += kVbqThreads) {
+    float4 f;
+    if (XBF16) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2 *>(x) + u);
+      f = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u), __uint_as_float(v.y << 16),
+                      __uint_as_float(v.y & 0xFFFF0000u));
+    } else {
+      f = __ldg(reinterpret_cast<const float4 *>(x) + u);
+    }
+    *reinterpret_cast<float4 *>(xs + (u >> 4) * kVbqPitch + (u & 15) * 16) = f;
   }
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (kLaneThreads / 32);
-  for (int64_t n = blockIdx.x * static_cast<int64_t>(kLaneThreads / 32) + (threadIdx.x >> 5); n < N; n += warps) {
+  __syncthreads();
+  uint16_t *list = reinterpret_cast<uint16_t *>(xs + static_cast<int64_t>(KG) * kVbqPitch) + warp * kVbqMaxGroups;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * kVbqWarps;
+  for (int64_t n = blockIdx.x * static_cast<int64_t>(kVbqWarps) + warp; n < N; n += warps) {
+    const int64_t g0 = n * KG;
     float acc = 0.0f;
-    for (int64_t gk = lane; gk < KG; gk += 32) {
-      const int64_t g = n * KG + gk;
-      const uint8_t *src[kPerLaunch];
-      float sv[kPerLaunch], zv[kPerLaunch];
-      int bv[kPerLaunch];
-#pragma unroll
-      for (int j = 0; j < kPerLaunch; ++j) {
-        if (j < count) {
-          int b = 4;
-          if (ss.bits[j]) {
-            b = __ldg(ss.bits[j] + g);
-            const int bb = width_ok(b) ? b : 1;
-            // offsets are multiples of 8 b by construction; the mask keeps a damaged map aligned
-            src[j] = ss.plane[j][width_slot(bb)] + (__ldg(ss.offset[j] + g) & ~static_cast<uint32_t>(8 * bb - 1));
-          } else {
-            src[j] = ss.plane[j][2] + g * 32;
-          }
-          bv[j] = width_ok(b) ? b : 0;             // a bad width in a map contributes nothing
-          sv[j] = f16_bits_to_f32(__ldg(ss.scale[j] + g));
-          zv[j] = 8388608.0f + static_cast<float>(__ldg(ss.zero[j] + g));   // 2^23 + z
-        }
-      }
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float wsum[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) wsum[t] = 0.0f;
-#pragma unroll
-        for (int j = 0; j < kPerLaunch; ++j) {
-          if (j < count && bv[j]) {
-            uint32_t q[16];
-            load_codes16(src[j], bv[j], c, q);
-#pragma unroll
-            for (int t = 0; t < 16; ++t) wsum[t] = fmaf(sv[j], __fsub_rn(__uint_as_float(q[t]), zv[j]), wsum[t]);
-          }
-        }
-        float xv[16];
-        if (XS) {
-          const uint8_t *p = xs + gk * kPitch + c * (XBF16 ? 32 : 64);
-          if (XBF16) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint4 u = *reinterpret_cast<const uint4 *>(p + 16 * h);
-              const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                xv[8 * h + 2 * e] = __uint_as_float(w[e] << 16);
-                xv[8 * h + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-              }
-            }
-          } else {
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const float4 f = *reinterpret_cast<const float4 *>(p + 16 * h);
-              xv[4 * h] = f.x; xv[4 * h + 1] = f.y; xv[4 * h + 2] = f.z; xv[4 * h + 3] = f.w;
-            }
-          }
-        } else {
-          load_x16<XBF16>(x, gk * 64 + 16 * c, xv);
-        }
-#pragma unroll
-        for (int t = 0; t < 16; ++t) acc = fmaf(wsum[t], xv[t], acc);
+    for (int j = 0; j < count; ++j) {
+      const uint8_t *bits = ss.bits[j];
+      const uint16_t *scale = ss.scale[j];
+      const uint8_t *zero = ss.zero[j];
+      if (!bits) {                 // fixed 4-bit: every group, 32 bytes at 32 g of plane 4
+        acc += width_pass<4>(nullptr, KG, lane, g0, ss.plane[j][2], nullptr, scale, zero, xs);
+        continue;
       }
+      const uint32_t *offset = ss.offset[j];
+      // list the row's groups by width: widths 1, 2, 4, 8 at list offsets base[0..3]
+      int cnt[4] = {0, 0, 0, 0};
+      for (int w0 = 0; w0 < KG; w0 += 32) {
+        const int b = w0 + lane < KG ? __ldg(bits + g0 + w0 + lane) : 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) cnt[c] += __popc(__ballot_sync(0xffffffffu, b == (1 << c)));
+      }
+      int fill[4] = {0, cnt[0], cnt[0] + cnt[1], cnt[0] + cnt[1] + cnt[2]};
+      const int base[4] = {fill[0], fill[1], fill[2], fill[3]};
+      __syncwarp();     // the previous stage's passes have read the list
+      for (int w0 = 0; w0 < KG; w0 += 32) {
+        const int b = w0 + lane < KG ? __ldg(bits + g0 + w0 + lane) : 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t mk = __ballot_sync(0xffffffffu, b == (1 << c));
+          if (b == (1 << c)) list[fill[c] + __popc(mk & lt)] = static_cast<uint16_t>(w0 + lane);
+          fill[c] += __popc(mk);
+        }
+      }
+      __syncwarp();
+      acc += width_pass<1>(list + base[0], cnt[0], lane, g0, ss.plane[j][0], offset, scale, zero, xs);
+      acc += width_pass<2>(list + base[1], cnt[1], lane, g0, ss.plane[j][1], offset, scale, zero, xs);
+      acc += width_pass<4>(list + base[2], cnt[2], lane, g0, ss.plane[j][2], offset, scale, zero, xs);
+      acc += width_pass<8>(list + base[3], cnt[3], lane, g0, ss.plane[j][3], offset, scale, zero, xs);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) y[n] = accumulate ? y[n] + acc : acc;
+    __syncwarp();       // the list is rewritten for the next row
   }
 }
 
 template <bool XBF16>
-cq_status launch_lane(const StageSet &ss, int count, const void *x, int64_t N, int64_t K, float *y, bool acc,
+cq_status launch_vbq1(const StageSet &ss, int count, const void *x, int64_t N, int64_t K, float *y, bool acc,
                       cudaStream_t s) {
-  const int64_t smem = (K >> 6) * lane_pitch(XBF16);
-  const bool xs = smem <= 160 * 1024;
-  const int64_t need = (N + 7) / 8, cap = static_cast<int64_t>(sm_count()) * 3;
+  const int64_t smem = vbq_smem(K >> 6);
+  cq_status st = cuda_check(cudaFuncSetAttribute(gemv_vbq1_kernel<XBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(smem)),
+                            "cq_dequant_gemv: shared memory attribute");
+  if (st != CQ_OK) return st;
+  // one wave of resident CTAs (grid-stride over rows): as many per SM as registers and the
+  // staged activations allow
+  int per_sm = 1;
+  st = cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_vbq1_kernel<XBF16>, kVbqThreads,
+                                                                static_cast<size_t>(smem)),
+                  "cq_dequant_gemv: occupancy");
+  if (st != CQ_OK) return st;
+  const int64_t need = (N + kVbqWarps - 1) / kVbqWarps;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
   const int blocks = static_cast<int>(need < cap ? need : cap);
-  if (xs) {
-    cq_status st = cuda_check(cudaFuncSetAttribute(gemv_lane_kernel<XBF16, true>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
-                              "cq_dequant_gemv: shared memory attribute");
-    if (st != CQ_OK) return st;
-    gemv_lane_kernel<XBF16, true><<<blocks, kLaneThreads, static_cast<size_t>(smem), s>>>(ss, count, x, N, K, y, acc);
-  } else {
-    gemv_lane_kernel<XBF16, false><<<blocks, kLaneThreads, 0, s>>>(ss, count, x, N, K, y, acc);
-  }
+  gemv_vbq1_kernel<XBF16><<<blocks, kVbqThreads, static_cast<size_t>(smem), s>>>(ss, count, x, N, K, y, acc);
   return launch_check("cq_dequant_gemv (batch 1, per-group widths / stages)");
 }
 
@@ -560,11 +565,11 @@ cq_status launch_gemv_stages(const cq_qweight *const *stages, int count, const v
       ss.scale[j] = q.scale;
       ss.zero[j] = q.zero;
     }
-    // batch 1 over a stack of stages: the lane-per-group kernel (measured faster there); any
-    // other batch, and a single matrix of per-group widths, the tensor-core kernel
-    if (m == 1 && count >= 2) {
-      cq_status st = xdt == CQ_BF16 ? launch_lane<true>(ss, cnt, x, N, K, y, j0 > 0, s)
-                                    : launch_lane<false>(ss, cnt, x, N, K, y, j0 > 0, s);
+    // batch 1 (measured faster there): width-sorted passes on CUDA cores; any other batch, or
+    // rows too long to stage, tensor cores
+    if (m == 1 && (K >> 6) <= kVbqMaxGroups && vbq_smem(K >> 6) <= 200 * 1024) {
+      cq_status st = xdt == CQ_BF16 ? launch_vbq1<true>(ss, cnt, x, N, K, y, j0 > 0, s)
+                                    : launch_vbq1<false>(ss, cnt, x, N, K, y, j0 > 0, s);
       if (st != CQ_OK) return st;
       continue;
     }
