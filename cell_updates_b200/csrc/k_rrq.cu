@@ -370,11 +370,12 @@ gemv_vb_kernel(const __grid_constant__ StageSet ss, int count, const void *__res
 // per group in fp32 and scaled by s.
 constexpr int kVbqWarps = 8;
 constexpr int kVbqThreads = 32 * kVbqWarps;
-constexpr int kVbqMaxGroups = 1024;        // per row (K <= 65536); longer rows use the tensor-core kernel
+constexpr int kVbqMaxGroups = 1024;        // per row (u16 list entries); longer rows use the tensor-core kernel
 constexpr int kVbqPitch = 272;             // fp32 x: 256 bytes per group + 16
 
+// staged x, then per warp a list of the row's group indices (u16), KG entries
 __host__ __device__ constexpr int64_t vbq_smem(int64_t KG) {
-  return KG * kVbqPitch + static_cast<int64_t>(kVbqWarps) * kVbqMaxGroups * 2;
+  return KG * kVbqPitch + ((static_cast<int64_t>(kVbqWarps) * KG * 2 + 15) & ~int64_t(15));
 }
 
 // the 8 B bytes of one group of width B
@@ -473,7 +474,7 @@ gemv_vbq1_kernel(const __grid_constant__ StageSet ss, int count, const void *__r
     *reinterpret_cast<float4 *>(xs + (u >> 4) * kVbqPitch + (u & 15) * 16) = f;
   }
   __syncthreads();
-  uint16_t *list = reinterpret_cast<uint16_t *>(xs + static_cast<int64_t>(KG) * kVbqPitch) + warp * kVbqMaxGroups;
+  uint16_t *list = reinterpret_cast<uint16_t *>(xs + static_cast<int64_t>(KG) * kVbqPitch) + warp * KG;
   const uint32_t lt = (1u << lane) - 1u;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * kVbqWarps;
   for (int64_t n = blockIdx.x * static_cast<int64_t>(kVbqWarps) + warp; n < N; n += warps) {
