@@ -425,25 +425,21 @@ __device__ __forceinline__ float group_dot(const GroupCodes<B> &gc, uint32_t z, 
 
 // One width pass of a row: lane i takes list entries i, i + 32, ... (the row's groups of width
 // B, or with list == nullptr every group of a fixed-4 stage) two at a time, both groups' loads
-// issued before either product.
+// issued before either product. The row's groups of one width are consecutive in the plane
+// (offsets are ranks among same-width groups in row-major order, times 8 B), so the i-th one
+// starts 8 B * i bytes after the first: one offset per pass, read by the caller, instead of one
+// dependent offset load per group.
 template <int B>
 __device__ __forceinline__ float width_pass(const uint16_t *list, int cnt, int lane, int64_t g0, const uint8_t *pl,
-                                           const uint32_t *offset, const uint16_t *scale, const uint8_t *zero,
-                                           const uint8_t *xs) {
+                                           const uint16_t *scale, const uint8_t *zero, const uint8_t *xs) {
   float acc = 0.0f;
   for (int i = lane; i < cnt; i += 64) {
     const bool two = i + 32 < cnt;
+    const int ib = two ? i + 32 : i;
     const int ga = list ? list[i] : i;
-    const int gb = two ? (list ? list[i + 32] : i + 32) : ga;
-    const uint8_t *sa, *sb;
-    if (offset) {
-      // offsets are multiples of 8 B by construction; the mask keeps a damaged map aligned
-      sa = pl + (__ldg(offset + g0 + ga) & ~static_cast<uint32_t>(8 * B - 1));
-      sb = pl + (__ldg(offset + g0 + gb) & ~static_cast<uint32_t>(8 * B - 1));
-    } else {
-      sa = pl + (g0 + ga) * 32;
-      sb = pl + (g0 + gb) * 32;
-    }
+    const int gb = list ? list[ib] : ib;
+    const uint8_t *sa = list ? pl + static_cast<int64_t>(i) * (8 * B) : pl + (g0 + ga) * 32;
+    const uint8_t *sb = list ? pl + static_cast<int64_t>(ib) * (8 * B) : pl + (g0 + gb) * 32;
     const uint32_t za = __ldg(zero + g0 + ga), zb = __ldg(zero + g0 + gb);
     const float fa = f16_bits_to_f32(__ldg(scale + g0 + ga)), fb = f16_bits_to_f32(__ldg(scale + g0 + gb));
     const GroupCodes<B> ca = load_group<B>(sa);
@@ -486,7 +482,7 @@ gemv_vbq1_kernel(const __grid_constant__ StageSet ss, int count, const void *__r
       const uint16_t *scale = ss.scale[j];
       const uint8_t *zero = ss.zero[j];
       if (!bits) {                 // fixed 4-bit: every group, 32 bytes at 32 g of plane 4
-        acc += width_pass<4>(nullptr, KG, lane, g0, ss.plane[j][2], nullptr, scale, zero, xs);
+        acc += width_pass<4>(nullptr, KG, lane, g0, ss.plane[j][2], scale, zero, xs);
         continue;
       }
       const uint32_t *offset = ss.offset[j];
@@ -510,10 +506,16 @@ gemv_vbq1_kernel(const __grid_constant__ StageSet ss, int count, const void *__r
         }
       }
       __syncwarp();
-      acc += width_pass<1>(list + base[0], cnt[0], lane, g0, ss.plane[j][0], offset, scale, zero, xs);
-      acc += width_pass<2>(list + base[1], cnt[1], lane, g0, ss.plane[j][1], offset, scale, zero, xs);
-      acc += width_pass<4>(list + base[2], cnt[2], lane, g0, ss.plane[j][2], offset, scale, zero, xs);
-      acc += width_pass<8>(list + base[3], cnt[3], lane, g0, ss.plane[j][3], offset, scale, zero, xs);
+      // where each width's run of this row starts in its plane (the offset of its first group;
+      // a multiple of 8 b by construction, the mask keeps a damaged map aligned)
+      uint32_t first[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        first[c] = cnt[c] ? (__ldg(offset + g0 + list[base[c]]) & ~((8u << c) - 1u)) : 0u;
+      acc += width_pass<1>(list + base[0], cnt[0], lane, g0, ss.plane[j][0] + first[0], scale, zero, xs);
+      acc += width_pass<2>(list + base[1], cnt[1], lane, g0, ss.plane[j][1] + first[1], scale, zero, xs);
+      acc += width_pass<4>(list + base[2], cnt[2], lane, g0, ss.plane[j][2] + first[2], scale, zero, xs);
+      acc += width_pass<8>(list + base[3], cnt[3], lane, g0, ss.plane[j][3] + first[3], scale, zero, xs);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
