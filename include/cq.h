@@ -121,10 +121,10 @@ cq_status cq_rrq_stage(float *r, int64_t rows, int64_t cols, int bits, uint8_t *
  * cq_dequant_gemv_stages -- the multiply over an RRQ stage stack ([RRQ] as above): y[m, rows]
  * (fp32, overwritten) = sum over k of (sum over stages j of s_j (q_j - z_j)) * x[m, k], for
  * 1 <= count <= 8 stages of the same shape, each fixed-4 or with a per-group width map, none
- * with a residual (CQ_ERR_UNSUPPORTED), 1 <= m <= 8, x fp32 or bf16 (16-byte aligned). At
- * m = 1 with two or more stages the stage sum of each weight is formed in fp32 before the
- * product (CUDA cores); otherwise each stage's group adds s_j * sum (q_j - z_j) x with exact
- * products (tensor cores, as cq_dequant_gemv). fp32 accumulation either way.
+ * with a residual (CQ_ERR_UNSUPPORTED), 1 <= m <= 8, x fp32 or bf16 (16-byte aligned). Each
+ * stage's group adds s_j * (sum over the group of (q_j - z_j) x), the group sum in fp32: at
+ * m = 1 on CUDA cores (x rounded to fp32, exact for bf16), at m >= 2 on tensor cores with exact
+ * products (as cq_dequant_gemv). fp32 accumulation either way.
  * Errors: CQ_ERR_ARG (count, NULL, m, dtype), CQ_ERR_SHAPE (unequal shapes), CQ_ERR_ALIGN.
  */
 cq_status cq_dequant_gemv_stages(const cq_qweight *const *stages, int count, const void *x, cq_dtype x_dtype,
@@ -195,12 +195,12 @@ cq_status cq_requant_verify_pair(const cq_qweight *qw, int64_t first_w, int64_t 
  * cq_dequant_gemv -- [VBQ] fused dequantize-and-multiply for decode:
  *     y[i, n] = sum_k (s*(q-z) + r)[n, k] * x[i, k],   i < m, 1 <= m <= 8,
  * products accumulated in fp32. x: [m, cols] of x_dtype (16-byte aligned); y: [m, rows] fp32.
- * y is overwritten. Without a residual every format runs on tensor cores (mma.sync, bf16
- * operands, fp32 accumulation) with exact products: fixed-4 weights with bf16 x as the integer
- * codes against x, the zero point folded in through the group sums of x; per-group widths, and
- * fp32 x, as the integer q - z of each group against x (fp32 x split into two bf16 parts, so
- * |x - hi - lo| <= 2^-17 |x|), the scale applied to each group's fp32 sum. Weights that carry a
- * residual run on an fp32 CUDA-core path.
+ * y is overwritten. Fixed-4 weights with bf16 x and no residual run on tensor cores (mma.sync,
+ * exact products, fp32 accumulation; the zero point enters through the group sums of x). Per-
+ * group widths, and fp32 x, without a residual: at m = 1 on CUDA cores, per group the fp32 sum of
+ * (q - z) x (q - z exact) scaled by s; at m >= 2 on tensor cores with q - z as exact bf16
+ * operands (fp32 x split into two bf16 parts, |x - hi - lo| <= 2^-17 |x|), the scale applied to
+ * each group's fp32 sum. Weights that carry a residual run on an fp32 CUDA-core path.
  */
 cq_status cq_dequant_gemv(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m,
                           float *y, cq_stream_t stream);
