@@ -400,27 +400,56 @@ __device__ __forceinline__ GroupCodes<B> load_group(const uint8_t *src) {
   return gc;
 }
 
-// sum over the group of (q - z) * x, fp32 (q - z exact from the 2^23 + q bit pattern)
+// sum over the group of (q - z) * x, fp32. Widths 1, 2, 4: the codes are read in windows of 8
+// (4 for width 4) that span at most 16 bits; code p of a window is masked in place, so its
+// float bit pattern is 2^23 + q * 2^(p b) (no shift: one LOP3), minus 2^23 + z * 2^(p b) gives
+// (q - z) * 2^(p b) exactly, and each window position has its own accumulator, scaled back by
+// 2^(-p b) once per group (exact). Width 8: byte p of a word is placed into 2^23 + q by PRMT.
 template <int B>
 __device__ __forceinline__ float group_dot(const GroupCodes<B> &gc, uint32_t z, const uint8_t *xg) {
-  const float zc = 8388608.0f + static_cast<float>(z);
-  constexpr int kPer = 32 / B;                         // codes per word
-  float d = 0.0f;
+  if (B == 8) {
+    const float zc = 8388608.0f + static_cast<float>(z);
+    float d = 0.0f;
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {                       // 4 codes per 16-byte x read
-    const float4 xv = *reinterpret_cast<const float4 *>(xg + 16 * c);
-    const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+    for (int c = 0; c < 16; ++c) {
+      const float4 f = *reinterpret_cast<const float4 *>(xg + 16 * c);
+      const float xa[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int t = 4 * c + e;
-      const uint32_t word = gc.w[t / kPer];
-      const int sh = (t % kPer) * B;
-      const uint32_t bitsq = B == 8 ? __byte_perm(word, 0x4B000000u, 0x7440u | (t % 4))
-                                    : and_or(word >> sh, (1u << B) - 1u, 0x4B000000u);
-      d = fmaf(__fsub_rn(__uint_as_float(bitsq), zc), xa[e], d);
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t bitsq = __byte_perm(gc.w[c], 0x4B000000u, 0x7440u | e);
+        d = fmaf(__fsub_rn(__uint_as_float(bitsq), zc), xa[e], d);
+      }
     }
+    return d;
+  } else {
+    constexpr int kWin = B == 4 ? 4 : 8;               // codes per window (8 or 16 bits)
+    float zc[kWin], dp[kWin];
+#pragma unroll
+    for (int p = 0; p < kWin; ++p) {
+      zc[p] = fmaf(static_cast<float>(z), static_cast<float>(1u << (p * B)), 8388608.0f);   // exact
+      dp[p] = 0.0f;
+    }
+#pragma unroll
+    for (int t0 = 0; t0 < 64; t0 += kWin) {
+      const int bit0 = t0 * B;                         // first bit of the window in the group
+      const uint32_t word = gc.w[bit0 / 32] >> (bit0 % 32);
+      float xa[kWin];
+#pragma unroll
+      for (int h = 0; h < kWin / 4; ++h) {
+        const float4 f = *reinterpret_cast<const float4 *>(xg + 4 * (t0 + 4 * h));
+        xa[4 * h] = f.x; xa[4 * h + 1] = f.y; xa[4 * h + 2] = f.z; xa[4 * h + 3] = f.w;
+      }
+#pragma unroll
+      for (int p = 0; p < kWin; ++p) {
+        const uint32_t bitsq = and_or(word, ((1u << B) - 1u) << (p * B), 0x4B000000u);
+        dp[p] = fmaf(__fsub_rn(__uint_as_float(bitsq), zc[p]), xa[p], dp[p]);
+      }
+    }
+    float d = 0.0f;
+#pragma unroll
+    for (int p = 0; p < kWin; ++p) d = fmaf(dp[p], __uint_as_float(static_cast<uint32_t>(127 - p * B) << 23), d);
+    return d;
   }
-  return d;
 }
 
 // One width pass of a row: lane i takes list entries i, i + 32, ... (the row's groups of width
@@ -451,7 +480,7 @@ __device__ __forceinline__ float width_pass(const uint16_t *list, int cnt, int l
 }
 
 template <bool XBF16>
-__global__ void __launch_bounds__(kVbqThreads, 2)
+__global__ void __launch_bounds__(kVbqThreads, 3)
 gemv_vbq1_kernel(const __grid_constant__ StageSet ss, int count, const void *__restrict__ x, int64_t N, int64_t K,
                  float *__restrict__ y, bool accumulate) {
   extern __shared__ __align__(16) uint8_t xs[];
