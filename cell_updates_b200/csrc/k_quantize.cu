@@ -30,10 +30,13 @@ constexpr int kSmem = 1024 + kWarps * kStages * kTileBytes + kWarps * kStages * 
 //
 // With kResid (one stage of recurrent residual quantization, [RRQ] the 2512.18934 listing
 // page, "Recurrent Residual Quantization" abstract: 2-bit round-to-nearest residual
-// corrections stacked on a 2-bit base) the thread then re-reads its group (L2-resident: the
-// tile was just loaded) and writes back, in place, what the stage does not represent:
-// r <- RN32(r - s (q - z)), the product exact; a flagged group keeps its values. w is then
-// read and written by the same thread only, reads first, so it carries no __restrict__.
+// corrections stacked on a 2-bit base) the warp keeps its tile buffer until the stage is done:
+// each thread replaces its group's row in the buffer by what the stage does not represent,
+// r <- RN32(r - s (q - z)) (the product exact; a flagged group keeps its values), and one lane
+// writes the two boxes back in place with TMA stores; the buffer is refilled once the stores
+// have read it. w is read and written through the tensor map only (tiles are disjoint), plus
+// a thread's own rare exact-division re-read of its group before its row is stored, so it
+// carries no __restrict__.
 template <bool kResid>
 __global__ void __launch_bounds__(kThreads, 1)
 quantize_kernel(const __grid_constant__ CUtensorMap tm_w, float *w, int64_t G, const uint8_t *__restrict__ bits,
@@ -96,11 +99,13 @@ quantize_kernel(const __grid_constant__ CUtensorMap tm_w, float *w, int64_t G, c
       asm("min.NaN.f32 %0, %0, %1;\n" : "+f"(lo) : "f"(v[j]));
       asm("max.NaN.f32 %0, %0, %1;\n" : "+f"(hi) : "f"(v[j]));
     }
-    // every lane's words of this slot are in registers (min/max consumed them): refill it
+    // every lane's words of this slot are in registers (min/max consumed them): refill it (a
+    // residual stage refills after writing the slot back)
     __syncwarp();
     ++n_done;
-    {
-      const int64_t next = tile + static_cast<int64_t>(kStages) * stride;
+    const int cur = slot;
+    const int64_t next = tile + static_cast<int64_t>(kStages) * stride;
+    if (!kResid) {
       if (next < n_tiles) {
         if (lane == 0) issue(slot, next);
         ++n_issued;
@@ -175,18 +180,40 @@ quantize_kernel(const __grid_constant__ CUtensorMap tm_w, float *w, int64_t G, c
         __stcs(dst + c, make_uint4(wd[0], wd[1], wd[2], wd[3]));
       }
       if (kResid && !bad) {
-        float4 *rg = reinterpret_cast<float4 *>(w + g * kGroup);
+        // the new residual replaces the group's row of the tile buffer (same swizzled chunks)
+        uint8_t *rrow = ring + cur * kTileBytes + lane * 128;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float4 o = rg[c];
-          __stcs(rg + c, make_float4(__fsub_rn(o.x, __fmul_rn(sf, v[4 * c])), __fsub_rn(o.y, __fmul_rn(sf, v[4 * c + 1])),
-                                     __fsub_rn(o.z, __fmul_rn(sf, v[4 * c + 2])), __fsub_rn(o.w, __fmul_rn(sf, v[4 * c + 3]))));
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            float4 *p4 = reinterpret_cast<float4 *>(rrow + h * kBoxBytes + ((c ^ (lane & 7)) << 4));
+            const float4 o = *p4;
+            const int j = 32 * h + 4 * c;
+            *p4 = make_float4(__fsub_rn(o.x, __fmul_rn(sf, v[j])), __fsub_rn(o.y, __fmul_rn(sf, v[j + 1])),
+                              __fsub_rn(o.z, __fmul_rn(sf, v[j + 2])), __fsub_rn(o.w, __fmul_rn(sf, v[j + 3])));
+          }
         }
       }
       scale[g] = bad ? 0 : s16;
       zero[g] = bad ? 0 : static_cast<uint8_t>(z);
     }
+    if (kResid) {
+      // write the tile back in place (rows past G are not written), then refill the buffer
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const uint8_t *src = ring + cur * kTileBytes;
+        tma_store_2d(&tm_w, src, 0, static_cast<int>(tile * kTileGroups));
+        tma_store_2d(&tm_w, src + kBoxBytes, 32, static_cast<int>(tile * kTileGroups));
+        bulk_commit();
+        bulk_wait_read_all();
+        if (next < n_tiles) issue(cur, next);
+      }
+      if (next < n_tiles) ++n_issued;
+      __syncwarp();
+    }
   }
+  if (kResid && lane == 0) bulk_wait_all();
   // a warp that gave up lets the copies it issued land before the CTA exits
   for (; n_done < n_issued; ++n_done) {
     mbar_wait(bars + slot, phase, abort_flag, nullptr, false);
