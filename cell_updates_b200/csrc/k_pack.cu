@@ -15,21 +15,56 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// 8 codes (one per byte of v) -> 8*b bits, code j at bits [j*b, (j+1)*b)
+// 8 codes (one per byte of v, as the two words lo, hi) -> 8*b bits, code j at bits [j*b, (j+1)*b).
+// Widths 1 and 2 gather four bytes' low bits with one multiply: with bytes c_i < 2^b at bit 8i,
+// x * K (K = 0x10204080 for b = 1, 0x01041040 for b = 2) puts c_i at bit 32 - 4b + b i and every cross
+// term at a distinct lower position (or past bit 31), so no carry reaches the top 4b bits.
+__device__ __forceinline__ uint32_t gather4(uint32_t x, int b) {
+  return b == 1 ? (x * 0x10204080u) >> 28 : (x * 0x01041040u) >> 24;
+}
 __device__ __forceinline__ uint64_t pack8(uint64_t v, int b) {
-  uint64_t out = 0;
-  const uint64_t mask = (1ull << b) - 1ull;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) out |= ((v >> (8 * j)) & mask) << (j * b);
-  return out;
+  const uint32_t lo = static_cast<uint32_t>(v), hi = static_cast<uint32_t>(v >> 32);
+  switch (b) {
+    case 1: return gather4(lo & 0x01010101u, 1) | (gather4(hi & 0x01010101u, 1) << 4);
+    case 2: return gather4(lo & 0x03030303u, 2) | (gather4(hi & 0x03030303u, 2) << 8);
+    case 4: {
+      // nibbles of four bytes -> 16 bits: (x | x >> 4) keeps pairs in each half word
+      const uint32_t a = lo & 0x0F0F0F0Fu, c = hi & 0x0F0F0F0Fu;
+      const uint32_t a2 = (a | (a >> 4)) & 0x00FF00FFu, c2 = (c | (c >> 4)) & 0x00FF00FFu;
+      return static_cast<uint64_t>(__byte_perm(a2, c2, 0x6420));
+    }
+    default: return v;
+  }
 }
 
+// 8*b bits -> 8 codes, one per byte (the inverse of pack8)
+__device__ __forceinline__ uint32_t spread4(uint32_t x, int b) {
+  // the low 4b bits of x -> four bytes of b bits each
+  if (b == 1) {
+    x &= 0xFu;
+    x = (x | (x << 14)) & 0x00030003u;
+    return (x | (x << 7)) & 0x01010101u;
+  }
+  x &= 0xFFu;
+  x = (x | (x << 12)) & 0x000F000Fu;
+  return (x | (x << 6)) & 0x03030303u;
+}
 __device__ __forceinline__ uint64_t unpack8(uint64_t p, int b) {
-  uint64_t out = 0;
-  const uint64_t mask = (1ull << b) - 1ull;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) out |= ((p >> (j * b)) & mask) << (8 * j);
-  return out;
+  const uint32_t w = static_cast<uint32_t>(p);
+  switch (b) {
+    case 1: return spread4(w, 1) | (static_cast<uint64_t>(spread4(w >> 4, 1)) << 32);
+    case 2: return spread4(w, 2) | (static_cast<uint64_t>(spread4(w >> 8, 2)) << 32);
+    case 4: {
+      // 16 bits -> four bytes of one nibble each, per 32-bit half
+      uint32_t a = w & 0xFFFFu, c = w >> 16;
+      a = (a | (a << 8)) & 0x00FF00FFu;
+      c = (c | (c << 8)) & 0x00FF00FFu;
+      a = (a | (a << 4)) & 0x0F0F0F0Fu;
+      c = (c | (c << 4)) & 0x0F0F0F0Fu;
+      return a | (static_cast<uint64_t>(c) << 32);
+    }
+    default: return p;
+  }
 }
 
 __device__ __forceinline__ void store_bytes(uint8_t *dst, uint64_t v, int b) {

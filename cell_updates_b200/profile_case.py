@@ -6,7 +6,9 @@ kernels: gemv (16384x16384, m=1), gemv8 (same, m=8), gemm (8192x28672, m=64), qu
 pack, project, verify (projected bf16 residual), revoke (no residual), pair (both checks),
 rrq (one 2-bit residual stage), stages / stages8 (the stage-stack GEMV over 4 two-bit stages,
 m=1 / m=8), vbq / vbq8 (the GEMV of a matrix of per-group widths drawn as in the VBQ
-configuration, m=1 / m=8) -- all but the first three on 8192x16384.
+configuration, m=1 / m=8), vpack / vunpack / vindex (pack, unpack and the offset index of the
+VBQ configuration's 2048x8192 width map) -- all but the first three and the last three on
+8192x16384.
 Each is preceded by the set-up launches (random weights, quantize, pack); capture the
 measured kernel with `ncu -k regex:<name> -s <set-up launches + warm-up> -c 1`.
 """
@@ -26,10 +28,11 @@ def main():
     dev = torch.device("cuda")
     torch.manual_seed(0)
     N, K, m = {"gemv": (16384, 16384, 1), "gemv8": (16384, 16384, 8), "gemm": (8192, 28672, 64),
-               "stages8": (8192, 16384, 8), "vbq8": (8192, 16384, 8)}.get(a.kernel, (8192, 16384, 1))
+               "stages8": (8192, 16384, 8), "vbq8": (8192, 16384, 8), "vpack": (2048, 8192, 1),
+               "vunpack": (2048, 8192, 1), "vindex": (2048, 8192, 1)}.get(a.kernel, (8192, 16384, 1))
     w = torch.randn(N, K, device=dev) * 0.02
     bits = None
-    if a.kernel in ("vbq", "vbq8"):
+    if a.kernel in ("vbq", "vbq8", "vpack", "vunpack", "vindex"):
         bits = torch.from_numpy(synth.vbq_bits(N * K // 64, seed=2)).to(dev)
     qw, codes, _ = ops.quantize_and_pack(w, bits)
     x = torch.randn(m, K, device=dev).to(torch.bfloat16)
@@ -72,6 +75,12 @@ def main():
             cq.cq_requant_verify_pair(qw.with_residual(r), 0, N * K, mism, first, m0, f0)
         elif a.kernel == "rrq":
             cq.cq_rrq_stage(rr, 2, codes, scale, zero, st)
+        elif a.kernel == "vpack":
+            cq.cq_pack_varbits(codes, N * K // 64, bits, qw.offset, qw.planes)
+        elif a.kernel == "vunpack":
+            cq.cq_unpack_varbits(qw, codes)
+        elif a.kernel == "vindex":
+            cq.cq_varbits_index(bits, qw.offset, torch.empty(4, dtype=torch.int64, device=dev))
         elif a.kernel in ("stages", "stages8"):
             cq.cq_dequant_gemv_stages(stages, x, y)
         else:
