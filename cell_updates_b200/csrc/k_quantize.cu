@@ -138,7 +138,11 @@ quantize_kernel(const __grid_constant__ CUtensorMap tm_w, float *w, int64_t G, c
 #pragma unroll
     for (int j = 0; j < 64; j += 2) {
       const float2 qt = __fmul2_rn(make_float2(v[j], v[j + 1]), make_float2(rc, rc));
-      const float2 t = make_float2(rintf(qt.x), rintf(qt.y));
+      // t = rne(qt) for |qt| < 2^22 as (qt + 1.5 2^23) - 1.5 2^23 (two packed adds, no rounding
+      // instruction); a larger or non-finite qt fails the certificate below (|qt| 2^-22 >= 1, or
+      // NaN) and takes the exact path, which rounds with rintf
+      const float2 t = __fadd2_rn(__fadd2_rn(qt, make_float2(12582912.0f, 12582912.0f)),
+                                  make_float2(-12582912.0f, -12582912.0f));
       const float2 d = __fadd2_rn(qt, make_float2(-t.x, -t.y));
       const float2 m = __ffma2_rn(make_float2(fabsf(qt.x), fabsf(qt.y)), make_float2(0x1p-22f, 0x1p-22f),
                                   make_float2(fabsf(d.x), fabsf(d.y)));
