@@ -6,26 +6,28 @@
 // thelatestinai.com/papers/2512.18934, "Recurrent Residual Quantization" abstract: the weights
 // are a low-bit base plus a sequence of quantized residual corrections (2-bit round-to-nearest
 // stages stacked to 4, 6 and 8 bits), so one artifact serves several precisions; a model of
-// 2(J+1) bits uses the first J+1 stages (made by cq_rrq_stage, k_quantize.cu). One kernel serves
-// both: for a list of stages of one shape, each fixed-4 or with a per-group width map,
+// 2(J+1) bits uses the first J+1 stages (made by cq_rrq_stage, k_quantize.cu). Two kernels serve
+// both, for a list of stages of one shape, each fixed-4 or with a per-group width map:
 //     y[i, n] = sum_j sum_g s_j[n, g] * sum_{k in g} (q_j[n, k] - z_j[n, g]) * x[i, k]
-// (a single VBQ matrix is a list of one stage).
+// (a single VBQ matrix is a list of one stage), chosen by batch size on measurement:
 //
-// Tensor cores, mma.sync m16n8k16 (bf16 operands, fp32 accumulation): a warp takes 16 rows of one
-// group at a time; A is the 16 x 64 block of q - z, B the group's 64 activations of up to 8
-// batch rows. q - z is an integer in [-255, 255], exact in bf16, so every product is exact; the
-// group's four MMAs start from zero and the group result is scaled by s (fp32) and added to the
-// running sums, so the only rounding is fp32 accumulation (fp32 activations enter as two bf16
-// parts, hi + lo, which leaves |x - hi - lo| <= 2^-17 |x|). The contraction over k is a sum, so
-// codes and activations may be paired in any order both operands share: lane (gid, tig) feeds the
-// 16 codes 16 tig .. 16 tig + 15 of rows gid and gid + 8, as the pairs (t, t + 8), and loads the
-// matching 16 activations of batch row gid.
-//
-// For widths 1, 2 and 4 the bf16 pair (128 + q_t, 128 + q_{t+8}) comes from the packed bytes
-// with one shift and one LOP3 whatever the width (the width only sets the shift step and the
-// mask), and one bf16x2 subtraction of 128 + z gives q - z; so rows of different widths in one
-// warp run the same instructions. 8-bit groups (128 + q is not exact in bf16 past q = 127) go
-// through fp32: (2^23 + q) - (2^23 + z), exact, then packed to bf16.
+//  * batch 1, gemv_vbq1_kernel (CUDA cores): a warp per row lists the row's groups by width and
+//    decodes one width per pass with constant masks (below, before the kernel).
+//  * batch 2..8, gemv_vb_kernel (tensor cores, mma.sync m16n8k16, bf16 operands, fp32
+//    accumulation): a warp takes 16 rows of one group at a time; A is the 16 x 64 block of
+//    q - z, B the group's 64 activations of up to 8 batch rows. q - z is an integer in
+//    [-255, 255], exact in bf16, so every product is exact; the group's four MMAs start from zero
+//    and the group result is scaled by s (fp32) and added to the running sums, so the only
+//    rounding is fp32 accumulation (fp32 activations enter as two bf16 parts, hi + lo, which
+//    leaves |x - hi - lo| <= 2^-17 |x|). The contraction over k is a sum, so codes and
+//    activations may be paired in any order both operands share: lane (gid, tig) feeds the 16
+//    codes 16 tig .. 16 tig + 15 of rows gid and gid + 8, as the pairs (t, t + 8), and loads the
+//    matching 16 activations of batch row gid. For widths 1, 2 and 4 the bf16 pair
+//    (128 + q_t, 128 + q_{t+8}) comes from the packed bytes with one shift and one LOP3 whatever
+//    the width (the width only sets the shift step and the mask), and one bf16x2 subtraction of
+//    128 + z gives q - z; so rows of different widths in one warp run the same instructions.
+//    8-bit groups (128 + q is not exact in bf16 past q = 127) go through fp32:
+//    (2^23 + q) - (2^23 + z), exact, then packed to bf16.
 #include "cq_internal.cuh"
 
 namespace cq {
