@@ -311,6 +311,7 @@ def isolated_components(torch, cq, ops, device, peaks, stream):
     out["cellfill_stack"] = cellfill_stack_verify(torch, cq, ops, synth_module(), device, peaks, stream)
     out["rrq"] = rrq_components(torch, cq, ops, device, peaks, stream)
     out["vbq"] = vbq_components(torch, cq, ops, synth_module(), device, peaks, stream)
+    out["scale_verify_2_4e10"] = scale_chunked_verify(torch, cq, ops, synth_module(), device, peaks, stream)
     return out
 
 
@@ -477,6 +478,55 @@ def cellfill_stack_verify(torch, cq, ops, synth, device, peaks, stream):
                      "frac_hbm": n * per_w[name] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
         del g
     del plane, scale, zero, r, qw_r, qw_0
+    torch.cuda.empty_cache()
+    return res
+
+
+def scale_chunked_verify(torch, cq, ops, synth, device, peaks, stream):
+    """The scale configuration's verify: 2.4e10 constrained 4-bit weights with bf16 residuals
+    (~61 GB resident: 12 GB codes, 1.1 GB scales and zeros, 48 GB residuals), built on the
+    device by the counter-based generator (seed 4), projected once, then both CellFill checks
+    (with the residual and revoked) over the whole artifact in chunks of 2^31 weights, the
+    chunks' calls captured in one graph. Rates in weights/s and GB/s (2.5 + 3/64 B per weight)."""
+    n = 24_000_000_000
+    chunk = 1 << 31
+    G = n // GROUP
+    torch.cuda.empty_cache()
+    plane = torch.empty(n // 2, dtype=torch.uint8, device=device)
+    scale = torch.empty(G, dtype=torch.int16, device=device)
+    zero = torch.empty(G, dtype=torch.uint8, device=device)
+    r = torch.empty(n, dtype=torch.bfloat16, device=device)
+    with torch.cuda.stream(stream):
+        cq.cqs_code_words(plane.view(torch.int64), 4, 0, stream)
+        cq.cqs_scales(scale, 4, 0, stream)
+        cq.cqs_zeros(zero, 4, 0, stream)
+        cq.cqs_residual_bf16(r, scale, 4, 0, float(synth.ih4_multiplier(0.3)), stream)
+        cq.cq_project_residual(r, scale, None, stream)
+    torch.cuda.synchronize()
+    qw = cq.QWeight(1, n, [None, None, plane, None], scale, zero, residual=r)
+    starts = list(range(0, n, chunk))
+    cnt = torch.zeros((len(starts), 4), dtype=torch.int64, device=device)
+
+    def run():
+        for i, c0 in enumerate(starts):
+            nw = min(chunk, n - c0)
+            cq.cq_requant_verify_pair(qw, c0, nw, cnt[i, 0:1], cnt[i, 1:2], cnt[i, 2:3], cnt[i, 3:4], None, stream)
+
+    with torch.cuda.stream(stream):
+        run()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            run()
+    g.replay()
+    ms = time_graph(torch, g, 5, stream)
+    c = cnt.cpu()
+    assert int(c[:, 0].sum()) == 0 and int(c[:, 2].sum()) == 0, "scale verify: mismatches after projection"
+    per_w = 2.5 + 3.0 / GROUP
+    res = {"weights": n, "chunks": len(starts), "ms": ms, "weights_per_s": n / (ms * 1e-3),
+           "GBps": n * per_w / (ms * 1e-3) / 1e9, "frac_hbm": n * per_w / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del g, plane, scale, zero, r, qw
     torch.cuda.empty_cache()
     return res
 
