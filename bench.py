@@ -720,10 +720,11 @@ def _sample_inputs(rows_per_matrix):
     return out
 
 
-def cpu_sample(rows_per_matrix):
-    """The same step on a row sample of each matrix, on the host cores, with the oracle."""
+def cpu_sample(rows_per_matrix, threads=None):
+    """The same step on a row sample of each matrix, on the host cores (all of them unless
+    `threads` is given), with the oracle."""
     from oracle import c_oracle as co
-    threads = co.default_threads()
+    threads = threads or co.default_threads()
     inputs = _sample_inputs(rows_per_matrix)
     nbytes = n_w = 0
     t0 = time.perf_counter()
@@ -750,10 +751,16 @@ def cpu_baseline(rows, min_seconds=10.0):
     while dt < min_seconds:
         b, n, t, threads = cpu_sample(rows)
         nbytes, n_w, dt, reps = nbytes + b, n_w + n, dt + t, reps + 1
+    # the same oracle on one thread, on a quarter of the row sample (one pass)
+    rows1 = max(64, rows // 4)
+    b1, n1, t1, _ = cpu_sample(rows1, threads=1)
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"first {rows} rows of each of the 3 matrices ({n_w // reps} weights), the whole step, "
                       f"repeated {reps}x ({dt:.1f} s)",
-            "seconds": dt}
+            "seconds": dt,
+            "single_thread": {"value": b1 / t1 / 1e9, "unit": "GB/s", "cores": 1,
+                              "sample": f"first {rows1} rows of each of the 3 matrices ({n1} weights), the whole "
+                                        f"step, once ({t1:.1f} s)"}}
 
 
 def run_reference(args, rank, world):
