@@ -353,6 +353,16 @@ def test_gemv_varbits_shapes(rows, cols, m, x_dtype, only):
     check_matmul(host(ops.gemv(qw, x_d)), y_ref, f"vbq {rows}x{cols} m={m} {x_dtype} only={only}")
 
 
+def test_gemv_varbits_rows_too_long_to_stage():
+    """Batch 1 with rows whose staged activations exceed the width-sorted kernel's shared
+    memory (760 groups): the tensor-core kernel takes them."""
+    rows, cols = 40, 64 * 760
+    bits = synth.vbq_bits(rows * cols // 64, seed=23)
+    for x_dtype in ("bf16", "f32"):
+        qw, x_d, y_ref, _ = _matmul_case(rows, cols, 1, x_dtype, bits=bits, seed=29)
+        check_matmul(host(ops.gemv(qw, x_d)), y_ref, f"vbq long rows m=1 {x_dtype}")
+
+
 def test_gemv_fixed4_fp32_activations():
     qw, x_d, y_ref, _ = _matmul_case(300, 64 * 21, 6, "f32", seed=17)
     check_matmul(host(ops.gemv(qw, x_d)), y_ref, "fixed-4 f32 x")
