@@ -199,7 +199,7 @@ cq_status cq_requant_verify_pair(const cq_qweight *qw, int64_t first_w, int64_t 
   const char *fn = "cq_requant_verify_pair";
   cq_status st = check_qweight(qw, fn, true);
   if (st != CQ_OK) return st;
-  if (!qw->residual && qw->rows * qw->cols) return fail(CQ_ERR_ARG, "%s: the pair needs a residual", fn);
+  if (!qw->residual && qw->rows > 0 && qw->cols > 0) return fail(CQ_ERR_ARG, "%s: the pair needs a residual", fn);
   if (!mismatches || !first_bad || !revoke_mismatches || !revoke_first_bad)
     return fail(CQ_ERR_ARG, "%s: a result pointer is NULL", fn);
   const int64_t total = qw->rows * qw->cols;
