@@ -600,6 +600,18 @@ def run_gpu(args, rank, world, local_rank):
         end.record(stream)
     torch.cuda.synchronize()
     t_marked = start.elapsed_time(end) / args.steps
+    # per-step spread: the one-step graph replayed with an event pair around each replay (its
+    # graph-launch latency included), reported as median and p10/p90 beside the K-step headline
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
+    with torch.cuda.stream(stream):
+        for a, b in pairs:
+            a.record(stream)
+            g1.replay()
+            b.record(stream)
+    torch.cuda.synchronize()
+    one = np.array(sorted(a.elapsed_time(b) for a, b in pairs))
+    spread = {"replays": len(pairs), "median_ms": float(np.median(one)), "p10_ms": float(np.percentile(one, 10)),
+              "p90_ms": float(np.percentile(one, 90)), "graph": "one step per replay"}
     per_kernel = {k: 0.0 for k in KERNELS}           # ms summed over every launch
     for mk in marks:
         for k, (a, b) in mk.items():
@@ -638,6 +650,7 @@ def run_gpu(args, rank, world, local_rank):
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_step, "ms_per_step_with_event_nodes": t_marked,
+            "step_spread": spread,
             "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "u4 codes / fp32 quantize / bf16 x, fp32 accumulate",
             "data": "synthetic (seeded Student-t weights, N(0,1) activations, N(0,(0.3s)^2) bf16 residuals)",
