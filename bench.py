@@ -239,6 +239,7 @@ def time_graph(torch, graph, reps, stream):
 
 def isolated_components(torch, cq, ops, device, peaks, stream):
     """Cold-L2 component rates: GEMV (rotating > 2x L2), the 32-layer decode proxy, verify."""
+    torch.manual_seed(2026)              # every draw below (weights, activations) is seeded
     out = {}
     L2 = torch.cuda.get_device_properties(device).L2_cache_size
     # 32-layer 7B-shaped decode: distinct weights per layer (3.54 GB), one graph per token. Per
