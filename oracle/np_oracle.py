@@ -142,13 +142,18 @@ def _rrq_residual(r, deq):
 
 # ---- packed storage ([VBQ]: per-group widths stored bit-packed) ----------------------
 
+def _width_rank(sel):
+    """Number of earlier groups (row-major group order) that have the same width."""
+    return np.cumsum(sel) - sel
+
+
 def varbits_index(bits):
     bits = np.asarray(bits, np.int64)
     off = np.zeros(bits.size, np.uint64)
     plane_bytes = []
     for b in WIDTHS:
         sel = bits == b
-        rank = np.cumsum(sel) - sel          # earlier groups of the same width
+        rank = _width_rank(sel)
         off[sel] = (rank[sel] * 8 * b).astype(np.uint64)
         plane_bytes.append(int(sel.sum()) * 8 * b)
     return off.astype(np.uint32), plane_bytes

@@ -253,6 +253,28 @@ def pin_pack_roundtrip_and_totals(impl, seed=5):
     assert np.array_equal(impl.unpack(planes, G, bits), codes)
 
 
+def pin_index_hand_example(impl):
+    # Widths 2,1,2,4,1,2 worked by hand from the layout (offset = 8b x the number of earlier
+    # groups of the same width, in row-major order): the 2-bit groups 0, 2, 5 are ranks 0, 1, 2
+    # -> 0, 16, 32; the 1-bit groups 1, 4 -> 0, 8; the 4-bit group 3 -> 0.  Plane sizes: two
+    # 1-bit groups (16 B), three 2-bit (48 B), one 4-bit (32 B), none at 8 bits.  A reversed or
+    # column-major rank, or offsets in bits or codes instead of bytes, changes these numbers.
+    bits = np.array([2, 1, 2, 4, 1, 2], np.uint8)
+    off, pbytes = impl.varbits_index(bits)
+    assert np.asarray(off).astype(np.int64).tolist() == [0, 0, 16, 0, 8, 32]
+    assert [int(v) for v in pbytes] == [16, 48, 32, 0]
+    # and pack puts each group's bytes there: constant codes give constant bytes
+    # (2-bit 1 -> 0x55, 2 -> 0xAA, 3 -> 0xFF; 1-bit 1 -> 0xFF, alternating 0,1 -> 0xAA;
+    # 4-bit 7 -> 0x77)
+    codes = np.zeros((6, GROUP), np.uint8)
+    codes[0], codes[1], codes[2], codes[3], codes[5] = 1, 1, 2, 7, 3
+    codes[4] = np.tile([0, 1], 32)
+    planes = impl.pack(codes.ravel(), bits)
+    assert planes[0][:16].tolist() == [0xFF] * 8 + [0xAA] * 8
+    assert planes[1][:48].tolist() == [0x55] * 16 + [0xAA] * 16 + [0xFF] * 16
+    assert planes[2][:32].tolist() == [0x77] * 32
+
+
 # ---- the CellFill invariants -------------------------------------------------------------------
 
 def _random_artifact(rng, G, bits=None, subnormal_scales=False):

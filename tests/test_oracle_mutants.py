@@ -32,6 +32,8 @@ MUTANTS = {
     "verify_drops_residual": ("_served_weight", lambda sf, k, r: sf * k, [P.pin_negative_control]),
     "dequant_zero_sign": ("_dequant_f64", lambda s, q, z: s * (q + z), [P.pin_matmul]),
     "msb_first": ("_BIT_ORDER", "big", [P.pin_pack_lsb_first]),
+    "index_rank_from_the_end": ("_width_rank", lambda sel: sel.sum() - np.cumsum(sel),
+                                [P.pin_index_hand_example]),
     "rrq_residual_sign": ("_rrq_residual", lambda r, deq: r + deq,
                           [P.pin_rrq_residual_inside_half_step, P.pin_rrq_telescopes]),
     "rrq_residual_not_updated": ("_rrq_residual", lambda r, deq: r + np.float32(0) * deq,
