@@ -50,7 +50,7 @@ def load_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-# algorithmic bytes per weight of each step (what the method must move)
+# algorithmic bytes per weight of each step: what the method must move, counted from the formats
 def kernel_bytes(n):
     G = n // GROUP
     meta = 3 * G                      # fp16 scale + u8 zero per group
@@ -798,6 +798,85 @@ def run_reference(args, rank, world):
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def profile_case(kernel, reps=3):
+    """Run one libcq kernel `reps` times on an input larger than the L2 cache, for ncu captures
+    (`ncu -k regex:<kernel name> -s <set-up launches + warm-up> -c 1 python bench.py --case
+    <case>`). Cases: gemv (16384x16384, m=1), gemv8 (same, m=8), gemm (8192x28672, m=64),
+    quantize, pack, project, verify (projected bf16 residual), revoke (no residual), pair (both
+    checks), rrq (one 2-bit residual stage), stages / stages8 (the stage-stack GEMV over four
+    2-bit stages, m=1 / m=8), vbq / vbq8 (the GEMV of a matrix of per-group widths drawn as in
+    the VBQ configuration, m=1 / m=8), vpack / vunpack / vindex (pack, unpack and the offset
+    index of the VBQ configuration's 2048x8192 width map); the others on 8192x16384. Each is
+    preceded by its set-up launches (random weights, quantize, pack)."""
+    import torch
+    from cell_updates_b200 import build, cq, ops, synth
+    from types import SimpleNamespace
+    a = SimpleNamespace(kernel=kernel, reps=reps)
+    build.build()
+    dev = torch.device("cuda")
+    torch.manual_seed(0)
+    N, K, m = {"gemv": (16384, 16384, 1), "gemv8": (16384, 16384, 8), "gemm": (8192, 28672, 64),
+               "stages8": (8192, 16384, 8), "vbq8": (8192, 16384, 8), "vpack": (2048, 8192, 1),
+               "vunpack": (2048, 8192, 1), "vindex": (2048, 8192, 1)}.get(a.kernel, (8192, 16384, 1))
+    w = torch.randn(N, K, device=dev) * 0.02
+    bits = None
+    if a.kernel in ("vbq", "vbq8", "vpack", "vunpack", "vindex"):
+        bits = torch.from_numpy(synth.vbq_bits(N * K // 64, seed=2)).to(dev)
+    qw, codes, _ = ops.quantize_and_pack(w, bits)
+    x = torch.randn(m, K, device=dev).to(torch.bfloat16)
+    y = torch.empty(m, N, device=dev)
+    ws = torch.empty(max(16, cq.cq_gemm_workspace(N, K, m)), dtype=torch.uint8, device=dev)
+    r = (torch.randn(N * K, device=dev) * 1e-3).to(torch.bfloat16)
+    mism = torch.empty(1, dtype=torch.int64, device=dev)
+    first = torch.empty(1, dtype=torch.int64, device=dev)
+    scale, zero = qw.scale, qw.zero
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    if a.kernel in ("verify", "pair"):
+        cq.cq_project_residual(r, scale, None)     # a residual inside its cells, as after an update
+    stages = None
+    if a.kernel in ("stages", "stages8"):
+        stages, _, _ = ops.rrq_build(w, 4)
+    if a.kernel == "rrq":
+        rr = w.clone()
+    if a.kernel in ("gemv", "gemv8", "gemm", "vbq", "vbq8"):
+        del w, r                                   # keep the device footprint small under the profiler
+        torch.cuda.empty_cache()
+    torch.cuda.synchronize()
+    for _ in range(a.reps):
+        if a.kernel in ("gemv", "gemv8", "vbq", "vbq8"):
+            cq.cq_dequant_gemv(qw, x, y)
+        elif a.kernel == "gemm":
+            cq.cq_dequant_gemm(qw, x, y, ws)
+        elif a.kernel == "quantize":
+            cq.cq_quantize(w, None, codes, scale, zero, st)
+        elif a.kernel == "pack":
+            cq.cq_pack_varbits(codes, N * K // 64, None, None, qw.planes)
+        elif a.kernel == "project":
+            cq.cq_project_residual(r, scale, None)
+        elif a.kernel == "verify":
+            cq.cq_requant_verify(qw.with_residual(r), 0, N * K, mism, first)
+        elif a.kernel == "revoke":
+            cq.cq_requant_verify(qw, 0, N * K, mism, first)
+        elif a.kernel == "pair":
+            m0 = torch.empty(1, dtype=torch.int64, device=dev)
+            f0 = torch.empty(1, dtype=torch.int64, device=dev)
+            cq.cq_requant_verify_pair(qw.with_residual(r), 0, N * K, mism, first, m0, f0)
+        elif a.kernel == "rrq":
+            cq.cq_rrq_stage(rr, 2, codes, scale, zero, st)
+        elif a.kernel == "vpack":
+            cq.cq_pack_varbits(codes, N * K // 64, bits, qw.offset, qw.planes)
+        elif a.kernel == "vunpack":
+            cq.cq_unpack_varbits(qw, codes)
+        elif a.kernel == "vindex":
+            cq.cq_varbits_index(bits, qw.offset, torch.empty(4, dtype=torch.int64, device=dev))
+        elif a.kernel in ("stages", "stages8"):
+            cq.cq_dequant_gemv_stages(stages, x, y)
+        else:
+            raise SystemExit(f"unknown kernel {a.kernel}")
+    torch.cuda.synchronize()
+    print("ok", a.kernel, N, K, m)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -807,7 +886,12 @@ def main():
     ap.add_argument("--cpu-sample-rows", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-components", dest="components", action="store_false")
+    ap.add_argument("--case", default=None, help="run one kernel for an ncu capture (see profile_case) and exit")
+    ap.add_argument("--reps", type=int, default=3, help="launches of the --case kernel")
     args = ap.parse_args()
+    if args.case:
+        profile_case(args.case, args.reps)
+        return
     args.warmup = max(args.warmup, 3) if args.impl == "cq" else args.warmup
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", args.gpus if args.gpus == 1 else 1))
