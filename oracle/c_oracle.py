@@ -37,6 +37,9 @@ def lib():
         L.oq_project_bf16.argtypes = [p, p, i64, p]; L.oq_project_bf16.restype = i32
         L.oq_verify.argtypes = [p, p, p, p, p, p, p, p, p, i32, i64, i64, p, p, p, i32]
         L.oq_verify.restype = i32
+        L.oq_reparam_phi.argtypes = [C.c_float]; L.oq_reparam_phi.restype = C.c_float
+        L.oq_reparam.argtypes = [p, p, i64, i32, p]; L.oq_reparam.restype = i32
+        L.oq_reparam_grad.argtypes = [p, p, p, i64, i32, p]; L.oq_reparam_grad.restype = i32
         L.oq_dequant_matmul_f64.argtypes = [p, p, p, p, p, p, p, p, p, i32, i64, i64, p, i32,
                                             i32, p, i32]
         L.oq_dequant_matmul_f64.restype = i32
@@ -197,6 +200,36 @@ def project_bf16(r_bits, scale):
     n = np.zeros(1, np.uint64)
     _check(lib().oq_project_bf16(_ptr(r), _ptr(scale), r.size, _ptr(n)), "oq_project_bf16")
     return r, int(n[0])
+
+
+# ---- bounded reparameterization of the residual ---------------------------------------
+
+def reparam_phi(theta):
+    """phi(theta) = theta / sqrt(1 + theta^2) in binary32, step by step (scalar)."""
+    return float(np.float32(lib().oq_reparam_phi(float(np.float32(theta)))))
+
+
+def reparam(theta, scale, r_dtype="bf16"):
+    """theta f32 [n] -> r = RN(c_dt * phi(theta)): f32 [n], or bf16 bit patterns u16 [n]."""
+    theta = _c(theta, np.float32)
+    scale = _c(scale, np.uint16)
+    assert theta.size == scale.size * 64
+    rd = 1 if r_dtype == "bf16" else 0
+    r = np.zeros(theta.size, np.uint16 if rd else np.float32)
+    _check(lib().oq_reparam(_ptr(theta), _ptr(scale), theta.size, rd, _ptr(r)), "oq_reparam")
+    return r
+
+
+def reparam_grad(theta, scale, grad_r, r_dtype="bf16"):
+    """dL/dtheta [n] f32 from dL/dr [n] f32 (straight through the final rounding)."""
+    theta = _c(theta, np.float32)
+    scale = _c(scale, np.uint16)
+    grad_r = _c(grad_r, np.float32)
+    rd = 1 if r_dtype == "bf16" else 0
+    g = np.zeros(theta.size, np.float32)
+    _check(lib().oq_reparam_grad(_ptr(theta), _ptr(scale), _ptr(grad_r), theta.size, rd, _ptr(g)),
+           "oq_reparam_grad")
+    return g
 
 
 # ---- requant verify -----------------------------------------------------------------

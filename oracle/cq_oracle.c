@@ -321,6 +321,74 @@ int oq_project_bf16(uint16_t *r, const uint16_t *scale, int64_t n, uint64_t *n_c
 }
 
 /* ------------------------------------------------------------------------------
+ * Bounded reparameterization of the residual ([CF] Abstract: CellFill is also offered as a
+ * bounded reparameterization, under which staying inside the cell holds by construction
+ * instead of being restored by a projection).  The pages do not print the bounded map.
+ * Reading: r = RN(c_dt * phi(theta)) with the algebraic sigmoid
+ *     phi(theta) = theta / sqrt(1 + theta^2)        (odd, increasing, |phi| < 1, phi(0) = 0)
+ * and c_dt the projection's bound for the residual's format (c for fp32, c_bf = RZ_bf16(c)
+ * for bf16).  Every step is one IEEE-754 binary32 operation rounded to nearest, in this
+ * order, so any IEEE machine reproduces the residual bit for bit:
+ *     u = RN(theta * theta);  d = RN(1 + u);  q = RN(sqrt(d));  phi = RN(theta / q)
+ * |phi| <= 1 (q >= |theta| in exact arithmetic and RN is monotone), so |r| <= c_dt.
+ * |theta| > 2^32 gives phi = +-1 (the value the formula rounds to there; it avoids the
+ * overflow of theta^2), and a NaN theta gives r = +0 (its update is revoked): no parameter
+ * value, infinities included, can leave the cell.  bf16 r is RN_bf16 of the fp32 product.
+ * Backward, straight through the final rounding:
+ *     dL/dtheta = RN(RN(dL/dr * c_dt) * phi'),  phi' = (1 + theta^2)^(-3/2) = RN(RN(1 / d) / q)
+ * with phi' = 0 for a NaN theta or |theta| > 2^32.
+ * ---------------------------------------------------------------------------- */
+#define REPARAM_SAT 0x1p32f
+
+float oq_reparam_phi(float theta)
+{
+    if (theta != theta) return 0.0f;
+    if (theta > REPARAM_SAT) return 1.0f;
+    if (theta < -REPARAM_SAT) return -1.0f;
+    float u = theta * theta;
+    float d = 1.0f + u;
+    float q = sqrtf(d);
+    return theta / q;
+}
+
+static float reparam_dphi(float theta)
+{
+    if (theta != theta || theta > REPARAM_SAT || theta < -REPARAM_SAT) return 0.0f;
+    float u = theta * theta;
+    float d = 1.0f + u;
+    float q = sqrtf(d);
+    float inv = 1.0f / d;
+    return inv / q;
+}
+
+/* the residual's bound in its format (r_dtype 0 = fp32: c, 1 = bf16: c_bf) */
+static float reparam_bound(uint16_t s16, int r_dtype)
+{
+    float c = cell_halfwidth(s16);
+    return r_dtype ? oq_bf16_to_f32(oq_f32_to_bf16_rz(c)) : c;
+}
+
+int oq_reparam(const float *theta, const uint16_t *scale, int64_t n, int r_dtype, void *r)
+{
+    for (int64_t i = 0; i < n; i++) {
+        float v = reparam_bound(scale[i / GROUP], r_dtype) * oq_reparam_phi(theta[i]);
+        if (r_dtype) ((uint16_t *)r)[i] = oq_f32_to_bf16_rn(v);
+        else ((float *)r)[i] = v;
+    }
+    return 0;
+}
+
+int oq_reparam_grad(const float *theta, const uint16_t *scale, const float *grad_r, int64_t n, int r_dtype,
+                    float *grad_theta)
+{
+    for (int64_t i = 0; i < n; i++) {
+        float gc = grad_r[i] * reparam_bound(scale[i / GROUP], r_dtype);
+        grad_theta[i] = gc * reparam_dphi(theta[i]);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------
  * Re-quantization check ([CF]: re-quantizing the served weights returns the
  * released artifact bit for bit; dropping the residual revokes exactly).
  * For weight i of group g (code q, scale s, zero z, width b, L = 2^b-1):

@@ -227,6 +227,55 @@ def project_bf16(r_bits, scale):
     return ob.ravel(), int((ob != rb).sum())
 
 
+# ---- bounded reparameterization ([CF] Abstract: the bounded-reparameterization form) -----
+# r = RN(c_dt * phi(theta)), phi(theta) = theta / sqrt(1 + theta^2) step by step in binary32
+# (see the C oracle for the reading); NaN -> 0, |theta| > 2^32 -> sign(theta).
+_SAT = np.float32(2.0 ** 32)
+
+
+def _reparam_phi(theta):
+    t = np.asarray(theta, np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        d = np.float32(1) + t * t
+        phi = t / np.sqrt(d)
+    phi = np.where(t > _SAT, np.float32(1), np.where(t < -_SAT, np.float32(-1), phi))
+    return np.where(np.isnan(t), np.float32(0), phi).astype(np.float32)
+
+
+def _reparam_dphi(theta):
+    t = np.asarray(theta, np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        d = np.float32(1) + t * t
+        dphi = (np.float32(1) / d) / np.sqrt(d)
+    dead = np.isnan(t) | (np.abs(t) > _SAT)
+    return np.where(dead, np.float32(0), dphi).astype(np.float32)
+
+
+def _reparam_bound(scale, r_dtype):
+    c = _halfwidth(scale)
+    return _bf16_bound(c) if r_dtype == "bf16" else c
+
+
+def _f32_to_bf16_rn(v):
+    """Finite binary32 -> bf16 bits, round to nearest, ties to even."""
+    u = np.asarray(v, np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def reparam(theta, scale, r_dtype="bf16"):
+    t = np.asarray(theta, np.float32).reshape(-1, GROUP)
+    c = _reparam_bound(scale, r_dtype)[:, None]
+    v = (c * _reparam_phi(t)).astype(np.float32).ravel()
+    return _f32_to_bf16_rn(v) if r_dtype == "bf16" else v
+
+
+def reparam_grad(theta, scale, grad_r, r_dtype="bf16"):
+    t = np.asarray(theta, np.float32).reshape(-1, GROUP)
+    c = _reparam_bound(scale, r_dtype)[:, None]
+    gc = np.asarray(grad_r, np.float32).reshape(-1, GROUP) * c
+    return (gc * _reparam_dphi(t)).astype(np.float32).ravel()
+
+
 # ---- requant verify ([CF]: bit-identical re-quantization, exact revocation) -------------
 
 def verify(planes, scale, zero, bits=None, r=None, r_dtype="f32"):

@@ -44,6 +44,15 @@ class COracle:
     def rrq_stage(self, r, b=2):
         return co.rrq_stage(r, b)
 
+    def reparam_phi(self, theta):
+        return co.reparam_phi(theta)
+
+    def reparam(self, theta, scale, r_dtype="bf16"):
+        return co.reparam(theta, scale, r_dtype)
+
+    def reparam_grad(self, theta, scale, grad_r, r_dtype="bf16"):
+        return co.reparam_grad(theta, scale, grad_r, r_dtype)
+
     def dequant_matmul_f64(self, planes, scale, zero, rows, cols, x, x_dtype="f32", bits=None,
                            r=None, r_dtype="f32"):
         off = None if bits is None else co.varbits_index(bits)[0]
@@ -77,6 +86,15 @@ class NpOracle:
 
     def rrq_stage(self, r, b=2):
         return no.rrq_stage(r, b)
+
+    def reparam_phi(self, theta):
+        return float(no._reparam_phi(np.float32(theta)))
+
+    def reparam(self, theta, scale, r_dtype="bf16"):
+        return no.reparam(theta, scale, r_dtype)
+
+    def reparam_grad(self, theta, scale, grad_r, r_dtype="bf16"):
+        return no.reparam_grad(theta, scale, grad_r, r_dtype)
 
     def dequant_matmul_f64(self, planes, scale, zero, rows, cols, x, x_dtype="f32", bits=None,
                            r=None, r_dtype="f32"):

@@ -511,4 +511,138 @@ def pin_rrq_base_is_the_2bit_quantizer(impl, seed=75):
     assert np.array_equal(r.reshape(-1, GROUP)[g].view(np.uint32), w.reshape(-1, GROUP)[g].view(np.uint32))
 
 
+
+# ---- bounded reparameterization of the residual ([CF] Abstract) -------------------------------
+
+def _rn32(fr):
+    """The binary32 nearest to the rational fr (ties to even), by exact comparison."""
+    x = np.float32(float(fr))
+    best = None
+    for cand in (np.nextafter(x, np.float32(-np.inf)), x, np.nextafter(x, np.float32(np.inf))):
+        d = abs(Fraction(float(cand)) - fr)
+        key = (d, int(np.float32(cand).view(np.uint32)) & 1)
+        if best is None or key < best[0]:
+            best = (key, cand)
+    return float(best[1])
+
+
+def pin_reparam_closed_forms(impl):
+    # theta = a/b with b a power of two and 1 + theta^2 a rational square (Pythagorean triples
+    # 3-4-5, 8-15-17, 16-63-65, 32-255-257): every step before the division is exact, so
+    # phi = RN32(a / c) exactly.
+    for a, b, c in ((3, 4, 5), (15, 8, 17), (63, 16, 65), (255, 32, 257)):
+        theta = a / b
+        assert impl.reparam_phi(theta) == _rn32(Fraction(a, c)), (a, b, c)
+        assert impl.reparam_phi(-theta) == -_rn32(Fraction(a, c)), (a, b, c)
+    assert impl.reparam_phi(0.0) == 0.0
+    assert impl.reparam_phi(np.inf) == 1.0 and impl.reparam_phi(-np.inf) == -1.0
+    assert impl.reparam_phi(3e38) == 1.0 and impl.reparam_phi(-3e38) == -1.0
+    assert impl.reparam_phi(np.nan) == 0.0
+    # theta^2 underflows for a subnormal theta: 1 + 0 = 1, sqrt(1) = 1, phi = theta exactly
+    tiny = float(np.float32(1e-40))
+    assert impl.reparam_phi(tiny) == tiny
+
+
+def _theta_sweep(rng, G):
+    t = rng.uniform(-6, 6, (G, GROUP)).astype(np.float32)
+    specials = np.array([0.0, -0.0, np.inf, -np.inf, np.nan, 3e38, -3e38, 2.0 ** 32, -(2.0 ** 33), 1e-40,
+                         -1e-40, 1e-3, 40.0, -4096.0], np.float32)
+    t[:, :specials.size] = specials
+    return t.ravel()
+
+
+def pin_reparam_stays_in_cell(impl, seed=81):
+    # whatever theta is, the residual is one the (pinned) projection leaves unchanged, and the
+    # artifact re-quantizes to its codes: the invariance needs no projection step
+    rng = np.random.default_rng(seed)
+    G = 300
+    codes, scale, zero = _random_artifact(rng, G, subnormal_scales=True)
+    planes = impl.pack(codes, None)
+    theta = _theta_sweep(rng, G)
+    for dt in ("f32", "bf16"):
+        r = impl.reparam(theta, scale, dt)
+        rp, n = (impl.project_bf16 if dt == "bf16" else impl.project_f32)(r.copy(), scale)
+        assert n == 0 and np.array_equal(np.asarray(rp).view(np.uint8), np.asarray(r).view(np.uint8)), dt
+        m, fb, _ = impl.verify(planes, scale, zero, r=r, r_dtype=dt)
+        assert m == 0 and fb == -1, (dt, m)
+        # NaN parameters revoke their weight's update: r = +0 exactly
+        bits = np.asarray(r).view(np.uint16 if dt == "bf16" else np.uint32)
+        assert not bits[np.isnan(theta)].any()
+        # the bound is reached at the infinities: r = +-c_dt, c_dt being what projecting a huge
+        # residual gives
+        big = np.full(G * GROUP, 1e30, np.float32)
+        if dt == "bf16":
+            big = (big.view(np.uint32) >> 16).astype(np.uint16)
+            cb, _ = impl.project_bf16(big, scale)
+            cf = (cb.astype(np.uint32) << 16).view(np.float32)
+            rf = (bits.astype(np.uint32) << 16).view(np.float32)
+        else:
+            cf, _ = impl.project_f32(big, scale)
+            rf = np.asarray(r, np.float32)
+        assert np.array_equal(rf[theta == np.inf], cf[theta == np.inf])
+        assert np.array_equal(rf[theta == -np.inf], -cf[theta == -np.inf])
+        assert (np.abs(rf) <= cf).all()
+
+
+def pin_reparam_zero_revokes(impl, seed=83):
+    # theta = 0 gives r = +0 everywhere: the served weights are the release's exactly
+    rng = np.random.default_rng(seed)
+    G, rows = 64, 16
+    codes, scale, zero = _random_artifact(rng, G)
+    planes = impl.pack(codes, None)
+    cols = G * GROUP // rows
+    x = rng.standard_normal((2, cols)).astype(np.float32)
+    for dt in ("f32", "bf16"):
+        r = impl.reparam(np.zeros(G * GROUP, np.float32), scale, dt)
+        assert not np.asarray(r).view(np.uint8).any()
+        y0 = impl.dequant_matmul_f64(planes, scale, zero, rows, cols, x)
+        y1 = impl.dequant_matmul_f64(planes, scale, zero, rows, cols, x, r=r, r_dtype=dt)
+        assert np.array_equal(y0, y1)
+
+
+def pin_reparam_monotone_odd(impl, seed=85):
+    rng = np.random.default_rng(seed)
+    G = 40
+    scale = np.full(G, 0x2E66, np.uint16)               # one scale: compare across the sweep
+    theta = np.sort(rng.uniform(-50, 50, G * GROUP).astype(np.float32))
+    for dt in ("f32", "bf16"):
+        r = impl.reparam(theta, scale, dt)
+        rf = ((np.asarray(r).astype(np.uint32) << 16).view(np.float32) if dt == "bf16" else np.asarray(r))
+        # increasing up to the rounding of the steps (the rounded square root can make two
+        # neighbouring quotients differ by an ulp the wrong way)
+        ulp = np.abs(rf[1:]).astype(np.float64) * 2.0 ** -22
+        assert (np.diff(rf.astype(np.float64)) >= -ulp).all(), dt
+        assert rf[0] < 0 < rf[-1]
+        rn = impl.reparam(-theta, scale, dt)
+        rnf = ((np.asarray(rn).astype(np.uint32) << 16).view(np.float32) if dt == "bf16" else np.asarray(rn))
+        assert np.array_equal(rnf, -rf), dt
+
+
+def pin_reparam_gradient(impl, seed=87):
+    # the backward pass against a central finite difference of the fp64 map c * t / sqrt(1 + t^2)
+    # (c = the bound the projection gives), not against the oracle's own derivative formula
+    rng = np.random.default_rng(seed)
+    G = 50
+    scale = np.asarray(rng.uniform(1e-3, 1e-1, G), np.float16).view(np.uint16)
+    theta = rng.uniform(-4, 4, G * GROUP).astype(np.float32)
+    g = rng.standard_normal(G * GROUP).astype(np.float32)
+    for dt in ("f32", "bf16"):
+        big = np.full(G * GROUP, 1e30, np.float32)
+        if dt == "bf16":
+            cb, _ = impl.project_bf16((big.view(np.uint32) >> 16).astype(np.uint16), scale)
+            c = (cb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        else:
+            c = impl.project_f32(big, scale)[0].astype(np.float64)
+        t = theta.astype(np.float64)
+        h = 1e-4
+        f = lambda u: u / np.sqrt(1.0 + u * u)
+        expect = g.astype(np.float64) * c * (f(t + h) - f(t - h)) / (2 * h)
+        got = impl.reparam_grad(theta, scale, g, dt).astype(np.float64)
+        assert np.allclose(got, expect, rtol=1e-5, atol=1e-12 * np.abs(c).max()), dt
+    # no gradient through a saturated or NaN parameter
+    sat = np.array([np.inf, -np.inf, np.nan, 1e30] + [0.5] * 60, np.float32)
+    gs = impl.reparam_grad(sat, scale[:1], np.ones(64, np.float32), "f32")
+    assert not gs[:4].any() and (gs[4:] > 0).all()
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

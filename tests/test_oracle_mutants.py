@@ -32,6 +32,17 @@ MUTANTS = {
     "verify_drops_residual": ("_served_weight", lambda sf, k, r: sf * k, [P.pin_negative_control]),
     "dequant_zero_sign": ("_dequant_f64", lambda s, q, z: s * (q + z), [P.pin_matmul]),
     "msb_first": ("_BIT_ORDER", "big", [P.pin_pack_lsb_first]),
+    "reparam_without_sqrt": ("_reparam_phi", lambda t: (np.asarray(t, np.float32) /
+                                                       (np.float32(1) + np.asarray(t, np.float32) ** 2)),
+                             [P.pin_reparam_closed_forms, P.pin_reparam_stays_in_cell]),
+    "reparam_derivative_power": ("_reparam_dphi", lambda t: (np.float32(1) / np.sqrt(
+                                     np.float32(1) + np.asarray(t, np.float32) ** 2)).astype(np.float32),
+                                 [P.pin_reparam_gradient]),
+    "reparam_nan_kept": ("_reparam_phi", lambda t: np.clip(np.asarray(t, np.float32) / np.sqrt(
+                             np.float32(1) + np.asarray(t, np.float32) ** 2), -1, 1).astype(np.float32),
+                         [P.pin_reparam_stays_in_cell]),
+    "reparam_bf16_bound_rounded_nearest": ("_reparam_bound", lambda s, dt: _rn_bf16(no._halfwidth(s)) if dt == "bf16"
+                                           else no._halfwidth(s), [P.pin_reparam_stays_in_cell]),
     "index_rank_from_the_end": ("_width_rank", lambda sel: sel.sum() - np.cumsum(sel),
                                 [P.pin_index_hand_example]),
     "rrq_residual_sign": ("_rrq_residual", lambda r, deq: r + deq,

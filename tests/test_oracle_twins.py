@@ -60,3 +60,19 @@ def test_chunked_verify_matches_whole():
         if fb >= 0:
             firsts.append(fb)
     assert parts == total and min(firsts) == first
+
+
+def test_reparam_twins_agree():
+    # the bounded reparameterization: C and NumPy give the same bits, forward and backward
+    from oracle import np_oracle as no
+    rng = np.random.default_rng(2027)
+    G = 500
+    scale = rng.integers(1, 0x7BFF, G).astype(np.uint16)
+    theta = (rng.standard_normal(G * 64) * rng.choice([1e-3, 1.0, 30.0, 1e6], G * 64)).astype(np.float32)
+    theta[:8] = [np.inf, -np.inf, np.nan, 0.0, -0.0, 1e-40, 2.0 ** 32, -3e38]
+    g = rng.standard_normal(G * 64).astype(np.float32)
+    for dt in ("f32", "bf16"):
+        a, b = co.reparam(theta, scale, dt), no.reparam(theta, scale, dt)
+        assert np.array_equal(np.asarray(a).view(np.uint8), np.asarray(b).view(np.uint8)), dt
+        ga, gb = co.reparam_grad(theta, scale, g, dt), no.reparam_grad(theta, scale, g, dt)
+        assert np.array_equal(ga.view(np.uint32), gb.view(np.uint32)), dt
