@@ -40,6 +40,8 @@ def lib():
         L.oq_reparam_phi.argtypes = [C.c_float]; L.oq_reparam_phi.restype = C.c_float
         L.oq_reparam.argtypes = [p, p, i64, i32, p]; L.oq_reparam.restype = i32
         L.oq_reparam_grad.argtypes = [p, p, p, i64, i32, p]; L.oq_reparam_grad.restype = i32
+        L.oq_requant_refine.argtypes = [p, i64, i64, p, p, p, i32, p, i32, p, p, p]
+        L.oq_requant_refine.restype = i32
         L.oq_dequant_matmul_f64.argtypes = [p, p, p, p, p, p, p, p, p, i32, i64, i64, p, i32,
                                             i32, p, i32]
         L.oq_dequant_matmul_f64.restype = i32
@@ -230,6 +232,26 @@ def reparam_grad(theta, scale, grad_r, r_dtype="bf16"):
     _check(lib().oq_reparam_grad(_ptr(theta), _ptr(scale), _ptr(grad_r), theta.size, rd, _ptr(g)),
            "oq_reparam_grad")
     return g
+
+
+# ---- ReQuant fixed-grid refinement --------------------------------------------------------
+
+def requant_refine(w, H, codes, scale, zero, b=4, sweeps=1):
+    """Refine codes (u8 [rows*cols], not modified) on the frozen grid against H = X^T X (fp64
+    [cols, cols]) -> (codes, err_before [rows], err_after [rows], moves [rows])."""
+    w = _c(w, np.float32)
+    rows, cols = w.shape
+    H = _c(H, np.float64)
+    assert H.shape == (cols, cols)
+    q = np.array(codes, np.uint8, copy=True).reshape(-1)
+    scale = _c(scale, np.uint16)
+    zero = _c(zero, np.uint8)
+    eb = np.zeros(rows, np.float64)
+    ea = np.zeros(rows, np.float64)
+    mv = np.zeros(rows, np.uint64)
+    _check(lib().oq_requant_refine(_ptr(w), rows, cols, _ptr(H), _ptr(scale), _ptr(zero), int(b), _ptr(q),
+                                   int(sweeps), _ptr(eb), _ptr(ea), _ptr(mv)), "oq_requant_refine")
+    return q, eb, ea, mv
 
 
 # ---- requant verify -----------------------------------------------------------------

@@ -685,3 +685,98 @@ int oq_dequant_matmul_f64(const uint8_t *bits, const uint32_t *offset, const uin
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------------
+ * ReQuant fixed-grid refinement (page 1, thelatestinai.com/papers/2608.20873, ReQuant
+ * abstract: a backpropagation-free stage after any initializer revisits the integer
+ * assignments on the fixed grid; an accepted update strictly lowers the mean squared
+ * reconstruction error and stays on the grid; several sweeps over a round-to-nearest start).
+ * Reading: the error is the layer's output reconstruction error on calibration activations X,
+ *     E(q) = sum_n d_n^T H d_n,   d_n = w_n - s (q_n - z),   H = X^T X   (fp64, K x K)
+ * (in weight space round-to-nearest is already optimal, so the abstract's gains need the output
+ * error); the grid is frozen (s, z unchanged); a candidate update moves one code to a neighbouring
+ * level, q +- 1 inside [0, L]. Rows are independent (E separates over rows). For each row, with
+ * g = H d kept current: one sweep visits k = 0 .. K-1 in order; with S = s of k's group (exact
+ * in fp64), t2 = (S*S)*H_kk, t4 = (2*S)*g_k, the two candidates change E by
+ *     up: t2 - t4 (if q_k < L),   down: t2 + t4 (if q_k > 0);
+ * the smaller one is taken if it is strictly negative (up on a tie); then q_k moves, and every
+ * g_j <- g_j - delta * H_jk with delta = +S or -S. Every operation is one IEEE-754 binary64
+ * operation rounded to nearest (no fused multiply-add) and every sum runs in increasing index
+ * order, so any implementation that keeps this order reproduces the codes exactly:
+ *     d_k = (double)w_k - S*(q_k - z)    (the product exact),
+ *     g_j = (...((0 + H_j0 d_0) + H_j1 d_1) ...) + H_j,K-1 d_K-1
+ * err_before / err_after (per row, may be NULL): sum_k of d_k * g_k in the same way, with d and
+ * g recomputed from scratch; moves (may be NULL): accepted updates per row.
+ * ---------------------------------------------------------------------------- */
+static void rq_residual(const float *w, const uint16_t *scale, const uint8_t *zero, const uint8_t *q, int64_t K,
+                        double *d)
+{
+    for (int64_t k = 0; k < K; k++) {
+        double S = (double)oq_f16_to_f32(scale[k / GROUP]);
+        d[k] = (double)w[k] - S * (double)((int)q[k] - (int)zero[k / GROUP]);
+    }
+}
+
+static void rq_gradient(const double *H, const double *d, int64_t K, double *g)
+{
+    for (int64_t j = 0; j < K; j++) {
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; k++) acc = acc + H[j * K + k] * d[k];
+        g[j] = acc;
+    }
+}
+
+static double rq_error(const double *d, const double *g, int64_t K)
+{
+    double e = 0.0;
+    for (int64_t k = 0; k < K; k++) e = e + d[k] * g[k];
+    return e;
+}
+
+int oq_requant_refine(const float *w, int64_t rows, int64_t cols, const double *H, const uint16_t *scale,
+                      const uint8_t *zero, int b, uint8_t *codes, int sweeps, double *err_before,
+                      double *err_after, uint64_t *moves)
+{
+    if (rows < 0 || cols < 0 || cols % GROUP || !valid_bits(b) || sweeps < 0) return 2;
+    int64_t K = cols, KG = cols / GROUP;
+    int L = (1 << b) - 1;
+    double *d = (double *)malloc((size_t)(K ? K : 1) * sizeof(double));
+    double *g = (double *)malloc((size_t)(K ? K : 1) * sizeof(double));
+    if (!d || !g) { free(d); free(g); return 3; }
+    for (int64_t n = 0; n < rows; n++) {
+        const float *wn = w + n * K;
+        const uint16_t *sn = scale + n * KG;
+        const uint8_t *zn = zero + n * KG;
+        uint8_t *qn = codes + n * K;
+        rq_residual(wn, sn, zn, qn, K, d);
+        rq_gradient(H, d, K, g);
+        if (err_before) err_before[n] = rq_error(d, g, K);
+        uint64_t mv = 0;
+        for (int sw = 0; sw < sweeps; sw++) {
+            for (int64_t k = 0; k < K; k++) {
+                double S = (double)oq_f16_to_f32(sn[k / GROUP]);
+                double t2 = (S * S) * H[k * K + k];
+                double t4 = (2.0 * S) * g[k];
+                double up = t2 - t4, down = t2 + t4;
+                int step = 0;
+                if (qn[k] < L && up < 0.0) step = 1;
+                if (qn[k] > 0 && down < 0.0 && (step == 0 || down < up)) step = -1;
+                if (step) {
+                    double delta = step > 0 ? S : -S;
+                    qn[k] = (uint8_t)(qn[k] + step);
+                    for (int64_t j = 0; j < K; j++) g[j] = g[j] - delta * H[j * K + k];
+                    mv++;
+                }
+            }
+        }
+        if (moves) moves[n] = mv;
+        if (err_after) {
+            rq_residual(wn, sn, zn, qn, K, d);
+            rq_gradient(H, d, K, g);
+            err_after[n] = rq_error(d, g, K);
+        }
+    }
+    free(d);
+    free(g);
+    return 0;
+}

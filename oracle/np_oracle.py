@@ -276,6 +276,74 @@ def reparam_grad(theta, scale, grad_r, r_dtype="bf16"):
     return (gc * _reparam_dphi(t)).astype(np.float32).ravel()
 
 
+# ---- ReQuant fixed-grid refinement (page 1, ReQuant abstract) --------------------------------
+# Output reconstruction error E = sum_n d_n^T H d_n, H = X^T X; one sweep visits the row's codes
+# in order and moves a code to a neighbouring level when that strictly lowers E (see the C
+# oracle for the reading and the order of the binary64 operations).
+
+def _rq_gradient(H, d):
+    """g = H d with the sum over k in increasing order (vectorised over j, sequential over k)."""
+    g = np.zeros(d.size, np.float64)
+    for k in range(d.size):
+        g = g + H[:, k] * d[k]
+    return g
+
+
+def _rq_error(d, g):
+    e = np.float64(0.0)
+    for k in range(d.size):
+        e = e + d[k] * g[k]
+    return float(e)
+
+
+def _rq_changes(sk, hkk, gk):
+    """The change of E for a move up (+s) and down (-s): (s s) H_kk -+ (2 s) g_k."""
+    t2 = (sk * sk) * hkk
+    t4 = (2.0 * sk) * gk
+    return t2 - t4, t2 + t4
+
+
+def _rq_update(g, delta, hk):
+    """g <- g - delta * H[:, k] after a move of delta."""
+    return g - delta * hk
+
+
+def _rq_accept(up, down, q, L):
+    """The move taken: +1, -1 or 0 (a strictly negative change only; up on a tie)."""
+    step = 1 if (q < L and up < 0.0) else 0
+    if q > 0 and down < 0.0 and (step == 0 or down < up):
+        step = -1
+    return step
+
+
+def requant_refine(w, H, codes, scale, zero, b=4, sweeps=1):
+    w = np.asarray(w, np.float32)
+    rows, cols = w.shape
+    H = np.asarray(H, np.float64)
+    q = np.array(codes, np.uint8, copy=True).reshape(rows, cols)
+    S = _f16_to_f32(scale).astype(np.float64).reshape(rows, -1).repeat(GROUP, axis=1)
+    Z = np.asarray(zero, np.int64).reshape(rows, -1).repeat(GROUP, axis=1)
+    L = (1 << b) - 1
+    eb, ea, mv = np.zeros(rows), np.zeros(rows), np.zeros(rows, np.uint64)
+    diag = np.diagonal(H).copy()
+    for n in range(rows):
+        d = w[n].astype(np.float64) - S[n] * (q[n].astype(np.int64) - Z[n]).astype(np.float64)
+        g = _rq_gradient(H, d)
+        eb[n] = _rq_error(d, g)
+        for _ in range(sweeps):
+            for k in range(cols):
+                sk = S[n, k]
+                up, down = _rq_changes(sk, diag[k], g[k])
+                step = _rq_accept(up, down, int(q[n, k]), L)
+                if step:
+                    q[n, k] = int(q[n, k]) + step
+                    g = _rq_update(g, sk if step > 0 else -sk, H[:, k])
+                    mv[n] += 1
+        d = w[n].astype(np.float64) - S[n] * (q[n].astype(np.int64) - Z[n]).astype(np.float64)
+        ea[n] = _rq_error(d, _rq_gradient(H, d))
+    return q.ravel(), eb, ea, mv
+
+
 # ---- requant verify ([CF]: bit-identical re-quantization, exact revocation) -------------
 
 def verify(planes, scale, zero, bits=None, r=None, r_dtype="f32"):

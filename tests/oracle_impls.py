@@ -53,6 +53,9 @@ class COracle:
     def reparam_grad(self, theta, scale, grad_r, r_dtype="bf16"):
         return co.reparam_grad(theta, scale, grad_r, r_dtype)
 
+    def requant_refine(self, w, H, codes, scale, zero, b=4, sweeps=1):
+        return co.requant_refine(w, H, codes, scale, zero, b, sweeps)
+
     def dequant_matmul_f64(self, planes, scale, zero, rows, cols, x, x_dtype="f32", bits=None,
                            r=None, r_dtype="f32"):
         off = None if bits is None else co.varbits_index(bits)[0]
@@ -95,6 +98,9 @@ class NpOracle:
 
     def reparam_grad(self, theta, scale, grad_r, r_dtype="bf16"):
         return no.reparam_grad(theta, scale, grad_r, r_dtype)
+
+    def requant_refine(self, w, H, codes, scale, zero, b=4, sweeps=1):
+        return no.requant_refine(w, H, codes, scale, zero, b, sweeps)
 
     def dequant_matmul_f64(self, planes, scale, zero, rows, cols, x, x_dtype="f32", bits=None,
                            r=None, r_dtype="f32"):

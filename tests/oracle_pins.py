@@ -645,4 +645,102 @@ def pin_reparam_gradient(impl, seed=87):
     assert not gs[:4].any() and (gs[4:] > 0).all()
 
 
+
+# ---- ReQuant fixed-grid refinement (page 1, ReQuant abstract) ---------------------------------
+
+def _calibration(rng, n, K):
+    """Synthetic calibration activations: N(0, 1) with a few outlier input channels (x10)."""
+    X = rng.standard_normal((n, K))
+    X[:, rng.choice(K, max(1, K // 32), replace=False)] *= 10.0
+    return X
+
+
+def _out_error(X, w, codes, scale, zero):
+    """||X (w - s (q - z))^T||^2 per row, straight from the definition (NumPy BLAS, fp64)."""
+    rows, cols = w.shape
+    S = np.asarray(scale, np.uint16).view(np.float16).astype(np.float64).reshape(rows, -1).repeat(GROUP, 1)
+    Z = np.asarray(zero, np.float64).reshape(rows, -1).repeat(GROUP, 1)
+    D = w.astype(np.float64) - S * (np.asarray(codes, np.float64).reshape(rows, cols) - Z)
+    return ((X @ D.T) ** 2).sum(axis=0)
+
+
+def pin_requant_weight_space_is_rtn(impl, seed=91):
+    # With H = I the error is the weight-space one, which round-to-nearest already minimizes:
+    # from the RTN start nothing moves, and from codes pushed one level off the refinement
+    # returns every code to the exact nearest level (brute force over the 16 levels in exact
+    # rational arithmetic; a level exactly half-way keeps its code: only strict gains move).
+    rng = np.random.default_rng(seed)
+    rows, cols = 3, 128
+    w = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    # a hand-made exact tie: group scale 0.25, zero 8, w = 0.125 lies half-way between 0 and 0.25
+    w[0, :64] = (0.25 * (np.arange(64) % 16) - 2.0).astype(np.float32)
+    w[0, 3] = np.float32(0.125)
+    codes, scale, zero, _ = impl.quantize(w)
+    H = np.eye(cols)
+    q, eb, ea, mv = impl.requant_refine(w, H, codes, scale, zero, 4, 1)
+    assert not mv.any() and np.array_equal(q, codes)
+    S = np.asarray(scale, np.uint16).view(np.float16).astype(np.float32)
+    pushed = np.array(codes, np.int64).reshape(rows, cols)
+    for n in range(rows):
+        for k in range(cols):
+            if rng.random() < 0.3 and (n, k) != (0, 3):
+                pushed[n, k] += 1 if pushed[n, k] < 15 else -1
+    q, eb, ea, mv = impl.requant_refine(w, H, pushed.astype(np.uint8).ravel(), scale, zero, 4, 1)
+    q = q.reshape(rows, cols)
+    for n in range(rows):
+        for k in range(cols):
+            g = n * (cols // GROUP) + k // GROUP
+            sf, zz, wf = Fraction(float(S[g])), int(zero[g]), Fraction(float(w[n, k]))
+            errs = [abs(wf - sf * (lv - zz)) for lv in range(16)]
+            best = min(errs)
+            assert errs[int(q[n, k])] == best, (n, k, int(q[n, k]), errs.index(best))
+    assert int(q[0, 3]) == int(codes[3])          # the tie stays where round-to-nearest put it
+
+
+def pin_requant_strictly_lowers_output_error(impl, seed=93):
+    rng = np.random.default_rng(seed)
+    rows, cols = 8, 192
+    w = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    codes, scale, zero, _ = impl.quantize(w)
+    X = _calibration(rng, 300, cols)
+    H = X.T @ X
+    e0 = _out_error(X, w, codes, scale, zero)
+    q, eb, ea, mv = impl.requant_refine(w, H, codes, scale, zero, 4, 2)
+    e1 = _out_error(X, w, q, scale, zero)
+    assert q.max() <= 15                              # still codes of the same 4-bit grid
+    assert mv.sum() > 0
+    assert (e1[mv > 0] < e0[mv > 0]).all() and np.array_equal(e1[mv == 0], e0[mv == 0])
+    assert np.allclose(eb, e0, rtol=1e-9) and np.allclose(ea, e1, rtol=1e-9)
+    # each sweep lowers it further or leaves it
+    q1 = impl.requant_refine(w, H, codes, scale, zero, 4, 1)[0]
+    assert (_out_error(X, w, q1, scale, zero) >= e1 - 1e-12 * e0).all()
+
+
+def pin_requant_local_optimum(impl, seed=95):
+    # swept until a sweep moves nothing, no single move to a neighbouring level lowers the
+    # output error (checked move by move from the definition)
+    rng = np.random.default_rng(seed)
+    rows, cols = 2, 128
+    w = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    codes, scale, zero, _ = impl.quantize(w)
+    X = _calibration(rng, 200, cols)
+    H = X.T @ X
+    q = codes
+    for _ in range(40):
+        q, _, _, mv = impl.requant_refine(w, H, q, scale, zero, 4, 1)
+        if not mv.any():
+            break
+    assert not mv.any()
+    e = _out_error(X, w, q, scale, zero)
+    qq = np.array(q, np.int64).reshape(rows, cols)
+    for n in range(rows):
+        for k in range(cols):
+            for step in (-1, 1):
+                if 0 <= qq[n, k] + step <= 15:
+                    t = qq.copy()
+                    t[n, k] += step
+                    e2 = _out_error(X, w, t.ravel(), scale, zero)
+                    assert e2[n] >= e[n] * (1 - 1e-12), (n, k, step)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

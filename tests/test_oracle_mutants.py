@@ -43,6 +43,13 @@ MUTANTS = {
                          [P.pin_reparam_stays_in_cell]),
     "reparam_bf16_bound_rounded_nearest": ("_reparam_bound", lambda s, dt: _rn_bf16(no._halfwidth(s)) if dt == "bf16"
                                            else no._halfwidth(s), [P.pin_reparam_stays_in_cell]),
+    "requant_accepts_ties": ("_rq_accept", lambda up, down, q, L: (1 if (q < L and up <= 0.0) else
+                                                               (-1 if (q > 0 and down <= 0.0) else 0)),
+                             [P.pin_requant_weight_space_is_rtn]),
+    "requant_change_sign": ("_rq_changes", lambda sk, hkk, gk: ((sk * sk) * hkk + (2.0 * sk) * gk,
+                                                                (sk * sk) * hkk - (2.0 * sk) * gk),
+                            [P.pin_requant_strictly_lowers_output_error]),
+    "requant_stale_gradient": ("_rq_update", lambda g, delta, hk: g, [P.pin_requant_local_optimum]),
     "index_rank_from_the_end": ("_width_rank", lambda sel: sel.sum() - np.cumsum(sel),
                                 [P.pin_index_hand_example]),
     "rrq_residual_sign": ("_rrq_residual", lambda r, deq: r + deq,
