@@ -313,6 +313,7 @@ def isolated_components(torch, cq, ops, device, peaks, stream):
     out["rrq"] = rrq_components(torch, cq, ops, device, peaks, stream)
     out["vbq"] = vbq_components(torch, cq, ops, synth_module(), device, peaks, stream)
     out["scale_verify_2_4e10"] = scale_chunked_verify(torch, cq, ops, synth_module(), device, peaks, stream)
+    out["requant"] = requant_components(torch, cq, ops, device, stream)
     return out
 
 
@@ -434,7 +435,9 @@ def cellfill_stack_verify(torch, cq, ops, synth, device, peaks, stream):
     """The CellFill configuration at its own size: a 28-layer 1.7B-shaped stack
     (1,526,726,656 weights, frozen 4-bit codes, bf16 residuals ~N(0,(0.3 s)^2)) built on the
     device by the counter-based generator; project, verify with the residual, verify without it
-    (revocation), each over the whole stack in one call. Rates in weights/s and GB/s."""
+    (revocation), each over the whole stack in one call; then the bounded reparameterization
+    (bf16 residual from an fp32 parameter theta ~ N(0, 2^2)) and its backward pass, whose
+    residual is verified once more. Rates in weights/s and GB/s."""
     n = 28 * (4 * 2048 * 2048 + 2 * 2048 * 6144 + 6144 * 2048)
     G = n // GROUP
     plane = torch.empty(n // 2, dtype=torch.uint8, device=device)
@@ -452,15 +455,26 @@ def cellfill_stack_verify(torch, cq, ops, synth, device, peaks, stream):
     first = torch.zeros(1, dtype=torch.int64, device=device)
     mism0 = torch.zeros(1, dtype=torch.int64, device=device)
     first0 = torch.zeros(1, dtype=torch.int64, device=device)
+    theta = torch.empty(n, dtype=torch.float32, device=device)
+    grad = torch.empty(n, dtype=torch.float32, device=device)
+    grad_theta = torch.empty(n, dtype=torch.float32, device=device)
+    with torch.cuda.stream(stream):
+        cq.cqs_normal_f32(theta, 3, 9, 0, float(synth.ih4_multiplier(2.0)), stream)
+        cq.cqs_normal_f32(grad, 3, 10, 0, float(synth.ih4_multiplier(1.0)), stream)
+    torch.cuda.synchronize()
     qw_r = cq.QWeight(1, n, [None, None, plane, None], scale, zero, residual=r)
     qw_0 = cq.QWeight(1, n, [None, None, plane, None], scale, zero)
     res = {"weights": n}
     calls = {"project": lambda: cq.cq_project_residual(r, scale, ncl, stream),
              "verify": lambda: cq.cq_requant_verify(qw_r, 0, n, mism, first, None, stream),
              "revoke_verify": lambda: cq.cq_requant_verify(qw_0, 0, n, mism, first, None, stream),
-             "verify_pair": lambda: cq.cq_requant_verify_pair(qw_r, 0, n, mism, first, mism0, first0, None, stream)}
+             "verify_pair": lambda: cq.cq_requant_verify_pair(qw_r, 0, n, mism, first, mism0, first0, None, stream),
+             "reparam": lambda: cq.cq_reparam_residual(theta, scale, r, stream),
+             "reparam_grad": lambda: cq.cq_reparam_residual_grad(theta, scale, grad, grad_theta, cq.CQ_BF16, stream)}
+    # bytes per weight: read theta (4), write the bf16 residual (2) / read theta and dL/dr, write
+    # dL/dtheta (12); plus the group's scale
     per_w = {"project": 4.0 + 2.0 / GROUP, "verify": 2.5 + 3.0 / GROUP, "revoke_verify": 0.5 + 3.0 / GROUP,
-             "verify_pair": 2.5 + 3.0 / GROUP}
+             "verify_pair": 2.5 + 3.0 / GROUP, "reparam": 6.0 + 2.0 / GROUP, "reparam_grad": 12.0 + 2.0 / GROUP}
     for name, fn in calls.items():
         with torch.cuda.stream(stream):
             fn()
@@ -471,16 +485,114 @@ def cellfill_stack_verify(torch, cq, ops, synth, device, peaks, stream):
                 fn()
         g.replay()
         ms = time_graph(torch, g, 10, stream)
-        if name != "project":
+        if name in ("verify", "revoke_verify", "verify_pair"):
             assert int(mism.item()) == 0, f"{name}: {int(mism.item())} mismatches"
         if name == "verify_pair":
             assert int(mism0.item()) == 0, f"{name}: {int(mism0.item())} revocation mismatches"
         res[name] = {"ms": ms, "weights_per_s": n / (ms * 1e-3), "GBps": n * per_w[name] / (ms * 1e-3) / 1e9,
                      "frac_hbm": n * per_w[name] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
         del g
-    del plane, scale, zero, r, qw_r, qw_0
+    # the reparameterized residual re-quantizes to the codes, and dropping it revokes
+    with torch.cuda.stream(stream):
+        cq.cq_requant_verify_pair(qw_r, 0, n, mism, first, mism0, first0, None, stream)
+    torch.cuda.synchronize()
+    assert int(mism.item()) == 0 and int(mism0.item()) == 0, "reparameterized residual left its cell"
+    res["decode_28_layers_served"] = cellfill_decode(torch, cq, plane, scale, zero, r, device, peaks, stream)
+    del plane, scale, zero, r, qw_r, qw_0, theta, grad, grad_theta
     torch.cuda.empty_cache()
     return res
+
+
+def cellfill_decode(torch, cq, plane, scale, zero, r, device, peaks, stream):
+    """Decode over the CellFill stack as served (W = s (q - z) + r, bf16 residual): the 28
+    layers' q, k, v, o (2048x2048), gate and up (6144x2048) and down (2048x6144) are consecutive
+    slices of the stack's artifact; one token = 196 GEMVs at batch 1 in one graph, every weight's
+    code, scale, zero point and residual read once (2.546875 B per weight, 3.89 GB per token)."""
+    shapes = [(2048, 2048)] * 4 + [(6144, 2048)] * 2 + [(2048, 6144)]
+    mats, off = [], 0
+    for _ in range(28):
+        for (N, K) in shapes:
+            n = N * K
+            mats.append(cq.QWeight(N, K, [None, None, plane[off // 2:(off + n) // 2], None],
+                                   scale[off // GROUP:(off + n) // GROUP], zero[off // GROUP:(off + n) // GROUP],
+                                   residual=r[off:off + n]))
+            off += n
+    assert off == plane.numel() * 2
+    xs = {K: torch.randn(1, K, device=device).to(torch.bfloat16) for K in (2048, 6144)}
+    ys = {N: torch.empty(1, N, device=device) for N in (2048, 6144)}
+    token_bytes = off * (2.5 + 3.0 / GROUP)
+
+    def token():
+        for q in mats:
+            cq.cq_dequant_gemv(q, xs[q.cols], ys[q.rows], stream)
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        token()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            token()
+    for _ in range(3):
+        g.replay()
+    t_ms = time_graph(torch, g, 10, stream)
+    out = {"tokens_per_s": 1e3 / t_ms, "ms_per_token": t_ms, "weight_bytes_per_token": token_bytes,
+           "GBps": token_bytes / t_ms / 1e6, "frac_hbm": token_bytes / t_ms / 1e6 / peaks["hbm_gbs"],
+           "ceiling_tokens_per_s": peaks["hbm_gbs"] * 1e9 / token_bytes, "launches_per_token": len(mats)}
+    # per shape over the 28 layers' copies (each shape's pool is larger than L2)
+    per = {}
+    for (N, K) in sorted(set(shapes)):
+        pool = [q for q in mats if q.rows == N and q.cols == K]
+        g1 = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g1, stream=stream):
+                for q in pool:
+                    cq.cq_dequant_gemv(q, xs[K], ys[N], stream)
+        g1.replay()
+        t = time_graph(torch, g1, 5, stream) / len(pool)
+        b = N * K * (2.5 + 3.0 / GROUP)
+        per[f"{N}x{K}"] = {"us": t * 1e3, "GBps": b / t / 1e6, "frac_hbm": b / t / 1e6 / peaks["hbm_gbs"]}
+        del g1
+    out["gemv_m1_cold"] = per
+    del g
+    return out
+
+
+def requant_components(torch, cq, ops, device, stream):
+    """ReQuant on the decode configuration's 4096x4096 shape: round-to-nearest codes of weights
+    ~0.02 t(5) (the same recipe), refined against H = X^T X from 1024 synthetic calibration rows
+    (N(0, 1) with 1/32 of the input channels x10); the gradient pass, one sweep and the closing
+    error pass, then four sweeps. Reports time, accepted moves and the output-error ratio."""
+    from cell_updates_b200 import synth
+    N, K = SHAPES[0]
+    w = torch.from_numpy(synth.student_t_weights(N, K, seed=1)).to(device)
+    codes, scale, zero, _ = ops.quantize(w)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(2027)
+    X = torch.randn(1024, K, device=device, dtype=torch.float64, generator=gen)
+    X[:, torch.randperm(K, device=device, generator=gen)[:K // 32]] *= 10.0
+    H = X.T @ X
+    H = (H + H.T) * 0.5
+    del X
+    out = {"shape": f"{N}x{K}", "calibration_rows": 1024}
+    for sweeps in (1, 4):
+        q = codes.clone()
+        eb = torch.empty(N, dtype=torch.float64, device=device)
+        ea = torch.empty(N, dtype=torch.float64, device=device)
+        mv = torch.empty(N, dtype=torch.int64, device=device)
+        ws = torch.empty(cq.cq_requant_workspace(N, K), dtype=torch.uint8, device=device)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            cq.cq_requant_refine(w, H, scale, zero, 4, q, sweeps, eb, ea, mv, ws, stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        out[f"sweeps_{sweeps}"] = {"ms": ms, "weights_per_s": N * K * sweeps / (ms * 1e-3),
+                                   "moves": int(mv.sum().item()),
+                                   "error_ratio_mean": float((ea / eb).mean().item())}
+    del H, w
+    torch.cuda.empty_cache()
+    return out
 
 
 def scale_chunked_verify(torch, cq, ops, synth, device, peaks, stream):
@@ -632,6 +744,13 @@ def run_gpu(args, rank, world, local_rank):
         comps[k] = {"us_per_step": t_k * 1e3, "GBps": bytes_step[k] / (t_k * 1e-3) / 1e9,
                     "frac_hbm": bytes_step[k] / (t_k * 1e-3) / 1e9 / peaks["hbm_gbs"],
                     "share": per_kernel[k] / max(sum(per_kernel.values()), 1e-12)}
+    # the batch-64 GEMM is a dense contraction: its tensor-core rate against the sustained bf16 peak
+    # (the kernel runs inside a long step) and the burst one
+    t_gemm = per_kernel["gemm"] / args.steps * 1e-3
+    gemm_flops = 2.0 * GEMM_M * wl.n_weights()
+    comps["gemm"]["TFLOPs"] = gemm_flops / t_gemm / 1e12
+    comps["gemm"]["frac_bf16_sustained"] = comps["gemm"]["TFLOPs"] / peaks["bf16_tflops_sustained"]
+    comps["gemm"]["frac_bf16_burst"] = comps["gemm"]["TFLOPs"] / peaks["bf16_tflops"]
     dominant = max(KERNELS, key=lambda k: per_kernel[k])
     achieved = comps[dominant]["GBps"]
     roofline = {"kernel": dominant, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
@@ -657,7 +776,10 @@ def run_gpu(args, rank, world, local_rank):
             "data": "synthetic (seeded Student-t weights, N(0,1) activations, N(0,(0.3s)^2) bf16 residuals)",
             "config": {"workload": WORKLOAD, "weights_per_step": n_w, "gemv_batch": 1, "gemm_batch": GEMM_M,
                        "residual": "bf16", "l2": "inputs larger than L2 (377 MB fp32 weights per step)",
-                       "parallelism": f"replicas x{world}", "step": "+".join(KERNELS)},
+                       "parallelism": f"replicas x{world}", "step": "+".join(KERNELS),
+                       "value_is": "composite: the algorithmic bytes of all six rows of one step over the step "
+                                   "time; the metric's own parts are the top-level dequant_gemv_*, tokens_per_s "
+                                   "and requant_verify_* keys"},
             "roofline": roofline,
             # weights checked per second by the pass that checks both (with r, and revoked)
             "requant_verify_weights_per_s": n_w / (per_kernel["verify_pair"] / args.steps * 1e-3),
@@ -671,7 +793,14 @@ def run_gpu(args, rank, world, local_rank):
         if iso:
             line["isolated"] = iso
             line["tokens_per_s"] = iso["decode_32_layers"]["tokens_per_s"]
+            line["tokens_per_s_frac_of_ceiling"] = (iso["decode_32_layers"]["tokens_per_s"] /
+                                                    iso["decode_32_layers"]["ceiling_tokens_per_s"])
+            line["dequant_gemv_GBps_cold"] = {k: v["GBps"] for k, v in iso["gemv_m1_cold"].items()}
+            served = iso["cellfill_stack"].get("decode_28_layers_served")
+            if served:
+                line["tokens_per_s_cellfill_served"] = served["tokens_per_s"]
             line["requant_verify_weights_per_s_cellfill_stack"] = iso["cellfill_stack"]["verify"]["weights_per_s"]
+            line["requant_verify_weights_per_s_2_4e10"] = iso["scale_verify_2_4e10"]["weights_per_s"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_sample_rows)
     if dist:
@@ -806,7 +935,9 @@ def profile_case(kernel, reps=3):
     checks), rrq (one 2-bit residual stage), stages / stages8 (the stage-stack GEMV over four
     2-bit stages, m=1 / m=8), vbq / vbq8 (the GEMV of a matrix of per-group widths drawn as in
     the VBQ configuration, m=1 / m=8), vpack / vunpack / vindex (pack, unpack and the offset
-    index of the VBQ configuration's 2048x8192 width map); the others on 8192x16384. Each is
+    index of the VBQ configuration's 2048x8192 width map), gemvr (the GEMV with a projected bf16
+    residual, m=1), reparam / reparam_grad (the bounded reparameterization, bf16 residual, and its
+    backward pass); the others on 8192x16384. Each is
     preceded by its set-up launches (random weights, quantize, pack)."""
     import torch
     from cell_updates_b200 import build, cq, ops, synth
@@ -838,8 +969,15 @@ def profile_case(kernel, reps=3):
         stages, _, _ = ops.rrq_build(w, 4)
     if a.kernel == "rrq":
         rr = w.clone()
-    if a.kernel in ("gemv", "gemv8", "gemm", "vbq", "vbq8"):
-        del w, r                                   # keep the device footprint small under the profiler
+    if a.kernel in ("gemvr", "reparam", "reparam_grad"):
+        r = (torch.randn(N * K, device=dev) * 1e-3).to(torch.bfloat16)
+        cq.cq_project_residual(r, scale, None)     # served weights with a residual inside its cells
+        theta = torch.randn(N * K, device=dev) * 2.0
+        g_theta = torch.empty_like(theta) if a.kernel == "reparam_grad" else None
+    if a.kernel in ("gemv", "gemv8", "gemm", "vbq", "vbq8", "gemvr"):
+        del w                                      # keep the device footprint small under the profiler
+        if a.kernel != "gemvr":
+            del r
         torch.cuda.empty_cache()
     torch.cuda.synchronize()
     for _ in range(a.reps):
@@ -871,6 +1009,12 @@ def profile_case(kernel, reps=3):
             cq.cq_varbits_index(bits, qw.offset, torch.empty(4, dtype=torch.int64, device=dev))
         elif a.kernel in ("stages", "stages8"):
             cq.cq_dequant_gemv_stages(stages, x, y)
+        elif a.kernel == "gemvr":
+            cq.cq_dequant_gemv(qw.with_residual(r), x, y)
+        elif a.kernel == "reparam":
+            cq.cq_reparam_residual(theta, scale, r)
+        elif a.kernel == "reparam_grad":
+            cq.cq_reparam_residual_grad(theta, scale, theta, g_theta, cq.CQ_BF16)
         else:
             raise SystemExit(f"unknown kernel {a.kernel}")
     torch.cuda.synchronize()

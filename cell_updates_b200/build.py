@@ -4,7 +4,7 @@
 * ``libcq_synth.so`` -- seeded device-side test inputs (include/cq_synth.h).
 
 Each translation unit is compiled separately so the IEEE-exact kernels (quantize,
-projection, verify) get ``-fmad=false`` on top of their explicit round-to-nearest
+projection, verify, reparameterization) get ``-fmad=false`` on top of their explicit round-to-nearest
 intrinsics, while the matmul kernels keep fused multiply-adds.
 """
 import os
@@ -30,8 +30,15 @@ LIBCQ_UNITS = {
     "k_gemv.cu": [],
     "k_gemm.cu": [],
     "k_rrq.cu": [],
+    "k_reparam.cu": EXACT,
+    "k_requant.cu": EXACT,
 }
 SYNTH_UNITS = {"synth.cu": EXACT}
+
+# test-only builds of libcq with a fault injected on the host side of a kernel's pipeline (a copy
+# that is never requested, so a bounded wait runs out and the abort path runs); the tests load
+# them by path, nothing else does
+TEST_VARIANTS = {"drop_first_copy": {"k_quantize.cu": ["-DCQ_TEST_DROP_FIRST_COPY"]}}
 
 LIBCQ = os.path.join(HERE, "libcq.so")
 LIBSYNTH = os.path.join(HERE, "libcq_synth.so")
@@ -46,9 +53,13 @@ def _newer(target, deps):
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
-def _compile(unit, extra, verbose):
+def test_variant_path(name):
+    return os.path.join(BUILD, f"libcq_{name}.so")
+
+
+def _compile(unit, extra, verbose, tag=""):
     src = os.path.join(CSRC, unit)
-    obj = os.path.join(BUILD, unit.replace(".cu", ".o"))
+    obj = os.path.join(BUILD, unit.replace(".cu", f"{tag}.o"))
     if _newer(obj, [src, *HEADERS, __file__]):
         cmd = [NVCC, *COMMON, *extra, "-c", src, "-o", obj]
         if verbose:
@@ -72,6 +83,10 @@ def build(verbose: bool = False) -> None:
     os.makedirs(BUILD, exist_ok=True)
     _link([_compile(u, f, verbose) for u, f in LIBCQ_UNITS.items()], LIBCQ, verbose)
     _link([_compile(u, f, verbose) for u, f in SYNTH_UNITS.items()], LIBSYNTH, verbose)
+    for name, units in TEST_VARIANTS.items():
+        objs = [_compile(u, f + units.get(u, []), verbose, tag=f"_{name}" if u in units else "")
+                for u, f in LIBCQ_UNITS.items()]
+        _link(objs, test_variant_path(name), verbose)
 
 
 if __name__ == "__main__":

@@ -18,13 +18,14 @@ LIBSYNTH_PATH = os.path.join(HERE, "libcq_synth.so")
 CQ_F32, CQ_BF16 = 0, 1
 STATUS = ["CQ_OK", "CQ_ERR_ARG", "CQ_ERR_SHAPE", "CQ_ERR_BITS", "CQ_ERR_ALIGN", "CQ_ERR_NONFINITE",
           "CQ_ERR_RANGE", "CQ_ERR_CUDA", "CQ_ERR_UNSUPPORTED"]
-QSTATUS_NONFINITE, QSTATUS_RANGE, QSTATUS_BADBITS = 1, 2, 4
+QSTATUS_NONFINITE, QSTATUS_RANGE, QSTATUS_BADBITS, QSTATUS_TIMEOUT = 1, 2, 4, 8
 
 # every symbol include/cq.h declares
 EXPORTS = ["cq_quantize", "cq_varbits_index", "cq_pack_varbits", "cq_unpack_varbits",
            "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemv_multi", "cq_dequant_gemm",
            "cq_dequant_gemm_static", "cq_gemm_workspace", "cq_last_error", "cq_status_string", "cq_rrq_stage",
-           "cq_dequant_gemv_stages", "cq_requant_verify_pair"]
+           "cq_dequant_gemv_stages", "cq_requant_verify_pair", "cq_reparam_residual", "cq_reparam_residual_grad", "cq_requant_refine",
+           "cq_requant_workspace"]
 SYNTH_EXPORTS = ["cqs_normal_f32", "cqs_code_words", "cqs_scales", "cqs_zeros", "cqs_residual_bf16"]
 
 
@@ -61,10 +62,15 @@ def lib():
         L.cq_dequant_gemv.argtypes = [p, p, i32, i32, p, p]
         L.cq_dequant_gemv_multi.argtypes = [p, i32, p, i32, i32, p, p]
         L.cq_dequant_gemm.argtypes = [p, p, i32, i32, p, p, C.c_size_t, p]
-        L.cq_dequant_gemm_static.argtypes = [p, p, i32, i32, p, p]
+        L.cq_dequant_gemm_static.argtypes = [p, p, i32, i32, p, p, p]
         L.cq_rrq_stage.argtypes = [p, i64, i64, i32, p, p, p, p, p]
         L.cq_requant_verify_pair.argtypes = [p, i64, i64, p, p, p, p, p, p]
         L.cq_dequant_gemv_stages.argtypes = [p, i32, p, i32, i32, p, p]
+        L.cq_reparam_residual.argtypes = [p, p, i64, p, i32, p]
+        L.cq_reparam_residual_grad.argtypes = [p, p, p, i64, i32, p, p]
+        L.cq_requant_refine.argtypes = [p, i64, i64, p, p, p, i32, p, i32, p, p, p, p, C.c_size_t, p]
+        L.cq_requant_workspace.argtypes = [i64, i64]
+        L.cq_requant_workspace.restype = C.c_size_t
         L.cq_gemm_workspace.argtypes = [i64, i64, i32]
         L.cq_gemm_workspace.restype = C.c_size_t
         L.cq_last_error.restype = C.c_char_p
@@ -73,7 +79,8 @@ def lib():
         for name in ("cq_quantize", "cq_varbits_index", "cq_pack_varbits", "cq_unpack_varbits",
                      "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemv_multi",
                      "cq_dequant_gemm", "cq_dequant_gemm_static", "cq_rrq_stage", "cq_dequant_gemv_stages",
-                     "cq_requant_verify_pair"):
+                     "cq_requant_verify_pair", "cq_reparam_residual", "cq_reparam_residual_grad",
+                     "cq_requant_refine"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -226,6 +233,32 @@ def cq_dequant_gemv_stages(stages, x, y, stream=None):
                                         _stream(stream)), "cq_dequant_gemv_stages")
 
 
+def cq_reparam_residual(theta, scale, r, stream=None):
+    """r = c * theta / sqrt(1 + theta^2), bounded into each weight's cell (see include/cq.h)."""
+    _check(lib().cq_reparam_residual(_ptr(theta), _ptr(scale), theta.numel(), _ptr(r), _dtype_code(r),
+                                     _stream(stream)), "cq_reparam_residual")
+
+
+def cq_reparam_residual_grad(theta, scale, grad_r, grad_theta, r_dtype, stream=None):
+    """dL/dtheta from dL/dr; r_dtype (CQ_F32 / CQ_BF16) picks the bound as in the forward pass."""
+    _check(lib().cq_reparam_residual_grad(_ptr(theta), _ptr(scale), _ptr(grad_r), theta.numel(), int(r_dtype),
+                                          _ptr(grad_theta), _stream(stream)), "cq_reparam_residual_grad")
+
+
+def cq_requant_workspace(rows, cols):
+    return int(lib().cq_requant_workspace(rows, cols))
+
+
+def cq_requant_refine(w, H, scale, zero, bits, codes, sweeps, err_before=None, err_after=None, moves=None,
+                      workspace=None, stream=None):
+    """ReQuant refinement of codes (in place) on the frozen grid against H (see include/cq.h)."""
+    rows, cols = w.shape
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().cq_requant_refine(_ptr(w), rows, cols, _ptr(H), _ptr(scale), _ptr(zero), int(bits), _ptr(codes),
+                                   int(sweeps), _ptr(err_before), _ptr(err_after), _ptr(moves), _ptr(workspace),
+                                   nbytes, _stream(stream)), "cq_requant_refine")
+
+
 def cq_gemm_workspace(rows, cols, m):
     return int(lib().cq_gemm_workspace(rows, cols, m))
 
@@ -238,11 +271,11 @@ def cq_dequant_gemm(qw, x, y, workspace=None, stream=None):
                                  _stream(stream)), "cq_dequant_gemm")
 
 
-def cq_dequant_gemm_static(qw, x, y, stream=None):
+def cq_dequant_gemm_static(qw, x, y, status_word=None, stream=None):
     """cq_dequant_gemm without a workspace: the library's own static scratch (see include/cq.h)."""
     s = qw.struct()
-    _check(lib().cq_dequant_gemm_static(C.byref(s), _ptr(x), _dtype_code(x), x.shape[0], _ptr(y), _stream(stream)),
-           "cq_dequant_gemm_static")
+    _check(lib().cq_dequant_gemm_static(C.byref(s), _ptr(x), _dtype_code(x), x.shape[0], _ptr(y),
+                                        _ptr(status_word), _stream(stream)), "cq_dequant_gemm_static")
 
 
 def cq_last_error():

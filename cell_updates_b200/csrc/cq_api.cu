@@ -80,6 +80,18 @@ cq_status check_qweight(const cq_qweight *qw, const char *fn, bool need_residual
 }
 
 }  // namespace
+
+cq_status check_matmul_args(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m, float *y, int max_m,
+                            const char *fn) {
+  cq_status st = check_qweight(qw, fn, false);
+  if (st != CQ_OK) return st;
+  if (m < 1 || m > max_m) return fail(CQ_ERR_ARG, "%s: m=%d outside [1, %d]", fn, m, max_m);
+  if (x_dtype != CQ_F32 && x_dtype != CQ_BF16) return fail(CQ_ERR_ARG, "%s: bad x dtype %d", fn, (int)x_dtype);
+  if (qw->rows && (!y || (qw->cols && !x))) return fail(CQ_ERR_ARG, "%s: NULL x or y", fn);
+  if (x && !aligned16(x)) return fail(CQ_ERR_ALIGN, "%s: x is not 16-byte aligned", fn);
+  return CQ_OK;
+}
+
 }  // namespace cq
 
 using namespace cq;
@@ -180,6 +192,55 @@ cq_status cq_project_residual(void *r, cq_dtype dtype, const uint16_t *scale, in
   return launch_project(r, dtype, scale, n, n_clamped, reinterpret_cast<cudaStream_t>(stream));
 }
 
+cq_status cq_reparam_residual(const float *theta, const uint16_t *scale, int64_t n, void *r, cq_dtype r_dtype,
+                              cq_stream_t stream) {
+  const char *fn = "cq_reparam_residual";
+  if (r_dtype != CQ_F32 && r_dtype != CQ_BF16) return fail(CQ_ERR_ARG, "%s: bad residual dtype %d", fn, (int)r_dtype);
+  if (n < 0 || n % kGroup) return fail(CQ_ERR_SHAPE, "%s: n=%lld must be a non-negative multiple of 64", fn, (long long)n);
+  if (n && (!theta || !scale || !r)) return fail(CQ_ERR_ARG, "%s: NULL buffer", fn);
+  if (n && (!aligned16(theta) || !aligned16(r))) return fail(CQ_ERR_ALIGN, "%s: theta and r must be 16-byte aligned", fn);
+  return launch_reparam(theta, scale, n, r, r_dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+cq_status cq_reparam_residual_grad(const float *theta, const uint16_t *scale, const float *grad_r, int64_t n,
+                                   cq_dtype r_dtype, float *grad_theta, cq_stream_t stream) {
+  const char *fn = "cq_reparam_residual_grad";
+  if (r_dtype != CQ_F32 && r_dtype != CQ_BF16) return fail(CQ_ERR_ARG, "%s: bad residual dtype %d", fn, (int)r_dtype);
+  if (n < 0 || n % kGroup) return fail(CQ_ERR_SHAPE, "%s: n=%lld must be a non-negative multiple of 64", fn, (long long)n);
+  if (n && (!theta || !scale || !grad_r || !grad_theta)) return fail(CQ_ERR_ARG, "%s: NULL buffer", fn);
+  if (n && (!aligned16(theta) || !aligned16(grad_r) || !aligned16(grad_theta)))
+    return fail(CQ_ERR_ALIGN, "%s: theta, grad_r and grad_theta must be 16-byte aligned", fn);
+  return launch_reparam_grad(theta, scale, grad_r, n, r_dtype, grad_theta, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t cq_requant_workspace(int64_t rows, int64_t cols) {
+  if (rows <= 0 || cols <= 0) return 0;
+  return requant_workspace(rows, cols);
+}
+
+cq_status cq_requant_refine(const float *w, int64_t rows, int64_t cols, const double *H, const uint16_t *scale,
+                            const uint8_t *zero, int bits, uint8_t *codes, int sweeps, double *err_before,
+                            double *err_after, uint64_t *moves, void *workspace, size_t workspace_bytes,
+                            cq_stream_t stream) {
+  const char *fn = "cq_requant_refine";
+  cq_status st = check_shape(rows, cols, fn);
+  if (st != CQ_OK) return st;
+  if (!width_ok_host(bits)) return fail(CQ_ERR_BITS, "%s: width %d is not 1, 2, 4 or 8", fn, bits);
+  if (sweeps < 0) return fail(CQ_ERR_ARG, "%s: negative sweep count", fn);
+  if (rows == 0 || cols == 0) return CQ_OK;
+  if (cols > requant_max_cols())
+    return fail(CQ_ERR_UNSUPPORTED, "%s: cols=%lld above the %lld a row's state can hold on chip", fn,
+                (long long)cols, (long long)requant_max_cols());
+  if (!w || !H || !scale || !zero || !codes) return fail(CQ_ERR_ARG, "%s: NULL buffer", fn);
+  const size_t need = requant_workspace(rows, cols);
+  if (!workspace || workspace_bytes < need)
+    return fail(CQ_ERR_RANGE, "%s: workspace of %zu bytes, %zu needed", fn, workspace_bytes, need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 7u) || (reinterpret_cast<uintptr_t>(H) & 7u))
+    return fail(CQ_ERR_ALIGN, "%s: H and the workspace must be 8-byte aligned", fn);
+  return launch_requant(w, rows, cols, H, scale, zero, bits, codes, sweeps, err_before, err_after, moves,
+                        static_cast<double *>(workspace), reinterpret_cast<cudaStream_t>(stream));
+}
+
 cq_status cq_requant_verify(const cq_qweight *qw, int64_t first_w, int64_t n_w, uint64_t *mismatches,
                             int64_t *first_bad, uint32_t *group_flags, cq_stream_t stream) {
   const char *fn = "cq_requant_verify";
@@ -210,20 +271,10 @@ cq_status cq_requant_verify_pair(const cq_qweight *qw, int64_t first_w, int64_t 
                             reinterpret_cast<cudaStream_t>(stream));
 }
 
-static cq_status check_matmul(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m, float *y,
-                              int max_m, const char *fn) {
-  cq_status st = check_qweight(qw, fn, false);
-  if (st != CQ_OK) return st;
-  if (m < 1 || m > max_m) return fail(CQ_ERR_ARG, "%s: m=%d outside [1, %d]", fn, m, max_m);
-  if (x_dtype != CQ_F32 && x_dtype != CQ_BF16) return fail(CQ_ERR_ARG, "%s: bad x dtype %d", fn, (int)x_dtype);
-  if (qw->rows && (!y || (qw->cols && !x))) return fail(CQ_ERR_ARG, "%s: NULL x or y", fn);
-  if (x && !aligned16(x)) return fail(CQ_ERR_ALIGN, "%s: x is not 16-byte aligned", fn);
-  return CQ_OK;
-}
 
 cq_status cq_dequant_gemv(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m, float *y,
                           cq_stream_t stream) {
-  cq_status st = check_matmul(qw, x, x_dtype, m, y, 8, "cq_dequant_gemv");
+  cq_status st = check_matmul_args(qw, x, x_dtype, m, y, 8, "cq_dequant_gemv");
   if (st != CQ_OK) return st;
   return launch_gemv(*qw, x, x_dtype, m, y, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -236,7 +287,7 @@ cq_status cq_dequant_gemv_multi(const cq_qweight *const *qws, int count, const v
   if (!qws || !ys) return fail(CQ_ERR_ARG, "%s: NULL matrix or output list", fn);
   for (int i = 0; i < count; ++i) {
     if (!qws[i]) return fail(CQ_ERR_ARG, "%s: matrix %d is NULL", fn, i);
-    cq_status st = check_matmul(qws[i], x, x_dtype, m, ys[i], 8, fn);
+    cq_status st = check_matmul_args(qws[i], x, x_dtype, m, ys[i], 8, fn);
     if (st != CQ_OK) return st;
     if (qws[i]->cols != qws[0]->cols)
       return fail(CQ_ERR_SHAPE, "%s: matrix %d has %lld cols, matrix 0 has %lld", fn, i,
@@ -253,7 +304,7 @@ cq_status cq_dequant_gemv_stages(const cq_qweight *const *stages, int count, con
   if (!stages) return fail(CQ_ERR_ARG, "%s: NULL stage list", fn);
   for (int j = 0; j < count; ++j) {
     if (!stages[j]) return fail(CQ_ERR_ARG, "%s: stage %d is NULL", fn, j);
-    cq_status st = check_matmul(stages[j], x, x_dtype, m, y, 8, fn);
+    cq_status st = check_matmul_args(stages[j], x, x_dtype, m, y, 8, fn);
     if (st != CQ_OK) return st;
     if (stages[j]->rows != stages[0]->rows || stages[j]->cols != stages[0]->cols)
       return fail(CQ_ERR_SHAPE, "%s: stage %d is %lldx%lld, stage 0 is %lldx%lld", fn, j, (long long)stages[j]->rows,
@@ -271,7 +322,7 @@ size_t cq_gemm_workspace(int64_t rows, int64_t cols, int m) {
 cq_status cq_dequant_gemm(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m, float *y, void *workspace,
                           size_t workspace_bytes, cq_stream_t stream) {
   const char *fn = "cq_dequant_gemm";
-  cq_status st = check_matmul(qw, x, x_dtype, m, y, 256, fn);
+  cq_status st = check_matmul_args(qw, x, x_dtype, m, y, 256, fn);
   if (st != CQ_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (gemm_tc_eligible(*qw, x_dtype, m)) {

@@ -48,6 +48,18 @@ constexpr int kMaxRrqStages = 8;
 cq_status launch_gemv_stages(const cq_qweight *const *stages, int count, const void *x, cq_dtype xdt, int m,
                              float *y, cudaStream_t s);
 bool gemm_tc_eligible(const cq_qweight &qw, cq_dtype xdt, int m);
+cq_status launch_requant(const float *w, int64_t N, int64_t K, const double *H, const uint16_t *scale,
+                         const uint8_t *zero, int b, uint8_t *codes, int sweeps, double *err_before, double *err_after,
+                         uint64_t *moves, double *g, cudaStream_t s);
+size_t requant_workspace(int64_t rows, int64_t cols);
+int64_t requant_max_cols();
+cq_status launch_reparam(const float *theta, const uint16_t *scale, int64_t n, void *r, cq_dtype dt,
+                         cudaStream_t s);
+cq_status launch_reparam_grad(const float *theta, const uint16_t *scale, const float *grad_r, int64_t n, cq_dtype dt,
+                              float *grad_theta, cudaStream_t s);
+// the argument checks every matmul entry point shares (cq_api.cu)
+cq_status check_matmul_args(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m, float *y, int max_m,
+                            const char *fn);
 
 // ---- device-side helpers -------------------------------------------------------------
 __device__ __forceinline__ float f16_bits_to_f32(uint16_t h) {

@@ -653,6 +653,146 @@ cq_status launch_gemv4_segs(const cq_qweight *const *qws, int count, const void 
 }
 
 // ------------------------------------------------------------------------------------
+// fixed 4-bit codes with a bf16 residual: the CellFill served weights W = s (q - z) + r
+// ------------------------------------------------------------------------------------
+// [CF] the served weight carries the residual, so decode streams 0.5 B of codes and 2 B of
+// residual per weight. A CTA of 8 warps owns one 16-row tile; warp w takes the w-th eighth of
+// the row's groups, so each warp streams contiguous runs of codes and residual of 16 rows.
+// Per group, on tensor cores (mma.sync m16n8k16, fp32 accumulation, exact products):
+//   codes:    sum_k (128 + q) x  with 128 + q = bf16 0x4300 | q, minus (128 + z) sum_k x (the group
+//             sum of x from an MMA with an all-ones A), times s;
+//   residual: sum_k r x straight into the row accumulator (bf16 r and x: exact products).
+// Both operands pair k the same way: lane (gid, tig) holds k = 16 tig .. 16 tig + 15 of the
+// group for rows gid and gid + 8 (one 8-byte code load and two 16-byte residual loads per row),
+// the codes in the nibble order (0,4) (1,5) (2,6) (3,7), the residual and x permuted to match.
+// Each lane keeps the next group's loads in flight (two groups of loads per warp: ~80 B per
+// lane). The warps' partial sums meet in shared memory; y is written once per tile.
+constexpr int kRWarps = 8;
+constexpr int kRThreads = 32 * kRWarps;
+
+struct RGroup {
+  uint2 c0, c1;          // codes of rows gid, gid + 8 (16 nibbles each)
+  uint4 r0l, r0h, r1l, r1h;   // residual of rows gid, gid + 8 (16 bf16 each)
+  uint4 xl, xh;          // 16 bf16 activations of batch row gid (row 0 for gid >= m)
+  uint32_t s0, s1, z0, z1;
+};
+
+__device__ __forceinline__ void rgroup_load(RGroup &b, const uint8_t *c0, const uint8_t *c1, const uint16_t *r0,
+                                            const uint16_t *r1, const __nv_bfloat16 *xr, const uint16_t *sc0,
+                                            const uint16_t *sc1, const uint8_t *zp0, const uint8_t *zp1, int g) {
+  b.c0 = __ldcs(reinterpret_cast<const uint2 *>(c0 + g * 32));
+  b.c1 = __ldcs(reinterpret_cast<const uint2 *>(c1 + g * 32));
+  const uint4 *p0 = reinterpret_cast<const uint4 *>(r0 + g * 64);
+  const uint4 *p1 = reinterpret_cast<const uint4 *>(r1 + g * 64);
+  b.r0l = __ldcs(p0);
+  b.r0h = __ldcs(p0 + 1);
+  b.r1l = __ldcs(p1);
+  b.r1h = __ldcs(p1 + 1);
+  const uint4 *xp = reinterpret_cast<const uint4 *>(xr + g * 64);
+  b.xl = __ldg(xp);
+  b.xh = __ldg(xp + 1);
+  b.s0 = __ldg(sc0 + g);
+  b.s1 = __ldg(sc1 + g);
+  b.z0 = __ldg(zp0 + g);
+  b.z1 = __ldg(zp1 + g);
+}
+
+__device__ __forceinline__ void rgroup_mma(const RGroup &b, float acc[4]) {
+  uint32_t bx[8], ra[8], rb[8];
+  permute16(b.xl, b.xh, bx);
+  permute16(b.r0l, b.r0h, ra);
+  permute16(b.r1l, b.r1h, rb);
+  const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};   // bf16 1.0
+  float p[4] = {0.0f, 0.0f, 0.0f, 0.0f}, q[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t u0 = h ? b.c0.y : b.c0.x, u1 = h ? b.c1.y : b.c1.x;
+    const uint32_t A0[4] = {nib_pair(u0), nib_pair(u1), nib_pair(u0 >> 4), nib_pair(u1 >> 4)};
+    mma_bf16_16816(p, A0, bx[4 * h + 0], bx[4 * h + 1]);
+    mma_bf16_16816(q, ones, bx[4 * h + 0], bx[4 * h + 1]);
+    const uint32_t A1[4] = {nib_pair(u0 >> 8), nib_pair(u1 >> 8), nib_pair(u0 >> 12), nib_pair(u1 >> 12)};
+    mma_bf16_16816(p, A1, bx[4 * h + 2], bx[4 * h + 3]);
+    mma_bf16_16816(q, ones, bx[4 * h + 2], bx[4 * h + 3]);
+  }
+  const float s0 = f16_bits_to_f32(static_cast<uint16_t>(b.s0)), s1 = f16_bits_to_f32(static_cast<uint16_t>(b.s1));
+  const float zc0 = 128.0f + static_cast<float>(b.z0), zc1 = 128.0f + static_cast<float>(b.z1);
+  acc[0] = fmaf(s0, fmaf(-zc0, q[0], p[0]), acc[0]);
+  acc[1] = fmaf(s0, fmaf(-zc0, q[1], p[1]), acc[1]);
+  acc[2] = fmaf(s1, fmaf(-zc1, q[2], p[2]), acc[2]);
+  acc[3] = fmaf(s1, fmaf(-zc1, q[3], p[3]), acc[3]);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t A0[4] = {ra[4 * h + 0], rb[4 * h + 0], ra[4 * h + 1], rb[4 * h + 1]};
+    mma_bf16_16816(acc, A0, bx[4 * h + 0], bx[4 * h + 1]);
+    const uint32_t A1[4] = {ra[4 * h + 2], rb[4 * h + 2], ra[4 * h + 3], rb[4 * h + 3]};
+    mma_bf16_16816(acc, A1, bx[4 * h + 2], bx[4 * h + 3]);
+  }
+}
+
+__global__ void __launch_bounds__(kRThreads, 2)
+gemv4r_kernel(const uint8_t *__restrict__ plane, const uint16_t *__restrict__ scale, const uint8_t *__restrict__ zero,
+              const uint16_t *__restrict__ res, const __nv_bfloat16 *__restrict__ x, int m, int64_t N, int64_t K,
+              float *__restrict__ y) {
+  __shared__ float red[kRWarps][kTileRows * 8];
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int KG = static_cast<int>(K >> 6);
+  const int g0 = KG * warp / kRWarps, g1 = KG * (warp + 1) / kRWarps;
+  const int64_t n_tiles = (N + kTileRows - 1) / kTileRows;
+  for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+    int64_t row0 = tile * kTileRows + gid, row1 = row0 + 8;
+    row0 = row0 < N ? row0 : N - 1;               // rows past the end: any valid row, never stored
+    row1 = row1 < N ? row1 : N - 1;
+    const uint8_t *c0 = plane + row0 * (K / 2) + tig * 8, *c1 = plane + row1 * (K / 2) + tig * 8;
+    const uint16_t *r0 = res + row0 * K + tig * 16, *r1 = res + row1 * K + tig * 16;
+    const uint16_t *sc0 = scale + row0 * KG, *sc1 = scale + row1 * KG;
+    const uint8_t *zp0 = zero + row0 * KG, *zp1 = zero + row1 * KG;
+    const __nv_bfloat16 *xr = x + static_cast<int64_t>(gid < m ? gid : 0) * K + tig * 16;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    // the weights do not depend on earlier kernels; x and y do
+    RGroup a, b;
+    if (tile == blockIdx.x) pdl_wait();
+    if (g0 < g1) rgroup_load(a, c0, c1, r0, r1, xr, sc0, sc1, zp0, zp1, g0);
+    for (int g = g0; g < g1; g += 2) {
+      if (g + 1 < g1) rgroup_load(b, c0, c1, r0, r1, xr, sc0, sc1, zp0, zp1, g + 1);
+      rgroup_mma(a, acc);
+      if (g + 1 >= g1) break;
+      if (g + 2 < g1) rgroup_load(a, c0, c1, r0, r1, xr, sc0, sc1, zp0, zp1, g + 2);
+      rgroup_mma(b, acc);
+    }
+    // partials of rows gid, gid + 8 and batch columns 2 tig, 2 tig + 1: [col][row]
+    float *rw = red[warp];
+    rw[(2 * tig) * 16 + gid] = acc[0];
+    rw[(2 * tig + 1) * 16 + gid] = acc[1];
+    rw[(2 * tig) * 16 + gid + 8] = acc[2];
+    rw[(2 * tig + 1) * 16 + gid + 8] = acc[3];
+    __syncthreads();
+    if (threadIdx.x < 16 * m) {
+      const int row = threadIdx.x & 15, col = threadIdx.x >> 4;
+      float v = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kRWarps; ++w) v += red[w][threadIdx.x];
+      const int64_t rr = tile * kTileRows + row;
+      if (rr < N) y[static_cast<int64_t>(col) * N + rr] = v;
+    }
+    __syncthreads();
+  }
+}
+
+cq_status launch_gemv4r(const cq_qweight &qw, const void *x, int m, float *y, cudaStream_t s) {
+  const int64_t N = qw.rows, K = qw.cols;
+  const int64_t tiles = (N + kTileRows - 1) / kTileRows;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 2;
+  const int64_t grid = tiles < cap ? tiles : cap;
+  return cuda_check(launch_pdl(gemv4r_kernel, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), 0, s,
+                               static_cast<const uint8_t *>(qw.plane[2]), qw.scale, qw.zero,
+                               static_cast<const uint16_t *>(qw.residual), static_cast<const __nv_bfloat16 *>(x), m,
+                               N, K, y),
+                    "cq_dequant_gemv (residual)");
+}
+
+// ------------------------------------------------------------------------------------
 // generic fp32 path
 // ------------------------------------------------------------------------------------
 constexpr int kGenThreads = 256;
@@ -740,6 +880,10 @@ cq_status launch_gemv(const cq_qweight &qw, const void *x, cq_dtype xdt, int m, 
     const cq_qweight *one = &qw;
     return launch_gemv_stages(&one, 1, x, xdt, m, y, s);
   }
+  // the CellFill served weights: fixed 4-bit codes and a bf16 residual with bf16 x
+  if (qw.bits == nullptr && qw.residual_dtype == CQ_BF16 && xdt == CQ_BF16 && aligned16(qw.residual) &&
+      aligned8(qw.plane[2]))
+    return launch_gemv4r(qw, x, m, y, s);
   const int64_t need = (N + 7) / 8;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const int blocks = static_cast<int>(need < cap ? need : cap);

@@ -110,13 +110,20 @@ def gemv_multi(qws, x, stream=None):
     return ys
 
 
-def gemm(qw, x, workspace=None, stream=None):
+def gemm(qw, x, workspace=None, stream=None, check=True):
+    """y = W x for a batch; with check, waits for the result and raises if the GEMM's status
+    word (first 4 bytes of its workspace) says an internal wait gave up."""
     m = x.shape[0]
     y = torch.empty((m, qw.rows), dtype=torch.float32, device=x.device)
     need = cq.cq_gemm_workspace(qw.rows, qw.cols, m)
     if need and (workspace is None or workspace.numel() < need):
-        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+        # zero-filled: the word stays 0 when the call is served by the GEMV kernels instead
+        workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
     cq.cq_dequant_gemm(qw, x, y, workspace if need else None, stream)
+    if check and need:
+        word = int(workspace[:4].view(torch.int32).cpu()[0])   # synchronizes with the stream
+        if word != 0:
+            raise cq.CQError(7, f"cq_dequant_gemm: status word {word:#x} (an internal wait gave up)")
     return y
 
 
@@ -146,3 +153,30 @@ def gemv_stages(stages, x, stream=None):
     y = torch.empty((x.shape[0], stages[0].rows), dtype=torch.float32, device=x.device)
     cq.cq_dequant_gemv_stages(stages, x, y, stream)
     return y
+
+
+def reparam(theta, scale, r_dtype=torch.bfloat16, stream=None):
+    """Bounded reparameterization: theta (fp32 [n]) -> a residual of r_dtype inside every cell."""
+    r = torch.empty(theta.numel(), dtype=r_dtype, device=theta.device)
+    cq.cq_reparam_residual(theta, scale, r, stream)
+    return r
+
+
+def reparam_grad(theta, scale, grad_r, r_dtype=torch.bfloat16, stream=None):
+    """dL/dtheta of reparam() from dL/dr (fp32 [n])."""
+    g = torch.empty_like(theta)
+    cq.cq_reparam_residual_grad(theta, scale, grad_r, g, cq.CQ_BF16 if r_dtype == torch.bfloat16 else cq.CQ_F32,
+                                stream)
+    return g
+
+
+def requant_refine(w, H, scale, zero, codes, sweeps=1, bits=4, stream=None):
+    """ReQuant on a copy of codes -> (codes, err_before, err_after, moves), all on the device."""
+    rows = w.shape[0]
+    q = codes.clone()
+    eb = torch.empty(rows, dtype=torch.float64, device=w.device)
+    ea = torch.empty(rows, dtype=torch.float64, device=w.device)
+    mv = torch.empty(rows, dtype=torch.int64, device=w.device)
+    ws = torch.empty(cq.cq_requant_workspace(*w.shape), dtype=torch.uint8, device=w.device)
+    cq.cq_requant_refine(w, H, scale, zero, bits, q, sweeps, eb, ea, mv, ws, stream)
+    return q, eb, ea, mv

@@ -163,6 +163,63 @@ cq_status cq_project_residual(void *r, cq_dtype dtype, const uint16_t *scale, in
                               uint64_t *n_clamped, cq_stream_t stream);
 
 /*
+ * cq_reparam_residual -- [CF] Abstract, CellFill as a bounded reparameterization: the update is
+ * trained as an unconstrained parameter theta and served as a residual that lies in its
+ * weight's cell whatever theta is, so the release re-quantizes to its codes with no projection
+ * step. The map is not printed on the page; this library's reading:
+ *     r_i = RN(c_dt * phi(theta_i)),   phi(t) = t / sqrt(1 + t^2)
+ * c_dt: the bound cq_project_residual clamps to ((0.5 - 2^-10) * s for fp32 r; that value
+ * rounded toward zero to bf16 for bf16 r); s the scale of weight i's group. phi is evaluated
+ * as the binary32 steps u = RN(t*t), d = RN(1 + u), q = RN(sqrt(d)), phi = RN(t / q) (correctly
+ * rounded, no contraction), then the fp32 product, then for bf16 r one round to nearest
+ * bf16: the same bits on any IEEE-754 machine. |r| <= c_dt for every theta: +-inf gives +-c_dt,
+ * |theta| > 2^32 gives phi = +-1, and a NaN theta gives r = +0 (that weight's update revoked).
+ * theta: [n] fp32; r: [n] of r_dtype (overwritten); both 16-byte aligned; n % 64 == 0; element
+ * i belongs to group i/64 of scale. Errors: CQ_ERR_SHAPE, CQ_ERR_ARG (NULL, dtype), CQ_ERR_ALIGN.
+ */
+cq_status cq_reparam_residual(const float *theta, const uint16_t *scale, int64_t n, void *r,
+                              cq_dtype r_dtype, cq_stream_t stream);
+
+/*
+ * cq_reparam_residual_grad -- the backward pass of cq_reparam_residual for training theta,
+ * straight through its final rounding: grad_theta_i = RN(RN(grad_r_i * c_dt) * phi'(theta_i)),
+ * phi'(t) = (1 + t^2)^(-3/2) evaluated as RN(RN(1 / d) / q) with d and q as in the forward
+ * pass; 0 for a NaN theta or |theta| > 2^32. grad_r: [n] fp32 (dL/dr); grad_theta: [n] fp32
+ * (overwritten); r_dtype selects c_dt as in the forward pass. Alignment and errors as there.
+ */
+cq_status cq_reparam_residual_grad(const float *theta, const uint16_t *scale, const float *grad_r,
+                                   int64_t n, cq_dtype r_dtype, float *grad_theta, cq_stream_t stream);
+
+/*
+ * cq_requant_refine -- ReQuant fixed-grid refinement (page 1, thelatestinai.com/papers/2608.20873,
+ * ReQuant abstract: a backpropagation-free stage that revisits an existing quantized model's
+ * integer assignments on its fixed grid, every accepted update strictly lowering the mean squared
+ * reconstruction error; several sweeps over a round-to-nearest start). This library's reading:
+ * the error is the layer's output error on calibration activations X,
+ *     E(q) = sum_n d_n^T H d_n,   d_n = w_n - s (q_n - z),   H = X^T X,
+ * the scales and zero points stay as they are, and an update moves one code to a neighbouring
+ * level of the grid (q +- 1 within [0, 2^bits - 1]). Each of `sweeps` sweeps visits every row's
+ * codes in order; a move is taken only if it lowers E strictly (of the two, the larger decrease;
+ * up on a tie). Rows are refined independently. All arithmetic is binary64 in a fixed order
+ * without fused multiply-adds, so the codes are the same on any IEEE-754 machine that keeps it.
+ * w: [rows, cols] fp32 (the weights before quantization); H: [cols, cols] fp64, symmetric
+ * (H[j, k] == H[k, j] bit for bit), 8-byte aligned; scale/zero: [G]; codes: [rows*cols], one code
+ * per byte, refined in place (pack them with cq_pack_varbits). err_before / err_after: NULL or
+ * [rows] fp64, E of each row before and after; moves: NULL or [rows] uint64, accepted updates.
+ * workspace: at least cq_requant_workspace(rows, cols) bytes of device scratch (8-byte aligned).
+ * One width `bits` for every group. cols may be at most 25600 (a row's state is kept on chip;
+ * CQ_ERR_UNSUPPORTED beyond). Errors: CQ_ERR_SHAPE, CQ_ERR_BITS, CQ_ERR_ARG, CQ_ERR_RANGE
+ * (workspace too small), CQ_ERR_ALIGN.
+ */
+cq_status cq_requant_refine(const float *w, int64_t rows, int64_t cols, const double *H,
+                            const uint16_t *scale, const uint8_t *zero, int bits, uint8_t *codes,
+                            int sweeps, double *err_before, double *err_after, uint64_t *moves,
+                            void *workspace, size_t workspace_bytes, cq_stream_t stream);
+
+/* Bytes of workspace cq_requant_refine needs (host function, no GPU work). */
+size_t cq_requant_workspace(int64_t rows, int64_t cols);
+
+/*
  * cq_requant_verify -- [CF] rounding the served weights again must give the released codes
  * exactly, and with the residual removed (qw->residual = NULL) the update is undone. For weight i in
  * [first_w, first_w + n_w) with code q, scale s, zero z, width b:
@@ -245,14 +302,19 @@ cq_status cq_dequant_gemm(const cq_qweight *qw, const void *x, cq_dtype x_dtype,
  * Its scratch is an 8 MiB array inside the library that every GPU which loads the library
  * keeps until the process exits. A shape that would need more scratch than that is refused
  * with CQ_ERR_RANGE: the tensor-core GEMM needs 512 + 2 * min(m, 64) * cols bytes, so with
- * m >= 64 cols may be at most 65532. The first call on a device
- * looks up the array's device address with that device current; make that first call before
- * any stream capture. All calls share the array and the call clears what must start at zero,
- * but calls that overlap on the GPU (other streams, other threads) race on it.
+ * m >= 64 cols may be at most 65532. Arguments are checked first, so a bad call does no CUDA
+ * work; the first valid call on a device then looks up the array's device address with that
+ * device current (make that first call before any stream capture). All calls share the array
+ * and the call clears what must start at zero, but calls that overlap on the GPU (other
+ * streams, other threads) race on it.
+ * status_word: NULL, or one uint32 (device) that receives, in stream order after the multiply,
+ * the tensor-core GEMM's status word: 0, or non-zero if an internal wait gave up (y is then
+ * incomplete). Shapes served by the GEMV kernels write 0 there (those mark an aborted output
+ * with NaN instead).
  * Arguments, results and errors are otherwise those of cq_dequant_gemm.
  */
 cq_status cq_dequant_gemm_static(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m,
-                                 float *y, cq_stream_t stream);
+                                 float *y, uint32_t *status_word, cq_stream_t stream);
 
 /* Bytes of workspace cq_dequant_gemm needs for this shape (host function, no GPU work). */
 size_t cq_gemm_workspace(int64_t rows, int64_t cols, int m);

@@ -422,3 +422,31 @@ def test_gemm_bf16_residual_uses_exact_formula():
     rb, _ = co.project_bf16(synth.normal_residual_bf16(scale, seed=22), scale)
     qw, x_d, y_ref, _ = _matmul_case(128, 1024, 20, "bf16", r=rb, seed=21)
     check_matmul(host(ops.gemm(qw, x_d)), y_ref, "gemm r bf16")
+
+
+# the CellFill served weights W = s (q - z) + r with a bf16 residual, on tensor cores: ragged
+# 16-row tiles, fewer groups than warps (K = 64, 320), groups that split unevenly over the warps,
+# the decode and CellFill-stack shapes, projected and unprojected residuals
+@pytest.mark.parametrize("rows,cols", [(16, 64), (47, 64 * 5), (300, 64 * 21), (1000, 4096), (2048, 2048),
+                                       (6144, 2048), (2048, 6144), (100, 11008)])
+@pytest.mark.parametrize("m", [1, 3, 8])
+def test_gemv_bf16_residual_tensor_core(rows, cols, m):
+    w = synth.normal_weights(rows, cols, seed=rows + cols)
+    _, scale, _, _ = co.quantize(w)
+    rb = synth.normal_residual_bf16(scale, seed=rows + 3, rel_sigma=0.3)
+    if rows % 2:
+        rb, _ = co.project_bf16(rb, scale)
+    qw, x_d, y_ref, _ = _matmul_case(rows, cols, m, "bf16", r=rb, seed=rows + cols)
+    check_matmul(host(ops.gemv(qw, x_d)), y_ref, f"gemv r bf16 {rows}x{cols} m={m}")
+
+
+# the batch GEMM with a bf16 residual (CellFill served weights): every batch slice size, ragged
+# row tiles, several K ranges per CTA
+@pytest.mark.parametrize("rows,cols,m", [(384, 64 * 40, 64), (1000, 4096, 33), (200, 64 * 8, 16),
+                                         (129, 64 * 24, 100)])
+def test_gemm_bf16_residual_batches(rows, cols, m):
+    w = synth.normal_weights(rows, cols, seed=rows + m)
+    _, scale, _, _ = co.quantize(w)
+    rb, _ = co.project_bf16(synth.normal_residual_bf16(scale, seed=rows + 1, rel_sigma=0.3), scale)
+    qw, x_d, y_ref, _ = _matmul_case(rows, cols, m, "bf16", r=rb, seed=rows + m)
+    check_matmul(host(ops.gemm(qw, x_d)), y_ref, f"gemm r bf16 {rows}x{cols} m={m}")

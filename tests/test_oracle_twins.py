@@ -76,3 +76,19 @@ def test_reparam_twins_agree():
         assert np.array_equal(np.asarray(a).view(np.uint8), np.asarray(b).view(np.uint8)), dt
         ga, gb = co.reparam_grad(theta, scale, g, dt), no.reparam_grad(theta, scale, g, dt)
         assert np.array_equal(ga.view(np.uint32), gb.view(np.uint32)), dt
+
+
+def test_requant_twins_agree():
+    # ReQuant refinement: C and NumPy give the same codes, moves and errors, bit for bit
+    rng = np.random.default_rng(2028)
+    rows, cols = 5, 192
+    w = synth.normal_weights(rows, cols, seed=12)
+    codes, scale, zero, _ = co.quantize(w)
+    X = rng.standard_normal((400, cols))
+    X[:, 7] *= 10.0
+    H = X.T @ X
+    a = co.requant_refine(w, H, codes, scale, zero, 4, 2)
+    b = no.requant_refine(w, H, codes, scale, zero, 4, 2)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[3], b[3]) and a[3].sum() > 0
+    assert np.array_equal(a[1].view(np.uint64), b[1].view(np.uint64))
+    assert np.array_equal(a[2].view(np.uint64), b[2].view(np.uint64))
