@@ -758,18 +758,30 @@ cq_status static_scratch(void **out) {
 }  // namespace cq
 
 extern "C" cq_status cq_dequant_gemm_static(const cq_qweight *qw, const void *x, cq_dtype x_dtype, int m, float *y,
-                                            cq_stream_t stream) {
+                                            uint32_t *status_word, cq_stream_t stream) {
   using namespace cq;
   const char *fn = "cq_dequant_gemm_static";
-  void *scratch = nullptr;
-  cq_status st = static_scratch(&scratch);
+  // the arguments first: a bad call does no CUDA work at all, not even the address look-up
+  cq_status st = check_matmul_args(qw, x, x_dtype, m, y, 256, fn);
   if (st != CQ_OK) return st;
-  if (qw && x_dtype == CQ_BF16 && m >= 16 && gemm_tc_eligible(*qw, x_dtype, m)) {
+  const bool tc = gemm_tc_eligible(*qw, x_dtype, m);
+  if (tc) {
     const size_t need = gemm_tc_workspace(qw->rows, qw->cols, m);
     if (need > kStaticScratchBytes)
       return fail(CQ_ERR_RANGE, "%s: this shape needs %zu bytes of scratch, the static buffer holds %zu", fn, need,
                   kStaticScratchBytes);
   }
-  // the regular entry point does the validation and dispatch; the scratch is the static array
-  return cq_dequant_gemm(qw, x, x_dtype, m, y, scratch, kStaticScratchBytes, stream);
+  void *scratch = nullptr;
+  st = static_scratch(&scratch);
+  if (st != CQ_OK) return st;
+  // the regular entry point does the dispatch; the scratch is the static array
+  st = cq_dequant_gemm(qw, x, x_dtype, m, y, scratch, kStaticScratchBytes, stream);
+  if (st != CQ_OK || !status_word) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the tensor-core GEMM leaves its status word in the first 4 bytes of the scratch; the GEMV
+  // kernels that serve the other cases have none (they mark an aborted output with NaN)
+  if (tc && qw->rows > 0)
+    return cuda_check(cudaMemcpyAsync(status_word, scratch, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s),
+                      "cq_dequant_gemm_static: status word");
+  return cuda_check(cudaMemsetAsync(status_word, 0, sizeof(uint32_t), s), "cq_dequant_gemm_static: status word");
 }
