@@ -48,3 +48,30 @@ def check_matmul(y_gpu, y_ref, what=""):
     mx = np.abs(err).max() / max(rms, 1e-300)
     assert fro <= REL_FRO and mx <= MAX_OVER_RMS, f"{what}: relF={fro:.3e} max/rms={mx:.3e}"
     return fro, mx
+
+
+# ---- guard bands: a stand-in for a memory checker -------------------------------------------
+GUARD_BYTES = 4096
+SENTINEL = 0xA5
+
+
+class Guarded:
+    """A device buffer of `numel` elements of `dtype` with GUARD_BYTES of sentinel bytes on each
+    side (the buffer itself keeps 16-byte alignment). After a call, check() asserts that no
+    kernel wrote outside the buffer."""
+
+    def __init__(self, numel, dtype, fill=None):
+        esize = torch.empty(0, dtype=dtype).element_size()
+        self.nbytes = int(numel) * esize
+        self.raw = torch.full((self.nbytes + 2 * GUARD_BYTES,), SENTINEL, dtype=torch.uint8, device="cuda")
+        self.t = self.raw[GUARD_BYTES:GUARD_BYTES + self.nbytes].view(dtype)
+        if fill is not None:
+            self.t.copy_(fill.reshape(-1).view(dtype) if torch.is_tensor(fill) else torch.as_tensor(fill))
+
+    def check(self, what):
+        torch.cuda.synchronize()
+        pre = self.raw[:GUARD_BYTES]
+        post = self.raw[GUARD_BYTES + self.nbytes:]
+        bad_pre = int((pre != SENTINEL).sum())
+        bad_post = int((post != SENTINEL).sum())
+        assert bad_pre == 0 and bad_post == 0, f"{what}: {bad_pre} bytes written before, {bad_post} after the buffer"
