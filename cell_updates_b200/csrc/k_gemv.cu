@@ -666,7 +666,8 @@ cq_status launch_gemv4_segs(const cq_qweight *const *qws, int count, const void 
 // group for rows gid and gid + 8 (one 8-byte code load and two 16-byte residual loads per row),
 // the codes in the nibble order (0,4) (1,5) (2,6) (3,7), the residual and x permuted to match.
 // Each lane keeps the next group's loads in flight (two groups of loads per warp: ~80 B per
-// lane). The warps' partial sums meet in shared memory; y is written once per tile.
+// lane); the first two groups' weight loads are issued before the wait for the previous kernel
+// in the stream. The warps' partial sums meet in shared memory; y is written once per tile.
 constexpr int kRWarps = 8;
 constexpr int kRThreads = 32 * kRWarps;
 
@@ -677,9 +678,10 @@ struct RGroup {
   uint32_t s0, s1, z0, z1;
 };
 
-__device__ __forceinline__ void rgroup_load(RGroup &b, const uint8_t *c0, const uint8_t *c1, const uint16_t *r0,
-                                            const uint16_t *r1, const __nv_bfloat16 *xr, const uint16_t *sc0,
-                                            const uint16_t *sc1, const uint8_t *zp0, const uint8_t *zp1, int g) {
+// the weight side of a group (codes, residual, scale, zero point): independent of earlier kernels
+__device__ __forceinline__ void rgroup_load_w(RGroup &b, const uint8_t *c0, const uint8_t *c1, const uint16_t *r0,
+                                              const uint16_t *r1, const uint16_t *sc0, const uint16_t *sc1,
+                                              const uint8_t *zp0, const uint8_t *zp1, int g) {
   b.c0 = __ldcs(reinterpret_cast<const uint2 *>(c0 + g * 32));
   b.c1 = __ldcs(reinterpret_cast<const uint2 *>(c1 + g * 32));
   const uint4 *p0 = reinterpret_cast<const uint4 *>(r0 + g * 64);
@@ -688,13 +690,16 @@ __device__ __forceinline__ void rgroup_load(RGroup &b, const uint8_t *c0, const 
   b.r0h = __ldcs(p0 + 1);
   b.r1l = __ldcs(p1);
   b.r1h = __ldcs(p1 + 1);
-  const uint4 *xp = reinterpret_cast<const uint4 *>(xr + g * 64);
-  b.xl = __ldg(xp);
-  b.xh = __ldg(xp + 1);
   b.s0 = __ldg(sc0 + g);
   b.s1 = __ldg(sc1 + g);
   b.z0 = __ldg(zp0 + g);
   b.z1 = __ldg(zp1 + g);
+}
+// the activation side: x may be the previous kernel's output
+__device__ __forceinline__ void rgroup_load_x(RGroup &b, const __nv_bfloat16 *xr, int g) {
+  const uint4 *xp = reinterpret_cast<const uint4 *>(xr + g * 64);
+  b.xl = __ldg(xp);
+  b.xh = __ldg(xp + 1);
 }
 
 __device__ __forceinline__ void rgroup_mma(const RGroup &b, float acc[4]) {
@@ -729,19 +734,34 @@ __device__ __forceinline__ void rgroup_mma(const RGroup &b, float acc[4]) {
   }
 }
 
+// several matrices that read the same x in one launch: their 16-row tiles are numbered one after
+// the other (segment s owns tiles tile0[s] .. tile0[s+1]-1)
+struct RSegs {
+  const uint8_t *plane[kMaxSegs];
+  const uint16_t *scale[kMaxSegs];
+  const uint8_t *zero[kMaxSegs];
+  const uint16_t *res[kMaxSegs];
+  float *y[kMaxSegs];
+  int64_t rows[kMaxSegs];
+  int64_t tile0[kMaxSegs + 1];              // tile0[count] = all tiles; unused entries = INT64_MAX
+};
+
 __global__ void __launch_bounds__(kRThreads, 2)
-gemv4r_kernel(const uint8_t *__restrict__ plane, const uint16_t *__restrict__ scale, const uint8_t *__restrict__ zero,
-              const uint16_t *__restrict__ res, const __nv_bfloat16 *__restrict__ x, int m, int64_t N, int64_t K,
-              float *__restrict__ y) {
+gemv4r_kernel(const __grid_constant__ RSegs sg, const __nv_bfloat16 *__restrict__ x, int m, int64_t K) {
   __shared__ float red[kRWarps][kTileRows * 8];
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gid = lane >> 2, tig = lane & 3;
   const int KG = static_cast<int>(K >> 6);
   const int g0 = KG * warp / kRWarps, g1 = KG * (warp + 1) / kRWarps;
-  const int64_t n_tiles = (N + kTileRows - 1) / kTileRows;
+  const int64_t n_tiles = sg.tile0[kMaxSegs];
   for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-    int64_t row0 = tile * kTileRows + gid, row1 = row0 + 8;
+    const int s = (tile >= sg.tile0[1]) + (tile >= sg.tile0[2]) + (tile >= sg.tile0[3]);
+    const uint8_t *plane = seg_pick(sg.plane, s);
+    const uint16_t *scale = seg_pick(sg.scale, s), *res = seg_pick(sg.res, s);
+    const uint8_t *zero = seg_pick(sg.zero, s);
+    const int64_t N = seg_pick(sg.rows, s), lrow0 = (tile - seg_pick(sg.tile0, s)) * kTileRows;
+    int64_t row0 = lrow0 + gid, row1 = row0 + 8;
     row0 = row0 < N ? row0 : N - 1;               // rows past the end: any valid row, never stored
     row1 = row1 < N ? row1 : N - 1;
     const uint8_t *c0 = plane + row0 * (K / 2) + tig * 8, *c1 = plane + row1 * (K / 2) + tig * 8;
@@ -750,16 +770,26 @@ gemv4r_kernel(const uint8_t *__restrict__ plane, const uint16_t *__restrict__ sc
     const uint8_t *zp0 = zero + row0 * KG, *zp1 = zero + row1 * KG;
     const __nv_bfloat16 *xr = x + static_cast<int64_t>(gid < m ? gid : 0) * K + tig * 16;
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    // the weights do not depend on earlier kernels; x and y do
+    // the weights do not depend on earlier kernels, so the first two groups' weight loads are
+    // issued before the wait for the previous kernel; x and y do depend on it
     RGroup a, b;
+    if (g0 < g1) rgroup_load_w(a, c0, c1, r0, r1, sc0, sc1, zp0, zp1, g0);
+    if (g0 + 1 < g1) rgroup_load_w(b, c0, c1, r0, r1, sc0, sc1, zp0, zp1, g0 + 1);
     if (tile == blockIdx.x) pdl_wait();
-    if (g0 < g1) rgroup_load(a, c0, c1, r0, r1, xr, sc0, sc1, zp0, zp1, g0);
+    if (g0 < g1) rgroup_load_x(a, xr, g0);
+    if (g0 + 1 < g1) rgroup_load_x(b, xr, g0 + 1);
     for (int g = g0; g < g1; g += 2) {
-      if (g + 1 < g1) rgroup_load(b, c0, c1, r0, r1, xr, sc0, sc1, zp0, zp1, g + 1);
       rgroup_mma(a, acc);
+      if (g + 2 < g1) {
+        rgroup_load_w(a, c0, c1, r0, r1, sc0, sc1, zp0, zp1, g + 2);
+        rgroup_load_x(a, xr, g + 2);
+      }
       if (g + 1 >= g1) break;
-      if (g + 2 < g1) rgroup_load(a, c0, c1, r0, r1, xr, sc0, sc1, zp0, zp1, g + 2);
       rgroup_mma(b, acc);
+      if (g + 3 < g1) {
+        rgroup_load_w(b, c0, c1, r0, r1, sc0, sc1, zp0, zp1, g + 3);
+        rgroup_load_x(b, xr, g + 3);
+      }
     }
     // partials of rows gid, gid + 8 and batch columns 2 tig, 2 tig + 1: [col][row]
     float *rw = red[warp];
@@ -773,22 +803,46 @@ gemv4r_kernel(const uint8_t *__restrict__ plane, const uint16_t *__restrict__ sc
       float v = 0.0f;
 #pragma unroll
       for (int w = 0; w < kRWarps; ++w) v += red[w][threadIdx.x];
-      const int64_t rr = tile * kTileRows + row;
-      if (rr < N) y[static_cast<int64_t>(col) * N + rr] = v;
+      const int64_t rr = lrow0 + row;
+      if (rr < N) seg_pick(sg.y, s)[static_cast<int64_t>(col) * N + rr] = v;
     }
     __syncthreads();
   }
 }
 
-cq_status launch_gemv4r(const cq_qweight &qw, const void *x, int m, float *y, cudaStream_t s) {
-  const int64_t N = qw.rows, K = qw.cols;
-  const int64_t tiles = (N + kTileRows - 1) / kTileRows;
+// fixed 4-bit codes with a 16-byte aligned bf16 residual and bf16 x: the served-weight kernel
+bool gemv_res_eligible(const cq_qweight &qw, cq_dtype xdt) {
+  return qw.bits == nullptr && qw.residual != nullptr && qw.residual_dtype == CQ_BF16 && xdt == CQ_BF16 &&
+         aligned16(qw.residual) && aligned8(qw.plane[2]) && qw.rows > 0 && qw.cols > 0;
+}
+
+// up to kMaxSegs served-weight matrices with the same cols in one launch
+cq_status launch_gemv4r(const cq_qweight *const *qws, int count, const void *x, int m, float *const *ys,
+                        cudaStream_t s) {
+  RSegs sg;
+  memset(&sg, 0, sizeof(sg));
+  int64_t t = 0;
+  for (int i = 0; i < kMaxSegs; ++i) {
+    if (i < count) {
+      const cq_qweight &qw = *qws[i];
+      sg.plane[i] = static_cast<const uint8_t *>(qw.plane[2]);
+      sg.scale[i] = qw.scale;
+      sg.zero[i] = qw.zero;
+      sg.res[i] = static_cast<const uint16_t *>(qw.residual);
+      sg.y[i] = ys[i];
+      sg.rows[i] = qw.rows;
+      sg.tile0[i] = t;
+      t += (qw.rows + kTileRows - 1) / kTileRows;
+    } else {
+      sg.tile0[i] = INT64_MAX;
+    }
+  }
+  sg.tile0[kMaxSegs] = t;
+  if (count < kMaxSegs) sg.tile0[count] = t;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 2;
-  const int64_t grid = tiles < cap ? tiles : cap;
-  return cuda_check(launch_pdl(gemv4r_kernel, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), 0, s,
-                               static_cast<const uint8_t *>(qw.plane[2]), qw.scale, qw.zero,
-                               static_cast<const uint16_t *>(qw.residual), static_cast<const __nv_bfloat16 *>(x), m,
-                               N, K, y),
+  const int64_t grid = t < cap ? t : cap;
+  return cuda_check(launch_pdl(gemv4r_kernel, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), 0, s, sg,
+                               static_cast<const __nv_bfloat16 *>(x), m, qws[0]->cols),
                     "cq_dequant_gemv (residual)");
 }
 
@@ -881,9 +935,10 @@ cq_status launch_gemv(const cq_qweight &qw, const void *x, cq_dtype xdt, int m, 
     return launch_gemv_stages(&one, 1, x, xdt, m, y, s);
   }
   // the CellFill served weights: fixed 4-bit codes and a bf16 residual with bf16 x
-  if (qw.bits == nullptr && qw.residual_dtype == CQ_BF16 && xdt == CQ_BF16 && aligned16(qw.residual) &&
-      aligned8(qw.plane[2]))
-    return launch_gemv4r(qw, x, m, y, s);
+  if (gemv_res_eligible(qw, xdt)) {
+    const cq_qweight *one = &qw;
+    return launch_gemv4r(&one, 1, x, m, &y, s);
+  }
   const int64_t need = (N + 7) / 8;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const int blocks = static_cast<int>(need < cap ? need : cap);
@@ -906,17 +961,22 @@ cq_status launch_gemv_multi(const cq_qweight *const *qws, int count, const void 
                             float *const *ys, cudaStream_t s) {
   // runs of up to kMaxSegs tensor-core-eligible matrices become one launch; anything else goes
   // through the single-matrix path
+  // (the same for runs of matrices that carry a bf16 residual, on the served-weight kernel)
   int i = 0;
   while (i < count) {
-    if (!gemv_tc_eligible(*qws[i], xdt)) {
+    const bool tc = gemv_tc_eligible(*qws[i], xdt), res = gemv_res_eligible(*qws[i], xdt);
+    if (!tc && !res) {
       cq_status st = launch_gemv(*qws[i], x, xdt, m, ys[i], s);
       if (st != CQ_OK) return st;
       ++i;
       continue;
     }
     int j = i + 1;
-    while (j < count && j - i < kMaxSegs && gemv_tc_eligible(*qws[j], xdt)) ++j;
-    cq_status st = launch_gemv4_segs(qws + i, j - i, x, m, ys + i, s);
+    while (j < count && j - i < kMaxSegs &&
+           (tc ? gemv_tc_eligible(*qws[j], xdt) : gemv_res_eligible(*qws[j], xdt)))
+      ++j;
+    cq_status st = tc ? launch_gemv4_segs(qws + i, j - i, x, m, ys + i, s)
+                      : launch_gemv4r(qws + i, j - i, x, m, ys + i, s);
     if (st != CQ_OK) return st;
     i = j;
   }

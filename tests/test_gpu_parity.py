@@ -450,3 +450,27 @@ def test_gemm_bf16_residual_batches(rows, cols, m):
     rb, _ = co.project_bf16(synth.normal_residual_bf16(scale, seed=rows + 1, rel_sigma=0.3), scale)
     qw, x_d, y_ref, _ = _matmul_case(rows, cols, m, "bf16", r=rb, seed=rows + m)
     check_matmul(host(ops.gemm(qw, x_d)), y_ref, f"gemm r bf16 {rows}x{cols} m={m}")
+
+
+# several served-weight matrices (bf16 residual) that share x in one launch: ragged tiles in every
+# segment, more than four matrices (two launches), and a matrix without a residual in the list
+@pytest.mark.parametrize("m", [1, 5])
+def test_gemv_multi_with_residuals(m):
+    cols = 64 * 21
+    specs = [(300, True), (47, True), (64, True), (129, True), (1000, True), (33, False), (16, True)]
+    x = synth.activations(m, cols, seed=191 + m, dtype="bf16")
+    qws, refs = [], []
+    for i, (rows, with_r) in enumerate(specs):
+        w = synth.normal_weights(rows, cols, seed=170 + i)
+        qw, _, _, oc = _quantize_both(w, None)
+        planes, off = _oracle_qw(oc[0], oc[1], oc[2], None)
+        rb = None
+        if with_r:
+            rb, _ = co.project_bf16(synth.normal_residual_bf16(oc[1], seed=180 + i, rel_sigma=0.3), oc[1])
+            qw = qw.with_residual(bf16_dev(rb))
+        qws.append(qw)
+        refs.append(co.dequant_matmul_f64(planes, oc[1], oc[2], rows, cols, x, "bf16", None, None, rb,
+                                          "bf16" if with_r else "f32"))
+    ys = ops.gemv_multi(qws, bf16_dev(x))
+    for i, (qw, y_ref) in enumerate(zip(qws, refs)):
+        check_matmul(host(ys[i]), y_ref, f"multi residual[{i}] {qw.rows}x{qw.cols} m={m}")
