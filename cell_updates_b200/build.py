@@ -38,7 +38,8 @@ SYNTH_UNITS = {"synth.cu": EXACT}
 # test-only builds of libcq with a fault injected on the host side of a kernel's pipeline (a copy
 # that is never requested, so a bounded wait runs out and the abort path runs); the tests load
 # them by path, nothing else does
-TEST_VARIANTS = {"drop_first_copy": {"k_quantize.cu": ["-DCQ_TEST_DROP_FIRST_COPY"]}}
+TEST_VARIANTS = {"drop_first_copy": {"k_quantize.cu": ["-DCQ_TEST_DROP_FIRST_COPY"],
+                                      "k_gemm.cu": ["-DCQ_TEST_DROP_FIRST_COPY"]}}
 
 LIBCQ = os.path.join(HERE, "libcq.so")
 LIBSYNTH = os.path.join(HERE, "libcq_synth.so")

@@ -20,25 +20,23 @@
 // Structure (one CTA per SM, persistent; work = (128-row tile, step of four groups) items
 // split evenly over the CTAs in row-major order, so a CTA covers a contiguous K range of one
 // or a few tiles; a maximal run of one tile's steps in one CTA is a "segment"):
-//   warps 10-13 epilogue, and warps 10-12 loaders: copy each step's codes (128 rows x 128 bytes, eight
-//               lanes per row, so every warp instruction reads four whole 128-byte lines) and
-//               the rows' scales and zero points with cp.async into an 8-stage ring, seven
-//               steps ahead; cp.async completion arrives on the stage's barrier. At a
-//               segment's end they tcgen05.ld their rows of the accumulator, scale and add to y
-//               with atomics (segments of one tile in two CTAs combine there). Per-thread
-//               copies keep many short row runs in flight: DRAM serves this 128-row pattern
-//               about twice as fast as 128-row TMA boxes of the same bytes.
-//   warps 2-9   dequantize: thread (row, part) turns half a row of a group into fp16
-//               s * (q - z) and stores it to tensor memory (its lane = its row)
+//   warps 2-9   dequantize: thread (row, part) loads 64 contiguous bytes of its row (two groups
+//               of a step) plus their scales and zero points straight into registers, three
+//               steps ahead, turns them into fp16 s * (q - z) and stores them to tensor memory
+//               (its lane = its row). Codes never pass through shared memory: its bandwidth
+//               (128 B per clock) goes to the activation tiles and the MMAs' operand reads.
 //   warp 0      TMA producer: per step the fp16 activations (m rows x 64 per group, 128-byte
-//               swizzled = the UMMA K-major layout), double-buffered
+//               swizzled = the UMMA K-major layout)
 //   warp 1      MMA issuer: per group four tcgen05.mma (M=128, N=NT, K=16), A from tensor
 //               memory and B from shared memory, into the segment's accumulator (two
 //               accumulators alternate between segments)
-// A step's A operand is stored to tensor memory only once the previous step's MMAs have
-// completed (the dequantization arithmetic still overlaps them): stores into other columns of
-// the same lanes while MMAs that read A from tensor memory were in flight gave wrong sums on
-// this part for N = 16 and 32.
+//   warps 10-13 epilogue: at a segment's end they tcgen05.ld their rows of the accumulator,
+//               scale and add to y with atomics (segments of one tile in two CTAs combine
+//               there), after adding the segment's slow groups in fp32
+// Three steps are in flight in tensor memory (A slots: a_full when stored, step_free when their
+// MMAs completed), so the dequantizers store steps i + 1 and i + 2 while the MMAs of step i run;
+// the activation tiles have their own deeper ring (x_full / x_free, 5 stages at N = 64, 8 below),
+// because their TMA latency from L2, not the MMAs, otherwise sets the pace of the steps.
 // The preparation kernel also zeroes y and the status word. Every barrier wait is bounded: on
 // timeout the CTA raises a status flag, drains what it issued, frees its tensor memory and
 // returns.
@@ -51,20 +49,13 @@ constexpr int kTileM = 128;
 constexpr int kXWarp = 0;                          // TMA producer of the activation tiles
 constexpr int kMmaWarp = 1;
 constexpr int kDeqWarp0 = 2;
-constexpr int kRowParts = 2;                       // dequantizers per row, each 64 / kRowParts columns of a group
-constexpr int kDeqWarps = 4 * kRowParts;           // kRowParts per TMEM lane quarter
+constexpr int kDeqWarps = 8;                       // two per TMEM lane quarter, two groups of a step each
 constexpr int kEpiWarp0 = kDeqWarp0 + kDeqWarps;
 constexpr int kEpiWarps = 4;                       // one per TMEM lane quarter
-constexpr int kLoadWarps = 3;                      // epilogue warps that also load (not warp 13)
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr int kG = 4;                              // groups per pipeline step
-constexpr int kSteps = 2;                          // A (tensor memory) and activation (shared) slots
+constexpr int kSlots = 3;                          // steps in flight: A slots (tensor memory), activation stages
 constexpr int kAccBufs = 2;                        // fp32 segment accumulators in tensor memory
-constexpr int kRing = 8;                           // code / metadata stages loaded ahead
-constexpr uint32_t kCodeStepBytes = kTileM * 128;           // 128 rows x 4 groups x 32 B, swizzled
-constexpr uint32_t kScaleOff = kCodeStepBytes;              // 128 rows x 4 scales
-constexpr uint32_t kZeroOff = kScaleOff + kTileM * 8;       // 128 rows x 4 zero points
-constexpr uint32_t kStageBytes = kZeroOff + kTileM * 4;
 constexpr int kFlagSlots = 8;                      // per-segment masks of rows with slow groups
 constexpr uint32_t kACols = 32;                    // one group of A: 128 lanes x 64 fp16
 constexpr uint32_t kMaxFastScale = 0x6C00u;        // 4096 in fp16 bits
@@ -76,13 +67,34 @@ struct Cfg {
   static constexpr uint32_t kXBytes = NT * 128;                     // one group of activations
   static constexpr uint32_t kAccCols = kAccBufs * NT;
   static constexpr uint32_t kACol0 = kAccCols;                     // A slots follow the accumulators
-  static constexpr uint32_t kCols = kAccCols + kSteps * kG * kACols;
+  static constexpr uint32_t kCols = kAccCols + kSlots * kG * kACols;
   static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
   static_assert(kCols <= 512, "tensor memory holds 512 columns");
-  static constexpr int kBars = 2 * kRing + 3 * kSteps + 2 * kAccBufs + kFlagSlots + 1;
-  static constexpr uint32_t kSmem =
-      1024 + kRing * kStageBytes + kSteps * kG * kXBytes + kBars * 8 + kFlagSlots * 16 + NT * 4 + 16;
+  // activation stages: as many as fit in ~160 KB, so the TMA latency of the activation tiles
+  // (from L2) is hidden behind several steps; at most 8
+  static constexpr int kXStages = (160 * 1024) / (kG * kXBytes) < 8 ? (160 * 1024) / (kG * kXBytes) : 8;
+  static_assert(kXStages >= kSlots, "activation stages");
+  static constexpr int kBars = 2 * kSlots + 2 * kXStages + 2 * kAccBufs + kFlagSlots + 1;
+  static constexpr uint32_t kSmem = 1024 + kXStages * kG * kXBytes + kBars * 8 + kFlagSlots * 16 + NT * 4 + 16;
   static_assert(kSmem <= 232448, "shared memory per CTA");
+};
+
+// one group's codes, residual and metadata for one dequantizer thread (residual variant)
+struct ResBuf {
+  uint4 c[2];
+  uint4 r[8];
+  uint32_t s, z;
+};
+
+__device__ __forceinline__ uint32_t word4c(const uint4 &v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// one step's codes and metadata for one dequantizer thread: 64 bytes (two groups) of its row,
+// the two groups' fp16 scales and zero points
+struct CodeBuf {
+  uint4 c[4];
+  uint32_t s2, z2;
 };
 
 // UMMA shared-memory descriptor: K-major operand in the 128-byte swizzled canonical layout
@@ -120,6 +132,16 @@ __device__ __forceinline__ void umma_ts_lean(uint32_t tmem_d, uint32_t tmem_a, u
         "r"(tmem_a), "r"(bdesc_lo), "r"(bdesc_hi), "r"(idesc));
 }
 
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
 [[maybe_unused]] __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
@@ -205,12 +227,6 @@ __device__ __forceinline__ void deq_word(uint32_t wd, uint32_t zz1, uint32_t nzz
 __device__ __forceinline__ bool slow_group(uint32_t sbits, uint32_t z) {
   return (sbits & 0x7FFFu) > kMaxFastScale || z > kMaxFastZero;
 }
-
-// 16-byte copy into shared memory that bypasses L1, and the wait for all of a thread's copies
-__device__ __forceinline__ void cp_async_16cg(void *dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
 // The work of one CTA: steps = (tile, kG groups) in row-major order; step p of a tile covers
 // groups kG*p .. kG*p + kG - 1 (the tensor-core path takes K a multiple of 4 groups).
@@ -298,23 +314,28 @@ gemm_prep_kernel(const uint16_t *__restrict__ x, int64_t K, uint16_t *__restrict
 }
 
 // ---- the GEMM kernel ----------------------------------------------------------------------------
-template <int NT>
+// One step = kG groups (256 columns) of one 128-row tile. A step's A operand occupies one of
+// kSlots slots of tensor memory and its activations one of XS shared-memory stages; two MMA
+// commits per step (step_free, x_free) release them. The dequantizers load their rows' codes straight
+// into registers (kPre steps in flight per thread: 16-byte loads of 64 contiguous bytes per
+// row and step), so codes never pass through shared memory, whose bandwidth the activation
+// tiles and the MMAs' operand reads need.
+template <int NT, bool RES>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restrict__ plane,
                 const uint16_t *__restrict__ scale, const uint8_t *__restrict__ zero,
-                const uint16_t *__restrict__ xb, const float *__restrict__ xmul, float *__restrict__ y, int m,
-                int64_t N, int64_t K, int KG, int64_t n_items, uint32_t *__restrict__ status) {
+                const uint16_t *__restrict__ res, const uint16_t *__restrict__ xb, const float *__restrict__ xmul,
+                float *__restrict__ y, int m, int64_t N, int64_t K, int KG, int64_t n_items,
+                uint32_t *__restrict__ status) {
   using C = Cfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sR = smem;                                   // code / metadata ring filled by the loader warps
-  uint8_t *sX = sR + kRing * kStageBytes;               // activation tiles (1024-aligned, swizzled)
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sX + kSteps * kG * C::kXBytes);
-  // a step (kG groups) has an A slot in tensor memory and an activation slot in shared memory,
-  // filled separately (a_full, x_full) and released together by one MMA commit (s_empty)
-  uint64_t *r_full = bars, *r_empty = r_full + kRing;   // ring stages: copies landed / stage read
-  uint64_t *a_full = r_empty + kRing, *x_full = a_full + kSteps, *s_empty = x_full + kSteps;
-  uint64_t *acc_full = s_empty + kSteps, *acc_empty = acc_full + kAccBufs;
+  uint8_t *sX = smem;                                   // activation stages (1024-aligned, swizzled)
+  constexpr int XS = C::kXStages;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sX + XS * kG * C::kXBytes);
+  uint64_t *a_full = bars, *step_free = a_full + kSlots;   // A slots: stored / MMAs done
+  uint64_t *x_full = step_free + kSlots, *x_free = x_full + XS;   // activation stages: landed / MMAs done
+  uint64_t *acc_full = x_free + XS, *acc_empty = acc_full + kAccBufs;
   uint64_t *seg_done = acc_empty + kAccBufs;            // dequantizers finished a segment's masks
   uint64_t *drain = seg_done + kFlagSlots;
   uint32_t *seg_mask = reinterpret_cast<uint32_t *>(drain + 1);   // [kFlagSlots][4 lane quarters]
@@ -329,14 +350,13 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
   const int P = KG / kG;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kRing; ++i) {
-      mbar_init(r_full + i, 32 * kLoadWarps);   // one cp.async arrival per loader thread
-      mbar_init(r_empty + i, kDeqWarps);
-    }
-    for (int i = 0; i < kSteps; ++i) {
+    for (int i = 0; i < kSlots; ++i) {
       mbar_init(a_full + i, kDeqWarps);
+      mbar_init(step_free + i, 1);
+    }
+    for (int i = 0; i < XS; ++i) {
       mbar_init(x_full + i, 1);
-      mbar_init(s_empty + i, 1);
+      mbar_init(x_free + i, 1);
     }
     for (int i = 0; i < kAccBufs; ++i) {
       mbar_init(acc_full + i, 1);
@@ -365,17 +385,29 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
       Walk w;
       walk_init(w, it_begin, P);
       int x_issued = 0;
+      bool dropped = false;
       for (int li = 0; li < n_local; ++li) {
-        const int st = li % kSteps;
-        if (!mbar_wait(s_empty + st, ((li / kSteps) & 1) ^ 1, abort_flag, status)) break;
+        const int st = li % XS;
+        if (!mbar_wait(x_free + st, ((li / XS) & 1) ^ 1, abort_flag, status)) break;
+#ifdef CQ_TEST_DROP_FIRST_COPY
+        // test build only (never in libcq.so): CTA 0 does not request its first activation
+        // tiles, so the MMA issuer's wait runs out and every role takes the abort path
+        if (blockIdx.x == 0 && li == 0) {
+          dropped = true;
+          x_issued = li + 1;
+          walk_next(w, P);
+          continue;
+        }
+#endif
         uint8_t *dst = sX + st * kG * C::kXBytes;
         mbar_arrive_expect_tx(x_full + st, kG * C::kXBytes);
         for (int jj = 0; jj < kG; ++jj) tma_load_2d(dst + jj * C::kXBytes, &tm_x, (kG * w.p + jj) * 64, 0, x_full + st);
         x_issued = li + 1;
         walk_next(w, P);
       }
-      for (int li = x_issued - kSteps > 0 ? x_issued - kSteps : 0; li < x_issued; ++li)
-        mbar_wait(x_full + (li % kSteps), (li / kSteps) & 1, abort_flag, status, false);
+      // every issued copy lands before the CTA exits
+      for (int li = x_issued - XS > 0 ? x_issued - XS : 0; li < x_issued; ++li)
+        if (!(dropped && li == 0)) mbar_wait(x_full + (li % XS), (li / XS) & 1, abort_flag, status, false);
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
@@ -390,15 +422,16 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
       int seg = 0;
       bool first = true;          // the next step opens a segment
       for (int li = 0; li < n_local; ++li) {
-        const int st = li % kSteps, b = seg % kAccBufs;
+        const int st = li % kSlots, b = seg % kAccBufs, xst = li % XS;
+        const uint32_t par = (li / kSlots) & 1;
         const bool seg_end = walk_seg_end(w, P, it_end);
         if (first && !mbar_wait(acc_empty + b, ((seg / kAccBufs) & 1) ^ 1, abort_flag, status)) break;
-        if (!mbar_wait(a_full + st, (li / kSteps) & 1, abort_flag, status)) break;
-        if (!mbar_wait(x_full + st, (li / kSteps) & 1, abort_flag, status)) break;
+        if (!mbar_wait(x_full + xst, (li / XS) & 1, abort_flag, status)) break;
+        if (!mbar_wait(a_full + st, par, abort_flag, status)) break;
         tc_fence_after();
         const uint32_t ta = tmem + C::kACol0 + st * kG * kACols;
         const uint32_t td = tmem + b * NT;
-        const uint32_t blo = dlo0 + ((st * kG * C::kXBytes) >> 4);
+        const uint32_t blo = dlo0 + ((xst * kG * C::kXBytes) >> 4);
         if (first) umma_ts_lean<false>(td, ta, blo, dhi, idesc);
         else umma_ts_lean<true>(td, ta, blo, dhi, idesc);
         umma_ts_lean<true>(td, ta + 8, blo + 2, dhi, idesc);
@@ -412,7 +445,8 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
           umma_ts_lean<true>(td, taj + 16, bj + 4, dhi, idesc);
           umma_ts_lean<true>(td, taj + 24, bj + 6, dhi, idesc);
         }
-        umma_commit(s_empty + st);
+        umma_commit(step_free + st);
+        umma_commit(x_free + xst);
         if (seg_end) {
           umma_commit(acc_full + b);
           ++seg;
@@ -425,128 +459,174 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
       mbar_wait(drain, 0, abort_flag, status, false);
     }
   } else if (warp < kEpiWarp0) {
-    // ---------------- dequantize: a part of a row per thread, into tensor memory ----------------
+    // ---------------- dequantize: two groups of a row per thread, into tensor memory ----------------
     // a warp may only touch TMEM lanes 32 * (warp % 4) .. + 31, so rows follow the warp index
-    constexpr int kW = 8 / kRowParts;             // code words per group and thread (4 columns each)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;               // tile row = TMEM lane
-    const int part = (warp - kDeqWarp0) >> 2;     // columns (64 / kRowParts) * part .. of each group
-    Walk w;
-    walk_init(w, it_begin, P);
+    const int part = (warp - kDeqWarp0) >> 2;     // groups 2 part, 2 part + 1 of each step
     const uint32_t tlane = static_cast<uint32_t>(quad * 32) << 16;
+    const int64_t row_bytes = K / 2;
+    Walk wl, wp;
+    walk_init(wl, it_begin, P);
+    walk_init(wp, it_begin, P);
     int seg = 0;
     bool slow = false;                            // this row has a slow group in the segment
-    for (int li = 0; li < n_local; ++li) {
-      const int st = li % kSteps, rs = li % kRing;
-      if (!warp_wait(r_full + rs, (li / kRing) & 1, abort_flag, status)) break;
-      const uint8_t *sb = sR + rs * kStageBytes;
-      const uint2 sm = *reinterpret_cast<const uint2 *>(sb + kScaleOff + r * 8);
-      const uint32_t zw = *reinterpret_cast<const uint32_t *>(sb + kZeroOff + r * 4);
-      uint32_t v[kG][4 * kW];
+    auto load = [&](CodeBuf &cb) {
+      int64_t row = static_cast<int64_t>(wl.tile) * kTileM + r;
+      row = row < N ? row : N - 1;                // rows past the end: any valid row, result unused
+      const int g = kG * wl.p + 2 * part;
+      const uint4 *src = reinterpret_cast<const uint4 *>(plane + row * row_bytes + g * 32);
+      cb.c[0] = __ldcs(src);
+      cb.c[1] = __ldcs(src + 1);
+      cb.c[2] = __ldcs(src + 2);
+      cb.c[3] = __ldcs(src + 3);
+      cb.s2 = __ldg(reinterpret_cast<const uint32_t *>(scale + row * KG + g));
+      cb.z2 = __ldg(reinterpret_cast<const uint16_t *>(zero + row * KG + g));
+      walk_next(wl, P);
+    };
+    // dequantize a loaded step into its A slot; false when a wait gave up
+    auto process = [&](const CodeBuf &cb, int li) -> bool {
+      const int st = li % kSlots;
+      uint32_t v[32];
 #pragma unroll
-      for (int jj = 0; jj < kG; ++jj) {
-        const uint32_t z = (zw >> (8 * jj)) & 0xFFu;
-        const uint32_t sbits = ((jj < 2 ? sm.x : sm.y) >> (16 * (jj & 1))) & 0xFFFFu;
+      for (int grp = 0; grp < 2; ++grp) {
+        const uint32_t z = (cb.z2 >> (8 * grp)) & 0xFFu;
+        const uint32_t sbits = (cb.s2 >> (16 * grp)) & 0xFFFFu;
         const bool sl = slow_group(sbits, z);
         slow |= sl;
         const uint32_t zc = sl ? 0u : z;
         const uint32_t zz1 = 0x64006400u | zc | (zc << 16);
         const uint32_t nzz16 = 0xD400D400u | (zc << 4) | (zc << 20);
         const uint32_t s2 = sl ? 0u : (sbits | (sbits << 16));
-        // bytes 32 jj + 4 kW part .. of row r: 16-byte chunk (32 jj + 4 kW part) / 16, swizzled by
-        // the row's low three bits
-        const int byte0 = jj * 32 + 4 * kW * part;
-        const uint8_t *cp = sb + r * 128 + ((((byte0 >> 4) ^ (r & 7))) << 4) + (byte0 & 15);
-        if constexpr (kW == 4) {
-          const uint4 cw = *reinterpret_cast<const uint4 *>(cp);
-          deq_word(cw.x, zz1, nzz16, s2, &v[jj][0]);
-          deq_word(cw.y, zz1, nzz16, s2, &v[jj][4]);
-          deq_word(cw.z, zz1, nzz16, s2, &v[jj][8]);
-          deq_word(cw.w, zz1, nzz16, s2, &v[jj][12]);
-        } else {
-          const uint2 cw = *reinterpret_cast<const uint2 *>(cp);
-          deq_word(cw.x, zz1, nzz16, s2, &v[jj][0]);
-          deq_word(cw.y, zz1, nzz16, s2, &v[jj][4]);
+        const uint4 lo = cb.c[2 * grp], hi = cb.c[2 * grp + 1];
+        deq_word(lo.x, zz1, nzz16, s2, &v[0]);
+        deq_word(lo.y, zz1, nzz16, s2, &v[4]);
+        deq_word(lo.z, zz1, nzz16, s2, &v[8]);
+        deq_word(lo.w, zz1, nzz16, s2, &v[12]);
+        deq_word(hi.x, zz1, nzz16, s2, &v[16]);
+        deq_word(hi.y, zz1, nzz16, s2, &v[20]);
+        deq_word(hi.z, zz1, nzz16, s2, &v[24]);
+        deq_word(hi.w, zz1, nzz16, s2, &v[28]);
+        if (grp == 0) {
+          // the slot is free once the MMAs of the step kSlots earlier have completed
+          if (li >= kSlots && !warp_wait(step_free + st, ((li / kSlots) & 1) ^ 1, abort_flag, status)) return false;
+          tc_fence_after();
         }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(r_empty + rs);   // the stage is in registers
-      // A is stored only while no MMA is in flight: the previous step's commit covers them all
-      if (li > 0 && !warp_wait(s_empty + (li - 1) % kSteps, ((li - 1) / kSteps) & 1, abort_flag, status)) break;
-      tc_fence_after();
-      const uint32_t ta = tmem + tlane + C::kACol0 + st * kG * kACols + part * 4 * kW;
-#pragma unroll
-      for (int jj = 0; jj < kG; ++jj) {
-        if constexpr (kW == 4) tmem_st16(ta + jj * kACols, v[jj]);
-        else tmem_st8(ta + jj * kACols, v[jj]);
+        tmem_st32(tmem + tlane + C::kACol0 + st * kG * kACols + (2 * part + grp) * kACols, v);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(a_full + st);
-      if (walk_seg_end(w, P, it_end)) {
+      if (walk_seg_end(wp, P, it_end)) {
         // rows whose slow groups the epilogue adds; then the segment's mask is complete
         const uint32_t bal = __ballot_sync(0xFFFFFFFFu, slow);
-        const int slot = seg % kFlagSlots;
+        const int fs = seg % kFlagSlots;
         if (lane == 0) {
-          if (bal) atomicOr(seg_mask + slot * 4 + quad, bal);
-          mbar_arrive(seg_done + slot);
+          if (bal) atomicOr(seg_mask + fs * 4 + quad, bal);
+          mbar_arrive(seg_done + fs);
         }
         slow = false;
         ++seg;
       }
-      walk_next(w, P);
+      walk_next(wp, P);
+      return true;
+    };
+    if constexpr (!RES) {
+      CodeBuf b0, b1, b2;
+      if (n_local > 0) load(b0);
+      if (n_local > 1) load(b1);
+      if (n_local > 2) load(b2);
+      for (int li = 0; li < n_local; li += 3) {
+        if (!process(b0, li)) break;
+        if (li + 3 < n_local) load(b0);
+        if (li + 1 >= n_local || !process(b1, li + 1)) break;
+        if (li + 4 < n_local) load(b1);
+        if (li + 2 >= n_local || !process(b2, li + 2)) break;
+        if (li + 5 < n_local) load(b2);
+      }
+    } else {
+      // with a bf16 residual: A = RN16(fma(s, q - z, r)) (q - z exact in fp32, one fp32 rounding,
+      // then one fp16 rounding), one group at a time with the next group's loads in flight (the
+      // residual is four times the codes' bytes, so fewer groups fit in registers)
+      const int n_grp = 2 * n_local;
+      auto rload = [&](ResBuf &b, int t) {
+        int64_t row = static_cast<int64_t>(wl.tile) * kTileM + r;
+        row = row < N ? row : N - 1;
+        const int g = kG * wl.p + 2 * part + (t & 1);
+        const uint4 *src = reinterpret_cast<const uint4 *>(plane + row * row_bytes + g * 32);
+        b.c[0] = __ldcs(src);
+        b.c[1] = __ldcs(src + 1);
+        const uint4 *rs = reinterpret_cast<const uint4 *>(res + row * K + g * 64);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) b.r[i] = __ldcs(rs + i);
+        b.s = __ldg(scale + row * KG + g);
+        b.z = __ldg(zero + row * KG + g);
+        if (t & 1) walk_next(wl, P);
+      };
+      auto rprocess = [&](const ResBuf &b, int t) -> bool {
+        const int li = t >> 1, grp = t & 1, st = li % kSlots;
+        const bool sl = slow_group(b.s, b.z);
+        slow |= sl;
+        const float sf = sl ? 0.0f : f16_bits_to_f32(static_cast<uint16_t>(b.s));
+        const float zb = 8388608.0f + static_cast<float>(sl ? 0u : b.z);
+        uint32_t v[32];
+#pragma unroll
+        for (int wd = 0; wd < 8; ++wd) {
+          const uint32_t cw = wd < 4 ? word4c(b.c[0], wd) : word4c(b.c[1], wd - 4);
+          const uint4 rr = b.r[wd];       // residuals of k = 8 wd .. 8 wd + 7
+          const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            // the pair (j, j + 4) of these eight: codes at nibbles j and j + 4
+            const float qa = __fsub_rn(__uint_as_float(0x4B000000u | ((cw >> (4 * j)) & 15u)), zb);
+            const float qb = __fsub_rn(__uint_as_float(0x4B000000u | ((cw >> (4 * j + 16)) & 15u)), zb);
+            const uint32_t w0 = rw[j >> 1], w1 = rw[2 + (j >> 1)];
+            const float ra = __uint_as_float((j & 1) ? (w0 & 0xFFFF0000u) : (w0 << 16));
+            const float rb = __uint_as_float((j & 1) ? (w1 & 0xFFFF0000u) : (w1 << 16));
+            const __half2 h = __floats2half2_rn(__fmaf_rn(sf, qa, ra), __fmaf_rn(sf, qb, rb));
+            v[4 * wd + j] = *reinterpret_cast<const uint32_t *>(&h);
+          }
+        }
+        if (grp == 0) {
+          if (li >= kSlots && !warp_wait(step_free + st, ((li / kSlots) & 1) ^ 1, abort_flag, status)) return false;
+          tc_fence_after();
+        }
+        tmem_st32(tmem + tlane + C::kACol0 + st * kG * kACols + (2 * part + grp) * kACols, v);
+        if (grp == 1) {
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(a_full + st);
+          if (walk_seg_end(wp, P, it_end)) {
+            const uint32_t bal = __ballot_sync(0xFFFFFFFFu, slow);
+            const int fs = seg % kFlagSlots;
+            if (lane == 0) {
+              if (bal) atomicOr(seg_mask + fs * 4 + quad, bal);
+              mbar_arrive(seg_done + fs);
+            }
+            slow = false;
+            ++seg;
+          }
+          walk_next(wp, P);
+        }
+        return true;
+      };
+      ResBuf a0, a1;
+      if (n_grp > 0) rload(a0, 0);
+      if (n_grp > 1) rload(a1, 1);
+      for (int t = 0; t < n_grp; t += 2) {
+        if (!rprocess(a0, t)) break;
+        if (t + 2 < n_grp) rload(a0, t + 2);
+        if (!rprocess(a1, t + 1)) break;
+        if (t + 3 < n_grp) rload(a1, t + 3);
+      }
     }
   } else {
     // ---------------- epilogue: one row per thread, all NT columns ----------------
     const int quad = warp & 3;                 // this warp may read TMEM lanes 32*quad .. +31
     const int r = quad * 32 + lane;
     const int et = threadIdx.x - 32 * kEpiWarp0;
-    // loader: step la's copies into ring stage la % kRing, once the dequantizers have read the
-    // step that used it before; lane l of a warp copies 16-byte chunk l % 8 of four rows per
-    // instruction, and the four scales and zero points of one or two rows
-    const int64_t row_bytes = K / 2;
-    Walk wl;
-    walk_init(wl, it_begin, P);
-    int la = 0;
-    bool ok = true;
-    // the warp on the MMA issuer's scheduler (warp % 4 == 1) does not load: it would slow the
-    // dequantizers that share that scheduler, which already lose issue slots to the MMA issuer
-    const bool loader = (warp & 3) != kMmaWarp;
-    const int lw = (warp & 3) == 0 ? 2 : (warp & 3) - 2;   // warps 10, 11, 12 -> 0, 1, 2
-    auto load_until = [&](int target) {
-      if (!loader) return;
-      const int lim = target < n_local ? target : n_local;
-      while (ok && la < lim) {
-        const int rs = la % kRing;
-        if (!warp_wait(r_empty + rs, ((la / kRing) & 1) ^ 1, abort_flag, status)) {
-          ok = false;
-          break;
-        }
-        uint8_t *sb = sR + rs * kStageBytes;
-        const int g = kG * wl.p;
-        const int64_t row0 = static_cast<int64_t>(wl.tile) * kTileM;
-#pragma unroll
-        for (int k = 0; k < (32 + kLoadWarps - 1) / kLoadWarps; ++k) {
-          const int rg = lw + kLoadWarps * k;     // group of four rows
-          if (rg >= 32) break;
-          const int rr = rg * 4 + (lane >> 3), c = lane & 7;
-          int64_t row = row0 + rr;
-          row = row < N ? row : N - 1;            // rows past the end: any valid row, result unused
-          cp_async_16cg(sb + rr * 128 + ((c ^ (rr & 7)) << 4), plane + row * row_bytes + g * 32 + c * 16);
-        }
-        for (int t = lw * 32 + lane; t < kTileM; t += 32 * kLoadWarps) {
-          int64_t row = row0 + t;
-          row = row < N ? row : N - 1;
-          cp_async_8(sb + kScaleOff + t * 8, scale + row * KG + g);
-          cp_async_4(sb + kZeroOff + t * 4, zero + row * KG + g);
-        }
-        cp_async_arrive_noinc(r_full + rs);
-        walk_next(wl, P);
-        ++la;
-      }
-    };
-    load_until(kRing);                         // fill the ring before anything else
     pdl_wait();                                // xmul and the zeroed y come from the preparation kernel
     if (et < NT) s_xmul[et] = et < m ? xmul[et] : 0.0f;
     epi_sync();
@@ -554,19 +634,18 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
     walk_init(w, it_begin, P);
     int seg = 0, ga = kG * w.p;
     bool open = true;                          // the next step opens a segment
-    for (int li = 0; li < n_local && ok; ++li) {
-      load_until(li + kRing);                  // refill the stage the dequantizers freed
+    for (int li = 0; li < n_local; ++li) {
       if (open) ga = kG * w.p;
       const bool seg_end = walk_seg_end(w, P, it_end);
       open = seg_end;
       if (seg_end) {
-        const int b = seg % kAccBufs, slot = seg % kFlagSlots;
+        const int b = seg % kAccBufs, fs = seg % kFlagSlots;
         const int gb = kG * w.p + kG;
         const int64_t row = static_cast<int64_t>(w.tile) * kTileM + r;
-        if (!warp_wait(seg_done + slot, (seg / kFlagSlots) & 1, abort_flag, status)) break;
-        const uint32_t mask = seg_mask[slot * 4 + quad];
+        if (!warp_wait(seg_done + fs, (seg / kFlagSlots) & 1, abort_flag, status)) break;
+        const uint32_t mask = seg_mask[fs * 4 + quad];
         __syncwarp();
-        if (lane == 0) seg_mask[slot * 4 + quad] = 0u;
+        if (lane == 0) seg_mask[fs * 4 + quad] = 0u;
         if (((mask >> lane) & 1u) && row < N) {
           // groups the tensor cores did not take: s * sum_k (q - z) x in fp32, straight to y
           for (int g = ga; g < gb; ++g) {
@@ -610,7 +689,6 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
       }
       walk_next(w, P);
     }
-    cp_async_wait_all();                       // no copy may land after the CTA has exited
   }
   __syncthreads();
   if (warp == kMmaWarp) {
@@ -626,7 +704,7 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
 constexpr size_t kWsXmul = 16, kWsX16 = 512;
 constexpr int kSliceRows = 64;
 
-template <int NT>
+template <int NT, bool RES>
 cq_status launch_nt(const cq_qweight &qw, const void *x, int m, float *y, uint8_t *ws, bool clear_status,
                     cudaStream_t s) {
   using C = Cfg<NT>;
@@ -661,7 +739,7 @@ cq_status launch_nt(const cq_qweight &qw, const void *x, int m, float *y, uint8_
   const int64_t tiles = (N + kTileM - 1) / kTileM;
   const int64_t items = tiles * (KG / kG);                // steps of kG groups
   const int64_t grid = items < sm_count() ? items : sm_count();
-  cq_status st = cuda_check(cudaFuncSetAttribute(gemm4_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cq_status st = cuda_check(cudaFuncSetAttribute(gemm4_tc_kernel<NT, RES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  static_cast<int>(C::kSmem)),
                             "cq_dequant_gemm: shared memory attribute");
   if (st != CQ_OK) return st;
@@ -675,20 +753,23 @@ cq_status launch_nt(const cq_qweight &qw, const void *x, int m, float *y, uint8_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_check(cudaLaunchKernelEx(&cfg, gemm4_tc_kernel<NT>, tm_x, static_cast<const uint8_t *>(qw.plane[2]),
-                                       qw.scale, qw.zero, static_cast<const uint16_t *>(x),
-                                       static_cast<const float *>(xmul), y, m, N, K, KG, items, status),
+  return cuda_check(cudaLaunchKernelEx(&cfg, gemm4_tc_kernel<NT, RES>, tm_x, static_cast<const uint8_t *>(qw.plane[2]),
+                                       qw.scale, qw.zero, static_cast<const uint16_t *>(qw.residual),
+                                       static_cast<const uint16_t *>(x), static_cast<const float *>(xmul), y, m, N, K,
+                                       KG, items, status),
                     "cq_dequant_gemm");
 }
 
 }  // namespace
 
-// fixed-4 weights without a residual, bf16 x, m >= 16, K a multiple of 4 groups, and the
-// alignments the per-thread copies need (16-byte codes, 8-byte scales, 4-byte zero points)
+// fixed-4 weights, no residual or a bf16 one, bf16 x, m >= 16, K a multiple of 4 groups, and the
+// alignments the per-thread loads need (16-byte codes and residual rows, 4-byte scale pairs,
+// 2-byte zero pairs)
 bool gemm_tc_eligible(const cq_qweight &qw, cq_dtype xdt, int m) {
-  return qw.bits == nullptr && qw.residual == nullptr && xdt == CQ_BF16 && m >= 16 && qw.rows > 0 && qw.cols > 0 &&
-         (qw.cols / kGroup) % kG == 0 && aligned16(qw.plane[2]) && aligned8(qw.scale) &&
-         (reinterpret_cast<uintptr_t>(qw.zero) & 3u) == 0;
+  const bool res_ok = qw.residual == nullptr || (qw.residual_dtype == CQ_BF16 && aligned16(qw.residual));
+  return qw.bits == nullptr && res_ok && xdt == CQ_BF16 && m >= 16 && qw.rows > 0 && qw.cols > 0 &&
+         (qw.cols / kGroup) % kG == 0 && aligned16(qw.plane[2]) && (reinterpret_cast<uintptr_t>(qw.scale) & 3u) == 0 &&
+         (reinterpret_cast<uintptr_t>(qw.zero) & 1u) == 0;
 }
 
 // the status word, the per-row powers of two and the fp16 activations of one batch slice
@@ -708,9 +789,15 @@ cq_status launch_gemm_tc(const cq_qweight &qw, const void *x, int m, float *y, v
     float *yi = y + static_cast<int64_t>(i0) * N;
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     cq_status st;
-    if (mi <= 16) st = launch_nt<16>(qw, xi, mi, yi, w8, i0 == 0, s);
-    else if (mi <= 32) st = launch_nt<32>(qw, xi, mi, yi, w8, i0 == 0, s);
-    else st = launch_nt<64>(qw, xi, mi, yi, w8, i0 == 0, s);
+    if (qw.residual) {
+      if (mi <= 16) st = launch_nt<16, true>(qw, xi, mi, yi, w8, i0 == 0, s);
+      else if (mi <= 32) st = launch_nt<32, true>(qw, xi, mi, yi, w8, i0 == 0, s);
+      else st = launch_nt<64, true>(qw, xi, mi, yi, w8, i0 == 0, s);
+    } else {
+      if (mi <= 16) st = launch_nt<16, false>(qw, xi, mi, yi, w8, i0 == 0, s);
+      else if (mi <= 32) st = launch_nt<32, false>(qw, xi, mi, yi, w8, i0 == 0, s);
+      else st = launch_nt<64, false>(qw, xi, mi, yi, w8, i0 == 0, s);
+    }
     if (st != CQ_OK) return st;
   }
   return CQ_OK;

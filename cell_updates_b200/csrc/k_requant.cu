@@ -31,7 +31,7 @@ namespace {
 constexpr int kRqTile = 64;          // gradient tile: 64 rows x 64 columns of g
 constexpr int kRqK = 16;             // k per shared-memory stage
 constexpr int kRqThreads = 256;      // 16 x 16 threads, 4 x 4 outputs each
-constexpr int kSweepMaxWarps = 4;    // rows per sweep CTA when their g fit in shared memory
+constexpr int kSweepMaxWarps = 8;    // rows per sweep CTA when their g fit in shared memory
 constexpr size_t kSweepSmem = 200 * 1024;
 
 __device__ __forceinline__ double code_residual(const float *w, const uint16_t *scale, const uint8_t *zero,
@@ -118,17 +118,20 @@ rq_sweep_kernel(const double *__restrict__ H, const uint16_t *__restrict__ scale
   const int64_t KG = K >> 6;
   uint8_t *qn = codes + n * K;
   unsigned long long mv = 0;
+  const int Ki = static_cast<int>(K);
   for (int sw = 0; sw < sweeps; ++sw) {
-    for (int64_t k0 = 0; k0 < K; k0 += 32) {
-      // the lanes fetch 32 codes at a time; every lane then walks them in order
+    for (int k0 = 0; k0 < Ki; k0 += 32) {
+      // the lanes fetch 32 codes and the 32 diagonal entries of H at a time; every lane then
+      // walks them in order
       int qv = qn[k0 + lane];
+      const double hdiag = H[static_cast<int64_t>(k0 + lane) * (K + 1)];
       const double S = static_cast<double>(f16_bits_to_f32(scale[n * KG + (k0 >> 6)]));
       const double SS = __dmul_rn(S, S), S2 = __dmul_rn(2.0, S);
       for (int i = 0; i < 32; ++i) {
-        const int64_t k = k0 + i;
+        const int k = k0 + i;
         const int q = __shfl_sync(0xffffffffu, qv, i);
         const double gk = gr[k];
-        const double t2 = __dmul_rn(SS, H[k * K + k]);
+        const double t2 = __dmul_rn(SS, __shfl_sync(0xffffffffu, hdiag, i));
         const double t4 = __dmul_rn(S2, gk);
         const double up = __dsub_rn(t2, t4), down = __dadd_rn(t2, t4);
         int step = (q < L && up < 0.0) ? 1 : 0;
@@ -136,9 +139,11 @@ rq_sweep_kernel(const double *__restrict__ H, const uint16_t *__restrict__ scale
         if (step) {                      // warp-uniform: every lane took the same decision
           const double delta = step > 0 ? S : -S;
           if (lane == i) qv = q + step;
-          const double *hk = H + k * K;
+          const double *hk = H + static_cast<int64_t>(k) * K;
           __syncwarp();
-          for (int64_t j = lane; j < K; j += 32) gr[j] = __dsub_rn(gr[j], __dmul_rn(delta, hk[j]));
+          // row k of H, lane-strided and coalesced (measured faster than explicitly batching
+          // the loads, which the compiler does on its own); each g_j receives this one update
+          for (int j = lane; j < Ki; j += 32) gr[j] = __dsub_rn(gr[j], __dmul_rn(delta, hk[j]));
           __syncwarp();
           ++mv;
         }

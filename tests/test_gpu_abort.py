@@ -57,3 +57,38 @@ def test_quantize_wait_runs_out_and_reports_timeout(cuda_ok):
     assert np.array_equal(host(codes2), oc)
     assert np.array_equal(host(scale2, np.uint16), osc)
     assert np.array_equal(host(zero2), oz)
+
+
+def test_gemm_wait_runs_out_and_reports_status(cuda_ok):
+    # the same test-only build omits CTA 0's first activation tiles in the tensor-core GEMM: the
+    # MMA issuer's wait gives up, every role of that CTA takes the abort path (the issued copies
+    # land, the issued MMAs drain, tensor memory is released), the status word in the workspace
+    # is non-zero, and the regular library then computes the same product correctly
+    build.build()
+    L = C.CDLL(build.test_variant_path("drop_first_copy"))
+    L.cq_dequant_gemm.argtypes = [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_size_t,
+                                  C.c_void_p]
+    L.cq_dequant_gemm.restype = C.c_int
+    rows, cols, m = 512, 4096, 64
+    w = synth.normal_weights(rows, cols, seed=3)
+    qw, _, _ = ops.quantize_and_pack(dev(w))
+    x = torch.from_numpy(synth.activations(m, cols, seed=4, dtype="bf16").view(np.int16)).cuda().view(torch.bfloat16)
+    y = torch.zeros((m, rows), device="cuda")
+    need = cq.cq_gemm_workspace(rows, cols, m)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    s = qw.struct()
+    torch.cuda.synchronize()
+    t0 = time.monotonic()
+    rc = L.cq_dequant_gemm(C.byref(s), x.data_ptr(), cq.CQ_BF16, m, y.data_ptr(), ws.data_ptr(), need,
+                           C.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    elapsed = time.monotonic() - t0
+    assert rc == 0
+    assert int(ws[:4].view(torch.int32).cpu()[0]) != 0
+    assert elapsed < 30.0, elapsed
+    ref = ops.gemm(qw, x)                          # regular library, same device: a correct product
+    planes = [np.zeros(1, np.uint8)] * 2 + [host(qw.planes[2]), np.zeros(1, np.uint8)]
+    from gpu_util import check_matmul
+    y_ref = co.dequant_matmul_f64(planes, host(qw.scale, np.uint16), host(qw.zero), rows, cols,
+                                  host(x.view(torch.int16)).view(np.uint16), "bf16")
+    check_matmul(host(ref).astype(np.float64), y_ref, "gemm after an aborted call")
