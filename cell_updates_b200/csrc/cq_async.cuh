@@ -59,18 +59,10 @@ constexpr uint32_t kSuspendLimit = 1u << 20;
 __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile uint32_t *abort_flag,
                                           uint32_t *status, bool honour_abort = true) {
   if (mbar_try_wait(b, parity)) return true;
-#ifdef CQ_SPIN_WAIT
-  // polling without a suspend hint (same limit in tries; each try is shorter)
-  for (uint32_t i = 0; i < kSuspendLimit * 16u; ++i) {
-    if (mbar_try_wait(b, parity)) return true;
-    if (honour_abort && *abort_flag) return false;
-  }
-#else
   for (uint32_t i = 0; i < kSuspendLimit; ++i) {
     if (mbar_try_wait_hint(b, parity, 1000u)) return true;
     if (honour_abort && *abort_flag) return false;
   }
-#endif
   *abort_flag = 1u;
   if (status) {
     // the status word may be cleared by the kernel this grid overlaps (programmatic dependent
