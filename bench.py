@@ -9,9 +9,11 @@ configuration (three weight matrices 4096x4096, 11008x4096, 4096x11008, drawn as
     without it (revocation), both in one pass -> dequant-GEMV at batch 1 (decode)
     -> dequant-GEMM at batch 64
 
-for each matrix (each row runs over the three matrices before the next row starts).  K steps
-are captured as one CUDA graph and replayed for the timed region; per-row durations come from a
-second K-step graph with an event pair around each row's three launches, replayed after it.
+The three matrices are one flat artifact (their buffers back to back), so quantize, pack,
+project and the verify pair each run as one call over all of them; the GEMV and the GEMM run per
+matrix.  K steps are captured as one CUDA graph and replayed for the timed region; per-row
+durations come from a second K-step graph with an event pair around each row's calls, replayed
+after it.
 Printed: one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cq|reference]
@@ -68,9 +70,10 @@ def kernel_bytes(n):
 KERNELS = ["quantize", "pack", "project", "verify_pair", "gemv", "gemm"]
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
-# the kernel's launches in one step of this workload (mean over the three matrices), taken with
-# the kernel as it is now; a kernel changed since its capture gets no entry (traffic null).
-MEASURED_TRAFFIC = {"quantize": 158.5e6}
+# the kernel's launch in a step of this workload (one launch over the three matrices' flat
+# artifact; mean of two steps), taken with the kernel as it is now; a kernel changed since its
+# capture gets no entry (traffic null).
+MEASURED_TRAFFIC = {"quantize": 518.6e6}
 
 
 # ---------------------------------------------------------------------------------------
@@ -144,60 +147,84 @@ def count_kernel_nodes(graph):
 
 
 class Workload:
+    """The three decode matrices as one flat artifact: their fp32 weights, codes, scales, zero
+    points, 4-bit plane and bf16 residuals are allocated back to back, so the streaming rows
+    (quantize, pack, project, both verify checks) each run as one call over all of them -- the
+    format is a flat sequence of 64-weight groups, whatever the matrix shapes -- while the GEMV
+    and the GEMM run per matrix on views of the same buffers."""
+
     def __init__(self, torch, cq, ops, synth, device, seed_base=1):
         self.torch, self.cq, self.ops = torch, cq, ops
-        self.mats = []
+        ns = [N * K for (N, K) in SHAPES]
+        n_all = sum(ns)
+        G_all = n_all // GROUP
+        self.n_all = n_all
+        w_parts, r_parts = [], []
+        self.w = torch.empty(n_all, dtype=torch.float32, device=device)
+        self.codes = torch.empty(n_all, dtype=torch.uint8, device=device)
+        self.scale = torch.empty(G_all, dtype=torch.int16, device=device)
+        self.zero = torch.empty(G_all, dtype=torch.uint8, device=device)
+        self.plane = torch.empty(n_all // 2, dtype=torch.uint8, device=device)
+        self.r = torch.empty(n_all, dtype=torch.bfloat16, device=device)
         for idx, (N, K) in enumerate(SHAPES):
-            w = synth.student_t_weights(N, K, seed=seed_base + 1000 * idx)
-            w_host = torch.from_numpy(w).pin_memory()
-            w_dev = w_host.to(device)
-            qw, codes, status = ops.quantize_and_pack(w_dev)
-            scale_np = qw.scale.cpu().view(torch.int16).numpy().view(np.uint16)
-            r = synth.normal_residual_bf16(scale_np, seed=seed_base + 1000 * idx + 7, rel_sigma=0.3)
-            r_host = torch.from_numpy(r.view(np.int16)).view(torch.bfloat16).pin_memory()
+            w_parts.append(synth.student_t_weights(N, K, seed=seed_base + 1000 * idx).ravel())
+        self.w_host = torch.from_numpy(np.concatenate(w_parts)).pin_memory()
+        self.w.copy_(self.w_host)
+        st = torch.zeros(1, dtype=torch.int32, device=device)
+        cq.cq_quantize(self.w.view(1, n_all), None, self.codes, self.scale, self.zero, st)
+        cq.cq_pack_varbits(self.codes, G_all, None, None, [None, None, self.plane, None])
+        scale_np = self.scale.cpu().view(torch.int16).numpy().view(np.uint16)
+        self.mats = []
+        off = 0
+        for idx, (N, K) in enumerate(SHAPES):
+            n = N * K
+            g0, g1 = off // GROUP, (off + n) // GROUP
+            r_parts.append(synth.normal_residual_bf16(scale_np[g0:g1], seed=seed_base + 1000 * idx + 7,
+                                                      rel_sigma=0.3).view(np.int16))
             x = synth.activations(1, K, seed=seed_base + 1000 * idx + 11, dtype="bf16")
             X = synth.activations(GEMM_M, K, seed=seed_base + 1000 * idx + 13, dtype="bf16")
             x_host = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
             X_host = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).pin_memory()
-            m = dict(N=N, K=K, n=N * K, w_host=w_host, w=w_dev, codes=codes, qw=qw,
-                     r_host=r_host, r=r_host.to(device), x_host=x_host, x=x_host.to(device),
-                     X_host=X_host, X=X_host.to(device),
-                     y=torch.empty(1, N, device=device), Y=torch.empty(GEMM_M, N, device=device),
-                     status=torch.zeros(1, dtype=torch.int32, device=device),
-                     mism=torch.zeros(1, dtype=torch.int64, device=device),
-                     first=torch.zeros(1, dtype=torch.int64, device=device),
-                     mism0=torch.zeros(1, dtype=torch.int64, device=device),
-                     first0=torch.zeros(1, dtype=torch.int64, device=device),
-                     nclamp=torch.zeros(1, dtype=torch.int64, device=device))
+            qw = cq.QWeight(N, K, [None, None, self.plane[off // 2:(off + n) // 2], None], self.scale[g0:g1],
+                            self.zero[g0:g1])
+            m = dict(N=N, K=K, n=n, qw=qw, x_host=x_host, x=x_host.to(device), X_host=X_host, X=X_host.to(device),
+                     y=torch.empty(1, N, device=device), Y=torch.empty(GEMM_M, N, device=device))
             need = cq.cq_gemm_workspace(N, K, GEMM_M)
             m["ws"] = torch.empty(max(need, 16), dtype=torch.uint8, device=device) if need else None
             self.mats.append(m)
+            off += n
+        self.r_host = torch.from_numpy(np.concatenate(r_parts)).view(torch.bfloat16).pin_memory()
+        self.r.copy_(self.r_host)
+        self.qw_all = cq.QWeight(1, n_all, [None, None, self.plane, None], self.scale, self.zero, residual=self.r)
+        z = lambda dt: torch.zeros(1, dtype=dt, device=device)
+        self.status, self.nclamp = z(torch.int32), z(torch.int64)
+        self.mism, self.first, self.mism0, self.first0 = z(torch.int64), z(torch.int64), z(torch.int64), z(torch.int64)
         torch.cuda.synchronize()
 
     def step(self, stream, marks=None):
-        """Enqueue one step: each row of the path over the three matrices, then the next row
-        (every matrix keeps its own order quantize -> pack -> project -> verify pair ->
-        GEMV -> GEMM). marks[kernel] = (start, end) external events around a row's three
-        launches: recorded inside a graph capture they become event nodes that time the row on
-        replay (one pair per row keeps their own cost out of the launches they time)."""
+        """Enqueue one step: quantize, pack, project and both verify checks each as one call over
+        the three matrices' flat artifact, then the GEMV and the GEMM per matrix. marks[kernel] =
+        (start, end) external events around a row's calls: recorded inside a graph capture they
+        become event nodes that time the row on replay (one pair per row keeps their own cost out
+        of the launches they time)."""
         cq = self.cq
 
         def row(name, fn):
             if marks is not None:
                 marks[name][0].record(stream)
-            for m in self.mats:
-                fn(m, m["qw"])
+            fn()
             if marks is not None:
                 marks[name][1].record(stream)
 
-        row("quantize", lambda m, qw: cq.cq_quantize(m["w"], None, m["codes"], qw.scale, qw.zero, m["status"], stream))
-        row("pack", lambda m, qw: cq.cq_pack_varbits(m["codes"], m["n"] // GROUP, None, None, qw.planes, stream))
-        row("project", lambda m, qw: cq.cq_project_residual(m["r"], qw.scale, m["nclamp"], stream))
-        row("verify_pair", lambda m, qw: cq.cq_requant_verify_pair(qw.with_residual(m["r"]), 0, m["n"], m["mism"],
-                                                                   m["first"], m["mism0"], m["first0"], None,
-                                                                   stream))
-        row("gemv", lambda m, qw: cq.cq_dequant_gemv(qw, m["x"], m["y"], stream))
-        row("gemm", lambda m, qw: cq.cq_dequant_gemm(qw, m["X"], m["Y"], m["ws"], stream))
+        row("quantize", lambda: cq.cq_quantize(self.w.view(1, self.n_all), None, self.codes, self.scale, self.zero,
+                                               self.status, stream))
+        row("pack", lambda: cq.cq_pack_varbits(self.codes, self.n_all // GROUP, None, None,
+                                               [None, None, self.plane, None], stream))
+        row("project", lambda: cq.cq_project_residual(self.r, self.scale, self.nclamp, stream))
+        row("verify_pair", lambda: cq.cq_requant_verify_pair(self.qw_all, 0, self.n_all, self.mism, self.first,
+                                                             self.mism0, self.first0, None, stream))
+        row("gemv", lambda: [cq.cq_dequant_gemv(m["qw"], m["x"], m["y"], stream) for m in self.mats])
+        row("gemm", lambda: [cq.cq_dequant_gemm(m["qw"], m["X"], m["Y"], m["ws"], stream) for m in self.mats])
 
     def n_weights(self):
         return sum(m["n"] for m in self.mats)
@@ -208,6 +235,12 @@ class Workload:
             for k, v in kernel_bytes(m["n"]).items():
                 tot[k] += v
         return tot
+
+
+def launches_of(kernel, wl):
+    """Main-kernel launches of a row per step: the streaming rows run once over the flat artifact,
+    the GEMV and the GEMM once per matrix."""
+    return len(wl.mats) if kernel in ("gemv", "gemm") else 1
 
 
 def max_over_ranks(value, dist, device):
@@ -739,8 +772,7 @@ def run_gpu(args, rank, world, local_rank):
         for k, (a, b) in mk.items():
             per_kernel[k] += a.elapsed_time(b)
     t_step = max_over_ranks(t_step, dist, device)
-    checks = [int(m["mism"].item()) for m in wl.mats] + [int(m["mism0"].item()) for m in wl.mats] + \
-             [int(m["status"].item()) for m in wl.mats]
+    checks = [int(wl.mism.item()), int(wl.mism0.item()), int(wl.status.item())]
     assert all(c == 0 for c in checks), f"hot-path results not clean: {checks}"
 
     bytes_step = wl.step_bytes()
@@ -765,8 +797,8 @@ def run_gpu(args, rank, world, local_rank):
     roofline = {"kernel": dominant, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": MEASURED_TRAFFIC.get(dominant),
                 "peak_source": peaks["source"],
-                "algorithmic_bytes_per_launch": bytes_step[dominant] / len(wl.mats),
-                "launches_timed": args.steps * len(wl.mats)}
+                "algorithmic_bytes_per_launch": bytes_step[dominant] / launches_of(dominant, wl),
+                "launches_timed": args.steps * launches_of(dominant, wl)}
     iso = isolated_components(torch, cq, ops, device, peaks, stream) if args.components else None
 
     # end to end: pinned host inputs -> device, the step, results -> host
@@ -821,27 +853,30 @@ def run_gpu(args, rank, world, local_rank):
 
 
 def run_e2e(torch, wl, graph, stream, steps):
-    """Same step with host buffers: H2D of W, r, x, X before and D2H of y, Y, counts after."""
-    h2d = d2h = 0
+    """Same step with host buffers: H2D of W, r, x, X before and D2H of y, Y and the counters after."""
+    h2d = wl.w_host.numel() * 4 + wl.r_host.numel() * 2
+    d2h = 2 * 8 + 4
     for m in wl.mats:
-        h2d += sum(t.numel() * t.element_size() for t in (m["w_host"], m["r_host"], m["x_host"], m["X_host"]))
-        d2h += m["y"].numel() * 4 + m["Y"].numel() * 4 + 2 * 8 * 2 + 4
-    outs = [{k: torch.empty_like(m[k], device="cpu").pin_memory() for k in ("y", "Y", "mism", "mism0", "status")}
-            for m in wl.mats]
+        h2d += sum(t.numel() * t.element_size() for t in (m["x_host"], m["X_host"]))
+        d2h += m["y"].numel() * 4 + m["Y"].numel() * 4
+    outs = [{k: torch.empty_like(m[k], device="cpu").pin_memory() for k in ("y", "Y")} for m in wl.mats]
+    counters = {k: torch.empty_like(getattr(wl, k), device="cpu").pin_memory() for k in ("mism", "mism0", "status")}
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         a.record(stream)
         for _ in range(steps):
+            wl.w.copy_(wl.w_host, non_blocking=True)
+            wl.r.copy_(wl.r_host, non_blocking=True)
             for m in wl.mats:
-                m["w"].copy_(m["w_host"], non_blocking=True)
-                m["r"].copy_(m["r_host"], non_blocking=True)
                 m["x"].copy_(m["x_host"], non_blocking=True)
                 m["X"].copy_(m["X_host"], non_blocking=True)
             graph.replay()
             for m, o in zip(wl.mats, outs):
                 for k in o:
                     o[k].copy_(m[k], non_blocking=True)
+            for k, t in counters.items():
+                t.copy_(getattr(wl, k), non_blocking=True)
         b.record(stream)
     torch.cuda.synchronize()
     return {"ms_per_step": a.elapsed_time(b) / steps, "h2d": h2d, "d2h": d2h}

@@ -16,15 +16,17 @@
 // Backward, straight through the final rounding: dL/dtheta = RN(RN(dL/dr * c_dt) * phi'),
 // phi' = (1 + t^2)^(-3/2) = RN(RN(1 / d) / q), and 0 for a NaN or saturated theta.
 //
-// Layout: one lane per eight weights (32 bytes of theta), four such units in flight per lane;
-// the eight lanes of a 64-weight group share its scale. Streaming, HBM-bound.
+// Layout: one lane per eight weights (32 bytes of theta), two such units in flight per lane and
+// four CTAs of 256 threads per SM (more warps hide the long dependent sequences of the correctly
+// rounded square root and division better than more units per lane: the backward pass went from
+// 66 to 97 % of HBM); the eight lanes of a 64-weight group share its scale. Streaming.
 #include "cq_async.cuh"
 
 namespace cq {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 2;
 constexpr float kSat = 0x1p32f;
 
 __device__ __forceinline__ float cell_bound(uint16_t s16, bool bf16) {
@@ -58,7 +60,7 @@ __device__ __forceinline__ void store8(float *p, int64_t u, const float v[8]) {
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
 reparam_kernel(const float *__restrict__ theta, const uint16_t *__restrict__ scale, int64_t n_units,
                void *__restrict__ r) {
   pdl_wait();
@@ -96,7 +98,7 @@ reparam_kernel(const float *__restrict__ theta, const uint16_t *__restrict__ sca
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
 reparam_grad_kernel(const float *__restrict__ theta, const uint16_t *__restrict__ scale,
                     const float *__restrict__ grad_r, int64_t n_units, float *__restrict__ grad_theta) {
   pdl_wait();
