@@ -411,27 +411,31 @@ __device__ __forceinline__ GroupCodes<B> load_group(const uint8_t *src) {
 // 2^(-p b) once per group (exact). Width 8: byte p of a word is placed into 2^23 + q by PRMT.
 template <int B>
 __device__ __forceinline__ float group_dot(const GroupCodes<B> &gc, uint32_t z, const uint8_t *xg) {
+  // pairs of window positions go through the two-wide fp32 add and FMA (each half rounds as the
+  // scalar operation would)
   if (B == 8) {
     const float zc = 8388608.0f + static_cast<float>(z);
-    float d = 0.0f;
+    const float2 nz = make_float2(-zc, -zc);
+    float2 d2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       const float4 f = *reinterpret_cast<const float4 *>(xg + 16 * c);
-      const float xa[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t bitsq = __byte_perm(gc.w[c], 0x4B000000u, 0x7440u | e);
-        d = fmaf(__fsub_rn(__uint_as_float(bitsq), zc), xa[e], d);
-      }
+      const float2 q01 = make_float2(__uint_as_float(__byte_perm(gc.w[c], 0x4B000000u, 0x7440u)),
+                                     __uint_as_float(__byte_perm(gc.w[c], 0x4B000000u, 0x7441u)));
+      const float2 q23 = make_float2(__uint_as_float(__byte_perm(gc.w[c], 0x4B000000u, 0x7442u)),
+                                     __uint_as_float(__byte_perm(gc.w[c], 0x4B000000u, 0x7443u)));
+      d2[0] = __ffma2_rn(__fadd2_rn(q01, nz), make_float2(f.x, f.y), d2[0]);
+      d2[1] = __ffma2_rn(__fadd2_rn(q23, nz), make_float2(f.z, f.w), d2[1]);
     }
-    return d;
+    return (d2[0].x + d2[0].y) + (d2[1].x + d2[1].y);
   } else {
     constexpr int kWin = B == 4 ? 4 : 8;               // codes per window (8 or 16 bits)
-    float zc[kWin], dp[kWin];
+    float2 nz[kWin / 2], dp[kWin / 2];
 #pragma unroll
-    for (int p = 0; p < kWin; ++p) {
-      zc[p] = fmaf(static_cast<float>(z), static_cast<float>(1u << (p * B)), 8388608.0f);   // exact
-      dp[p] = 0.0f;
+    for (int h = 0; h < kWin / 2; ++h) {
+      nz[h] = make_float2(-fmaf(static_cast<float>(z), static_cast<float>(1u << (2 * h * B)), 8388608.0f),
+                          -fmaf(static_cast<float>(z), static_cast<float>(1u << ((2 * h + 1) * B)), 8388608.0f));
+      dp[h] = make_float2(0.0f, 0.0f);
     }
 #pragma unroll
     for (int t0 = 0; t0 < 64; t0 += kWin) {
@@ -444,14 +448,18 @@ __device__ __forceinline__ float group_dot(const GroupCodes<B> &gc, uint32_t z, 
         xa[4 * h] = f.x; xa[4 * h + 1] = f.y; xa[4 * h + 2] = f.z; xa[4 * h + 3] = f.w;
       }
 #pragma unroll
-      for (int p = 0; p < kWin; ++p) {
-        const uint32_t bitsq = and_or(word, ((1u << B) - 1u) << (p * B), 0x4B000000u);
-        dp[p] = fmaf(__fsub_rn(__uint_as_float(bitsq), zc[p]), xa[p], dp[p]);
+      for (int h = 0; h < kWin / 2; ++h) {
+        const float2 q = make_float2(__uint_as_float(and_or(word, ((1u << B) - 1u) << (2 * h * B), 0x4B000000u)),
+                                     __uint_as_float(and_or(word, ((1u << B) - 1u) << ((2 * h + 1) * B), 0x4B000000u)));
+        dp[h] = __ffma2_rn(__fadd2_rn(q, nz[h]), make_float2(xa[2 * h], xa[2 * h + 1]), dp[h]);
       }
     }
     float d = 0.0f;
 #pragma unroll
-    for (int p = 0; p < kWin; ++p) d = fmaf(dp[p], __uint_as_float(static_cast<uint32_t>(127 - p * B) << 23), d);
+    for (int h = 0; h < kWin / 2; ++h) {
+      d = fmaf(dp[h].x, __uint_as_float(static_cast<uint32_t>(127 - 2 * h * B) << 23), d);
+      d = fmaf(dp[h].y, __uint_as_float(static_cast<uint32_t>(127 - (2 * h + 1) * B) << 23), d);
+    }
     return d;
   }
 }

@@ -339,18 +339,33 @@ def test_gemv_varbits(m):
     check_matmul(host(ops.gemv(qw, x_d)), y_ref, f"vbq m={m}")
 
 
-# the per-group-width kernel: ragged 16-row tiles, group runs that do not split evenly over the
-# CTA's warps (fewer groups than warps, too), fp32 activations (two bf16 parts), and width maps
-# of one width only (8-bit groups take their own operand path)
+# the per-group-width kernels: ragged 16-row tiles, group runs that do not split evenly over the
+# CTA's warps (fewer groups than warps, too), fp32 activations (two bf16 parts), width maps of one
+# width only (8-bit groups take their own operand path), and at batch 1 long rows whose width
+# runs take several passes of 64 (300, 257, 129, 128 groups)
 @pytest.mark.parametrize("rows,cols,m,x_dtype,only", [(47, 64 * 9, 3, "f32", None), (300, 64 * 21, 8, "bf16", None),
                                                       (16, 64, 1, "bf16", None), (1000, 4096, 1, "f32", None),
                                                       (129, 64 * 37, 5, "bf16", 8), (64, 64 * 40, 8, "f32", 8),
-                                                      (200, 64 * 16, 2, "bf16", 1), (33, 64 * 5, 7, "bf16", 2)])
+                                                      (200, 64 * 16, 2, "bf16", 1), (33, 64 * 5, 7, "bf16", 2),
+                                                      (70, 64 * 300, 1, "bf16", None), (50, 64 * 257, 1, "f32", 8),
+                                                      (45, 64 * 129, 1, "bf16", 1), (9, 64 * 128, 1, "bf16", 2)])
 def test_gemv_varbits_shapes(rows, cols, m, x_dtype, only):
     G = rows * cols // 64
     bits = np.full(G, only, np.uint8) if only else synth.vbq_bits(G, seed=rows + cols)
     qw, x_d, y_ref, _ = _matmul_case(rows, cols, m, x_dtype, bits=bits, seed=rows + m)
     check_matmul(host(ops.gemv(qw, x_d)), y_ref, f"vbq {rows}x{cols} m={m} {x_dtype} only={only}")
+
+
+@pytest.mark.parametrize("rows,cols,m", [(70, 64 * 300, 1), (33, 64 * 40, 1), (33, 64 * 40, 3)])
+def test_gemv_stages_fixed4_and_varbits(rows, cols, m):
+    """A stack of a fixed-4 matrix and a per-group-width matrix of the same shape, multiplied with
+    the same activations: the sum of the two products, the fixed-4 stage at batch 1 included."""
+    bits = synth.vbq_bits(rows * cols // 64, seed=cols)
+    q4, x_d, y4, _ = _matmul_case(rows, cols, m, "bf16", seed=41)
+    qv, x_dv, yv, _ = _matmul_case(rows, cols, m, "bf16", bits=bits, seed=41)
+    assert torch.equal(x_d, x_dv)
+    check_matmul(host(ops.gemv_stages([q4, qv], x_d)), y4 + yv, f"fixed-4 + vbq stack {rows}x{cols} m={m}")
+    check_matmul(host(ops.gemv_stages([qv, q4, qv], x_d)), y4 + 2 * yv, f"vbq + fixed-4 + vbq {rows}x{cols} m={m}")
 
 
 def test_gemv_varbits_rows_too_long_to_stage():

@@ -78,7 +78,7 @@ def _oracle_stack(w, n_stages):
 
 
 @pytest.mark.parametrize("rows,cols,n_stages", [(256, 512, 1), (333, 64 * 21, 2), (1000, 4096, 3), (512, 2048, 4),
-                                                 (96, 1024, 6)])
+                                                 (96, 1024, 6), (40, 64 * 200, 3)])
 @pytest.mark.parametrize("m,x_dtype", [(1, "bf16"), (3, "f32"), (8, "bf16")])
 def test_rrq_gemv_stages(rows, cols, n_stages, m, x_dtype):
     w = synth.normal_weights(rows, cols, seed=7 * rows + n_stages)
