@@ -39,12 +39,14 @@ SYNTH_UNITS = {"synth.cu": EXACT}
 # that is never requested, so a bounded wait runs out and the abort path runs); the tests load
 # them by path, nothing else does
 TEST_VARIANTS = {"drop_first_copy": {"k_quantize.cu": ["-DCQ_TEST_DROP_FIRST_COPY"],
-                                      "k_gemm.cu": ["-DCQ_TEST_DROP_FIRST_COPY"]}}
+                                      "k_gemm.cu": ["-DCQ_TEST_DROP_FIRST_COPY"]},
+                 # every unit with its in-kernel index checks compiled in (cq_debug.cuh)
+                 "debug": {u: ["-DCQ_DEBUG"] for u in LIBCQ_UNITS}}
 
 LIBCQ = os.path.join(HERE, "libcq.so")
 LIBSYNTH = os.path.join(HERE, "libcq_synth.so")
-HEADERS = [os.path.join(CSRC, "cq_internal.cuh"), os.path.join(HERE, "..", "include", "cq.h"),
-           os.path.join(HERE, "..", "include", "cq_synth.h")]
+HEADERS = [*(os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith(".cuh")),
+           os.path.join(HERE, "..", "include", "cq.h"), os.path.join(HERE, "..", "include", "cq_synth.h")]
 
 
 def _newer(target, deps):

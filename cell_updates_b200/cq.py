@@ -25,7 +25,7 @@ EXPORTS = ["cq_quantize", "cq_varbits_index", "cq_pack_varbits", "cq_unpack_varb
            "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemv_multi", "cq_dequant_gemm",
            "cq_dequant_gemm_static", "cq_gemm_workspace", "cq_last_error", "cq_status_string", "cq_rrq_stage",
            "cq_dequant_gemv_stages", "cq_requant_verify_pair", "cq_reparam_residual", "cq_reparam_residual_grad", "cq_requant_refine",
-           "cq_requant_workspace"]
+           "cq_requant_workspace", "cq_debug_word", "cq_debug_selftest"]
 SYNTH_EXPORTS = ["cqs_normal_f32", "cqs_code_words", "cqs_scales", "cqs_zeros", "cqs_residual_bf16"]
 
 
@@ -71,6 +71,8 @@ def lib():
         L.cq_requant_refine.argtypes = [p, i64, i64, p, p, p, i32, p, i32, p, p, p, p, C.c_size_t, p]
         L.cq_requant_workspace.argtypes = [i64, i64]
         L.cq_requant_workspace.restype = C.c_size_t
+        L.cq_debug_word.argtypes = [p]
+        L.cq_debug_selftest.argtypes = [p]
         L.cq_gemm_workspace.argtypes = [i64, i64, i32]
         L.cq_gemm_workspace.restype = C.c_size_t
         L.cq_last_error.restype = C.c_char_p
@@ -80,7 +82,7 @@ def lib():
                      "cq_project_residual", "cq_requant_verify", "cq_dequant_gemv", "cq_dequant_gemv_multi",
                      "cq_dequant_gemm", "cq_dequant_gemm_static", "cq_rrq_stage", "cq_dequant_gemv_stages",
                      "cq_requant_verify_pair", "cq_reparam_residual", "cq_reparam_residual_grad",
-                     "cq_requant_refine"):
+                     "cq_requant_refine", "cq_debug_word", "cq_debug_selftest"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -257,6 +259,18 @@ def cq_requant_refine(w, H, scale, zero, bits, codes, sweeps, err_before=None, e
     _check(lib().cq_requant_refine(_ptr(w), rows, cols, _ptr(H), _ptr(scale), _ptr(zero), int(bits), _ptr(codes),
                                    int(sweeps), _ptr(err_before), _ptr(err_after), _ptr(moves), _ptr(workspace),
                                    nbytes, _stream(stream)), "cq_requant_refine")
+
+
+def cq_debug_word():
+    """The first failed in-kernel index check since the last call (a debug build's site number),
+    or 0; waits for the device. A release build raises CQError(CQ_ERR_UNSUPPORTED)."""
+    w = C.c_uint32(0)
+    _check(lib().cq_debug_word(C.byref(w)), "cq_debug_word")
+    return int(w.value)
+
+
+def cq_debug_selftest(stream=None):
+    _check(lib().cq_debug_selftest(_stream(stream)), "cq_debug_selftest")
 
 
 def cq_gemm_workspace(rows, cols, m):

@@ -92,11 +92,64 @@ cq_status check_matmul_args(const cq_qweight *qw, const void *x, cq_dtype x_dtyp
   return CQ_OK;
 }
 
+#ifdef CQ_DEBUG
+// every unit's debug word, registered by its static initializer (cq_debug.cuh); the table is
+// zero-initialized before any initializer runs
+namespace {
+constexpr int kMaxDebugUnits = 32;
+uint32_t (*g_debug_takers[kMaxDebugUnits])();
+int g_debug_units = 0;
+std::mutex g_debug_mu;
+
+__global__ void debug_selftest_kernel() {
+  __shared__ uint32_t slot[1];
+  if (threadIdx.x == 0) slot[0] = 0u;
+  __syncthreads();
+  const uint32_t i = threadIdx.x + 1;                 // one past the slot
+  if (CQ_CHECK(i < 1, 0x0F01u)) slot[i] = 1u;
+  __syncthreads();
+  if (slot[0] != 0u) __threadfence();                 // keeps the slot live
+}
+}  // namespace
+
+void register_debug_word(uint32_t (*take)()) {
+  if (g_debug_units < kMaxDebugUnits) g_debug_takers[g_debug_units++] = take;
+}
+#endif
+
 }  // namespace cq
 
 using namespace cq;
 
 extern "C" {
+
+cq_status cq_debug_word(uint32_t *word) {
+  if (!word) return fail(CQ_ERR_ARG, "cq_debug_word: NULL word");
+  *word = 0;
+#ifdef CQ_DEBUG
+  std::lock_guard<std::mutex> lock(g_debug_mu);
+  cq_status st = cuda_check(cudaDeviceSynchronize(), "cq_debug_word: synchronize");
+  if (st != CQ_OK) return st;
+  for (int u = 0; u < g_debug_units; ++u) {
+    const uint32_t v = g_debug_takers[u]();
+    if (v == 0xFFFFFFFFu) return fail(CQ_ERR_CUDA, "cq_debug_word: could not read a unit's word");
+    if (!*word) *word = v;
+  }
+  return CQ_OK;
+#else
+  return fail(CQ_ERR_UNSUPPORTED, "cq_debug_word: a release build (no -DCQ_DEBUG) has no index checks");
+#endif
+}
+
+cq_status cq_debug_selftest(cq_stream_t stream) {
+#ifdef CQ_DEBUG
+  debug_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+  return launch_check("cq_debug_selftest");
+#else
+  (void)stream;
+  return fail(CQ_ERR_UNSUPPORTED, "cq_debug_selftest: a release build (no -DCQ_DEBUG) has no index checks");
+#endif
+}
 
 const char *cq_last_error(void) { return g_last_error; }
 

@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include "../../include/cq.h"
+#include "cq_debug.cuh"
 
 namespace cq {
 

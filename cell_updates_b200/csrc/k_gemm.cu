@@ -400,6 +400,7 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
         }
 #endif
         uint8_t *dst = sX + st * kG * C::kXBytes;
+        (void)CQ_CHECK(static_cast<int64_t>(kG) * (w.p + 1) * 64 <= K, 0x0604u);
         mbar_arrive_expect_tx(x_full + st, kG * C::kXBytes);
         for (int jj = 0; jj < kG; ++jj) tma_load_2d(dst + jj * C::kXBytes, &tm_x, (kG * w.p + jj) * 64, 0, x_full + st);
         x_issued = li + 1;
@@ -429,6 +430,7 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
         if (!mbar_wait(x_full + xst, (li / XS) & 1, abort_flag, status)) break;
         if (!mbar_wait(a_full + st, par, abort_flag, status)) break;
         tc_fence_after();
+        (void)CQ_CHECK(C::kACol0 + (st + 1) * kG * kACols <= C::kTmemCols && (b + 1) * NT <= C::kAccCols, 0x0603u);
         const uint32_t ta = tmem + C::kACol0 + st * kG * kACols;
         const uint32_t td = tmem + b * NT;
         const uint32_t blo = dlo0 + ((xst * kG * C::kXBytes) >> 4);
@@ -475,13 +477,17 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
       int64_t row = static_cast<int64_t>(wl.tile) * kTileM + r;
       row = row < N ? row : N - 1;                // rows past the end: any valid row, result unused
       const int g = kG * wl.p + 2 * part;
-      const uint4 *src = reinterpret_cast<const uint4 *>(plane + row * row_bytes + g * 32);
-      cb.c[0] = __ldcs(src);
-      cb.c[1] = __ldcs(src + 1);
-      cb.c[2] = __ldcs(src + 2);
-      cb.c[3] = __ldcs(src + 3);
-      cb.s2 = __ldg(reinterpret_cast<const uint32_t *>(scale + row * KG + g));
-      cb.z2 = __ldg(reinterpret_cast<const uint16_t *>(zero + row * KG + g));
+      if (CQ_CHECK(static_cast<int64_t>(wl.tile) * kTileM < N && g + 2 <= KG, 0x0601u)) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(plane + row * row_bytes + g * 32);
+        cb.c[0] = __ldcs(src);
+        cb.c[1] = __ldcs(src + 1);
+        cb.c[2] = __ldcs(src + 2);
+        cb.c[3] = __ldcs(src + 3);
+        cb.s2 = __ldg(reinterpret_cast<const uint32_t *>(scale + row * KG + g));
+        cb.z2 = __ldg(reinterpret_cast<const uint16_t *>(zero + row * KG + g));
+      } else {
+        cb = CodeBuf{};
+      }
       walk_next(wl, P);
     };
     // dequantize a loaded step into its A slot; false when a wait gave up
@@ -641,7 +647,8 @@ gemm4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t *__restr
       if (seg_end) {
         const int b = seg % kAccBufs, fs = seg % kFlagSlots;
         const int gb = kG * w.p + kG;
-        const int64_t row = static_cast<int64_t>(w.tile) * kTileM + r;
+        const bool seg_ok = CQ_CHECK(gb <= KG && ga >= 0 && static_cast<int64_t>(w.tile) * kTileM < N, 0x0602u);
+        const int64_t row = seg_ok ? static_cast<int64_t>(w.tile) * kTileM + r : N;
         if (!warp_wait(seg_done + fs, (seg / kFlagSlots) & 1, abort_flag, status)) break;
         const uint32_t mask = seg_mask[fs * 4 + quad];
         __syncwarp();

@@ -321,7 +321,8 @@ gemv4_kernel(const __grid_constant__ GemvSegs segs, const __nv_bfloat16 *__restr
         }
         const float in_scale = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
         const float in_scale16 = in_scale * 0.0625f;
-        if (b < nblk) {
+        if (b < nblk && CQ_CHECK(nn[u] < m && kk[u] < bpr &&
+                                     (xst - smem) + nn[u] * xpitch + kk[u] * 32 + 32 <= dynamic_smem_bytes(), 0x0501u)) {
           uint32_t f[8];
           permute16(v[u][0], v[u][1], f);
 #pragma unroll
@@ -423,6 +424,7 @@ gemv4_kernel(const __grid_constant__ GemvSegs segs, const __nv_bfloat16 *__restr
     const int64_t lrow0 = (tile - seg_pick(segs.tile0, sg)) * kTileRows, N = seg_pick(segs.rows, sg);
     float *y = seg_pick(segs.y, sg);
     const bool bad = *abort_flag != 0u;
+    const bool tile_ok = CQ_CHECK(sg >= 0 && sg < kMaxSegs && lrow0 >= 0 && lrow0 < N, 0x0502u);
     for (int idx = lane; idx < 16 * m; idx += 32) {
       float v = 0.0f;
 #pragma unroll
@@ -432,7 +434,7 @@ gemv4_kernel(const __grid_constant__ GemvSegs segs, const __nv_bfloat16 *__restr
       }
       const int row = idx & 15, col = idx >> 4;
       const int64_t r = lrow0 + row;
-      if (r < N) y[static_cast<int64_t>(col) * N + r] = bad ? __int_as_float(0x7fc00000) : v;
+      if (r < N && tile_ok) y[static_cast<int64_t>(col) * N + r] = bad ? __int_as_float(0x7fc00000) : v;
     }
     __threadfence_block();
     __syncwarp();
@@ -465,6 +467,7 @@ gemv4_kernel(const __grid_constant__ GemvSegs segs, const __nv_bfloat16 *__restr
     const uint8_t *box = ring + slot * kChunkBytes;
     const int g0 = cons.c * kCG;
     const int ng = KG - g0 < kCG ? KG - g0 : kCG;
+    (void)CQ_CHECK(ng > 0, 0x0503u);
     const uint8_t *xb = xs_base + g0 * 128;
     const uint32_t *sb = sum_base + g0 * 3;
     const float *fb = fsc_lane + g0 * 8;
@@ -761,6 +764,7 @@ gemv4r_kernel(const __grid_constant__ RSegs sg, const __nv_bfloat16 *__restrict_
     const uint16_t *scale = seg_pick(sg.scale, s), *res = seg_pick(sg.res, s);
     const uint8_t *zero = seg_pick(sg.zero, s);
     const int64_t N = seg_pick(sg.rows, s), lrow0 = (tile - seg_pick(sg.tile0, s)) * kTileRows;
+    (void)CQ_CHECK(s >= 0 && s < kMaxSegs && lrow0 >= 0 && lrow0 < N, 0x0504u);
     int64_t row0 = lrow0 + gid, row1 = row0 + 8;
     row0 = row0 < N ? row0 : N - 1;               // rows past the end: any valid row, never stored
     row1 = row1 < N ? row1 : N - 1;
@@ -883,6 +887,7 @@ gemv_generic_kernel(const uint8_t *__restrict__ bits, const uint32_t *__restrict
         src = p2 + g * 32;
       }
       if (!width_ok(b)) continue;
+      if (bits && !CQ_CHECK(offset[g] % (8u * b) == 0u && offset[g] / (8u * b) <= g, 0x0505u)) continue;
       const float s = f16_bits_to_f32(scale[g]);
       const float z = static_cast<float>(zero[g]);
       for (int jb = 0; jb < 8; ++jb) {

@@ -108,7 +108,11 @@ pack_kernel(const uint8_t *__restrict__ codes, int64_t n_units, const uint8_t *_
     if (bits) {
       b = __ldg(bits + g);
       if (!width_ok(b)) continue;   // nothing to store; quantize reports the width
-      base = planes.of(b) + __ldg(offset + g);
+      const uint32_t o = __ldg(offset + g);
+      // debug build: an offset off its 8 b grid, or a rank above the group's own index (a rank
+      // counts earlier groups of the same width), is recorded and its group not stored
+      if (!CQ_CHECK(o % (8u * b) == 0u && static_cast<int64_t>(o / (8u * b)) <= g, 0x0201u)) continue;
+      base = planes.of(b) + o;
     } else {
       base = planes.p[2] + g * 32;
     }
@@ -128,8 +132,9 @@ unpack_kernel(uint8_t *__restrict__ codes, int64_t n_units, const uint8_t *__res
     uint64_t v = 0;
     if (bits) {
       b = __ldg(bits + g);
-      if (width_ok(b)) {
-        base = planes.of(b) + __ldg(offset + g);
+      const uint32_t o = width_ok(b) ? __ldg(offset + g) : 0u;
+      if (width_ok(b) && CQ_CHECK(o % (8u * b) == 0u && static_cast<int64_t>(o / (8u * b)) <= g, 0x0202u)) {
+        base = planes.of(b) + o;
         v = unpack8(load_bytes(base + sub * b, b), b);
       }
     } else {

@@ -210,7 +210,7 @@ quantize_kernel(const __grid_constant__ CUtensorMap tm_w, float *w, int64_t G, c
       // write the tile back in place (rows past G are not written), then refill the buffer
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
+      if (lane == 0 && CQ_CHECK(tile * kTileGroups < G, 0x0101u)) {
         const uint8_t *src = ring + cur * kTileBytes;
         tma_store_2d(&tm_w, src, 0, static_cast<int>(tile * kTileGroups));
         tma_store_2d(&tm_w, src + kBoxBytes, 32, static_cast<int>(tile * kTileGroups));

@@ -113,6 +113,7 @@ rq_sweep_kernel(const double *__restrict__ H, const uint16_t *__restrict__ scale
   const int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
   if (n >= N) return;
   double *gr = sg + static_cast<int64_t>(warp) * K;
+  if (!CQ_CHECK(static_cast<int64_t>(warp + 1) * K * 8 <= dynamic_smem_bytes(), 0x0901u)) return;
   for (int64_t j = lane; j < K; j += 32) gr[j] = g[n * K + j];
   __syncwarp();
   const int64_t KG = K >> 6;
@@ -136,6 +137,7 @@ rq_sweep_kernel(const double *__restrict__ H, const uint16_t *__restrict__ scale
         const double up = __dsub_rn(t2, t4), down = __dadd_rn(t2, t4);
         int step = (q < L && up < 0.0) ? 1 : 0;
         if (q > 0 && down < 0.0 && (step == 0 || down < up)) step = -1;
+        (void)CQ_CHECK(q + step >= 0 && q + step <= L, 0x0902u);
         if (step) {                      // warp-uniform: every lane took the same decision
           const double delta = step > 0 ? S : -S;
           if (lane == i) qv = q + step;

@@ -94,7 +94,10 @@ __device__ __forceinline__ RowCodes load_codes(const StageSet &ss, int j, int64_
   RowCodes c;
   c.b = m.b;
   c.w = make_uint4(0u, 0u, 0u, 0u);
-  if (m.b) {
+  // debug build: an offset off its 8 b grid, or a rank above the group's own index (a rank
+  // counts earlier groups of the same width), is recorded (and the latter's load skipped)
+  (void)CQ_CHECK(!ss.bits[j] || !m.b || (m.off & (8u * m.b - 1u)) == 0u, 0x0701u);
+  if (m.b && CQ_CHECK(!ss.bits[j] || static_cast<int64_t>(m.off / (8u * m.b)) <= gabs, 0x0702u)) {
     const uint8_t *src;
     if (ss.bits[j]) {
       // offsets are multiples of 8 b by construction; the mask keeps a damaged map aligned
@@ -512,6 +515,7 @@ gemv_vbq1_kernel(const __grid_constant__ StageSet ss, int count, const void *__r
   }
   __syncthreads();
   uint16_t *list = reinterpret_cast<uint16_t *>(xs + static_cast<int64_t>(KG) * kVbqPitch) + warp * KG;
+  (void)CQ_CHECK(static_cast<int64_t>(KG) * kVbqPitch + (warp + 1) * KG * 2 <= dynamic_smem_bytes(), 0x0706u);
   const uint32_t lt = (1u << lane) - 1u;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * kVbqWarps;
   for (int64_t n = blockIdx.x * static_cast<int64_t>(kVbqWarps) + warp; n < N; n += warps) {
@@ -542,7 +546,8 @@ gemv_vbq1_kernel(const __grid_constant__ StageSet ss, int count, const void *__r
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const uint32_t mk = __ballot_sync(0xffffffffu, b == (1 << c));
-          if (b == (1 << c)) list[fill[c] + __popc(mk & lt)] = static_cast<uint16_t>(w0 + lane);
+          if (b == (1 << c) && CQ_CHECK(fill[c] + __popc(mk & lt) < KG, 0x0703u))
+            list[fill[c] + __popc(mk & lt)] = static_cast<uint16_t>(w0 + lane);
           fill[c] += __popc(mk);
         }
       }
@@ -551,8 +556,14 @@ gemv_vbq1_kernel(const __grid_constant__ StageSet ss, int count, const void *__r
       // a multiple of 8 b by construction, the mask keeps a damaged map aligned)
       uint32_t first[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        first[c] = cnt[c] ? (__ldg(offset + g0 + list[base[c]]) & ~((8u << c) - 1u)) : 0u;
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t o = cnt[c] ? __ldg(offset + g0 + list[base[c]]) : 0u;
+        first[c] = o & ~((8u << c) - 1u);
+        // debug build: the run must start on its 8 b grid, at a rank no higher than its first
+        // group's index (else the pass is skipped)
+        (void)CQ_CHECK((o & ((8u << c) - 1u)) == 0u, 0x0704u);
+        if (cnt[c] && !CQ_CHECK(static_cast<int64_t>(o >> (3 + c)) <= g0 + list[base[c]], 0x0705u)) cnt[c] = 0;
+      }
       acc += width_pass<1>(list + base[0], cnt[0], lane, g0, ss.plane[j][0] + first[0], scale, zero, xs);
       acc += width_pass<2>(list + base[1], cnt[1], lane, g0, ss.plane[j][1] + first[1], scale, zero, xs);
       acc += width_pass<4>(list + base[2], cnt[2], lane, g0, ss.plane[j][2] + first[2], scale, zero, xs);

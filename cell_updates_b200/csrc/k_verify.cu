@@ -112,7 +112,11 @@ __global__ void __launch_bounds__(kThreads) verify_kernel(VerifyArgs a) {
         if (b) {
           // select the plane without indexing the parameter array (keeps it out of local memory)
           const uint8_t *pl = b == 1 ? a.plane[0] : b == 2 ? a.plane[1] : b == 4 ? a.plane[2] : a.plane[3];
-          const uint8_t *src = pl + __ldg(a.offset + g) + ((i0 >> 3) & 7) * b;
+          const uint32_t o = __ldg(a.offset + g);
+          // debug build: an offset off its grid or with a rank above the group's index is
+          // recorded and read as rank 0
+          const uint32_t oc = CQ_CHECK(o % (8u * b) == 0u && static_cast<int64_t>(o / (8u * b)) <= g, 0x0401u) ? o : 0u;
+          const uint8_t *src = pl + oc + ((i0 >> 3) & 7) * b;
           switch (b) {
             case 1: word = __ldg(src); break;
             case 2: word = __ldg(reinterpret_cast<const uint16_t *>(src)); break;

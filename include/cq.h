@@ -319,6 +319,25 @@ cq_status cq_dequant_gemm_static(const cq_qweight *qw, const void *x, cq_dtype x
 /* Bytes of workspace cq_dequant_gemm needs for this shape (host function, no GPU work). */
 size_t cq_gemm_workspace(int64_t rows, int64_t cols, int m);
 
+/*
+ * cq_debug_word -- the debug build's record of a failed in-kernel index check. A library built
+ * with -DCQ_DEBUG checks the derived indices of its kernels (rows and columns of outputs,
+ * shared-memory and tensor-memory slots, group indices, packed-offset alignment); a failing
+ * check skips the access it guards and records its site, (unit << 8) | n, in a device word (the
+ * first failure wins) instead of trapping. This call waits for the device to finish
+ * (cudaDeviceSynchronize), stores in *word (host) the first non-zero site over all units, or 0,
+ * and clears every unit's record. A release build (the default) has no checks: *word = 0 and
+ * CQ_ERR_UNSUPPORTED. Errors: CQ_ERR_ARG (word NULL), CQ_ERR_CUDA.
+ */
+cq_status cq_debug_word(uint32_t *word);
+
+/*
+ * cq_debug_selftest -- debug build only: enqueues one kernel whose index check fails on purpose
+ * (site 0x0F01, the access it guards skipped), so that a test can see cq_debug_word report it.
+ * A release build returns CQ_ERR_UNSUPPORTED and enqueues nothing.
+ */
+cq_status cq_debug_selftest(cq_stream_t stream);
+
 /* Text of the last non-OK status returned on the calling thread (thread-local, host). */
 const char *cq_last_error(void);
 

@@ -30,6 +30,27 @@ def test_libcq_exports_header_symbols():
         assert hasattr(lib, n), n
 
 
+def test_test_builds_export_the_same_symbols():
+    names = _declared("cq.h")
+    for variant in build.TEST_VARIANTS:
+        lib = C.CDLL(build.test_variant_path(variant))
+        for n in names:
+            assert hasattr(lib, n), (variant, n)
+
+
+def test_debug_word_needs_a_debug_build():
+    """Release: no checks compiled in, CQ_ERR_UNSUPPORTED with the word zeroed; both builds
+    reject a NULL word on the host (no GPU is touched on either path)."""
+    rel = cq.lib()
+    w = C.c_uint32(0xDEAD)
+    assert rel.cq_debug_word(C.byref(w)) == 8 and w.value == 0
+    assert rel.cq_debug_word(None) == 1
+    assert rel.cq_debug_selftest(None) == 8
+    dbg = C.CDLL(build.test_variant_path("debug"))
+    dbg.cq_debug_word.argtypes = [C.c_void_p]
+    assert dbg.cq_debug_word(None) == 1
+
+
 def test_libcq_synth_exports_header_symbols():
     names = _declared("cq_synth.h")
     assert names == sorted(cq.SYNTH_EXPORTS)
