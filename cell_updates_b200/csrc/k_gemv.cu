@@ -580,7 +580,9 @@ gemv4_kernel(const __grid_constant__ GemvSegs segs, const __nv_bfloat16 *__restr
         }
       }
     }
-    // every lane's reads of this slot have fed the MMAs above; refill it
+    // every lane's reads of this slot have fed the MMAs above; refill it (the proxy fence orders
+    // those generic reads before the TMA write into the slot)
+    fence_proxy_async_smem();
     __syncwarp();
     ++n_done;
     if (e + kStages * kWarps < total) {

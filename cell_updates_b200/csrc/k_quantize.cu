@@ -105,7 +105,9 @@ quantize_kernel(const __grid_constant__ CUtensorMap tm_w, float *w, int64_t G, c
       asm("max.NaN.f32 %0, %0, %1;\n" : "+f"(hi) : "f"(v[j]));
     }
     // every lane's words of this slot are in registers (min/max consumed them): refill it (a
-    // residual stage refills after writing the slot back)
+    // residual stage refills after writing the slot back); the proxy fence orders these generic
+    // reads before the TMA write into the slot
+    fence_proxy_async_smem();
     __syncwarp();
     ++n_done;
     const int cur = slot;
