@@ -41,7 +41,9 @@ def test_test_builds_export_the_same_symbols():
 def test_debug_word_needs_a_debug_build():
     """Release: no checks compiled in, CQ_ERR_UNSUPPORTED with the word zeroed; both builds
     reject a NULL word on the host (no GPU is touched on either path)."""
-    rel = cq.lib()
+    rel = C.CDLL(build.LIBCQ)
+    rel.cq_debug_word.argtypes = [C.c_void_p]
+    rel.cq_debug_selftest.argtypes = [C.c_void_p]
     w = C.c_uint32(0xDEAD)
     assert rel.cq_debug_word(C.byref(w)) == 8 and w.value == 0
     assert rel.cq_debug_word(None) == 1
