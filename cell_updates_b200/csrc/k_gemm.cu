@@ -317,7 +317,7 @@ gemm_prep_kernel(const uint16_t *__restrict__ x, int64_t K, uint16_t *__restrict
 // One step = kG groups (256 columns) of one 128-row tile. A step's A operand occupies one of
 // kSlots slots of tensor memory and its activations one of XS shared-memory stages; two MMA
 // commits per step (step_free, x_free) release them. The dequantizers load their rows' codes straight
-// into registers (kPre steps in flight per thread: 16-byte loads of 64 contiguous bytes per
+// into registers (three steps in flight per thread: 16-byte loads of 64 contiguous bytes per
 // row and step), so codes never pass through shared memory, whose bandwidth the activation
 // tiles and the MMAs' operand reads need.
 template <int NT, bool RES>
