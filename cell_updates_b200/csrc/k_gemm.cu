@@ -35,8 +35,7 @@
 //               there), after adding the segment's slow groups in fp32
 // Three steps are in flight in tensor memory (A slots: a_full when stored, step_free when their
 // MMAs completed), so the dequantizers store steps i + 1 and i + 2 while the MMAs of step i run;
-// the activation tiles have their own deeper ring (x_full / x_free, 5 stages at N = 64, 8 below),
-// because their TMA latency from L2, not the MMAs, otherwise sets the pace of the steps.
+// the activation tiles have their own deeper ring (x_full / x_free, 5 stages at N = 64, 8 below).
 // The preparation kernel also zeroes y and the status word. Every barrier wait is bounded: on
 // timeout the CTA raises a status flag, drains what it issued, frees its tensor memory and
 // returns.
