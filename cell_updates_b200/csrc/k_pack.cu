@@ -250,6 +250,8 @@ __device__ __forceinline__ uint32_t field16(uint64_t v, int slot) {
 
 __global__ void __launch_bounds__(kIndexThreads)
 index_count_kernel(const uint8_t *__restrict__ bits, int64_t G, uint32_t *__restrict__ offset) {
+  pdl_wait();                     // the widths and the offset slots' earlier readers
+  pdl_launch_dependents();        // after the wait: a dependent may read the widths before its own
   const int64_t t = blockIdx.x;   // a full tile that is not the last one
   int widths[kIndexPer];
   uint64_t total;
@@ -260,6 +262,14 @@ index_count_kernel(const uint8_t *__restrict__ bits, int64_t G, uint32_t *__rest
 __global__ void __launch_bounds__(kIndexThreads)
 index_scan_kernel(const uint8_t *__restrict__ bits, int64_t G, int64_t n_tiles,
                   uint32_t *__restrict__ offset, uint64_t *__restrict__ plane_bytes) {
+  // the last tile's counts need only the widths, which the count pass's wait has made safe to
+  // read (single launch: this kernel's own wait comes first)
+  int widths[kIndexPer];
+  uint64_t last;
+  if (n_tiles == 1) pdl_wait();
+  block_exclusive_scan(thread_counts(bits, G, n_tiles - 1, threadIdx.x, widths), &last);
+  pdl_wait();                     // the count pass's slots
+  pdl_launch_dependents();
   // prefix over the first n_tiles-1 tiles, 32-bit counts (G <= 2^26 keeps them exact)
   __shared__ uint32_t base[4];
   if (threadIdx.x < 4) base[threadIdx.x] = 0;
@@ -293,9 +303,6 @@ index_scan_kernel(const uint8_t *__restrict__ bits, int64_t G, int64_t n_tiles,
     }
     __syncthreads();
   }
-  int widths[kIndexPer];
-  uint64_t last;
-  block_exclusive_scan(thread_counts(bits, G, n_tiles - 1, threadIdx.x, widths), &last);
   if (threadIdx.x < 4) {
     const int b = 1 << threadIdx.x;
     plane_bytes[threadIdx.x] = static_cast<uint64_t>(base[threadIdx.x] + field16(last, threadIdx.x)) * 8u * b;
@@ -308,7 +315,10 @@ index_write_kernel(const uint8_t *__restrict__ bits, int64_t G, int64_t n_tiles,
   const int64_t t = blockIdx.x;
   int widths[kIndexPer];
   uint64_t total;
+  // the widths were safe to read once the scan pass started (its predecessors had completed)
   const uint64_t excl = block_exclusive_scan(thread_counts(bits, G, t, threadIdx.x, widths), &total);
+  pdl_wait();                     // the scan pass's bases and plane sizes
+  pdl_launch_dependents();
   __shared__ uint32_t base[4];
   if (threadIdx.x < 4) {
     if (t < n_tiles - 1) {
@@ -350,16 +360,19 @@ cq_status launch_varbits_index(const uint8_t *bits, int64_t G, uint32_t *offset,
                                uint64_t *plane_bytes, cudaStream_t s) {
   if (G == 0) return cuda_check(cudaMemsetAsync(plane_bytes, 0, 4 * sizeof(uint64_t), s), "cq_varbits_index");
   const int64_t n_tiles = (G + kTile - 1) / kTile;
+  // programmatic dependent launches: each pass is scheduled while the one before it finishes
   if (n_tiles > 1) {
-    index_count_kernel<<<static_cast<unsigned>(n_tiles - 1), kIndexThreads, 0, s>>>(bits, G, offset);
-    cq_status st = launch_check("cq_varbits_index: count");
+    cq_status st = cuda_check(launch_pdl(index_count_kernel, dim3(static_cast<unsigned>(n_tiles - 1)),
+                                         dim3(kIndexThreads), 0, s, bits, G, offset), "cq_varbits_index: count");
     if (st != CQ_OK) return st;
   }
-  index_scan_kernel<<<1, kIndexThreads, 0, s>>>(bits, G, n_tiles, offset, plane_bytes);
-  cq_status st = launch_check("cq_varbits_index: scan");
+  cq_status st = cuda_check(launch_pdl(index_scan_kernel, dim3(1), dim3(kIndexThreads), 0, s, bits, G, n_tiles,
+                                       offset, plane_bytes), "cq_varbits_index: scan");
   if (st != CQ_OK) return st;
-  index_write_kernel<<<static_cast<unsigned>(n_tiles), kIndexThreads, 0, s>>>(bits, G, n_tiles, offset, plane_bytes);
-  return launch_check("cq_varbits_index: write");
+  st = cuda_check(launch_pdl(index_write_kernel, dim3(static_cast<unsigned>(n_tiles)), dim3(kIndexThreads), 0, s,
+                             bits, G, n_tiles, offset, plane_bytes), "cq_varbits_index: write");
+  if (st != CQ_OK) return st;
+  return launch_check("cq_varbits_index");
 }
 
 cq_status launch_pack(const uint8_t *codes, int64_t G, const uint8_t *bits, const uint32_t *offset,

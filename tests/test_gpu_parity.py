@@ -125,6 +125,36 @@ def test_varbits_index_and_pack_bit_exact(G):
     assert np.array_equal(host(ops.unpack(qw)), codes)
 
 
+@pytest.mark.parametrize("G", [262143, 262144, 262145, 600001, 1 << 20, (1 << 20) + 1, 1300001])
+def test_varbits_index_both_forms_unaligned_and_invalid(G):
+    """The index in both of its forms: one cluster launch up to 2^20 groups (rounds of 262144
+    groups) and three passes beyond; with the width map and the offsets off their 16-byte
+    boundaries (the element-wise paths); and with widths outside {1, 2, 4, 8}, which take no
+    bytes and get offset 0 while the valid groups keep the offsets of the valid subsequence."""
+    bits = synth.vbq_bits(G, seed=G)
+    off, pb = co.varbits_index(bits)
+    off_d, pb_d = ops.varbits_index(dev(bits))
+    assert np.array_equal(host(off_d, np.uint32), off) and pb_d == pb
+    bbuf = torch.zeros(G + 16, dtype=torch.uint8, device="cuda")
+    bbuf[1:G + 1] = dev(bits)
+    obuf = torch.full((G + 4,), -1, dtype=torch.int32, device="cuda")
+    pbt = torch.empty(4, dtype=torch.int64, device="cuda")
+    cq.cq_varbits_index(bbuf[1:G + 1], obuf[1:G + 1], pbt)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(obuf[1:G + 1], np.uint32), off) and [int(v) for v in pbt.cpu()] == pb
+    assert int(obuf[0].item()) == -1 and int(obuf[G + 1].item()) == -1
+    rng = np.random.default_rng(G)
+    bad = bits.copy()
+    idx = rng.choice(G, G // 97 + 1, replace=False)
+    bad[idx] = rng.choice(np.array([0, 3, 5, 16, 255], np.uint8), idx.size)
+    valid = np.ones(G, bool)
+    valid[idx] = False
+    off_v, pb_v = co.varbits_index(bits[valid])
+    off_b, pb_b = ops.varbits_index(dev(bad))
+    got = host(off_b, np.uint32)
+    assert np.all(got[~valid] == 0) and np.array_equal(got[valid], off_v) and pb_b == pb_v
+
+
 # ---- projection ---------------------------------------------------------------------------------
 
 def _residual_cases(scale, seed):
