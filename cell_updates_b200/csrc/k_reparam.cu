@@ -16,17 +16,21 @@
 // Backward, straight through the final rounding: dL/dtheta = RN(RN(dL/dr * c_dt) * phi'),
 // phi' = (1 + t^2)^(-3/2) = RN(RN(1 / d) / q), and 0 for a NaN or saturated theta.
 //
-// Layout: one lane per eight weights (32 bytes of theta), two such units in flight per lane and
-// four CTAs of 256 threads per SM (more warps hide the long dependent sequences of the correctly
-// rounded square root and division better than more units per lane: the backward pass went from
-// 66 to 97 % of HBM); the eight lanes of a 64-weight group share its scale. Streaming.
+// Layout: one lane per eight weights (32 bytes of theta); the eight lanes of a 64-weight group
+// share its scale. Streaming. The backward pass keeps two such units in flight per lane at four
+// CTAs of 256 threads per SM (more warps hide the long dependent sequences of the correctly
+// rounded square root and divisions better than more units per lane: it went from 66 to 97 % of
+// HBM); the forward pass, with one division fewer per weight, runs one unit per lane at six CTAs
+// per SM (74.5 % of HBM against 72.5 % in the backward pass's shape, and 65 % at four CTAs).
 #include "cq_async.cuh"
 
 namespace cq {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 2;
+constexpr int kUnroll = 2;          // backward: units in flight per lane, four CTAs per SM
+constexpr int kFwdUnroll = 1;       // forward: one unit per lane, kFwdCtas CTAs per SM
+constexpr int kFwdCtas = 6;          // and the grid's CTAs per SM
 constexpr float kSat = 0x1p32f;
 
 __device__ __forceinline__ float cell_bound(uint16_t s16, bool bf16) {
@@ -60,15 +64,15 @@ __device__ __forceinline__ void store8(float *p, int64_t u, const float v[8]) {
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kThreads, kFwdCtas)
 reparam_kernel(const float *__restrict__ theta, const uint16_t *__restrict__ scale, int64_t n_units,
                void *__restrict__ r) {
   pdl_wait();
   const int64_t step = static_cast<int64_t>(gridDim.x) * kThreads;
-  for (int64_t u0 = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; u0 < n_units; u0 += kUnroll * step) {
-    float t[kUnroll][8], c[kUnroll];
+  for (int64_t u0 = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; u0 < n_units; u0 += kFwdUnroll * step) {
+    float t[kFwdUnroll][8], c[kFwdUnroll];
 #pragma unroll
-    for (int k = 0; k < kUnroll; ++k) {
+    for (int k = 0; k < kFwdUnroll; ++k) {
       const int64_t u = u0 + k * step;
       if (u < n_units) {
         load8(theta, u, t[k]);
@@ -76,7 +80,7 @@ reparam_kernel(const float *__restrict__ theta, const uint16_t *__restrict__ sca
       }
     }
 #pragma unroll
-    for (int k = 0; k < kUnroll; ++k) {
+    for (int k = 0; k < kFwdUnroll; ++k) {
       const int64_t u = u0 + k * step;
       if (u >= n_units) continue;
       float v[8];
@@ -126,9 +130,9 @@ reparam_grad_kernel(const float *__restrict__ theta, const uint16_t *__restrict_
   }
 }
 
-int grid_for(int64_t units) {
-  const int64_t need = (units + kUnroll * kThreads - 1) / (kUnroll * kThreads);
-  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+int grid_for(int64_t units, int unroll, int per_sm) {
+  const int64_t need = (units + unroll * kThreads - 1) / (unroll * kThreads);
+  const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
   return static_cast<int>(need < cap ? need : cap);
 }
 
@@ -138,7 +142,7 @@ cq_status launch_reparam(const float *theta, const uint16_t *scale, int64_t n, v
                          cudaStream_t s) {
   if (n == 0) return CQ_OK;
   const int64_t units = n / 8;
-  const dim3 grid(grid_for(units));
+  const dim3 grid(grid_for(units, kFwdUnroll, kFwdCtas));
   const cudaError_t e = dt == CQ_BF16 ? launch_pdl(reparam_kernel<true>, grid, dim3(kThreads), 0, s, theta, scale,
                                                    units, r)
                                       : launch_pdl(reparam_kernel<false>, grid, dim3(kThreads), 0, s, theta, scale,
@@ -152,7 +156,7 @@ cq_status launch_reparam_grad(const float *theta, const uint16_t *scale, const f
                               float *grad_theta, cudaStream_t s) {
   if (n == 0) return CQ_OK;
   const int64_t units = n / 8;
-  const dim3 grid(grid_for(units));
+  const dim3 grid(grid_for(units, kUnroll, 8));   // two rounds of four resident CTAs per SM
   const cudaError_t e = dt == CQ_BF16 ? launch_pdl(reparam_grad_kernel<true>, grid, dim3(kThreads), 0, s, theta,
                                                    scale, grad_r, units, grad_theta)
                                       : launch_pdl(reparam_grad_kernel<false>, grid, dim3(kThreads), 0, s, theta,
