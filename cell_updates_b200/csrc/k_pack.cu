@@ -120,28 +120,56 @@ pack_kernel(const uint8_t *__restrict__ codes, int64_t n_units, const uint8_t *_
   }
 }
 
+// Unpack takes kPackUnroll units per lane and iteration and issues each phase's loads for all of
+// them before using any (width and offset together, then the plane bytes, which depend on the
+// offset), so a lane overlaps several dependent round trips: with one unit per iteration it ran
+// at 1.6 TB/s on 2048x8192 (13.9 us; 12.4 us unrolled).
+constexpr int kPackUnroll = 4;
+
 __global__ void __launch_bounds__(kThreads)
 unpack_kernel(uint8_t *__restrict__ codes, int64_t n_units, const uint8_t *__restrict__ bits,
               const uint32_t *__restrict__ offset, Planes planes) {
-  for (int64_t u = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; u < n_units;
-       u += static_cast<int64_t>(gridDim.x) * kThreads) {
-    const int64_t g = u >> 3;
-    const int sub = static_cast<int>(u & 7);
-    int b = 4;
-    const uint8_t *base;
-    uint64_t v = 0;
-    if (bits) {
-      b = __ldg(bits + g);
-      const uint32_t o = width_ok(b) ? __ldg(offset + g) : 0u;
-      if (width_ok(b) && CQ_CHECK(o % (8u * b) == 0u && static_cast<int64_t>(o / (8u * b)) <= g, 0x0202u)) {
-        base = planes.of(b) + o;
-        v = unpack8(load_bytes(base + sub * b, b), b);
+  pdl_wait();                     // the planes and the map come from earlier work; codes is written
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kThreads;
+  for (int64_t u0 = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; u0 < n_units;
+       u0 += kPackUnroll * step) {
+    int b[kPackUnroll];
+    uint32_t o[kPackUnroll];
+#pragma unroll
+    for (int k = 0; k < kPackUnroll; ++k) {
+      const int64_t u = u0 + k * step;
+      b[k] = 4;
+      o[k] = 0;
+      if (bits && u < n_units) {
+        b[k] = __ldg(bits + (u >> 3));
+        o[k] = __ldg(offset + (u >> 3));
       }
-    } else {
-      base = planes.p[2] + g * 32;
-      v = unpack8(load_bytes(base + sub * 4, 4), 4);
     }
-    reinterpret_cast<uint2 *>(codes)[u] = make_uint2(static_cast<uint32_t>(v), static_cast<uint32_t>(v >> 32));
+    uint64_t v[kPackUnroll];
+#pragma unroll
+    for (int k = 0; k < kPackUnroll; ++k) {
+      const int64_t u = u0 + k * step;
+      v[k] = 0;
+      if (u >= n_units) continue;
+      const int64_t g = u >> 3;
+      const int sub = static_cast<int>(u & 7);
+      if (bits) {
+        if (width_ok(b[k]) &&
+            CQ_CHECK(o[k] % (8u * b[k]) == 0u && static_cast<int64_t>(o[k] / (8u * b[k])) <= g, 0x0202u))
+          v[k] = load_bytes(planes.of(b[k]) + o[k] + sub * b[k], b[k]);
+        else
+          b[k] = 0;                  // no group here: the codes are written as zeros
+      } else {
+        v[k] = load_bytes(planes.p[2] + g * 32 + sub * 4, 4);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kPackUnroll; ++k) {
+      const int64_t u = u0 + k * step;
+      if (u >= n_units) break;
+      const uint64_t c = b[k] ? unpack8(v[k], b[k]) : 0ull;
+      reinterpret_cast<uint2 *>(codes)[u] = make_uint2(static_cast<uint32_t>(c), static_cast<uint32_t>(c >> 32));
+    }
   }
 }
 
@@ -387,6 +415,8 @@ cq_status launch_pack(const uint8_t *codes, int64_t G, const uint8_t *bits, cons
     return launch_check("cq_pack_varbits");
   }
   Planes P{{plane[0], plane[1], plane[2], plane[3]}};
+  // an ordinary launch, one unit per lane and iteration: unrolled like unpack and launched as a
+  // programmatic dependent, pack measured slower (9.9 -> 11.6 us on 2048x8192)
   pack_kernel<<<grid_for(G * 8), kThreads, 0, s>>>(codes, G * 8, bits, offset, P);
   return launch_check("cq_pack_varbits");
 }
@@ -396,7 +426,10 @@ cq_status launch_unpack(const cq_qweight &qw, uint8_t *codes, cudaStream_t s) {
   if (G == 0) return CQ_OK;
   Planes P{{const_cast<uint8_t *>(qw.plane[0]), const_cast<uint8_t *>(qw.plane[1]),
             const_cast<uint8_t *>(qw.plane[2]), const_cast<uint8_t *>(qw.plane[3])}};
-  unpack_kernel<<<grid_for(G * 8), kThreads, 0, s>>>(codes, G * 8, qw.bits, qw.offset, P);
+  cq_status st = cuda_check(launch_pdl(unpack_kernel, dim3(grid_for((G * 8 + kPackUnroll - 1) / kPackUnroll)),
+                                       dim3(kThreads), 0, s, codes, G * 8, qw.bits, qw.offset, P),
+                            "cq_unpack_varbits");
+  if (st != CQ_OK) return st;
   return launch_check("cq_unpack_varbits");
 }
 
