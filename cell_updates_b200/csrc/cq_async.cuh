@@ -104,13 +104,20 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 
 // result words set to zero by one thread (either may be NULL) before the kernel that
 // accumulates into them, which is launched as this kernel's programmatic dependent (one copy
-// per translation unit)
+// per translation unit). Itself launched as a programmatic dependent (launch_clear_results): it
+// waits for the kernel before it, and only then lets its dependent start, so a dependent that
+// reads its inputs before its own wait never sees them before their producer has finished.
 static __global__ void clear_results_kernel(uint32_t *w32, unsigned long long *w64) {
+  pdl_wait();
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
     if (w32) *w32 = 0u;
     if (w64) *w64 = 0ull;
   }
+}
+
+static inline cudaError_t launch_clear_results(uint32_t *w32, unsigned long long *w64, cudaStream_t s) {
+  return launch_pdl(clear_results_kernel, dim3(1), dim3(32), 0, s, w32, w64);
 }
 
 // 2-D tiled TMA load into this CTA's shared memory, completing on an mbarrier (no multicast)

@@ -257,7 +257,10 @@ __device__ __forceinline__ bool walk_seg_end(const Walk &w, int P, int64_t it_en
 __global__ void __launch_bounds__(kPrepThreads)
 gemm_prep_kernel(const uint16_t *__restrict__ x, int64_t K, uint16_t *__restrict__ x16, float *__restrict__ xmul,
                  float *__restrict__ y, int64_t N, uint32_t *__restrict__ status) {
-  pdl_launch_dependents();     // the GEMM may set up (barriers, tensor memory, code loads) meanwhile
+  pdl_wait();                  // x, and the earlier readers of x16, xmul, y and the status word
+  // the GEMM may set up (barriers, tensor memory, code loads) meanwhile: only after the wait, so
+  // its early code loads never overtake the codes' producer
+  pdl_launch_dependents();
   __shared__ uint32_t red[kPrepThreads / 32];
   const int64_t i = blockIdx.y;
   const uint4 *xr = reinterpret_cast<const uint4 *>(x + i * K);
@@ -735,9 +738,12 @@ cq_status launch_nt(const cq_qweight &qw, const void *x, int m, float *y, uint8_
   {
     const int64_t want = (2 * static_cast<int64_t>(sm_count()) + m - 1) / m;
     const int64_t splits = want < 1 ? 1 : want > 64 ? 64 : want;
-    gemm_prep_kernel<<<dim3(static_cast<unsigned>(splits), static_cast<unsigned>(m)), kPrepThreads, 0, s>>>(
-        static_cast<const uint16_t *>(x), K, x16, xmul, y, N, clear_status ? status : nullptr);
-    cq_status st = launch_check("cq_dequant_gemm: preparation");
+    cq_status st = cuda_check(launch_pdl(gemm_prep_kernel, dim3(static_cast<unsigned>(splits), static_cast<unsigned>(m)),
+                                         dim3(kPrepThreads), 0, s, static_cast<const uint16_t *>(x), K, x16, xmul, y, N,
+                                         clear_status ? status : nullptr),
+                              "cq_dequant_gemm: preparation");
+    if (st != CQ_OK) return st;
+    st = launch_check("cq_dequant_gemm: preparation");
     if (st != CQ_OK) return st;
   }
   // 2. the GEMM, allowed to start while the preparation runs (it waits for it where it must)

@@ -111,8 +111,10 @@ project_kernel(void *__restrict__ rv, const uint16_t *__restrict__ scale, int64_
 cq_status launch_project(void *r, cq_dtype dt, const uint16_t *scale, int64_t n, uint64_t *n_clamped,
                          cudaStream_t s) {
   if (n_clamped) {
-    clear_results_kernel<<<1, 32, 0, s>>>(nullptr, reinterpret_cast<unsigned long long *>(n_clamped));
-    cq_status st = launch_check("cq_project_residual: clear count");
+    cq_status st = cuda_check(launch_clear_results(nullptr, reinterpret_cast<unsigned long long *>(n_clamped), s),
+                              "cq_project_residual: clear count");
+    if (st != CQ_OK) return st;
+    st = launch_check("cq_project_residual: clear count");
     if (st != CQ_OK) return st;
   }
   if (n == 0) return CQ_OK;

@@ -238,8 +238,9 @@ template <bool kResid>
 cq_status launch_quantize_impl(float *w, int64_t G, const uint8_t *bits, int uniform_b, uint8_t *codes,
                                uint16_t *scale, uint8_t *zero, uint32_t *status, cudaStream_t s, const char *who) {
   if (status) {
-    clear_results_kernel<<<1, 32, 0, s>>>(status, nullptr);
-    cq_status st = launch_check(who);
+    cq_status st = cuda_check(launch_clear_results(status, nullptr, s), who);
+    if (st != CQ_OK) return st;
+    st = launch_check(who);
     if (st != CQ_OK) return st;
   }
   if (G == 0) return CQ_OK;

@@ -42,9 +42,12 @@ struct VerifyArgs {
 };
 
 // the results start at 0 mismatches and first index -1; one thread, then the verify grid
-// (launched as its programmatic dependent) may start
+// (launched as its programmatic dependent) may start. Itself a programmatic dependent: it lets
+// the verify grid start only after its own wait, when the kernel before it (which may have
+// written the residual the verify grid reads) has finished.
 __global__ void verify_clear_kernel(unsigned long long *mism, unsigned long long *first,
                                     unsigned long long *mism0, unsigned long long *first0) {
+  pdl_wait();
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
     *mism = 0ull;
@@ -461,11 +464,15 @@ cq_status launch_verify_impl(const cq_qweight &qw, int64_t first_w, int64_t n_w,
     cq_status st = cuda_check(cudaMemsetAsync(flags, 0, static_cast<size_t>((n_groups + 31) / 32) * 4, s), who);
     if (st != CQ_OK) return st;
   }
-  verify_clear_kernel<<<1, 32, 0, s>>>(reinterpret_cast<unsigned long long *>(mism),
-                                       reinterpret_cast<unsigned long long *>(first_bad),
-                                       reinterpret_cast<unsigned long long *>(mism0),
-                                       reinterpret_cast<unsigned long long *>(first0));
-  cq_status st = launch_check(who);
+  // the library-wide launcher (this file's launch_pdl above takes verify arguments)
+  cq_status st = cuda_check(::cq::launch_pdl(verify_clear_kernel, dim3(1), dim3(32), 0, s,
+                                             reinterpret_cast<unsigned long long *>(mism),
+                                             reinterpret_cast<unsigned long long *>(first_bad),
+                                             reinterpret_cast<unsigned long long *>(mism0),
+                                             reinterpret_cast<unsigned long long *>(first0)),
+                            who);
+  if (st != CQ_OK) return st;
+  st = launch_check(who);
   if (st != CQ_OK || n_w == 0) return st;
   VerifyArgs a;
   a.bits = qw.bits;
