@@ -20,6 +20,8 @@
 //  * gemv_generic: any format (per-group widths), fp32 or bf16 x, with a residual; one warp
 //    per row, fp32 CUDA-core math. Used for residual-carrying weights only: without a residual,
 //    per-group widths and fp32 activations go to the tensor-core kernel of k_rrq.cu.
+#include <cooperative_groups.h>
+
 #include "cq_async.cuh"
 
 namespace cq {
@@ -751,16 +753,26 @@ struct RSegs {
   int64_t tile0[kMaxSegs + 1];              // tile0[count] = all tiles; unused entries = INT64_MAX
 };
 
+// SPLIT = 2 (matrices with no more tiles than SMs): a thread-block cluster of two CTAs owns a
+// tile, each CTA taking half of the row's groups, so twice as many SMs stream the matrix and each
+// CTA's run is half as long. The two CTAs' tile sums meet in the first CTA's hands through
+// distributed shared memory between two cluster barriers (hardware barriers of co-scheduled
+// CTAs, nothing polled), in a fixed order, so y stays deterministic.
+template <int SPLIT>
 __global__ void __launch_bounds__(kRThreads, 2)
 gemv4r_kernel(const __grid_constant__ RSegs sg, const __nv_bfloat16 *__restrict__ x, int m, int64_t K) {
   __shared__ float red[kRWarps][kTileRows * 8];
+  __shared__ float part[kTileRows * 8];          // SPLIT > 1: this CTA's tile sums
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gid = lane >> 2, tig = lane & 3;
   const int KG = static_cast<int>(K >> 6);
-  const int g0 = KG * warp / kRWarps, g1 = KG * (warp + 1) / kRWarps;
+  const int rank = SPLIT > 1 ? static_cast<int>(cooperative_groups::this_cluster().block_rank()) : 0;
+  const int64_t unit = blockIdx.x / SPLIT, n_units = gridDim.x / SPLIT;
+  const int q0 = KG * rank / SPLIT, q1 = KG * (rank + 1) / SPLIT;     // this CTA's groups
+  const int g0 = q0 + (q1 - q0) * warp / kRWarps, g1 = q0 + (q1 - q0) * (warp + 1) / kRWarps;
   const int64_t n_tiles = sg.tile0[kMaxSegs];
-  for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+  for (int64_t tile = unit; tile < n_tiles; tile += n_units) {
     const int s = (tile >= sg.tile0[1]) + (tile >= sg.tile0[2]) + (tile >= sg.tile0[3]);
     const uint8_t *plane = seg_pick(sg.plane, s);
     const uint16_t *scale = seg_pick(sg.scale, s), *res = seg_pick(sg.res, s);
@@ -781,7 +793,7 @@ gemv4r_kernel(const __grid_constant__ RSegs sg, const __nv_bfloat16 *__restrict_
     RGroup a, b;
     if (g0 < g1) rgroup_load_w(a, c0, c1, r0, r1, sc0, sc1, zp0, zp1, g0);
     if (g0 + 1 < g1) rgroup_load_w(b, c0, c1, r0, r1, sc0, sc1, zp0, zp1, g0 + 1);
-    if (tile == blockIdx.x) pdl_wait();
+    if (tile == unit) pdl_wait();
     if (g0 < g1) rgroup_load_x(a, xr, g0);
     if (g0 + 1 < g1) rgroup_load_x(b, xr, g0 + 1);
     for (int g = g0; g < g1; g += 2) {
@@ -804,11 +816,20 @@ gemv4r_kernel(const __grid_constant__ RSegs sg, const __nv_bfloat16 *__restrict_
     rw[(2 * tig) * 16 + gid + 8] = acc[2];
     rw[(2 * tig + 1) * 16 + gid + 8] = acc[3];
     __syncthreads();
+    float v = 0.0f;
     if (threadIdx.x < 16 * m) {
-      const int row = threadIdx.x & 15, col = threadIdx.x >> 4;
-      float v = 0.0f;
 #pragma unroll
       for (int w = 0; w < kRWarps; ++w) v += red[w][threadIdx.x];
+    }
+    if (SPLIT > 1) {
+      if (threadIdx.x < 16 * m) part[threadIdx.x] = v;
+      cooperative_groups::this_cluster().sync();        // every CTA's sums are in place
+      if (rank == 0 && threadIdx.x < 16 * m)
+        for (int r = 1; r < SPLIT; ++r) v += cooperative_groups::this_cluster().map_shared_rank(part, r)[threadIdx.x];
+      cooperative_groups::this_cluster().sync();        // read before any CTA rewrites its sums
+    }
+    if (rank == 0 && threadIdx.x < 16 * m) {
+      const int row = threadIdx.x & 15, col = threadIdx.x >> 4;
       const int64_t rr = lrow0 + row;
       if (rr < N) seg_pick(sg.y, s)[static_cast<int64_t>(col) * N + rr] = v;
     }
@@ -845,9 +866,28 @@ cq_status launch_gemv4r(const cq_qweight *const *qws, int count, const void *x, 
   }
   sg.tile0[kMaxSegs] = t;
   if (count < kMaxSegs) sg.tile0[count] = t;
+  if (t <= sm_count()) {
+    // a cluster of two CTAs per tile (see gemv4r_kernel), one tile per cluster
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * t));
+    cfg.blockDim = dim3(kRThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cuda_check(cudaLaunchKernelEx(&cfg, gemv4r_kernel<2>, sg, static_cast<const __nv_bfloat16 *>(x), m,
+                                         qws[0]->cols),
+                      "cq_dequant_gemv (residual, split)");
+  }
   const int64_t cap = static_cast<int64_t>(sm_count()) * 2;
   const int64_t grid = t < cap ? t : cap;
-  return cuda_check(launch_pdl(gemv4r_kernel, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), 0, s, sg,
+  return cuda_check(launch_pdl(gemv4r_kernel<1>, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), 0, s, sg,
                                static_cast<const __nv_bfloat16 *>(x), m, qws[0]->cols),
                     "cq_dequant_gemv (residual)");
 }
