@@ -663,8 +663,9 @@ cq_status launch_gemv4_segs(const cq_qweight *const *qws, int count, const void 
 // fixed 4-bit codes with a bf16 residual: the CellFill served weights W = s (q - z) + r
 // ------------------------------------------------------------------------------------
 // [CF] the served weight carries the residual, so decode streams 0.5 B of codes and 2 B of
-// residual per weight. A CTA of 8 warps owns one 16-row tile; warp w takes the w-th eighth of
-// the row's groups, so each warp streams contiguous runs of codes and residual of 16 rows.
+// residual per weight. A CTA of 8 warps owns one 16-row tile (or, when the tiles do not fill
+// the SMs, half of its groups, in a two-CTA cluster); warp w takes the w-th eighth of the CTA's
+// groups, so each warp streams contiguous runs of codes and residual of 16 rows.
 // Per group, on tensor cores (mma.sync m16n8k16, fp32 accumulation, exact products):
 //   codes:    sum_k (128 + q) x  with 128 + q = bf16 0x4300 | q, minus (128 + z) sum_k x (the group
 //             sum of x from an MMA with an all-ones A), times s;
