@@ -156,7 +156,7 @@ cq_status launch_reparam_grad(const float *theta, const uint16_t *scale, const f
                               float *grad_theta, cudaStream_t s) {
   if (n == 0) return CQ_OK;
   const int64_t units = n / 8;
-  const dim3 grid(grid_for(units, kUnroll, 8));   // two rounds of four resident CTAs per SM
+  const dim3 grid(grid_for(units, kUnroll, 8));   // two waves of four resident CTAs per SM
   const cudaError_t e = dt == CQ_BF16 ? launch_pdl(reparam_grad_kernel<true>, grid, dim3(kThreads), 0, s, theta,
                                                    scale, grad_r, units, grad_theta)
                                       : launch_pdl(reparam_grad_kernel<false>, grid, dim3(kThreads), 0, s, theta,
