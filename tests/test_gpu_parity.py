@@ -126,11 +126,11 @@ def test_varbits_index_and_pack_bit_exact(G):
 
 
 @pytest.mark.parametrize("G", [262143, 262144, 262145, 600001, 1 << 20, (1 << 20) + 1, 1300001])
-def test_varbits_index_both_forms_unaligned_and_invalid(G):
-    """The index in both of its forms: one cluster launch up to 2^20 groups (rounds of 262144
-    groups) and three passes beyond; with the width map and the offsets off their 16-byte
-    boundaries (the element-wise paths); and with widths outside {1, 2, 4, 8}, which take no
-    bytes and get offset 0 while the valid groups keep the offsets of the valid subsequence."""
+def test_varbits_index_large_unaligned_and_invalid(G):
+    """The index's three chained passes over 64 to 318 tiles of 4096 groups (a ragged last tile
+    on both sides of the power-of-two sizes); with the width map and the offsets off their
+    16-byte boundaries; and with widths outside {1, 2, 4, 8}, which take no bytes and get offset
+    0 while the valid groups keep the offsets of the valid subsequence."""
     bits = synth.vbq_bits(G, seed=G)
     off, pb = co.varbits_index(bits)
     off_d, pb_d = ops.varbits_index(dev(bits))
